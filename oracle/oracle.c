@@ -1,0 +1,898 @@
+/*
+ * oracle.c - TEST INFRASTRUCTURE ONLY.
+ *
+ * A plain, slow, obviously-correct CPU reference of one small-batch decode
+ * step of a transformer decoder, in fp64 arithmetic.  It exists to check the
+ * GPU megakernel; nothing in the product library links, loads or calls it.
+ * Only the test-suite, the smoke check and the bench's CPU-baseline leg use
+ * it.  It shares no code with the CUDA path: the single shared piece is the
+ * seeded input generator (synth/synth.h), which holds none of the method's
+ * arithmetic.
+ *
+ * What it computes (source: "700 TPS on Kimi K3: A Case for TPU Megakernels",
+ * Inferact blog, section "Why megakernels?" and "Our Kimi K3 megakernel":
+ * the megakernel evaluates the whole decoder step - attention, router,
+ * shared expert, routed experts - in one program; it changes the schedule,
+ * not the result).  So the oracle is the textbook pre-norm decoder forward
+ * pass, step by step, with no blocking or fusion:
+ *
+ *   x = E[token]                                  (bf16 table widened exactly)
+ *   per layer:
+ *     h = RMSNorm(x) * g_attn
+ *     q, k, v = W_qkv h ; RoPE(q, k) at the token's position
+ *     cache[pos] = bf16(k), bf16(v)               (KV stored in bf16, RNE)
+ *     o = softmax(q K^T / sqrt(d)) V  over cached positions 0..pos (GQA)
+ *     x += W_o o
+ *     h = RMSNorm(x) * g_ffn
+ *     x += W_d (silu(W_g h) * (W_u h))            (dense)
+ *       or shared experts + sum_j w_j Expert_{idx_j}(h) (top-k softmax router,
+ *          weights renormalised over the selected k)
+ *   logits = W_lm RMSNorm(x) * g_final ; token = argmax (ties -> lower index)
+ *
+ * Multi-head latent attention (the post's Kimi K3 layers choose MLA by layer
+ * index; its math is not printed there): per head q = [q_nope | q_rope],
+ * latent c = W_dkv h plus one shared rope key k_r; cache holds [c | k_r];
+ * score = (q_nope . (W_uk,h c_t) + q_rope . k_r,t) / sqrt(dn + dr);
+ * o_h = sum_t p_t W_uv,h c_t.  The explicit form is the definition; the
+ * absorbed form (W_uk,h^T q_nope) . c_t is the same number by associativity
+ * and is offered for full-size runs, with a pin that the two agree.
+ *
+ * Speculative verify (section "DSpark": one launch evaluates 1 anchor and 7
+ * proposed continuations): Q consecutive positions of one sequence in one
+ * step, causal within the chunk; greedy acceptance.
+ *
+ * Readings where the post is silent (plainest choice): RMSNorm eps inside the
+ * sqrt, gain multiplies directly; rotate-half RoPE pairs (i, i + d/2) with
+ * inv_freq_i = theta^(-2i/d); no biases, no QK-norm, no soft-cap; untied LM
+ * head; silu(z) = z / (1 + e^-z); every MoE layer routes; routed scale 1;
+ * shared expert added with weight 1; fp8 = OCP E4M3 with one fp32 scale per
+ * 128x128 block of each [out, in] matrix.
+ *
+ * Build: gcc -O2 -fopenmp -ffp-contract=off -shared -fPIC (see build.py).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <float.h>
+
+#include "../synth/synth.h"
+
+/* ------------------------------------------------------------------------ */
+/* configuration                                                             */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+  int32_t layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
+  int32_t n_routed, n_shared, top_k, expert_ffn;
+  int32_t kv_lora_rank, rope_dim; /* kv_lora_rank > 0 selects MLA */
+  int32_t expert_fp8;
+  int32_t max_seqs, max_ctx;
+  double rope_theta, rms_eps;
+  double w_sigma, router_sigma, gain_sigma, kv_sigma, fp8_block_base;
+  uint64_t seed;
+} orc_cfg;
+
+typedef struct {
+  orc_cfg c;
+  uint16_t* kv_k;   /* [L][S][Hkv][Tmax][d]  bf16 bits (GQA) */
+  uint16_t* kv_v;
+  uint16_t* kv_lat; /* [L][S][Tmax][R + dr]   bf16 bits (MLA) */
+} orc_model;
+
+int32_t orc_argmax(int64_t n, const double* r, double* margin);
+
+/* ------------------------------------------------------------------------ */
+/* number formats                                                            */
+/* ------------------------------------------------------------------------ */
+
+static double bf16_to_double(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return (double)f;
+}
+
+/* double -> bf16, round to nearest even on the exact value. */
+static uint16_t double_to_bf16(double v) {
+  /* bf16 has 8 significant bits; find the two neighbours and pick. */
+  if (v == 0.0) return signbit(v) ? 0x8000 : 0;
+  int e;
+  double m = frexp(fabs(v), &e);          /* |v| = m * 2^e, m in [0.5, 1) */
+  double scaled = ldexp(m, 8);            /* in [128, 256) */
+  double fl = floor(scaled);
+  double frac = scaled - fl;
+  double q = fl;
+  if (frac > 0.5 || (frac == 0.5 && fmod(fl, 2.0) != 0.0)) q = fl + 1.0;
+  double r = ldexp(q, e - 8);
+  float f = (float)r; /* exact: r has at most 8 significant bits */
+  if (v < 0) f = -f;
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  return (uint16_t)(u >> 16);
+}
+
+/* OCP FP8 E4M3 decode: bias 7, subnormals 2^-6 * m/8, S.1111.111 = NaN. */
+double orc_e4m3_value(uint8_t code) {
+  int s = code >> 7, e = (code >> 3) & 0xF, m = code & 7;
+  double v;
+  if (e == 0xF && m == 7) return NAN;
+  if (e == 0) v = ldexp((double)m / 8.0, -6);
+  else v = ldexp(1.0 + (double)m / 8.0, e - 7);
+  return s ? -v : v;
+}
+
+uint16_t orc_bf16_round(double v) { return double_to_bf16(v); }
+
+/* ------------------------------------------------------------------------ */
+/* weight sources: an explicit array or a seeded synthetic tensor            */
+/* ------------------------------------------------------------------------ */
+
+enum { ORC_MAT_ARRAY = 0, ORC_MAT_BF16 = 1, ORC_MAT_FP8 = 2, ORC_MAT_GAIN = 3 };
+
+typedef struct {
+  int64_t rows, cols;
+  int32_t kind;
+  const double* a; /* ORC_MAT_ARRAY: row-major [rows][cols] */
+  uint64_t key, skey;
+  float scale, base;
+} orc_mat;
+
+static void mat_row(const orc_mat* W, int64_t r, double* out) {
+  int64_t C = W->cols;
+  switch (W->kind) {
+    case ORC_MAT_ARRAY:
+      memcpy(out, W->a + r * C, (size_t)C * sizeof(double));
+      break;
+    case ORC_MAT_BF16:
+      for (int64_t c = 0; c < C; ++c) out[c] = bf16_to_double(syn_bf16_normal(W->key, (uint64_t)(r * C + c), W->scale));
+      break;
+    case ORC_MAT_GAIN:
+      for (int64_t c = 0; c < C; ++c) out[c] = bf16_to_double(syn_bf16_gain(W->key, (uint64_t)c, W->scale));
+      break;
+    case ORC_MAT_FP8: {
+      int64_t nbc = (C + 127) / 128;
+      for (int64_t c = 0; c < C; ++c) {
+        double w = orc_e4m3_value(syn_e4m3_normal(W->key, (uint64_t)(r * C + c), W->scale));
+        double s = (double)syn_block_scale(W->skey, (uint64_t)((r / 128) * nbc + c / 128), W->base);
+        out[c] = w * s;
+      }
+      break;
+    }
+  }
+}
+
+/* y[m][r] = sum_c W[r][c] x[m][c] for m < M.  fp64 accumulation, c ascending. */
+static void matvec(const orc_mat* W, int M, const double* x, double* y) {
+  int64_t R = W->rows, C = W->cols;
+#pragma omp parallel
+  {
+    double* row = (double*)malloc((size_t)C * sizeof(double));
+#pragma omp for schedule(static)
+    for (int64_t r = 0; r < R; ++r) {
+      mat_row(W, r, row);
+      for (int m = 0; m < M; ++m) {
+        const double* xm = x + (int64_t)m * C;
+        double acc = 0.0;
+        for (int64_t c = 0; c < C; ++c) acc += row[c] * xm[c];
+        y[(int64_t)m * R + r] = acc;
+      }
+    }
+    free(row);
+  }
+}
+
+void orc_matvec_dense(int64_t rows, int64_t cols, const double* W, int M, const double* x, double* y) {
+  orc_mat m = {rows, cols, ORC_MAT_ARRAY, W, 0, 0, 0.f, 0.f};
+  matvec(&m, M, x, y);
+}
+
+/* ------------------------------------------------------------------------ */
+/* building blocks                                                           */
+/* ------------------------------------------------------------------------ */
+
+/* RMSNorm: y = x / sqrt(mean(x^2) + eps) * g. */
+void orc_rmsnorm(int n, const double* x, const double* g, double eps, double* y) {
+  double ss = 0.0;
+  for (int i = 0; i < n; ++i) ss += x[i] * x[i];
+  double inv = 1.0 / sqrt(ss / (double)n + eps);
+  for (int i = 0; i < n; ++i) y[i] = x[i] * inv * g[i];
+}
+
+/* Rotate-half RoPE on a d-vector at position pos: pairs (i, i + d/2),
+ * angle = pos * theta^(-2i/d). */
+void orc_rope_apply(int d, double* x, int32_t pos, double theta) {
+  int h = d / 2;
+  for (int i = 0; i < h; ++i) {
+    double inv_freq = pow(theta, -2.0 * (double)i / (double)d);
+    double ang = (double)pos * inv_freq;
+    double c = cos(ang), s = sin(ang);
+    double a = x[i], b = x[i + h];
+    x[i] = a * c - b * s;
+    x[i + h] = a * s + b * c;
+  }
+}
+
+/* Numerically safe softmax: subtract the max, exponentiate, normalise. */
+void orc_softmax(int n, const double* x, double* y) {
+  double mx = -INFINITY;
+  for (int i = 0; i < n; ++i) mx = x[i] > mx ? x[i] : mx;
+  double s = 0.0;
+  for (int i = 0; i < n; ++i) { y[i] = exp(x[i] - mx); s += y[i]; }
+  for (int i = 0; i < n; ++i) y[i] /= s;
+}
+
+/* One query head against T keys/values (row-major [T][d]):
+ * out = softmax(scale * q.K^T) V. */
+void orc_attention_head(int T, int d, const double* q, const double* K, const double* V,
+                        double scale, double* out) {
+  double* sc = (double*)malloc((size_t)T * sizeof(double));
+  double* p = (double*)malloc((size_t)T * sizeof(double));
+  for (int t = 0; t < T; ++t) {
+    double a = 0.0;
+    for (int i = 0; i < d; ++i) a += q[i] * K[(int64_t)t * d + i];
+    sc[t] = a * scale;
+  }
+  orc_softmax(T, sc, p);
+  for (int i = 0; i < d; ++i) out[i] = 0.0;
+  for (int t = 0; t < T; ++t)
+    for (int i = 0; i < d; ++i) out[i] += p[t] * V[(int64_t)t * d + i];
+  free(sc);
+  free(p);
+}
+
+double orc_silu(double z) { return z / (1.0 + exp(-z)); }
+
+/* Router: softmax over all E logits, top-k by probability (a stable
+ * descending order: equal values keep the lower index first), weights
+ * renormalised over the selected k.  margin = logit gap at the boundary. */
+void orc_router_select(int E, int k, const double* logits, int32_t* idx, double* w, double* margin) {
+  double* p = (double*)malloc((size_t)E * sizeof(double));
+  int32_t* ord = (int32_t*)malloc((size_t)E * sizeof(int32_t));
+  orc_softmax(E, logits, p);
+  for (int i = 0; i < E; ++i) ord[i] = i;
+  /* insertion sort, stable, descending by logit (softmax is monotone) */
+  for (int i = 1; i < E; ++i) {
+    int32_t v = ord[i];
+    int j = i - 1;
+    while (j >= 0 && logits[ord[j]] < logits[v]) { ord[j + 1] = ord[j]; --j; }
+    ord[j + 1] = v;
+  }
+  double s = 0.0;
+  for (int j = 0; j < k; ++j) { idx[j] = ord[j]; s += p[ord[j]]; }
+  for (int j = 0; j < k; ++j) w[j] = p[ord[j]] / s;
+  if (margin) *margin = (k < E) ? logits[ord[k - 1]] - logits[ord[k]] : INFINITY;
+  free(p);
+  free(ord);
+}
+
+/* SwiGLU expert: y = W_d (silu(W_g x) * (W_u x)). */
+static void swiglu(const orc_mat* Wg, const orc_mat* Wu, const orc_mat* Wd, int M, const double* x, double* y) {
+  int64_t I = Wg->rows;
+  double* g = (double*)malloc((size_t)M * I * sizeof(double));
+  double* u = (double*)malloc((size_t)M * I * sizeof(double));
+  matvec(Wg, M, x, g);
+  matvec(Wu, M, x, u);
+  for (int64_t i = 0; i < (int64_t)M * I; ++i) g[i] = orc_silu(g[i]) * u[i];
+  matvec(Wd, M, g, y);
+  free(g);
+  free(u);
+}
+
+void orc_swiglu_dense(int H, int I, const double* Wg, const double* Wu, const double* Wd, int M,
+                      const double* x, double* y) {
+  orc_mat g = {I, H, ORC_MAT_ARRAY, Wg, 0, 0, 0.f, 0.f};
+  orc_mat u = {I, H, ORC_MAT_ARRAY, Wu, 0, 0, 0.f, 0.f};
+  orc_mat d = {H, I, ORC_MAT_ARRAY, Wd, 0, 0, 0.f, 0.f};
+  swiglu(&g, &u, &d, M, x, y);
+}
+
+/* MoE FFN for one token x[H]: shared experts (weight 1) + routed top-k. */
+static void moe_ffn(int H, int E, int k, int n_shared, const orc_mat* Wr,
+                    const orc_mat* sg, const orc_mat* su, const orc_mat* sd, /* [n_shared] */
+                    const orc_mat* eg, const orc_mat* eu, const orc_mat* ed, /* [E] */
+                    const double* x, double* y, int32_t* idx, double* w, double* margin) {
+  double* lg = (double*)malloc((size_t)E * sizeof(double));
+  double* t = (double*)malloc((size_t)H * sizeof(double));
+  matvec(Wr, 1, x, lg);
+  orc_router_select(E, k, lg, idx, w, margin);
+  for (int i = 0; i < H; ++i) y[i] = 0.0;
+  for (int j = 0; j < n_shared; ++j) {
+    swiglu(&sg[j], &su[j], &sd[j], 1, x, t);
+    for (int i = 0; i < H; ++i) y[i] += t[i];
+  }
+  for (int j = 0; j < k; ++j) {
+    int e = idx[j];
+    swiglu(&eg[e], &eu[e], &ed[e], 1, x, t);
+    for (int i = 0; i < H; ++i) y[i] += w[j] * t[i];
+  }
+  free(lg);
+  free(t);
+}
+
+/* Array form for pins: router [E][H]; experts gate/up [E][I][H], down [E][H][I];
+ * shared likewise with n_shared entries. */
+void orc_moe_ffn_dense(int H, int I, int E, int k, int n_shared, const double* Wr,
+                       const double* g, const double* u, const double* d,
+                       const double* shg, const double* shu, const double* shd,
+                       const double* x, double* y, int32_t* idx, double* w) {
+  orc_mat r = {E, H, ORC_MAT_ARRAY, Wr, 0, 0, 0.f, 0.f};
+  orc_mat* eg = (orc_mat*)calloc((size_t)E, sizeof(orc_mat));
+  orc_mat* eu = (orc_mat*)calloc((size_t)E, sizeof(orc_mat));
+  orc_mat* ed = (orc_mat*)calloc((size_t)E, sizeof(orc_mat));
+  orc_mat* sg = (orc_mat*)calloc((size_t)(n_shared + 1), sizeof(orc_mat));
+  orc_mat* su = (orc_mat*)calloc((size_t)(n_shared + 1), sizeof(orc_mat));
+  orc_mat* sd = (orc_mat*)calloc((size_t)(n_shared + 1), sizeof(orc_mat));
+  for (int e = 0; e < E; ++e) {
+    eg[e] = (orc_mat){I, H, ORC_MAT_ARRAY, g + (int64_t)e * I * H, 0, 0, 0.f, 0.f};
+    eu[e] = (orc_mat){I, H, ORC_MAT_ARRAY, u + (int64_t)e * I * H, 0, 0, 0.f, 0.f};
+    ed[e] = (orc_mat){H, I, ORC_MAT_ARRAY, d + (int64_t)e * H * I, 0, 0, 0.f, 0.f};
+  }
+  for (int j = 0; j < n_shared; ++j) {
+    sg[j] = (orc_mat){I, H, ORC_MAT_ARRAY, shg + (int64_t)j * I * H, 0, 0, 0.f, 0.f};
+    su[j] = (orc_mat){I, H, ORC_MAT_ARRAY, shu + (int64_t)j * I * H, 0, 0, 0.f, 0.f};
+    sd[j] = (orc_mat){H, I, ORC_MAT_ARRAY, shd + (int64_t)j * H * I, 0, 0, 0.f, 0.f};
+  }
+  moe_ffn(H, E, k, n_shared, &r, sg, su, sd, eg, eu, ed, x, y, idx, w, NULL);
+  free(eg); free(eu); free(ed); free(sg); free(su); free(sd);
+}
+
+/* MLA attention of one query row over T cached latent rows [c(R) | k_r(dr)].
+ * q_full: per head [q_nope(dn) | q_rope(dr)] (RoPE already applied).
+ * W_uk: [Hq*dn][R], W_uv: [Hq*dv][R].  out: [Hq*dv].
+ * explicit: score_h,t = q_nope.(W_uk,h c_t) + q_rope.k_r,t, v_h,t = W_uv,h c_t;
+ * absorbed: score via (W_uk,h^T q_nope).c_t and o_h = W_uv,h sum_t p_t c_t. */
+static void mla_attend(int Hq, int dn, int dr, int dv, int R, int T, const double* q_full,
+                       const double* lat /*[T][R+dr]*/, const double* Wuk, const double* Wuv,
+                       int absorbed, double* out) {
+  int W = R + dr;
+  double scale = 1.0 / sqrt((double)(dn + dr));
+#pragma omp parallel for schedule(dynamic)
+  for (int h = 0; h < Hq; ++h) {
+    const double* qn = q_full + (int64_t)h * (dn + dr);
+    const double* qr = qn + dn;
+    const double* uk = Wuk + (int64_t)h * dn * R;
+    const double* uv = Wuv + (int64_t)h * dv * R;
+    double* sc = (double*)malloc((size_t)T * sizeof(double));
+    double* p = (double*)malloc((size_t)T * sizeof(double));
+    double* o = out + (int64_t)h * dv;
+    if (!absorbed) {
+      double* kn = (double*)malloc((size_t)dn * sizeof(double));
+      for (int t = 0; t < T; ++t) {
+        const double* c = lat + (int64_t)t * W;
+        for (int i = 0; i < dn; ++i) {
+          double a = 0.0;
+          for (int r = 0; r < R; ++r) a += uk[(int64_t)i * R + r] * c[r];
+          kn[i] = a;
+        }
+        double s = 0.0;
+        for (int i = 0; i < dn; ++i) s += qn[i] * kn[i];
+        for (int i = 0; i < dr; ++i) s += qr[i] * c[R + i];
+        sc[t] = s * scale;
+      }
+      free(kn);
+      orc_softmax(T, sc, p);
+      for (int i = 0; i < dv; ++i) o[i] = 0.0;
+      double* vt = (double*)malloc((size_t)dv * sizeof(double));
+      for (int t = 0; t < T; ++t) {
+        const double* c = lat + (int64_t)t * W;
+        for (int i = 0; i < dv; ++i) {
+          double a = 0.0;
+          for (int r = 0; r < R; ++r) a += uv[(int64_t)i * R + r] * c[r];
+          vt[i] = a;
+        }
+        for (int i = 0; i < dv; ++i) o[i] += p[t] * vt[i];
+      }
+      free(vt);
+    } else {
+      double* ql = (double*)calloc((size_t)R, sizeof(double));
+      for (int i = 0; i < dn; ++i)
+        for (int r = 0; r < R; ++r) ql[r] += qn[i] * uk[(int64_t)i * R + r];
+      for (int t = 0; t < T; ++t) {
+        const double* c = lat + (int64_t)t * W;
+        double s = 0.0;
+        for (int r = 0; r < R; ++r) s += ql[r] * c[r];
+        for (int i = 0; i < dr; ++i) s += qr[i] * c[R + i];
+        sc[t] = s * scale;
+      }
+      orc_softmax(T, sc, p);
+      double* ol = (double*)calloc((size_t)R, sizeof(double));
+      for (int t = 0; t < T; ++t) {
+        const double* c = lat + (int64_t)t * W;
+        for (int r = 0; r < R; ++r) ol[r] += p[t] * c[r];
+      }
+      for (int i = 0; i < dv; ++i) {
+        double a = 0.0;
+        for (int r = 0; r < R; ++r) a += uv[(int64_t)i * R + r] * ol[r];
+        o[i] = a;
+      }
+      free(ql);
+      free(ol);
+    }
+    free(sc);
+    free(p);
+  }
+}
+
+void orc_mla_attention(int Hq, int dn, int dr, int dv, int R, int T, const double* q_full,
+                       const double* lat, const double* Wuk, const double* Wuv, int absorbed, double* out) {
+  mla_attend(Hq, dn, dr, dv, R, T, q_full, lat, Wuk, Wuv, absorbed, out);
+}
+
+/* Greedy acceptance of a verify step: tokens[0] is the anchor, tokens[1..n-1]
+ * the proposals, g[i] the greedy token after position i.  Accept the longest
+ * prefix of proposals that matches the greedy chain. */
+/* Greedy token: the largest logit, ties to the lower index; margin = top1 - top2. */
+int32_t orc_argmax(int64_t n, const double* r, double* margin) {
+  int64_t best = 0;
+  for (int64_t v = 1; v < n; ++v) if (r[v] > r[best]) best = v;
+  double second = -INFINITY;
+  for (int64_t v = 0; v < n; ++v) if (v != best && r[v] > second) second = r[v];
+  if (margin) *margin = r[best] - second;
+  return (int32_t)best;
+}
+
+int32_t orc_accept(int n, const int32_t* tokens, const int32_t* g) {
+  int32_t a = 0;
+  while (a + 1 < n && tokens[a + 1] == g[a]) ++a;
+  return a;
+}
+
+/* ------------------------------------------------------------------------ */
+/* model: synthetic weights from the seed                                    */
+/* ------------------------------------------------------------------------ */
+
+static orc_mat syn_mat(const orc_cfg* c, uint32_t kind, uint32_t layer, uint32_t expert,
+                       int64_t rows, int64_t cols, double sigma) {
+  orc_mat m;
+  memset(&m, 0, sizeof m);
+  m.rows = rows; m.cols = cols; m.kind = ORC_MAT_BF16;
+  m.key = syn_key(c->seed, syn_stream(kind, layer, expert));
+  m.scale = syn_normal_scale(sigma);
+  return m;
+}
+
+static orc_mat syn_expert_mat(const orc_cfg* c, uint32_t kind, uint32_t layer, uint32_t expert,
+                              int64_t rows, int64_t cols) {
+  if (!c->expert_fp8) return syn_mat(c, kind, layer, expert, rows, cols, c->w_sigma);
+  orc_mat m;
+  memset(&m, 0, sizeof m);
+  m.rows = rows; m.cols = cols; m.kind = ORC_MAT_FP8;
+  m.key = syn_key(c->seed, syn_stream(kind, layer, expert));
+  m.skey = syn_key(c->seed, syn_stream(SYN_FP8_SCALE, layer, (kind << 12) | expert));
+  m.scale = syn_normal_scale(16.0);
+  m.base = (float)c->fp8_block_base;
+  return m;
+}
+
+static void syn_gain(const orc_cfg* c, uint32_t kind, uint32_t layer, int64_t n, double* g) {
+  orc_mat m;
+  memset(&m, 0, sizeof m);
+  m.rows = 1; m.cols = n; m.kind = ORC_MAT_GAIN;
+  m.key = syn_key(c->seed, syn_stream(kind, layer, 0));
+  m.scale = syn_normal_scale(c->gain_sigma);
+  mat_row(&m, 0, g);
+}
+
+static int is_mla(const orc_cfg* c) { return c->kv_lora_rank > 0; }
+static int lat_width(const orc_cfg* c) { return c->kv_lora_rank + c->rope_dim; }
+
+orc_model* orc_create(const orc_cfg* cfg) {
+  orc_model* m = (orc_model*)calloc(1, sizeof(orc_model));
+  m->c = *cfg;
+  const orc_cfg* c = &m->c;
+  if (is_mla(c)) {
+    size_t n = (size_t)c->layers * c->max_seqs * c->max_ctx * lat_width(c);
+    m->kv_lat = (uint16_t*)calloc(n, 2);
+    if (!m->kv_lat) { free(m); return NULL; }
+  } else {
+    size_t n = (size_t)c->layers * c->max_seqs * c->n_kv_heads * c->max_ctx * c->head_dim;
+    m->kv_k = (uint16_t*)calloc(n, 2);
+    m->kv_v = (uint16_t*)calloc(n, 2);
+    if (!m->kv_k || !m->kv_v) { free(m->kv_k); free(m->kv_v); free(m); return NULL; }
+  }
+  return m;
+}
+
+void orc_destroy(orc_model* m) {
+  if (!m) return;
+  free(m->kv_k); free(m->kv_v); free(m->kv_lat); free(m);
+}
+
+uint16_t* orc_kv_k(orc_model* m) { return m->kv_k; }
+uint16_t* orc_kv_v(orc_model* m) { return m->kv_v; }
+uint16_t* orc_kv_lat(orc_model* m) { return m->kv_lat; }
+
+/* Synthetic pre-filled context: positions [0, T) of every sequence get
+ * seeded bf16 values ~ N(0, kv_sigma^2).  The element index does not depend
+ * on the cache capacity. */
+void orc_kv_fill_synthetic(orc_model* m, uint64_t kv_seed, int32_t T) {
+  const orc_cfg* c = &m->c;
+  float sc = syn_normal_scale(c->kv_sigma);
+  if (is_mla(c)) {
+    int W = lat_width(c);
+    for (int l = 0; l < c->layers; ++l) {
+      uint64_t key = syn_key(kv_seed, syn_stream(SYN_KV_LAT, (uint32_t)l, 0));
+      for (int s = 0; s < c->max_seqs; ++s)
+        for (int t = 0; t < T; ++t)
+          for (int i = 0; i < W; ++i)
+            m->kv_lat[(((size_t)l * c->max_seqs + s) * c->max_ctx + t) * W + i] =
+                syn_bf16_normal(key, ((uint64_t)s << 32) + (uint64_t)t * W + i, sc);
+    }
+    return;
+  }
+  int d = c->head_dim, G = c->n_kv_heads;
+  for (int l = 0; l < c->layers; ++l) {
+    uint64_t kk = syn_key(kv_seed, syn_stream(SYN_KV_K, (uint32_t)l, 0));
+    uint64_t kv = syn_key(kv_seed, syn_stream(SYN_KV_V, (uint32_t)l, 0));
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int s = 0; s < c->max_seqs; ++s)
+      for (int g = 0; g < G; ++g)
+        for (int t = 0; t < T; ++t)
+          for (int i = 0; i < d; ++i) {
+            size_t o = ((((size_t)l * c->max_seqs + s) * G + g) * c->max_ctx + t) * d + i;
+            uint64_t idx = ((uint64_t)(s * G + g) << 32) + (uint64_t)t * d + i;
+            m->kv_k[o] = syn_bf16_normal(kk, idx, sc);
+            m->kv_v[o] = syn_bf16_normal(kv, idx, sc);
+          }
+  }
+}
+
+/* Attention of one query row (all Hq heads, RoPE applied) of sequence s at
+ * position p over cached positions 0..p of layer l.  GQA: query head hq reads
+ * kv head hq / (Hq / Hkv). */
+void orc_gqa_attend_row(orc_model* mdl, int l, int s, int p, const double* q, double* out) {
+  const orc_cfg* c = &mdl->c;
+  int Hq = c->n_q_heads, G = c->n_kv_heads, d = c->head_dim, grp = Hq / G, T = p + 1;
+  double* K = (double*)malloc((size_t)T * d * sizeof(double));
+  double* Vv = (double*)malloc((size_t)T * d * sizeof(double));
+  for (int hq = 0; hq < Hq; ++hq) {
+    int g = hq / grp;
+    size_t base = ((((size_t)l * c->max_seqs + s) * G + g) * c->max_ctx) * d;
+    for (int64_t i = 0; i < (int64_t)T * d; ++i) {
+      K[i] = bf16_to_double(mdl->kv_k[base + i]);
+      Vv[i] = bf16_to_double(mdl->kv_v[base + i]);
+    }
+    orc_attention_head(T, d, q + (int64_t)hq * d, K, Vv, 1.0 / sqrt((double)d), out + (int64_t)hq * d);
+  }
+  free(K);
+  free(Vv);
+}
+
+/* Row r of a synthetic weight tensor as the oracle sees it (fp8 tensors
+ * include their block scale).  fp8 != 0 selects the expert fp8 format. */
+void orc_debug_mat_row(const orc_cfg* cfg, uint32_t kind, uint32_t layer, uint32_t expert, int64_t rows,
+                       int64_t cols, int fp8, double sigma, int64_t r, double* out) {
+  orc_mat m;
+  memset(&m, 0, sizeof m);
+  m.rows = rows; m.cols = cols;
+  if (fp8) {
+    m.kind = ORC_MAT_FP8;
+    m.key = syn_key(cfg->seed, syn_stream(kind, layer, expert));
+    m.skey = syn_key(cfg->seed, syn_stream(SYN_FP8_SCALE, layer, (kind << 12) | expert));
+    m.scale = syn_normal_scale(16.0);
+    m.base = (float)cfg->fp8_block_base;
+  } else {
+    m.kind = ORC_MAT_BF16;
+    m.key = syn_key(cfg->seed, syn_stream(kind, layer, expert));
+    m.scale = syn_normal_scale(sigma);
+  }
+  mat_row(&m, r, out);
+}
+
+/*
+ * One decode (Q = 1) or verify (Q > 1) step for S sequences.
+ * Row m = s*Q + j is sequence s at position pos0[s] + j with input tokens[m].
+ * Outputs: logits [S*Q][V] (may be NULL), argmax [S*Q], argmax margin
+ * (top1 - top2 logit), and per layer router trace [L][S*Q][k] when non-NULL.
+ * Returns 0, or -1 on an argument error.
+ */
+int orc_step(orc_model* mdl, int S, int Q, const int32_t* tokens, const int32_t* pos0,
+             double* logits, int32_t* amax, double* amargin,
+             int32_t* ridx, double* rw, double* rmargin, int mla_absorbed) {
+  const orc_cfg* c = &mdl->c;
+  int M = S * Q, H = c->hidden, L = c->layers, V = c->vocab;
+  int Hq = c->n_q_heads, G = c->n_kv_heads, d = c->head_dim;
+  if (S < 1 || Q < 1 || S > c->max_seqs) return -1;
+  for (int s = 0; s < S; ++s)
+    if (pos0[s] < 0 || pos0[s] + Q > c->max_ctx) return -1;
+  for (int m = 0; m < M; ++m)
+    if (tokens[m] < 0 || tokens[m] >= V) return -1;
+
+  double* x = (double*)malloc((size_t)M * H * sizeof(double));
+  double* h = (double*)malloc((size_t)M * H * sizeof(double));
+  double* t = (double*)malloc((size_t)M * H * sizeof(double));
+  double* gain = (double*)malloc((size_t)H * sizeof(double));
+
+  /* embedding gather */
+  {
+    orc_mat E = syn_mat(c, SYN_EMBED, 0, 0, V, H, c->w_sigma);
+    for (int m = 0; m < M; ++m) mat_row(&E, tokens[m], x + (int64_t)m * H);
+  }
+
+  for (int l = 0; l < L; ++l) {
+    syn_gain(c, SYN_ATTN_NORM, (uint32_t)l, H, gain);
+    for (int m = 0; m < M; ++m) orc_rmsnorm(H, x + (int64_t)m * H, gain, c->rms_eps, h + (int64_t)m * H);
+
+    int64_t ao_w; /* attention output width */
+    double* ao;
+    if (!is_mla(c)) {
+      int64_t QW = (int64_t)(Hq + 2 * G) * d;
+      ao_w = (int64_t)Hq * d;
+      double* qkv = (double*)malloc((size_t)M * QW * sizeof(double));
+      ao = (double*)malloc((size_t)M * ao_w * sizeof(double));
+      orc_mat Wqkv = syn_mat(c, SYN_WQKV, (uint32_t)l, 0, QW, H, c->w_sigma);
+      matvec(&Wqkv, M, h, qkv);
+      /* RoPE and cache append for every row first (verify rows see each other) */
+      for (int m = 0; m < M; ++m) {
+        int s = m / Q, p = pos0[s] + m % Q;
+        double* r = qkv + (int64_t)m * QW;
+        for (int hh = 0; hh < Hq + G; ++hh) orc_rope_apply(d, r + (int64_t)hh * d, p, c->rope_theta);
+        for (int g = 0; g < G; ++g) {
+          size_t o = ((((size_t)l * c->max_seqs + s) * G + g) * c->max_ctx + p) * d;
+          for (int i = 0; i < d; ++i) {
+            mdl->kv_k[o + i] = double_to_bf16(r[(int64_t)(Hq + g) * d + i]);
+            mdl->kv_v[o + i] = double_to_bf16(r[(int64_t)(Hq + G + g) * d + i]);
+          }
+        }
+      }
+#pragma omp parallel for schedule(dynamic)
+      for (int m = 0; m < M; ++m) {
+        int s = m / Q, p = pos0[s] + m % Q;
+        orc_gqa_attend_row(mdl, l, s, p, qkv + (int64_t)m * QW, ao + (int64_t)m * ao_w);
+      }
+      free(qkv);
+    } else {
+      int R = c->kv_lora_rank, dr = c->rope_dim, dn = d, dv = d, W = lat_width(c);
+      int64_t QW = (int64_t)Hq * (dn + dr);
+      ao_w = (int64_t)Hq * dv;
+      double* q = (double*)malloc((size_t)M * QW * sizeof(double));
+      double* ckr = (double*)malloc((size_t)M * W * sizeof(double));
+      ao = (double*)malloc((size_t)M * ao_w * sizeof(double));
+      orc_mat Wq = syn_mat(c, SYN_MLA_WQ, (uint32_t)l, 0, QW, H, c->w_sigma);
+      orc_mat Wdkv = syn_mat(c, SYN_MLA_WDKV, (uint32_t)l, 0, W, H, c->w_sigma);
+      matvec(&Wq, M, h, q);
+      matvec(&Wdkv, M, h, ckr);
+      for (int m = 0; m < M; ++m) {
+        int s = m / Q, p = pos0[s] + m % Q;
+        for (int hh = 0; hh < Hq; ++hh) orc_rope_apply(dr, q + (int64_t)m * QW + (int64_t)hh * (dn + dr) + dn, p, c->rope_theta);
+        orc_rope_apply(dr, ckr + (int64_t)m * W + R, p, c->rope_theta);
+        size_t o = (((size_t)l * c->max_seqs + s) * c->max_ctx + p) * W;
+        for (int i = 0; i < W; ++i) mdl->kv_lat[o + i] = double_to_bf16(ckr[(int64_t)m * W + i]);
+      }
+      /* materialise W_uk, W_uv for this layer */
+      double* Wuk = (double*)malloc((size_t)Hq * dn * R * sizeof(double));
+      double* Wuv = (double*)malloc((size_t)Hq * dv * R * sizeof(double));
+      {
+        orc_mat A = syn_mat(c, SYN_MLA_WUK, (uint32_t)l, 0, (int64_t)Hq * dn, R, c->w_sigma);
+        orc_mat B = syn_mat(c, SYN_MLA_WUV, (uint32_t)l, 0, (int64_t)Hq * dv, R, c->w_sigma);
+#pragma omp parallel for schedule(static)
+        for (int64_t r = 0; r < (int64_t)Hq * dn; ++r) mat_row(&A, r, Wuk + r * R);
+#pragma omp parallel for schedule(static)
+        for (int64_t r = 0; r < (int64_t)Hq * dv; ++r) mat_row(&B, r, Wuv + r * R);
+      }
+      for (int m = 0; m < M; ++m) {
+        int s = m / Q, p = pos0[s] + m % Q, T = p + 1;
+        double* lat = (double*)malloc((size_t)T * W * sizeof(double));
+        size_t base = (((size_t)l * c->max_seqs + s) * c->max_ctx) * W;
+        for (int64_t i = 0; i < (int64_t)T * W; ++i) lat[i] = bf16_to_double(mdl->kv_lat[base + i]);
+        mla_attend(Hq, dn, dr, dv, R, T, q + (int64_t)m * QW, lat, Wuk, Wuv, mla_absorbed, ao + (int64_t)m * ao_w);
+        free(lat);
+      }
+      free(Wuk); free(Wuv); free(q); free(ckr);
+    }
+
+    /* output projection + residual */
+    {
+      orc_mat Wo = syn_mat(c, SYN_WO, (uint32_t)l, 0, H, ao_w, c->w_sigma);
+      matvec(&Wo, M, ao, t);
+      for (int64_t i = 0; i < (int64_t)M * H; ++i) x[i] += t[i];
+      free(ao);
+    }
+
+    /* FFN */
+    syn_gain(c, SYN_FFN_NORM, (uint32_t)l, H, gain);
+    for (int m = 0; m < M; ++m) orc_rmsnorm(H, x + (int64_t)m * H, gain, c->rms_eps, h + (int64_t)m * H);
+    if (c->n_routed == 0) {
+      orc_mat Wg = syn_mat(c, SYN_WGATE, (uint32_t)l, 0, c->ffn, H, c->w_sigma);
+      orc_mat Wu = syn_mat(c, SYN_WUP, (uint32_t)l, 0, c->ffn, H, c->w_sigma);
+      orc_mat Wd = syn_mat(c, SYN_WDOWN, (uint32_t)l, 0, H, c->ffn, c->w_sigma);
+      swiglu(&Wg, &Wu, &Wd, M, h, t);
+      for (int64_t i = 0; i < (int64_t)M * H; ++i) x[i] += t[i];
+    } else {
+      int E = c->n_routed, k = c->top_k, Ie = c->expert_ffn, NS = c->n_shared;
+      orc_mat Wr = syn_mat(c, SYN_ROUTER, (uint32_t)l, 0, E, H, c->router_sigma);
+      orc_mat* eg = (orc_mat*)calloc((size_t)E, sizeof(orc_mat));
+      orc_mat* eu = (orc_mat*)calloc((size_t)E, sizeof(orc_mat));
+      orc_mat* ed = (orc_mat*)calloc((size_t)E, sizeof(orc_mat));
+      orc_mat* sg = (orc_mat*)calloc((size_t)NS + 1, sizeof(orc_mat));
+      orc_mat* su = (orc_mat*)calloc((size_t)NS + 1, sizeof(orc_mat));
+      orc_mat* sd = (orc_mat*)calloc((size_t)NS + 1, sizeof(orc_mat));
+      for (int e = 0; e < E; ++e) {
+        eg[e] = syn_expert_mat(c, SYN_EX_GATE, (uint32_t)l, (uint32_t)e, Ie, H);
+        eu[e] = syn_expert_mat(c, SYN_EX_UP, (uint32_t)l, (uint32_t)e, Ie, H);
+        ed[e] = syn_expert_mat(c, SYN_EX_DOWN, (uint32_t)l, (uint32_t)e, H, Ie);
+      }
+      for (int j = 0; j < NS; ++j) {
+        sg[j] = syn_expert_mat(c, SYN_SH_GATE, (uint32_t)l, (uint32_t)j, Ie, H);
+        su[j] = syn_expert_mat(c, SYN_SH_UP, (uint32_t)l, (uint32_t)j, Ie, H);
+        sd[j] = syn_expert_mat(c, SYN_SH_DOWN, (uint32_t)l, (uint32_t)j, H, Ie);
+      }
+      int32_t* idx = (int32_t*)malloc((size_t)k * sizeof(int32_t));
+      double* w = (double*)malloc((size_t)k * sizeof(double));
+      for (int m = 0; m < M; ++m) {
+        double mg;
+        moe_ffn(H, E, k, NS, &Wr, sg, su, sd, eg, eu, ed, h + (int64_t)m * H, t, idx, w, &mg);
+        for (int i = 0; i < H; ++i) x[(int64_t)m * H + i] += t[i];
+        if (ridx) for (int j = 0; j < k; ++j) ridx[((int64_t)l * M + m) * k + j] = idx[j];
+        if (rw) for (int j = 0; j < k; ++j) rw[((int64_t)l * M + m) * k + j] = w[j];
+        if (rmargin) rmargin[(int64_t)l * M + m] = mg;
+      }
+      free(idx); free(w); free(eg); free(eu); free(ed); free(sg); free(su); free(sd);
+    }
+  }
+
+  /* final norm, LM head, greedy argmax */
+  syn_gain(c, SYN_FINAL_NORM, 0, H, gain);
+  for (int m = 0; m < M; ++m) orc_rmsnorm(H, x + (int64_t)m * H, gain, c->rms_eps, h + (int64_t)m * H);
+  double* lg = (double*)malloc((size_t)M * V * sizeof(double));
+  orc_mat Wlm = syn_mat(c, SYN_LM_HEAD, 0, 0, V, H, c->w_sigma);
+  matvec(&Wlm, M, h, lg);
+  for (int m = 0; m < M; ++m) {
+    double mg;
+    amax[m] = orc_argmax(V, lg + (int64_t)m * V, &mg);
+    if (amargin) amargin[m] = mg;
+  }
+  if (logits) memcpy(logits, lg, (size_t)M * V * sizeof(double));
+  free(lg); free(x); free(h); free(t); free(gain);
+  return 0;
+}
+
+/*
+ * Full-sequence causal forward with no cache (the recompute side of the
+ * "cached decode == recompute" identity): every layer materialises K and V
+ * (rounded to bf16, as stored) for all T positions and evaluates the naive
+ * masked softmax over the full score matrix.  logits: [T][V].
+ */
+int orc_forward_full(const orc_cfg* cfg, int T, const int32_t* tokens, double* logits) {
+  orc_cfg cc = *cfg;
+  const orc_cfg* c = &cc;
+  int H = c->hidden, L = c->layers, V = c->vocab, Hq = c->n_q_heads, G = c->n_kv_heads, d = c->head_dim;
+  double* x = (double*)malloc((size_t)T * H * sizeof(double));
+  double* h = (double*)malloc((size_t)T * H * sizeof(double));
+  double* t = (double*)malloc((size_t)T * H * sizeof(double));
+  double* gain = (double*)malloc((size_t)H * sizeof(double));
+  orc_mat E = syn_mat(c, SYN_EMBED, 0, 0, V, H, c->w_sigma);
+  for (int p = 0; p < T; ++p) mat_row(&E, tokens[p], x + (int64_t)p * H);
+  for (int l = 0; l < L; ++l) {
+    syn_gain(c, SYN_ATTN_NORM, (uint32_t)l, H, gain);
+    for (int p = 0; p < T; ++p) orc_rmsnorm(H, x + (int64_t)p * H, gain, c->rms_eps, h + (int64_t)p * H);
+    int64_t ao_w;
+    double* ao;
+    if (!is_mla(c)) {
+      int64_t QW = (int64_t)(Hq + 2 * G) * d;
+      ao_w = (int64_t)Hq * d;
+      double* qkv = (double*)malloc((size_t)T * QW * sizeof(double));
+      ao = (double*)malloc((size_t)T * ao_w * sizeof(double));
+      orc_mat Wqkv = syn_mat(c, SYN_WQKV, (uint32_t)l, 0, QW, H, c->w_sigma);
+      matvec(&Wqkv, T, h, qkv);
+      /* K, V for all positions, per kv head: [G][T][d] */
+      double* K = (double*)malloc((size_t)G * T * d * sizeof(double));
+      double* Vv = (double*)malloc((size_t)G * T * d * sizeof(double));
+      for (int p = 0; p < T; ++p) {
+        double* r = qkv + (int64_t)p * QW;
+        for (int hh = 0; hh < Hq + G; ++hh) orc_rope_apply(d, r + (int64_t)hh * d, p, c->rope_theta);
+        for (int g = 0; g < G; ++g)
+          for (int i = 0; i < d; ++i) {
+            K[((int64_t)g * T + p) * d + i] = bf16_to_double(double_to_bf16(r[(int64_t)(Hq + g) * d + i]));
+            Vv[((int64_t)g * T + p) * d + i] = bf16_to_double(double_to_bf16(r[(int64_t)(Hq + G + g) * d + i]));
+          }
+      }
+      int grp = Hq / G;
+      double scale = 1.0 / sqrt((double)d);
+#pragma omp parallel for collapse(2) schedule(dynamic)
+      for (int p = 0; p < T; ++p)
+        for (int hq = 0; hq < Hq; ++hq) {
+          int g = hq / grp;
+          const double* q = qkv + (int64_t)p * QW + (int64_t)hq * d;
+          /* full score row with the causal mask applied (j > p excluded) */
+          double* sc = (double*)malloc((size_t)T * sizeof(double));
+          double* pr = (double*)malloc((size_t)T * sizeof(double));
+          for (int j = 0; j < T; ++j) {
+            if (j > p) { sc[j] = -INFINITY; continue; }
+            double a = 0.0;
+            for (int i = 0; i < d; ++i) a += q[i] * K[((int64_t)g * T + j) * d + i];
+            sc[j] = a * scale;
+          }
+          orc_softmax(T, sc, pr);
+          double* o = ao + (int64_t)p * ao_w + (int64_t)hq * d;
+          for (int i = 0; i < d; ++i) o[i] = 0.0;
+          for (int j = 0; j < T; ++j)
+            for (int i = 0; i < d; ++i) o[i] += pr[j] * Vv[((int64_t)g * T + j) * d + i];
+          free(sc);
+          free(pr);
+        }
+      free(K); free(Vv); free(qkv);
+    } else {
+      int R = c->kv_lora_rank, dr = c->rope_dim, dn = d, dv = d, W = lat_width(c);
+      int64_t QW = (int64_t)Hq * (dn + dr);
+      ao_w = (int64_t)Hq * dv;
+      double* q = (double*)malloc((size_t)T * QW * sizeof(double));
+      double* lat = (double*)malloc((size_t)T * W * sizeof(double));
+      ao = (double*)malloc((size_t)T * ao_w * sizeof(double));
+      orc_mat Wq = syn_mat(c, SYN_MLA_WQ, (uint32_t)l, 0, QW, H, c->w_sigma);
+      orc_mat Wdkv = syn_mat(c, SYN_MLA_WDKV, (uint32_t)l, 0, W, H, c->w_sigma);
+      matvec(&Wq, T, h, q);
+      matvec(&Wdkv, T, h, lat);
+      for (int p = 0; p < T; ++p) {
+        for (int hh = 0; hh < Hq; ++hh) orc_rope_apply(dr, q + (int64_t)p * QW + (int64_t)hh * (dn + dr) + dn, p, c->rope_theta);
+        orc_rope_apply(dr, lat + (int64_t)p * W + R, p, c->rope_theta);
+        for (int i = 0; i < W; ++i) lat[(int64_t)p * W + i] = bf16_to_double(double_to_bf16(lat[(int64_t)p * W + i]));
+      }
+      double* Wuk = (double*)malloc((size_t)Hq * dn * R * sizeof(double));
+      double* Wuv = (double*)malloc((size_t)Hq * dv * R * sizeof(double));
+      orc_mat A = syn_mat(c, SYN_MLA_WUK, (uint32_t)l, 0, (int64_t)Hq * dn, R, c->w_sigma);
+      orc_mat B = syn_mat(c, SYN_MLA_WUV, (uint32_t)l, 0, (int64_t)Hq * dv, R, c->w_sigma);
+      for (int64_t r = 0; r < (int64_t)Hq * dn; ++r) mat_row(&A, r, Wuk + r * R);
+      for (int64_t r = 0; r < (int64_t)Hq * dv; ++r) mat_row(&B, r, Wuv + r * R);
+      /* position p sees rows 0..p (causal prefix of the full latent matrix) */
+      for (int p = 0; p < T; ++p)
+        mla_attend(Hq, dn, dr, dv, R, p + 1, q + (int64_t)p * QW, lat, Wuk, Wuv, 0, ao + (int64_t)p * ao_w);
+      free(Wuk); free(Wuv); free(q); free(lat);
+    }
+    orc_mat Wo = syn_mat(c, SYN_WO, (uint32_t)l, 0, H, ao_w, c->w_sigma);
+    matvec(&Wo, T, ao, t);
+    for (int64_t i = 0; i < (int64_t)T * H; ++i) x[i] += t[i];
+    free(ao);
+    syn_gain(c, SYN_FFN_NORM, (uint32_t)l, H, gain);
+    for (int p = 0; p < T; ++p) orc_rmsnorm(H, x + (int64_t)p * H, gain, c->rms_eps, h + (int64_t)p * H);
+    if (c->n_routed == 0) {
+      orc_mat Wg = syn_mat(c, SYN_WGATE, (uint32_t)l, 0, c->ffn, H, c->w_sigma);
+      orc_mat Wu = syn_mat(c, SYN_WUP, (uint32_t)l, 0, c->ffn, H, c->w_sigma);
+      orc_mat Wd = syn_mat(c, SYN_WDOWN, (uint32_t)l, 0, H, c->ffn, c->w_sigma);
+      swiglu(&Wg, &Wu, &Wd, T, h, t);
+    } else {
+      int Ex = c->n_routed, k = c->top_k, Ie = c->expert_ffn, NS = c->n_shared;
+      orc_mat Wr = syn_mat(c, SYN_ROUTER, (uint32_t)l, 0, Ex, H, c->router_sigma);
+      orc_mat* eg = (orc_mat*)calloc((size_t)Ex, sizeof(orc_mat));
+      orc_mat* eu = (orc_mat*)calloc((size_t)Ex, sizeof(orc_mat));
+      orc_mat* ed = (orc_mat*)calloc((size_t)Ex, sizeof(orc_mat));
+      orc_mat* sg = (orc_mat*)calloc((size_t)NS + 1, sizeof(orc_mat));
+      orc_mat* su = (orc_mat*)calloc((size_t)NS + 1, sizeof(orc_mat));
+      orc_mat* sd = (orc_mat*)calloc((size_t)NS + 1, sizeof(orc_mat));
+      for (int e = 0; e < Ex; ++e) {
+        eg[e] = syn_expert_mat(c, SYN_EX_GATE, (uint32_t)l, (uint32_t)e, Ie, H);
+        eu[e] = syn_expert_mat(c, SYN_EX_UP, (uint32_t)l, (uint32_t)e, Ie, H);
+        ed[e] = syn_expert_mat(c, SYN_EX_DOWN, (uint32_t)l, (uint32_t)e, H, Ie);
+      }
+      for (int j = 0; j < NS; ++j) {
+        sg[j] = syn_expert_mat(c, SYN_SH_GATE, (uint32_t)l, (uint32_t)j, Ie, H);
+        su[j] = syn_expert_mat(c, SYN_SH_UP, (uint32_t)l, (uint32_t)j, Ie, H);
+        sd[j] = syn_expert_mat(c, SYN_SH_DOWN, (uint32_t)l, (uint32_t)j, H, Ie);
+      }
+      int32_t* idx = (int32_t*)malloc((size_t)k * sizeof(int32_t));
+      double* w = (double*)malloc((size_t)k * sizeof(double));
+      for (int p = 0; p < T; ++p)
+        moe_ffn(H, Ex, k, NS, &Wr, sg, su, sd, eg, eu, ed, h + (int64_t)p * H, t + (int64_t)p * H, idx, w, NULL);
+      free(idx); free(w); free(eg); free(eu); free(ed); free(sg); free(su); free(sd);
+    }
+    for (int64_t i = 0; i < (int64_t)T * H; ++i) x[i] += t[i];
+  }
+  syn_gain(c, SYN_FINAL_NORM, 0, H, gain);
+  for (int p = 0; p < T; ++p) orc_rmsnorm(H, x + (int64_t)p * H, gain, c->rms_eps, h + (int64_t)p * H);
+  orc_mat Wlm = syn_mat(c, SYN_LM_HEAD, 0, 0, V, H, c->w_sigma);
+  matvec(&Wlm, T, h, logits);
+  free(x); free(h); free(t); free(gain);
+  return 0;
+}
+
+/* Bytes the oracle's model-level step reads from a weight source row by row;
+ * used only to label the CPU baseline. */
+int orc_num_threads(void) {
+#ifdef _OPENMP
+  extern int omp_get_max_threads(void);
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
