@@ -1,0 +1,185 @@
+/*
+ * mk.h - C ABI of the persistent decode megakernel for NVIDIA B200 (sm_100a).
+ *
+ * One call evaluates one whole decoder step (embedding -> every layer's
+ * attention and FFN / MoE -> final norm -> LM head -> greedy argmax) as a
+ * single persistent kernel.  Source of the operation: "700 TPS on Kimi K3:
+ * A Case for TPU Megakernels" (Inferact blog), section "Why megakernels?"
+ * (the whole decoder step inside one program, weight loads decoupled from
+ * their consumers), section "Our Kimi K3 megakernel" (phase order attention
+ * -> router -> shared expert -> routed experts; the next layer's attention
+ * weights are fetched while the current layer's MoE runs) and section
+ * "DSpark" (one launch checks 1 anchor + 7 proposals).
+ *
+ * Conventions for every entry point:
+ *   - Return MK_OK or an error code; no exception crosses the ABI.
+ *   - Argument errors are detected on the host and returned synchronously;
+ *     nothing is launched then.
+ *   - Compute calls are asynchronous on the caller's stream.  Errors found
+ *     on the device (a bounds violation in device-resident inputs, a
+ *     dependency wait that timed out) are recorded in a device status word
+ *     and read with mk_sync_status() after the stream has been synchronised.
+ *     They are sticky: later compute calls return MK_ERR_STATE until
+ *     mk_reset() is called.
+ *   - Pointers marked "dev" are CUDA device pointers owned by the caller;
+ *     "host" pointers are host memory owned by the caller.  The library never
+ *     frees caller memory and never keeps a caller pointer after a call
+ *     returns.  Weights, KV caches and scratch are owned by the library.
+ *   - mk_last_error() returns a static description of the last failure of a
+ *     handle (valid until the next call on that handle).
+ */
+#ifndef MK_H
+#define MK_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MK_OK = 0,
+  MK_ERR_INVALID = 1,        /* bad argument or unsupported shape */
+  MK_ERR_OOM = 2,            /* device allocation failed */
+  MK_ERR_CUDA = 3,           /* a CUDA runtime call failed */
+  MK_ERR_DEVICE_TIMEOUT = 4, /* a dependency wait inside the kernel ran out */
+  MK_ERR_DEVICE_BOUNDS = 5,  /* token / position out of range in device inputs */
+  MK_ERR_STATE = 6           /* handle is in the sticky error state, or wrong order of calls */
+} mk_status;
+
+/* Shape of the decoder.  A dense model has n_routed == 0 (then ffn > 0).
+ * A MoE model has n_routed > 0, top_k in [1, 8], expert_ffn > 0, n_shared >= 0.
+ * kv_lora_rank > 0 selects multi-head latent attention: query heads have
+ * head_dim "nope" dims + rope_dim rotary dims, values have head_dim dims, and
+ * the cache keeps kv_lora_rank + rope_dim values per position (n_kv_heads is
+ * ignored).  expert_fp8 != 0 stores shared and routed expert weights as OCP
+ * FP8 E4M3 with one fp32 scale per 128x128 block of each [out, in] matrix.
+ * max_batch (<= 8) bounds S * Q rows of one step; max_ctx bounds positions. */
+typedef struct {
+  int32_t layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
+  float rope_theta, rms_eps;
+  int32_t n_routed, n_shared, top_k, expert_ffn;
+  int32_t kv_lora_rank, rope_dim;
+  int32_t expert_fp8;
+  int32_t max_batch, max_ctx;
+} mk_model_desc;
+
+/* Parameters of the seeded synthetic weights (see synth/synth.h for the
+ * counter-based generator): weights ~ N(0, w_sigma^2) rounded to bf16, router
+ * ~ N(0, router_sigma^2), norm gains 1 + N(0, gain_sigma^2), fp8 expert codes
+ * e4m3(16 N(0,1)) with block scales fp8_block_base * (1 + j/8). */
+typedef struct {
+  uint64_t seed;
+  float w_sigma, router_sigma, gain_sigma, fp8_block_base;
+} mk_synth_params;
+
+typedef struct mk_handle mk_handle;
+typedef struct mk_kv mk_kv;
+
+/* Create a model on `device` (weights allocated, not initialised).
+ * Fails with MK_ERR_INVALID for unsupported shapes (e.g. head_dim other than
+ * 64 or 128, hidden not a multiple of 16, n_q_heads not a multiple of
+ * n_kv_heads) and MK_ERR_OOM when the weights do not fit. */
+mk_status mk_create(const mk_model_desc* desc, int device, mk_handle** out);
+
+/* Fill every weight from the seeded generator, directly on the device and
+ * already in the kernel's streaming layout.  Synchronous. */
+mk_status mk_init_random(mk_handle* h, const mk_synth_params* p);
+
+/* Weight tensor for mk_load_weights, in logical row-major [rows][cols]
+ * layout ([out, in] for projections).  `kind` and `layer`/`expert` name the
+ * tensor with the same ids as synth/synth.h (SYN_WQKV, SYN_EX_GATE, ...).
+ * data: bf16 bits (uint16) for bf16 tensors, e4m3 bytes for fp8 expert
+ * tensors (then `scales` = fp32 [ceil(rows/128)][ceil(cols/128)]).
+ * on_device != 0 means data/scales are device pointers, else host. */
+typedef struct {
+  int32_t kind, layer, expert;
+  int64_t rows, cols;
+  const void* data;
+  const float* scales;
+  int32_t on_device;
+} mk_tensor_src;
+
+/* Copy and re-tile `n` tensors into the model's weights.  The caller keeps
+ * ownership of the sources.  Shapes must match the descriptor exactly.
+ * Synchronous. */
+mk_status mk_load_weights(mk_handle* h, const mk_tensor_src* tensors, int n);
+
+/* A KV cache for up to `max_seqs` sequences of `max_ctx` positions, owned by
+ * the library, zero-filled.  Layout (device, bf16): GQA keys and values
+ * [layers][max_seqs][n_kv_heads][max_ctx][head_dim] each; MLA latent
+ * [layers][max_seqs][max_ctx][kv_lora_rank + rope_dim]. */
+mk_status mk_kv_create(mk_handle* h, int max_seqs, int max_ctx, mk_kv** out);
+
+/* Fill positions [0, length) of every sequence with seeded bf16 values
+ * ~ N(0, sigma^2) (a synthetic pre-filled context).  Synchronous. */
+mk_status mk_kv_fill_random(mk_kv* kv, uint64_t seed, float sigma, int32_t length);
+
+/* Copy the whole cache, in the layout above, into caller device memory of
+ * mk_kv_bytes() bytes (keys first, then values, for GQA).  Synchronous. */
+mk_status mk_kv_copy_out(mk_kv* kv, void* dst_dev);
+int64_t mk_kv_bytes(const mk_kv* kv);
+
+/* One decode step for B sequences (B <= max_batch): sequence b consumes
+ * tokens[b] at positions[b], writes its K/V there and attends over
+ * positions 0..positions[b].
+ *   tokens, positions: dev int32 [B]
+ *   logits_out: dev fp32 [B][vocab], or NULL
+ *   argmax_out: dev int32 [B] (greedy token; ties -> lower index)
+ *   stream: a cudaStream_t (NULL = default stream)
+ * Device-side bounds errors: token outside [0, vocab) or position outside
+ * [0, kv max_ctx). */
+mk_status mk_decode_step(mk_handle* h, const int32_t* tokens, const int32_t* positions, int B,
+                         mk_kv* kv, float* logits_out, int32_t* argmax_out, void* stream);
+
+/* Speculative verify of one sequence (sequence 0 of the cache): tokens8 =
+ * anchor followed by n_prop (<= 7) proposals, dev int32 [n_prop + 1], placed
+ * at positions position .. position + n_prop, causal within the chunk.  K/V
+ * are written for every position; the caller rewinds its length to
+ * position + accepted + 1 (later entries are overwritten by the next step).
+ *   logits_out: dev fp32 [n_prop + 1][vocab] or NULL
+ *   argmax_out: dev int32 [n_prop + 1] (greedy token after each position)
+ *   accepted_out: dev int32 [1] = largest n <= n_prop with
+ *                 tokens8[j] == argmax_out[j - 1] for all 1 <= j <= n. */
+mk_status mk_verify(mk_handle* h, const int32_t* tokens8, int n_prop, int32_t position, mk_kv* kv,
+                    float* logits_out, int32_t* argmax_out, int32_t* accepted_out, void* stream);
+
+/* Debug outputs of the next compute calls (dev pointers, or NULL to stop):
+ * router expert indices int32 [layers][rows][top_k] and weights fp32 (same
+ * shape) in top-k order. */
+mk_status mk_set_router_trace(mk_handle* h, int32_t* idx_dev, float* w_dev);
+
+/* Debug trace of the next compute calls: for every task of every CTA the
+ * kernel writes 8 int64 into trace_dev[cta][task][8]: %globaltimer (ns) at
+ * task start, when its dependency was satisfied, and at its end; SM clock
+ * cycles spent waiting for weight tiles, for activation slices; chunks and
+ * weight bytes consumed; the task's type.  Tasks beyond max_tasks_per_cta
+ * are not recorded.  NULL disables. */
+mk_status mk_set_trace(mk_handle* h, int64_t* trace_dev, int32_t max_tasks_per_cta);
+
+/* Read the device status word (call after the stream has been synchronised).
+ * Returns MK_OK or the recorded device error; errors stay until mk_reset. */
+mk_status mk_sync_status(mk_handle* h);
+
+/* Clear a sticky device error and all inter-CTA counters.  Synchronous. */
+mk_status mk_reset(mk_handle* h);
+
+/* Number of persistent CTAs (one per SM) and dynamic shared memory per CTA. */
+mk_status mk_launch_info(mk_handle* h, int32_t* ctas, int32_t* smem_bytes, int32_t* threads);
+
+/* Bytes of device memory held for weights. */
+int64_t mk_weight_bytes(const mk_handle* h);
+
+/* Test hook: make the next compute call wait on a dependency counter that
+ * nothing signals, with a wait limit of `timeout_ns`, so that it returns
+ * MK_ERR_DEVICE_TIMEOUT through mk_sync_status.  0 disables. */
+mk_status mk_debug_inject_stall(mk_handle* h, int64_t timeout_ns);
+
+const char* mk_last_error(const mk_handle* h);
+void mk_kv_destroy(mk_kv* kv);
+void mk_destroy(mk_handle* h);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MK_H */

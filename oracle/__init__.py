@@ -210,8 +210,8 @@ class OracleModel:
             raise MemoryError("oracle: cache allocation failed")
 
     def close(self):
-        if self.h:
-            lib().orc_destroy(self.h)
+        if getattr(self, "h", None) and _lib is not None:
+            _lib.orc_destroy(self.h)
             self.h = None
 
     def __del__(self):

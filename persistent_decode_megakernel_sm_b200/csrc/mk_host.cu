@@ -1,0 +1,958 @@
+// mk_host.cu - C ABI of the decode megakernel: model creation, weight
+// layout (seeded fill and loading from caller buffers), KV caches, the
+// static task planner and the cooperative launch.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
+#include <map>
+#include <string>
+#include <utility>
+#include <vector>
+
+#include "../../include/mk.h"
+#include "../../synth/synth.h"
+#include "mk_internal.h"
+
+namespace mk {
+__global__ void mk_step_kernel(const __grid_constant__ Launch P);
+}
+
+using namespace mk;
+
+// ---------------------------------------------------------------------------
+// logical source of every element of a tiled matrix
+// ---------------------------------------------------------------------------
+enum MapType { MAP_PLAIN = 0, MAP_GU = 1, MAP_CONCAT = 2, MAP_UKT = 3 };
+
+struct MatMap {
+  int32_t type;
+  int32_t kindA, kindB;   // tensor kinds (synth ids)
+  int32_t layer, expert;
+  int32_t rowsA;          // MAP_CONCAT: rows taken from kindA
+  int32_t lcolsA, lcolsB; // logical column count of the source tensors
+  int32_t Hq, dn, R;      // MAP_UKT
+  float sigA, sigB;
+};
+
+// tiled (row, col) -> logical (kind selector 0/1, lrow, lcol)
+__host__ __device__ static inline void map_elem(const MatMap& mp, int row, int col, int& which, int64_t& lrow,
+                                                int64_t& lcol) {
+  switch (mp.type) {
+    case MAP_GU: {
+      const int rt = row >> 4, rr = row & 15;
+      which = rr < 8 ? 0 : 1;
+      lrow = (int64_t)rt * 8 + (rr & 7);
+      lcol = col;
+      break;
+    }
+    case MAP_CONCAT:
+      if (row < mp.rowsA) { which = 0; lrow = row; }
+      else { which = 1; lrow = row - mp.rowsA; }
+      lcol = col;
+      break;
+    case MAP_UKT: {
+      // tiled row = h * R + c, tiled col = i  <->  W_uk[h * dn + i][c]
+      const int h = row / mp.R, c = row % mp.R;
+      which = 0;
+      lrow = (int64_t)h * mp.dn + col;
+      lcol = c;
+      break;
+    }
+    default:
+      which = 0;
+      lrow = row;
+      lcol = col;
+  }
+}
+
+__host__ __device__ static inline void frag_elem(int rt, int ct, int lane, int e, int& row, int& col) {
+  const int g = lane >> 2, t = lane & 3;
+  row = rt * 16 + g + 8 * ((e >> 1) & 1);
+  col = ct * 16 + 2 * t + (e & 1) + 8 * (e >> 2);
+}
+
+// Seeded fill, directly in tile order.
+__global__ void fill_tiles_kernel(uint8_t* w, int RT, int KT, int rows, int cols, int fp8, MatMap mp, uint64_t keyA,
+                                  uint64_t keyB, float scA, float scB) {
+  const int64_t n = (int64_t)RT * KT * 32;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int lane = (int)(i & 31);
+    const int64_t tile = i >> 5;
+    const int rt = (int)(tile / KT), ct = (int)(tile % KT);
+    if (!fp8) {
+      uint16_t v[8];
+      for (int e = 0; e < 8; ++e) {
+        int row, col;
+        frag_elem(rt, ct, lane, e, row, col);
+        v[e] = 0;
+        if (row < rows && col < cols) {
+          int which;
+          int64_t lr, lc;
+          map_elem(mp, row, col, which, lr, lc);
+          const int64_t lcols = which ? mp.lcolsB : mp.lcolsA;
+          v[e] = syn_bf16_normal(which ? keyB : keyA, (uint64_t)(lr * lcols + lc), which ? scB : scA);
+        }
+      }
+      uint4 o;
+      o.x = v[0] | ((uint32_t)v[1] << 16);
+      o.y = v[2] | ((uint32_t)v[3] << 16);
+      o.z = v[4] | ((uint32_t)v[5] << 16);
+      o.w = v[6] | ((uint32_t)v[7] << 16);
+      reinterpret_cast<uint4*>(w)[i] = o;
+    } else {
+      uint8_t v[8];
+      for (int e = 0; e < 8; ++e) {
+        int row, col;
+        frag_elem(rt, ct, lane, e, row, col);
+        v[e] = 0;
+        if (row < rows && col < cols) {
+          int which;
+          int64_t lr, lc;
+          map_elem(mp, row, col, which, lr, lc);
+          const int64_t lcols = which ? mp.lcolsB : mp.lcolsA;
+          v[e] = syn_e4m3_normal(which ? keyB : keyA, (uint64_t)(lr * lcols + lc), scA);
+        }
+      }
+      uint2 o;
+      o.x = v[0] | ((uint32_t)v[1] << 8) | ((uint32_t)v[2] << 16) | ((uint32_t)v[3] << 24);
+      o.y = v[4] | ((uint32_t)v[5] << 8) | ((uint32_t)v[6] << 16) | ((uint32_t)v[7] << 24);
+      reinterpret_cast<uint2*>(w)[i] = o;
+    }
+  }
+}
+
+// Re-tile one logical source tensor (row-major, on the device) into the
+// elements of a tiled matrix that it owns.
+__global__ void retile_kernel(uint8_t* w, int RT, int KT, int rows, int cols, int fp8, MatMap mp, int which_src,
+                              const uint8_t* src, int64_t src_cols) {
+  const int64_t n = (int64_t)RT * KT * 32;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int lane = (int)(i & 31);
+    const int64_t tile = i >> 5;
+    const int rt = (int)(tile / KT), ct = (int)(tile % KT);
+    for (int e = 0; e < 8; ++e) {
+      int row, col;
+      frag_elem(rt, ct, lane, e, row, col);
+      if (row >= rows || col >= cols) continue;
+      int which;
+      int64_t lr, lc;
+      map_elem(mp, row, col, which, lr, lc);
+      if (which != which_src) continue;
+      if (!fp8) {
+        reinterpret_cast<uint16_t*>(w)[i * 8 + e] = reinterpret_cast<const uint16_t*>(src)[lr * src_cols + lc];
+      } else {
+        w[i * 8 + e] = src[lr * src_cols + lc];
+      }
+    }
+  }
+}
+
+__global__ void fill_bf16_kernel(uint16_t* dst, int64_t n, uint64_t key, float sc, int gain) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    dst[i] = gain ? syn_bf16_gain(key, (uint64_t)i, sc) : syn_bf16_normal(key, (uint64_t)i, sc);
+}
+
+__global__ void fill_scales_kernel(float* dst, int64_t n, uint64_t key, float base) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    dst[i] = syn_block_scale(key, (uint64_t)i, base);
+}
+
+// Synthetic KV context: sequence s, kv head g, position t, element i of
+// layer l has index ((s * G + g) << 32) + t * d + i in stream (KV_K|KV_V, l).
+__global__ void fill_kv_kernel(uint16_t* dst, int L, int S, int G, int Tmax, int d, int T, uint64_t seed, int kind,
+                               float sc) {
+  const int64_t n = (int64_t)L * S * G * T * d;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int e = (int)(i % d);
+    int64_t r = i / d;
+    const int t = (int)(r % T);
+    r /= T;
+    const int g = (int)(r % G);
+    r /= G;
+    const int s = (int)(r % S);
+    const int l = (int)(r / S);
+    const uint64_t key = syn_key(seed, syn_stream((uint32_t)kind, (uint32_t)l, 0));
+    const uint64_t idx = ((uint64_t)(s * G + g) << 32) + (uint64_t)t * d + e;
+    dst[((((int64_t)l * S + s) * G + g) * Tmax + t) * d + e] = syn_bf16_normal(key, idx, sc);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// handle
+// ---------------------------------------------------------------------------
+struct MatHost {
+  Mat m;
+  MatMap map;
+  size_t bytes;
+};
+
+struct PlanKey {
+  int S, Q;
+  bool operator<(const PlanKey& o) const { return S < o.S || (S == o.S && Q < o.Q); }
+};
+
+struct Plan {
+  Task* d_tasks = nullptr;
+  int32_t* d_off = nullptr;
+  int n_items = 0, n_pairs = 0;
+  int n_tasks = 0;
+};
+
+struct mk_handle {
+  mk_model_desc desc{};
+  int device = 0;
+  int ncta = 0;
+  std::vector<void*> allocs;
+  std::vector<MatHost> mats;
+  std::vector<Layer> layers;
+  Model model{};
+  Model* d_model = nullptr;
+  Mat* d_mats = nullptr;
+  Layer* d_layers = nullptr;
+  uint16_t* embed = nullptr;
+  uint16_t* final_norm = nullptr;
+  std::vector<uint16_t*> attn_norm, ffn_norm;
+  float2* rope = nullptr;
+  int64_t weight_bytes = 0;
+  // scratch
+  float* buf[NBUF] = {};
+  int32_t ld[NBUF] = {};
+  float* ss_part = nullptr;
+  float* am_val = nullptr;
+  int32_t* am_idx = nullptr;
+  float* att_part = nullptr;
+  int att_rows_max = 0;
+  int n_items_max = 0;
+  int max_pairs = 0;
+  uint32_t* ctr = nullptr;
+  int n_ctr = 0;
+  int32_t* status = nullptr;
+  float* logits_tmp = nullptr;
+  int32_t* argmax_tmp = nullptr;
+  std::map<PlanKey, Plan> plans;
+  int32_t* trace_idx = nullptr;
+  float* trace_w = nullptr;
+  int64_t* task_trace = nullptr;
+  int32_t task_trace_cap = 0;
+  int64_t stall_ns = 0;
+  int64_t timeout_ns = 1000000000LL;
+  bool sticky = false;
+  bool initialised = false;
+  std::string err;
+};
+
+struct mk_kv {
+  mk_handle* h;
+  int max_seqs, max_ctx;
+  uint16_t* k = nullptr;
+  uint16_t* v = nullptr;
+  int64_t bytes = 0;
+};
+
+static mk_status fail(mk_handle* h, mk_status s, const std::string& msg) {
+  if (h) h->err = msg;
+  return s;
+}
+
+#define CK(call)                                                                                     \
+  do {                                                                                               \
+    cudaError_t e_ = (call);                                                                         \
+    if (e_ != cudaSuccess) return fail(h, MK_ERR_CUDA, std::string(#call) + ": " + cudaGetErrorString(e_)); \
+  } while (0)
+
+static mk_status dalloc(mk_handle* h, void** p, size_t bytes) {
+  if (bytes == 0) bytes = 16;
+  cudaError_t e = cudaMalloc(p, bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(h, MK_ERR_OOM, "cudaMalloc of " + std::to_string(bytes) + " bytes failed");
+  }
+  h->allocs.push_back(*p);
+  return MK_OK;
+}
+
+static int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+static mk_status add_mat(mk_handle* h, int rows, int cols, int fp8, int gu, const MatMap& mp, int* out_idx) {
+  MatHost mh{};
+  mh.m.rows = rows;
+  mh.m.cols = cols;
+  mh.m.RT = cdiv(rows, 16);
+  mh.m.KT = cdiv(cols, 16);
+  mh.m.fp8 = fp8;
+  mh.m.gu = gu;
+  mh.map = mp;
+  const size_t tb = fp8 ? TILE_FP8 : TILE_BF16;
+  mh.bytes = (size_t)mh.m.RT * mh.m.KT * tb;
+  void* p = nullptr;
+  mk_status s = dalloc(h, &p, mh.bytes);
+  if (s != MK_OK) return s;
+  mh.m.w = reinterpret_cast<const uint8_t*>(p);
+  h->weight_bytes += (int64_t)mh.bytes;
+  if (fp8) {
+    const int lrows = gu ? rows / 2 : rows;
+    mh.m.nbr = cdiv(lrows, 128);
+    mh.m.nbc = cdiv(cols, 128);
+    const size_t sb = (size_t)(gu ? 2 : 1) * mh.m.nbr * mh.m.nbc * sizeof(float);
+    s = dalloc(h, &p, sb);
+    if (s != MK_OK) return s;
+    mh.m.scales = reinterpret_cast<const float*>(p);
+    h->weight_bytes += (int64_t)sb;
+  }
+  *out_idx = (int)h->mats.size();
+  h->mats.push_back(mh);
+  return MK_OK;
+}
+
+static bool desc_ok(const mk_model_desc* d, std::string& why) {
+  if (!d) { why = "null descriptor"; return false; }
+  if (d->layers < 1 || d->hidden < 16 || d->hidden % 16) { why = "hidden must be a positive multiple of 16"; return false; }
+  if (d->vocab < 2) { why = "vocab < 2"; return false; }
+  if (d->max_batch < 1 || d->max_batch > MAXM) { why = "max_batch must be in [1, 8]"; return false; }
+  if (d->max_ctx < 2) { why = "max_ctx < 2"; return false; }
+  if (d->kv_lora_rank > 0) { why = "latent attention is not supported by this build"; return false; }
+  if (d->head_dim != 64 && d->head_dim != 128) { why = "head_dim must be 64 or 128"; return false; }
+  if (d->n_kv_heads < 1 || d->n_q_heads % d->n_kv_heads) { why = "n_q_heads must be a multiple of n_kv_heads"; return false; }
+  if ((d->n_q_heads / d->n_kv_heads) * MAXM > 48) { why = "query heads per kv head must be <= 6"; return false; }
+  if (d->n_routed == 0) {
+    if (d->ffn < 8 || d->ffn % 8) { why = "ffn must be a positive multiple of 8"; return false; }
+  } else {
+    why = "mixture-of-experts layers are not supported by this build";
+    return false;
+  }
+  return true;
+}
+
+extern "C" {
+
+mk_status mk_create(const mk_model_desc* desc, int device, mk_handle** out) {
+  if (!out) return MK_ERR_INVALID;
+  *out = nullptr;
+  std::string why;
+  if (!desc_ok(desc, why)) return MK_ERR_INVALID;
+  mk_handle* h = new mk_handle();
+  h->desc = *desc;
+  h->device = device;
+  mk_status s;
+#define TRY(x)                      \
+  do {                              \
+    s = (x);                        \
+    if (s != MK_OK) goto fail_out;  \
+  } while (0)
+  {
+    if (cudaSetDevice(device) != cudaSuccess) { s = MK_ERR_CUDA; h->err = "cudaSetDevice failed"; goto fail_out; }
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, device) != cudaSuccess) { s = MK_ERR_CUDA; goto fail_out; }
+    if (prop.major < 10) { s = MK_ERR_INVALID; h->err = "needs an sm_100 device"; goto fail_out; }
+    h->ncta = prop.multiProcessorCount;
+    const mk_model_desc& d = *desc;
+    const int L = d.layers, H = d.hidden, Hq = d.n_q_heads, G = d.n_kv_heads, hd = d.head_dim;
+    // ---- weights ----
+    TRY(dalloc(h, (void**)&h->embed, (size_t)d.vocab * H * 2));
+    TRY(dalloc(h, (void**)&h->final_norm, (size_t)H * 2));
+    h->weight_bytes += (int64_t)d.vocab * H * 2 + H * 2;
+    h->layers.resize(L);
+    h->attn_norm.resize(L);
+    h->ffn_norm.resize(L);
+    for (int l = 0; l < L; ++l) {
+      Layer& ly = h->layers[l];
+      TRY(dalloc(h, (void**)&h->attn_norm[l], (size_t)H * 2));
+      TRY(dalloc(h, (void**)&h->ffn_norm[l], (size_t)H * 2));
+      h->weight_bytes += 4LL * H;
+      ly.attn_norm = h->attn_norm[l];
+      ly.ffn_norm = h->ffn_norm[l];
+      MatMap mp{};
+      mp.layer = l;
+      mp.type = MAP_PLAIN;
+      mp.kindA = SYN_WQKV;
+      mp.lcolsA = H;
+      TRY(add_mat(h, (Hq + 2 * G) * hd, H, 0, 0, mp, &ly.m_qkv));
+      mp = MatMap{};
+      mp.layer = l;
+      mp.kindA = SYN_WO;
+      mp.lcolsA = Hq * hd;
+      TRY(add_mat(h, H, Hq * hd, 0, 0, mp, &ly.m_o));
+      mp = MatMap{};
+      mp.layer = l;
+      mp.type = MAP_GU;
+      mp.kindA = SYN_WGATE;
+      mp.kindB = SYN_WUP;
+      mp.lcolsA = mp.lcolsB = H;
+      TRY(add_mat(h, 2 * d.ffn, H, 0, 1, mp, &ly.m_gu));
+      mp = MatMap{};
+      mp.layer = l;
+      mp.kindA = SYN_WDOWN;
+      mp.lcolsA = d.ffn;
+      TRY(add_mat(h, H, d.ffn, 0, 0, mp, &ly.m_down));
+    }
+    {
+      MatMap mp{};
+      mp.kindA = SYN_LM_HEAD;
+      mp.lcolsA = H;
+      TRY(add_mat(h, d.vocab, H, 0, 0, mp, &h->model.m_lm));
+    }
+    // ---- RoPE table, double precision angles rounded to fp32 ----
+    {
+      const int half = hd / 2;
+      std::vector<float2> tab((size_t)d.max_ctx * half);
+      for (int p = 0; p < d.max_ctx; ++p)
+        for (int i = 0; i < half; ++i) {
+          const double inv = pow((double)d.rope_theta, -2.0 * i / (double)hd);
+          const double ang = (double)p * inv;
+          tab[(size_t)p * half + i] = make_float2((float)cos(ang), (float)sin(ang));
+        }
+      TRY(dalloc(h, (void**)&h->rope, tab.size() * sizeof(float2)));
+      if (cudaMemcpy(h->rope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice) != cudaSuccess) {
+        s = MK_ERR_CUDA;
+        goto fail_out;
+      }
+    }
+    // ---- device model tables ----
+    std::vector<Mat> mv;
+    for (auto& m : h->mats) mv.push_back(m.m);
+    TRY(dalloc(h, (void**)&h->d_mats, mv.size() * sizeof(Mat)));
+    TRY(dalloc(h, (void**)&h->d_layers, (size_t)L * sizeof(Layer)));
+    TRY(dalloc(h, (void**)&h->d_model, sizeof(Model)));
+    Model& md = h->model;
+    md.L = L;
+    md.H = H;
+    md.Hq = Hq;
+    md.Hkv = G;
+    md.d = hd;
+    md.I = d.ffn;
+    md.V = d.vocab;
+    md.E = d.n_routed;
+    md.NS = d.n_shared;
+    md.K = d.top_k;
+    md.Ie = d.expert_ffn;
+    md.R = d.kv_lora_rank;
+    md.dr = d.rope_dim;
+    md.fp8 = d.expert_fp8;
+    md.eps = d.rms_eps;
+    md.embed = h->embed;
+    md.final_norm = h->final_norm;
+    md.rope = h->rope;
+    md.rope_ctx = d.max_ctx;
+    md.layers = h->d_layers;
+    md.mats = h->d_mats;
+    if (cudaMemcpy(h->d_mats, mv.data(), mv.size() * sizeof(Mat), cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(h->d_layers, h->layers.data(), (size_t)L * sizeof(Layer), cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(h->d_model, &md, sizeof(Model), cudaMemcpyHostToDevice) != cudaSuccess) {
+      s = MK_ERR_CUDA;
+      goto fail_out;
+    }
+    // ---- scratch ----
+    const int MB = MAXM;
+    const int widths[NBUF] = {H, (Hq + 2 * G) * hd, Hq * hd, std::max(d.ffn, 8), 64};
+    for (int b = 0; b < NBUF; ++b) {
+      h->ld[b] = (widths[b] + 3) & ~3;
+      TRY(dalloc(h, (void**)&h->buf[b], (size_t)MB * h->ld[b] * sizeof(float)));
+    }
+    TRY(dalloc(h, (void**)&h->ss_part, (size_t)2 * h->ncta * MAXM * sizeof(float)));
+    TRY(dalloc(h, (void**)&h->am_val, (size_t)h->ncta * MAXM * sizeof(float)));
+    TRY(dalloc(h, (void**)&h->am_idx, (size_t)h->ncta * MAXM * sizeof(int32_t)));
+    h->max_pairs = d.max_batch * G;
+    h->n_items_max = std::max(h->ncta, h->max_pairs);
+    h->att_rows_max = MAXM * (Hq / G);
+    TRY(dalloc(h, (void**)&h->att_part, (size_t)h->n_items_max * h->att_rows_max * (hd + 2) * sizeof(float)));
+    h->n_ctr = (L + 1) * NCTR_LAYER + L * h->max_pairs + 2;
+    TRY(dalloc(h, (void**)&h->ctr, (size_t)h->n_ctr * sizeof(uint32_t)));
+    TRY(dalloc(h, (void**)&h->status, 4 * sizeof(int32_t)));
+    TRY(dalloc(h, (void**)&h->logits_tmp, 16));
+    TRY(dalloc(h, (void**)&h->argmax_tmp, MAXM * sizeof(int32_t)));
+    if (cudaMemset(h->ctr, 0, (size_t)h->n_ctr * 4) != cudaSuccess || cudaMemset(h->status, 0, 16) != cudaSuccess) {
+      s = MK_ERR_CUDA;
+      goto fail_out;
+    }
+    if (cudaFuncSetAttribute(mk_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess) {
+      s = MK_ERR_CUDA;
+      h->err = "cannot reserve dynamic shared memory";
+      goto fail_out;
+    }
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, mk_step_kernel, NTHREADS, SMEM_BYTES) != cudaSuccess ||
+        occ < 1) {
+      s = MK_ERR_CUDA;
+      h->err = "kernel does not fit one CTA per SM";
+      goto fail_out;
+    }
+  }
+#undef TRY
+  *out = h;
+  return MK_OK;
+fail_out:
+  for (void* p : h->allocs) cudaFree(p);
+  delete h;
+  return s;
+}
+
+void mk_destroy(mk_handle* h) {
+  if (!h) return;
+  cudaSetDevice(h->device);
+  cudaDeviceSynchronize();
+  for (auto& kv : h->plans) {
+    cudaFree(kv.second.d_tasks);
+    cudaFree(kv.second.d_off);
+  }
+  for (void* p : h->allocs) cudaFree(p);
+  delete h;
+}
+
+const char* mk_last_error(const mk_handle* h) { return h ? h->err.c_str() : "null handle"; }
+int64_t mk_weight_bytes(const mk_handle* h) { return h ? h->weight_bytes : 0; }
+
+mk_status mk_launch_info(mk_handle* h, int32_t* ctas, int32_t* smem_bytes, int32_t* threads) {
+  if (!h) return MK_ERR_INVALID;
+  if (ctas) *ctas = h->ncta;
+  if (smem_bytes) *smem_bytes = SMEM_BYTES;
+  if (threads) *threads = NTHREADS;
+  return MK_OK;
+}
+
+// ---------------------------------------------------------------------------
+// weights
+// ---------------------------------------------------------------------------
+static void launch_fill(const MatHost& mh, uint64_t seed, float sigA, float sigB) {
+  const uint64_t kA = syn_key(seed, syn_stream((uint32_t)mh.map.kindA, (uint32_t)mh.map.layer, (uint32_t)mh.map.expert));
+  const uint64_t kB = syn_key(seed, syn_stream((uint32_t)mh.map.kindB, (uint32_t)mh.map.layer, (uint32_t)mh.map.expert));
+  const float sA = mh.m.fp8 ? syn_normal_scale(16.0) : syn_normal_scale(sigA);
+  const float sB = mh.m.fp8 ? syn_normal_scale(16.0) : syn_normal_scale(sigB);
+  const int64_t n = (int64_t)mh.m.RT * mh.m.KT * 32;
+  const int blocks = (int)std::min<int64_t>((n + 255) / 256, 148 * 16);
+  fill_tiles_kernel<<<blocks, 256>>>(const_cast<uint8_t*>(mh.m.w), mh.m.RT, mh.m.KT, mh.m.rows, mh.m.cols, mh.m.fp8,
+                                     mh.map, kA, kB, sA, sB);
+}
+
+static void launch_fill_vec(uint16_t* dst, int64_t n, uint64_t key, float sc, int gain) {
+  const int blocks = (int)std::min<int64_t>((n + 255) / 256, 148 * 16);
+  fill_bf16_kernel<<<blocks, 256>>>(dst, n, key, sc, gain);
+}
+
+mk_status mk_init_random(mk_handle* h, const mk_synth_params* p) {
+  if (!h || !p) return fail(h, MK_ERR_INVALID, "null argument");
+  cudaSetDevice(h->device);
+  const mk_model_desc& d = h->desc;
+  const uint64_t seed = p->seed;
+  launch_fill_vec(h->embed, (int64_t)d.vocab * d.hidden, syn_key(seed, syn_stream(SYN_EMBED, 0, 0)),
+                  syn_normal_scale(p->w_sigma), 0);
+  launch_fill_vec(h->final_norm, d.hidden, syn_key(seed, syn_stream(SYN_FINAL_NORM, 0, 0)),
+                  syn_normal_scale(p->gain_sigma), 1);
+  for (int l = 0; l < d.layers; ++l) {
+    launch_fill_vec(h->attn_norm[l], d.hidden, syn_key(seed, syn_stream(SYN_ATTN_NORM, (uint32_t)l, 0)),
+                    syn_normal_scale(p->gain_sigma), 1);
+    launch_fill_vec(h->ffn_norm[l], d.hidden, syn_key(seed, syn_stream(SYN_FFN_NORM, (uint32_t)l, 0)),
+                    syn_normal_scale(p->gain_sigma), 1);
+  }
+  for (auto& mh : h->mats) {
+    const float sig = (mh.map.kindA == SYN_ROUTER) ? p->router_sigma : p->w_sigma;
+    launch_fill(mh, seed, sig, p->w_sigma);
+  }
+  CK(cudaGetLastError());
+  CK(cudaDeviceSynchronize());
+  h->initialised = true;
+  return MK_OK;
+}
+
+static int find_mat(mk_handle* h, int kind, int layer, int expert, int* which) {
+  for (size_t i = 0; i < h->mats.size(); ++i) {
+    const MatMap& mp = h->mats[i].map;
+    if (mp.layer != layer || mp.expert != expert) continue;
+    if (mp.kindA == kind) { *which = 0; return (int)i; }
+    if ((mp.type == MAP_GU || mp.type == MAP_CONCAT) && mp.kindB == kind) { *which = 1; return (int)i; }
+  }
+  return -1;
+}
+
+mk_status mk_load_weights(mk_handle* h, const mk_tensor_src* ts, int n) {
+  if (!h || (!ts && n > 0)) return fail(h, MK_ERR_INVALID, "null argument");
+  cudaSetDevice(h->device);
+  const mk_model_desc& d = h->desc;
+  for (int i = 0; i < n; ++i) {
+    const mk_tensor_src& t = ts[i];
+    if (!t.data) return fail(h, MK_ERR_INVALID, "tensor " + std::to_string(i) + ": null data");
+    const cudaMemcpyKind kind = t.on_device ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
+    // vectors
+    uint16_t* vec = nullptr;
+    int64_t vlen = 0;
+    if (t.kind == SYN_EMBED) { vec = h->embed; vlen = (int64_t)d.vocab * d.hidden; }
+    else if (t.kind == SYN_FINAL_NORM) { vec = h->final_norm; vlen = d.hidden; }
+    else if (t.kind == SYN_ATTN_NORM || t.kind == SYN_FFN_NORM) {
+      if (t.layer < 0 || t.layer >= d.layers) return fail(h, MK_ERR_INVALID, "layer out of range");
+      vec = (t.kind == SYN_ATTN_NORM ? h->attn_norm : h->ffn_norm)[t.layer];
+      vlen = d.hidden;
+    }
+    if (vec) {
+      if (t.rows * t.cols != vlen) return fail(h, MK_ERR_INVALID, "tensor " + std::to_string(i) + ": wrong size");
+      CK(cudaMemcpy(vec, t.data, (size_t)vlen * 2, kind));
+      continue;
+    }
+    int which = 0;
+    const int mi = find_mat(h, t.kind, t.layer, t.expert, &which);
+    if (mi < 0) return fail(h, MK_ERR_INVALID, "tensor " + std::to_string(i) + ": unknown kind/layer/expert");
+    MatHost& mh = h->mats[mi];
+    int64_t lrows = mh.m.rows, lcols = mh.m.cols;
+    if (mh.map.type == MAP_GU) lrows = mh.m.rows / 2;
+    if (mh.map.type == MAP_CONCAT) lrows = which ? mh.m.rows - mh.map.rowsA : mh.map.rowsA;
+    if (t.rows != lrows || t.cols != lcols)
+      return fail(h, MK_ERR_INVALID, "tensor " + std::to_string(i) + ": shape mismatch");
+    const size_t eb = mh.m.fp8 ? 1 : 2;
+    const size_t nbytes = (size_t)lrows * lcols * eb;
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(t.data);
+    void* staging = nullptr;
+    if (!t.on_device) {
+      CK(cudaMalloc(&staging, nbytes));
+      cudaError_t e = cudaMemcpy(staging, t.data, nbytes, cudaMemcpyHostToDevice);
+      if (e != cudaSuccess) { cudaFree(staging); return fail(h, MK_ERR_CUDA, "weight upload failed"); }
+      src = reinterpret_cast<const uint8_t*>(staging);
+    }
+    const int64_t nthr = (int64_t)mh.m.RT * mh.m.KT * 32;
+    const int blocks = (int)std::min<int64_t>((nthr + 255) / 256, 148 * 16);
+    retile_kernel<<<blocks, 256>>>(const_cast<uint8_t*>(mh.m.w), mh.m.RT, mh.m.KT, mh.m.rows, mh.m.cols, mh.m.fp8,
+                                   mh.map, which, src, lcols);
+    cudaError_t e = cudaDeviceSynchronize();
+    if (staging) cudaFree(staging);
+    if (e != cudaSuccess) return fail(h, MK_ERR_CUDA, std::string("retile: ") + cudaGetErrorString(e));
+    if (mh.m.fp8) {
+      if (!t.scales) return fail(h, MK_ERR_INVALID, "fp8 tensor without scales");
+      const size_t sn = (size_t)mh.m.nbr * mh.m.nbc;
+      float* dst = const_cast<float*>(mh.m.scales) + (mh.m.gu && which ? sn : 0);
+      CK(cudaMemcpy(dst, t.scales, sn * sizeof(float), kind));
+    }
+  }
+  h->initialised = true;
+  return MK_OK;
+}
+
+// ---------------------------------------------------------------------------
+// KV caches
+// ---------------------------------------------------------------------------
+mk_status mk_kv_create(mk_handle* h, int max_seqs, int max_ctx, mk_kv** out) {
+  if (!h || !out) return fail(h, MK_ERR_INVALID, "null argument");
+  *out = nullptr;
+  if (max_seqs < 1 || max_seqs > MAXM || max_ctx < 2 || max_ctx > h->desc.max_ctx)
+    return fail(h, MK_ERR_INVALID, "kv: max_seqs in [1, 8] and max_ctx in [2, model max_ctx] required");
+  cudaSetDevice(h->device);
+  const mk_model_desc& d = h->desc;
+  mk_kv* kv = new mk_kv();
+  kv->h = h;
+  kv->max_seqs = max_seqs;
+  kv->max_ctx = max_ctx;
+  const size_t n = (size_t)d.layers * max_seqs * d.n_kv_heads * max_ctx * d.head_dim;
+  if (cudaMalloc(&kv->k, n * 2) != cudaSuccess || cudaMalloc(&kv->v, n * 2) != cudaSuccess) {
+    cudaGetLastError();
+    cudaFree(kv->k);
+    cudaFree(kv->v);
+    delete kv;
+    return fail(h, MK_ERR_OOM, "kv cache allocation failed");
+  }
+  kv->bytes = (int64_t)n * 4;
+  cudaMemset(kv->k, 0, n * 2);
+  cudaMemset(kv->v, 0, n * 2);
+  CK(cudaDeviceSynchronize());
+  *out = kv;
+  return MK_OK;
+}
+
+void mk_kv_destroy(mk_kv* kv) {
+  if (!kv) return;
+  cudaSetDevice(kv->h->device);
+  cudaDeviceSynchronize();
+  cudaFree(kv->k);
+  cudaFree(kv->v);
+  delete kv;
+}
+
+int64_t mk_kv_bytes(const mk_kv* kv) { return kv ? kv->bytes : 0; }
+
+mk_status mk_kv_fill_random(mk_kv* kv, uint64_t seed, float sigma, int32_t length) {
+  if (!kv) return MK_ERR_INVALID;
+  mk_handle* h = kv->h;
+  if (length < 0 || length > kv->max_ctx) return fail(h, MK_ERR_INVALID, "kv fill length out of range");
+  if (length == 0) return MK_OK;
+  cudaSetDevice(h->device);
+  const mk_model_desc& d = h->desc;
+  const int blocks = 148 * 16;
+  const float sc = syn_normal_scale(sigma);
+  fill_kv_kernel<<<blocks, 256>>>(kv->k, d.layers, kv->max_seqs, d.n_kv_heads, kv->max_ctx, d.head_dim, length, seed,
+                                  SYN_KV_K, sc);
+  fill_kv_kernel<<<blocks, 256>>>(kv->v, d.layers, kv->max_seqs, d.n_kv_heads, kv->max_ctx, d.head_dim, length, seed,
+                                  SYN_KV_V, sc);
+  CK(cudaGetLastError());
+  CK(cudaDeviceSynchronize());
+  return MK_OK;
+}
+
+mk_status mk_kv_copy_out(mk_kv* kv, void* dst) {
+  if (!kv || !dst) return MK_ERR_INVALID;
+  mk_handle* h = kv->h;
+  cudaSetDevice(h->device);
+  const size_t half = (size_t)kv->bytes / 2;
+  CK(cudaMemcpy(dst, kv->k, half, cudaMemcpyDeviceToDevice));
+  CK(cudaMemcpy(reinterpret_cast<uint8_t*>(dst) + half, kv->v, half, cudaMemcpyDeviceToDevice));
+  return MK_OK;
+}
+
+// ---------------------------------------------------------------------------
+// planner: per-CTA task lists for a step of S sequences x Q positions
+// ---------------------------------------------------------------------------
+// Row tiles of one matrix over the CTAs: contiguous ranges, the remainder
+// tiles placed starting at a rotating CTA so that cumulative bytes balance.
+static std::vector<std::pair<int, int>> split_rows(int RT, int ncta, int& rot) {
+  std::vector<std::pair<int, int>> r(ncta);
+  const int base = RT / ncta, rem = RT % ncta;
+  int cur = 0;
+  for (int c = 0; c < ncta; ++c) {
+    const int extra = (((c - rot) % ncta + ncta) % ncta) < rem ? 1 : 0;
+    r[c] = {cur, cur + base + extra};
+    cur += base + extra;
+  }
+  rot = (rot + rem) % ncta;
+  return r;
+}
+
+static Task gemv(int layer, int mat, int rt0, int rt1, int in_kind, int in_buf, int epi, int out_buf, int gain,
+                 int wait_ctr, int wait_tgt, int sig) {
+  Task t{};
+  t.type = T_GEMV;
+  t.layer = (int16_t)layer;
+  t.mat = mat;
+  t.rt0 = rt0;
+  t.rt1 = rt1;
+  t.in_kind = (int16_t)in_kind;
+  t.in_buf = (int16_t)in_buf;
+  t.epi = (int16_t)epi;
+  t.out_buf = (int16_t)out_buf;
+  t.gain = (int16_t)gain;
+  t.wait_ctr = wait_ctr;
+  t.wait_tgt = wait_tgt;
+  t.sig_ctr = sig;
+  return t;
+}
+
+static mk_status get_plan(mk_handle* h, int S, int Q, Plan** out) {
+  auto it = h->plans.find(PlanKey{S, Q});
+  if (it != h->plans.end()) {
+    *out = &it->second;
+    return MK_OK;
+  }
+  const mk_model_desc& d = h->desc;
+  const int ncta = h->ncta, L = d.layers;
+  const int n_pairs = S * d.n_kv_heads;
+  const int n_items = std::max(n_pairs, ncta);
+  auto C = [&](int l, int slot) { return l * NCTR_LAYER + slot; };
+  std::vector<std::vector<Task>> per(ncta);
+  int rot = 0;
+  for (int l = 0; l < L; ++l) {
+    const Layer& ly = h->layers[l];
+    // QKV projection (layer 0 reads the embedding rows directly)
+    {
+      auto rr = split_rows(h->mats[ly.m_qkv].m.RT, ncta, rot);
+      for (int c = 0; c < ncta; ++c) {
+        Task t = gemv(l, ly.m_qkv, rr[c].first, rr[c].second, l == 0 ? IN_EMB_NORM : IN_X_NORM, 0, EPI_STORE, B_QKV,
+                      0, l == 0 ? -1 : C(l - 1, C_DOWN), ncta, C(l, C_QKV));
+        t.ss_src = 1;
+        per[c].push_back(t);
+      }
+    }
+    // attention items
+    for (int i = 0; i < n_items; ++i) {
+      Task t{};
+      t.type = T_ATTN;
+      t.layer = (int16_t)l;
+      t.rt0 = i;
+      t.wait_ctr = C(l, C_QKV);
+      t.wait_tgt = ncta;
+      t.sig_ctr = -1;
+      per[i % ncta].push_back(t);
+    }
+    // output projection + residual
+    {
+      auto rr = split_rows(h->mats[ly.m_o].m.RT, ncta, rot);
+      for (int c = 0; c < ncta; ++c) {
+        Task t = gemv(l, ly.m_o, rr[c].first, rr[c].second, IN_BUF, B_ATTN, EPI_RESID, 0, 0, C(l, C_ATTN), n_pairs,
+                      C(l, C_O));
+        t.resid_emb = (l == 0);
+        t.ss_dst = 0;
+        per[c].push_back(t);
+      }
+    }
+    // gate/up + SwiGLU
+    {
+      auto rr = split_rows(h->mats[ly.m_gu].m.RT, ncta, rot);
+      for (int c = 0; c < ncta; ++c) {
+        Task t = gemv(l, ly.m_gu, rr[c].first, rr[c].second, IN_X_NORM, 0, EPI_SWIGLU, B_H, 1, C(l, C_O), ncta,
+                      C(l, C_GU));
+        t.ss_src = 0;
+        per[c].push_back(t);
+      }
+    }
+    // down projection + residual
+    {
+      auto rr = split_rows(h->mats[ly.m_down].m.RT, ncta, rot);
+      for (int c = 0; c < ncta; ++c) {
+        Task t = gemv(l, ly.m_down, rr[c].first, rr[c].second, IN_BUF, B_H, EPI_RESID, 0, 0, C(l, C_GU), ncta,
+                      C(l, C_DOWN));
+        t.ss_dst = 1;
+        per[c].push_back(t);
+      }
+    }
+  }
+  // final norm + LM head + argmax
+  {
+    auto rr = split_rows(h->mats[h->model.m_lm].m.RT, ncta, rot);
+    for (int c = 0; c < ncta; ++c) {
+      Task t = gemv(L - 1, h->model.m_lm, rr[c].first, rr[c].second, IN_X_NORM, 0, EPI_LOGITS, 0, 2,
+                    C(L - 1, C_DOWN), ncta, -1);
+      t.ss_src = 1;
+      per[c].push_back(t);
+    }
+  }
+  std::vector<Task> flat;
+  std::vector<int32_t> off(ncta + 1, 0);
+  for (int c = 0; c < ncta; ++c) {
+    off[c] = (int32_t)flat.size();
+    flat.insert(flat.end(), per[c].begin(), per[c].end());
+  }
+  off[ncta] = (int32_t)flat.size();
+  Plan p;
+  p.n_items = n_items;
+  p.n_pairs = n_pairs;
+  p.n_tasks = (int)flat.size();
+  CK(cudaMalloc(&p.d_tasks, flat.size() * sizeof(Task)));
+  CK(cudaMalloc(&p.d_off, off.size() * sizeof(int32_t)));
+  CK(cudaMemcpy(p.d_tasks, flat.data(), flat.size() * sizeof(Task), cudaMemcpyHostToDevice));
+  CK(cudaMemcpy(p.d_off, off.data(), off.size() * sizeof(int32_t), cudaMemcpyHostToDevice));
+  auto res = h->plans.emplace(PlanKey{S, Q}, p);
+  *out = &res.first->second;
+  return MK_OK;
+}
+
+// ---------------------------------------------------------------------------
+// compute entry points
+// ---------------------------------------------------------------------------
+static mk_status launch_step(mk_handle* h, mk_kv* kv, int S, int Q, const int32_t* tokens, const int32_t* positions,
+                             int32_t pos_const, float* logits, int32_t* argmax, int32_t* accepted, void* stream) {
+  if (h->sticky) return fail(h, MK_ERR_STATE, "a previous device error is pending; call mk_reset");
+  if (!h->initialised) return fail(h, MK_ERR_STATE, "weights not initialised");
+  cudaSetDevice(h->device);
+  Plan* plan = nullptr;
+  mk_status s = get_plan(h, S, Q, &plan);
+  if (s != MK_OK) return s;
+  Launch P{};
+  P.model = h->d_model;
+  P.tasks = plan->d_tasks;
+  P.task_off = plan->d_off;
+  P.tokens = tokens;
+  P.positions = positions;
+  P.pos_const = pos_const;
+  P.S = S;
+  P.Q = Q;
+  P.M = S * Q;
+  P.kv_k = kv->k;
+  P.kv_v = kv->v;
+  P.kv_seqs = kv->max_seqs;
+  P.kv_ctx = kv->max_ctx;
+  P.logits = logits;
+  P.argmax = argmax ? argmax : h->argmax_tmp;
+  P.accepted = accepted;
+  P.router_idx = h->trace_idx;
+  P.router_w = h->trace_w;
+  for (int b = 0; b < NBUF; ++b) {
+    P.buf[b] = h->buf[b];
+    P.ld[b] = h->ld[b];
+  }
+  P.ss_part = h->ss_part;
+  P.am_val = h->am_val;
+  P.am_idx = h->am_idx;
+  P.att_part = h->att_part;
+  P.att_rows_max = h->att_rows_max;
+  P.ctr = h->ctr;
+  P.ctr_layer_stride = NCTR_LAYER;
+  P.ctr_pair_base = (h->desc.layers + 1) * NCTR_LAYER;
+  P.ctr_lm = P.ctr_pair_base + h->desc.layers * h->max_pairs;
+  P.ctr_done = P.ctr_lm + 1;
+  P.n_ctr = h->n_ctr;
+  P.status = h->status;
+  P.timeout_ns = h->stall_ns > 0 ? h->stall_ns : h->timeout_ns;
+  P.stall_ctr = h->stall_ns > 0 ? (h->desc.layers * NCTR_LAYER + C_STALL) : -1;
+  P.n_items = plan->n_items;
+  P.n_pairs = plan->n_pairs;
+  P.trace = h->task_trace;
+  P.trace_cap = h->task_trace_cap;
+  h->stall_ns = 0;
+  void* args[] = {&P};
+  cudaError_t e = cudaLaunchCooperativeKernel((const void*)mk_step_kernel, dim3(h->ncta), dim3(NTHREADS), args,
+                                              SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(h, MK_ERR_CUDA, std::string("launch: ") + cudaGetErrorString(e));
+  return MK_OK;
+}
+
+mk_status mk_decode_step(mk_handle* h, const int32_t* tokens, const int32_t* positions, int B, mk_kv* kv,
+                         float* logits_out, int32_t* argmax_out, void* stream) {
+  if (!h) return MK_ERR_INVALID;
+  if (!tokens || !positions || !kv || !argmax_out) return fail(h, MK_ERR_INVALID, "null argument");
+  if (kv->h != h) return fail(h, MK_ERR_INVALID, "kv cache belongs to another model");
+  if (B < 1 || B > h->desc.max_batch || B > kv->max_seqs) return fail(h, MK_ERR_INVALID, "B out of range");
+  return launch_step(h, kv, B, 1, tokens, positions, 0, logits_out, argmax_out, nullptr, stream);
+}
+
+mk_status mk_verify(mk_handle* h, const int32_t* tokens8, int n_prop, int32_t position, mk_kv* kv, float* logits_out,
+                    int32_t* argmax_out, int32_t* accepted_out, void* stream) {
+  if (!h) return MK_ERR_INVALID;
+  if (!tokens8 || !kv || !argmax_out || !accepted_out) return fail(h, MK_ERR_INVALID, "null argument");
+  if (kv->h != h) return fail(h, MK_ERR_INVALID, "kv cache belongs to another model");
+  if (n_prop < 0 || n_prop + 1 > h->desc.max_batch || n_prop + 1 > MAXM)
+    return fail(h, MK_ERR_INVALID, "n_prop out of range");
+  if (position < 0 || position + n_prop + 1 > kv->max_ctx) return fail(h, MK_ERR_INVALID, "position out of range");
+  return launch_step(h, kv, 1, n_prop + 1, tokens8, nullptr, position, logits_out, argmax_out, accepted_out, stream);
+}
+
+mk_status mk_set_router_trace(mk_handle* h, int32_t* idx_dev, float* w_dev) {
+  if (!h) return MK_ERR_INVALID;
+  h->trace_idx = idx_dev;
+  h->trace_w = w_dev;
+  return MK_OK;
+}
+
+mk_status mk_set_trace(mk_handle* h, int64_t* trace_dev, int32_t max_tasks_per_cta) {
+  if (!h || max_tasks_per_cta < 0) return MK_ERR_INVALID;
+  h->task_trace = trace_dev;
+  h->task_trace_cap = trace_dev ? max_tasks_per_cta : 0;
+  return MK_OK;
+}
+
+mk_status mk_sync_status(mk_handle* h) {
+  if (!h) return MK_ERR_INVALID;
+  cudaSetDevice(h->device);
+  int32_t st[4] = {0, 0, 0, 0};
+  CK(cudaMemcpy(st, h->status, sizeof st, cudaMemcpyDeviceToHost));
+  if (st[0] != 0) {
+    h->sticky = true;
+    h->err = std::string(st[0] == DERR_TIMEOUT ? "device dependency wait timed out" : "device bounds error") +
+             " (detail " + std::to_string(st[2]) + ")";
+    return (mk_status)st[0];
+  }
+  return MK_OK;
+}
+
+mk_status mk_reset(mk_handle* h) {
+  if (!h) return MK_ERR_INVALID;
+  cudaSetDevice(h->device);
+  CK(cudaDeviceSynchronize());
+  CK(cudaMemset(h->status, 0, 16));
+  CK(cudaMemset(h->ctr, 0, (size_t)h->n_ctr * 4));
+  CK(cudaDeviceSynchronize());
+  h->sticky = false;
+  return MK_OK;
+}
+
+mk_status mk_debug_inject_stall(mk_handle* h, int64_t timeout_ns) {
+  if (!h || timeout_ns < 0) return MK_ERR_INVALID;
+  h->stall_ns = timeout_ns;
+  return MK_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,154 @@
+// mk_internal.h - structures shared by the host planner and the persistent
+// kernel.  Nothing here is part of the public ABI.
+#pragma once
+#include <stdint.h>
+
+namespace mk {
+
+// ---------------------------------------------------------------------------
+// kernel geometry
+// ---------------------------------------------------------------------------
+constexpr int NCW = 8;                       // consumer warps
+constexpr int WARP_WP = NCW;                 // weight producer warp
+constexpr int WARP_XP = NCW + 1;             // activation producer warp
+constexpr int NTHREADS = (NCW + 2) * 32;
+constexpr int NCT = NCW * 32;                // consumer threads
+constexpr int STAGE_BYTES = 34816;           // one ring stage (= 2 x 64 rows x 272 B)
+constexpr int TILE_CAP = 32768;              // weight tile bytes per GEMV chunk (gains follow)
+constexpr int NSTAGE = 4;                    // weight ring depth
+constexpr int XSLOTS = 4;                    // activation ring depth
+constexpr int XSLOT_BYTES = 8192;            // one activation slice: M rows x (cols + pad)
+constexpr int XROW_PAD = 32;                 // bytes between activation rows (bank spread)
+constexpr int ATT_BYTES = 40960;             // GEMV reduction / attention scratch
+constexpr int NEWKV_BYTES = 8704;            // K/V rows of the step's own new positions
+constexpr int MISC_BYTES = 4096;
+constexpr int SMEM_BYTES =
+    NSTAGE * STAGE_BYTES + XSLOTS * XSLOT_BYTES + ATT_BYTES + NEWKV_BYTES + MISC_BYTES;
+constexpr int RMAX = 8;                      // row tiles per chunk
+constexpr int CPW = 4;                       // col tiles per warp per chunk
+constexpr int MAXM = 8;                      // activation rows per step (S * Q)
+constexpr int ATT_CT = 64;                   // cache positions per attention chunk
+constexpr int TILE_BF16 = 512;               // 16x16 bf16 tile in A-fragment order
+constexpr int TILE_FP8 = 256;                // 16x16 e4m3 tile in A-fragment order
+
+// ---------------------------------------------------------------------------
+// tasks
+// ---------------------------------------------------------------------------
+enum TaskType : int16_t {
+  T_GEMV = 1,      // out rows [rt0, rt1) of a matrix
+  T_ATTN = 2,      // one split-KV attention item (GQA)
+  T_MOE_GU = 3,    // routed expert gate/up tiles (data dependent)
+  T_MOE_DOWN = 4,  // down projection over shared + selected experts
+  T_TOPK = 5,      // (unused placeholder)
+};
+
+enum InKind : int16_t {
+  IN_X_NORM = 0,   // residual x [M][H] with RMSNorm (scales from per-CTA partial sums)
+  IN_EMB_NORM = 1, // embedding rows of the tokens, RMSNorm computed in the prologue
+  IN_BUF = 2,      // plain fp32 buffer [M][ld]
+};
+
+enum Epi : int16_t {
+  EPI_STORE = 0,   // out[m][row] = v
+  EPI_RESID = 1,   // x[m][row] = base + v, base = x or the embedding (layer 0)
+  EPI_SWIGLU = 2,  // tile rows 0..7 gate, 8..15 up: h[m][i] = silu(g) u
+  EPI_LOGITS = 3,  // logits + per-CTA argmax partial
+};
+
+enum BufId : int16_t {
+  B_X = 0, B_QKV = 1, B_ATTN = 2, B_H = 3, B_RLOG = 4, NBUF = 5
+};
+
+struct Task {
+  int16_t type, layer;
+  int16_t in_kind, epi;
+  int16_t in_buf, out_buf;
+  int16_t resid_emb, gain;   // resid base = embedding; gain: 0 attn, 1 ffn, 2 final
+  int32_t mat;               // matrix table index
+  int32_t rt0, rt1;          // row tiles (GEMV) / item index (ATTN)
+  int32_t wait_ctr, wait_tgt;
+  int32_t sig_ctr;           // counter incremented when the task is done (-1: none)
+  int32_t ss_src;            // IN_X_NORM: which partial-sum array (0: after O, 1: after down)
+  int32_t ss_dst;            // EPI_RESID: partial-sum array written
+};
+
+// ---------------------------------------------------------------------------
+// device-resident model description
+// ---------------------------------------------------------------------------
+struct Mat {
+  const uint8_t* w;          // tiles [RT][KT][tile]
+  const float* scales;       // fp8: [nbr][nbc] (GU: [2][nbr][nbc], gate then up)
+  int32_t rows, cols, RT, KT;
+  int32_t fp8;
+  int32_t nbr, nbc;
+  int32_t gu;                // rows interleaved gate/up by 8
+};
+
+struct Layer {
+  const uint16_t* attn_norm;
+  const uint16_t* ffn_norm;
+  int32_t m_qkv, m_o, m_gu, m_down;
+};
+
+struct Model {
+  int32_t L, H, Hq, Hkv, d, I, V;
+  int32_t E, NS, K, Ie;
+  int32_t R, dr, fp8;
+  float eps;
+  const uint16_t* embed;     // [V][H] row-major bf16
+  const uint16_t* final_norm;
+  int32_t m_lm;
+  const float2* rope;        // [max_ctx][d/2] (cos, sin)
+  int32_t rope_ctx;
+  const Layer* layers;
+  const Mat* mats;
+};
+
+// Per-launch arguments (passed by value).
+struct Launch {
+  const Model* model;
+  const Task* tasks;
+  const int32_t* task_off;   // [nCTA + 1]
+  // step inputs
+  const int32_t* tokens;     // dev [M]
+  const int32_t* positions;  // dev [S] or null (then pos_const)
+  int32_t pos_const;
+  int32_t S, Q, M;
+  // KV cache
+  uint16_t* kv_k;
+  uint16_t* kv_v;
+  int32_t kv_seqs, kv_ctx;
+  // outputs
+  float* logits;             // [M][V] or null
+  int32_t* argmax;           // [M]
+  int32_t* accepted;         // [1] or null
+  int32_t* router_idx;       // trace or null
+  float* router_w;
+  // scratch
+  float* buf[NBUF];
+  int32_t ld[NBUF];
+  float* ss_part;            // [2][nCTA][MAXM]
+  float* am_val;             // [nCTA][MAXM]
+  int32_t* am_idx;
+  float* att_part;           // [items][rows][d + 2]
+  int32_t att_rows_max;
+  uint32_t* ctr;             // counters
+  int32_t ctr_layer_stride;  // counters per layer
+  int32_t ctr_pair_base;     // offset of per-(layer, pair) counters
+  int32_t ctr_lm, ctr_done;
+  int32_t n_ctr;
+  int32_t* status;           // [0] error code, [1] abort flag, [2] detail
+  int64_t timeout_ns;
+  int32_t stall_ctr;         // test hook: >= 0 -> first consumer waits on this counter
+  int32_t n_items;           // attention items per layer
+  int32_t n_pairs;           // S * Hkv
+  int64_t* trace;            // [nCTA][trace_cap][8] or null
+  int32_t trace_cap;
+};
+
+// counter slots inside one layer
+enum CtrSlot { C_QKV = 0, C_ATTN = 1, C_O = 2, C_GU = 3, C_DOWN = 4, C_ROUTER = 5, C_STALL = 6, NCTR_LAYER = 8 };
+
+enum DevErr { DERR_NONE = 0, DERR_TIMEOUT = 4, DERR_BOUNDS = 5 };
+
+}  // namespace mk

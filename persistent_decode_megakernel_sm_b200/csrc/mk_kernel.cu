@@ -1,0 +1,1422 @@
+// mk_kernel.cu - the persistent decode-step kernel for sm_100a.
+//
+// One launch evaluates a whole decoder step ("700 TPS on Kimi K3: A Case for
+// TPU Megakernels", section "Why megakernels?": the whole decoder step is one
+// program, so a weight load is not tied to the kernel that consumes it).
+//
+// B200 mapping:
+//   - grid = one CTA per SM (cooperative launch guarantees co-residency);
+//   - each CTA runs a host-planned task list (GEMV row tiles, attention items);
+//   - warp 8 is a producer: it walks the same task list and streams every
+//     weight tile and KV-cache row the CTA will consume into a 5-stage shared
+//     memory ring with cp.async.bulk (TMA) + mbarrier complete_tx.  Weights do
+//     not depend on activations, so the producer never waits on another CTA:
+//     it runs ahead across task and layer boundaries (the cross-layer
+//     prefetch of section "Our Kimi K3 megakernel");
+//   - warps 0..7 consume: they wait on a global dependency counter (acquire),
+//     compute with mma.sync m16n8k16 on the tile in shared memory, write
+//     their outputs and release-increment the next counter.  Activations are
+//     fp32; tensor-core operands carry them as a bf16 hi + lo pair (about 16
+//     significant bits), so accumulation matches fp32 GEMV to ~1e-5.
+//   - every wait is bounded by %globaltimer; on expiry a CTA records the
+//     error, raises a global abort flag that all CTAs poll, drains its own
+//     in-flight bulk copies and returns.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+#include "mk_internal.h"
+
+namespace mk {
+
+// ---------------------------------------------------------------------------
+// PTX helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bulk (non-tensor) TMA copy global -> shared, completion on an mbarrier,
+// with an L2 policy (weights and cache rows are streamed once per step).
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void bar_consumers() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ int ld_volatile_i32(const int32_t* p) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t atom_add_acqrel(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint4 lds128(const void* p) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(smem_u32(p)));
+  return v;
+}
+__device__ __forceinline__ uint2 lds64(const void* p) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(smem_u32(p)));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds32(const void* p) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds16(const void* p) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(smem_u32(p)));
+  return v;
+}
+
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint4 a, uint32_t b0, uint32_t b1) {
+  asm(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_f16(float (&d)[4], uint4 a, uint32_t b0, uint32_t b1) {
+  asm(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo_elem, float hi_elem) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo_elem, hi_elem);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+// fp32 pair -> bf16 hi pair + bf16 residual pair.
+__device__ __forceinline__ void split_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  float2 hf = __bfloat1622float2(h);
+  __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+  hi = *reinterpret_cast<uint32_t*>(&h);
+  lo = *reinterpret_cast<uint32_t*>(&l);
+}
+__device__ __forceinline__ void split_f16(float a, float b, uint32_t& hi, uint32_t& lo) {
+  __half2 h = __floats2half2_rn(a, b);
+  float2 hf = __half22float2(h);
+  __half2 l = __floats2half2_rn(a - hf.x, b - hf.y);
+  hi = *reinterpret_cast<uint32_t*>(&h);
+  lo = *reinterpret_cast<uint32_t*>(&l);
+}
+__device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+__device__ __forceinline__ uint32_t fp8x2_to_f16x2(uint32_t two) {
+  __half2_raw r = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xFFFFu), __NV_E4M3);
+  return (uint32_t)r.x | ((uint32_t)r.y << 16);
+}
+__device__ __forceinline__ uint4 fp8_frag_to_f16(uint2 v) {
+  uint4 a;
+  a.x = fp8x2_to_f16x2(v.x);
+  a.y = fp8x2_to_f16x2(v.x >> 16);
+  a.z = fp8x2_to_f16x2(v.y);
+  a.w = fp8x2_to_f16x2(v.y >> 16);
+  return a;
+}
+
+// ---------------------------------------------------------------------------
+// shared state
+// ---------------------------------------------------------------------------
+struct Misc {
+  uint64_t full[NSTAGE];
+  uint64_t empty[NSTAGE];
+  uint64_t xfull[XSLOTS];
+  uint64_t xempty[XSLOTS];
+  float scale[MAXM];
+  volatile int abort;
+  int flag;
+  int pad[2];
+  // per-task trace accumulators (consumer thread 0)
+  long long tr_wf, tr_wx, tr_bytes;
+  int tr_chunks;
+};
+
+struct Ctx {
+  const Launch* P;
+  const Model* md;
+  Misc* ms;
+  uint8_t* ring;
+  uint8_t* xring;
+  uint8_t* att;
+  uint8_t* newkv;
+  int ncta;
+};
+
+__device__ __forceinline__ bool global_abort(const Launch& P) { return ld_volatile_i32(P.status + 1) != 0; }
+
+__device__ void raise_error(const Launch& P, Misc* ms, int code, int detail) {
+  atomicCAS(P.status, 0, code);
+  atomicExch(P.status + 2, detail);
+  atomicExch(P.status + 1, 1);
+  ms->abort = 1;
+}
+
+// ---------------------------------------------------------------------------
+// chunk iteration (identical in producer and consumers)
+// ---------------------------------------------------------------------------
+struct ChunkIt {
+  int rt1, KT, tb, gsz, xcap;
+  int g0, nr, KC, c0, nc;
+  __device__ __forceinline__ void set_group() {
+    nr = min(RMAX, rt1 - g0);
+    if (gsz > 0) {
+      int nb = (g0 / gsz + 1) * gsz;
+      nr = min(nr, nb - g0);
+    }
+    KC = min(min(KT, TILE_CAP / (nr * tb)), min(NCW * CPW, xcap));
+  }
+  // xcap: most col tiles whose activation slice (M rows) fits one x slot
+  __device__ __forceinline__ bool init(int rt0_, int rt1_, int KT_, int tb_, int gsz_, int xcap_) {
+    rt1 = rt1_;
+    KT = KT_;
+    tb = tb_;
+    gsz = gsz_;
+    xcap = xcap_;
+    g0 = rt0_;
+    if (g0 >= rt1) return false;
+    set_group();
+    c0 = 0;
+    nc = min(KC, KT);
+    return true;
+  }
+  __device__ __forceinline__ bool next() {
+    c0 += KC;
+    if (c0 >= KT) {
+      g0 += nr;
+      if (g0 >= rt1) return false;
+      set_group();
+      c0 = 0;
+    }
+    nc = min(KC, KT - c0);
+    return true;
+  }
+  __device__ __forceinline__ bool group_done() const { return c0 + KC >= KT; }
+  __device__ __forceinline__ uint32_t bytes() const { return (uint32_t)(nr * nc * tb); }
+};
+
+// Activation element size and the x-slot column cap of a GEMV task.
+__device__ __forceinline__ int x_esize(const Task& t) { return t.in_kind == IN_EMB_NORM ? 2 : 4; }
+__device__ __forceinline__ int x_cap(const Task& t, int M) {
+  return (XSLOT_BYTES / M - XROW_PAD) / (16 * x_esize(t));
+}
+__device__ __forceinline__ int x_rowbytes(const Task& t, int nc) { return nc * 16 * x_esize(t) + XROW_PAD; }
+__device__ __forceinline__ const uint16_t* task_gain(const Model& md, const Task& t) {
+  if (t.in_kind == IN_BUF) return nullptr;
+  const Layer* ly = md.layers + t.layer;
+  return t.gain == 0 ? ly->attn_norm : (t.gain == 1 ? ly->ffn_norm : md.final_norm);
+}
+
+// Attention item -> (pair, split index, number of splits, first item of pair).
+struct Item {
+  int pair, j, ns, first;
+};
+__device__ __forceinline__ Item decode_item(int item, int n_pairs, int n_items) {
+  Item it;
+  if (n_pairs >= n_items) {
+    it.pair = item;
+    it.j = 0;
+    it.ns = 1;
+    it.first = item;
+  } else {
+    it.pair = (int)(((int64_t)item * n_pairs) / n_items);
+    it.first = (int)(((int64_t)it.pair * n_items + n_pairs - 1) / n_pairs);
+    int nxt = (int)(((int64_t)(it.pair + 1) * n_items + n_pairs - 1) / n_pairs);
+    it.ns = nxt - it.first;
+    it.j = item - it.first;
+  }
+  return it;
+}
+
+__device__ __forceinline__ int seq_pos0(const Launch& P, int s) {
+  return P.positions ? __ldg(P.positions + s) : P.pos_const;
+}
+
+__device__ __forceinline__ int att_pitch(int d) { return d * 2 + 16; }
+
+// ---------------------------------------------------------------------------
+// producer warp
+// ---------------------------------------------------------------------------
+// Reserve ring slot `it` for `bytes` (lane 0 waits for the consumers to free
+// it, then arms the full barrier).  Returns false on abort.
+__device__ bool prod_reserve(const Ctx& C, uint32_t it, uint32_t bytes) {
+  const int lane = threadIdx.x & 31;
+  int ok = 1;
+  if (lane == 0) {
+    const int s = it % NSTAGE;
+    if (it >= (uint32_t)NSTAGE) {
+      const uint32_t par = ((it / NSTAGE) + 1) & 1;
+      uint64_t t0 = 0;
+      uint32_t spins = 0;
+      while (!mbar_try_wait(&C.ms->empty[s], par)) {
+        if (++spins >= 64) {
+          spins = 0;
+          if (C.ms->abort || global_abort(*C.P)) { ok = 0; break; }
+          uint64_t now = globaltimer();
+          if (t0 == 0) t0 = now;
+          else if (now - t0 > (uint64_t)C.P->timeout_ns * 2) {
+            raise_error(*C.P, C.ms, DERR_TIMEOUT, 0x10000 | s);
+            ok = 0;
+            break;
+          }
+        }
+      }
+    }
+    if (ok) mbar_arrive_expect_tx(&C.ms->full[s], bytes);
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  return ok != 0;
+}
+
+__device__ void producer(const Ctx& C) {
+  const Launch& P = *C.P;
+  const Model& md = *C.md;
+  const int lane = threadIdx.x & 31;
+  const uint64_t pol = policy_evict_first();
+  uint32_t it = 0;
+  const int beg = P.task_off[blockIdx.x], end = P.task_off[blockIdx.x + 1];
+  for (int ti = beg; ti < end; ++ti) {
+    const Task t = P.tasks[ti];
+    if (t.type == T_GEMV) {
+      const Mat& m = md.mats[t.mat];
+      const int tb = m.fp8 ? TILE_FP8 : TILE_BF16;
+      const uint16_t* gain = task_gain(md, t);
+      ChunkIt ci;
+      if (ci.init(t.rt0, t.rt1, m.KT, tb, 0, x_cap(t, P.M))) {
+        do {
+          const uint32_t gbytes = gain ? (uint32_t)(ci.nc * 32) : 0u;
+          if (!prod_reserve(C, it, ci.bytes() + gbytes)) goto drain;
+          uint8_t* dst = C.ring + (size_t)(it % NSTAGE) * STAGE_BYTES;
+          if (lane < ci.nr) {
+            const uint8_t* src = m.w + ((size_t)(ci.g0 + lane) * m.KT + ci.c0) * tb;
+            bulk_g2s(dst + (size_t)lane * ci.nc * tb, src, (uint32_t)(ci.nc * tb), &C.ms->full[it % NSTAGE], pol);
+          } else if (lane == 31 && gain) {
+            // the norm gain slice of these columns follows the tiles
+            bulk_g2s(dst + ci.bytes(), gain + ci.c0 * 16, gbytes, &C.ms->full[it % NSTAGE], pol);
+          }
+          __syncwarp();
+          ++it;
+        } while (ci.next());
+      }
+    } else if (t.type == T_ATTN) {
+      const Item itm = decode_item(t.rt0, P.n_pairs, P.n_items);
+      const int s = itm.pair / md.Hkv, g = itm.pair % md.Hkv;
+      const int T0 = seq_pos0(P, s);
+      const int a = (int)(((int64_t)itm.j * T0) / itm.ns), b = (int)(((int64_t)(itm.j + 1) * T0) / itm.ns);
+      const int d = md.d, pitch = att_pitch(d);
+      const size_t head = (((size_t)t.layer * P.kv_seqs + s) * md.Hkv + g) * (size_t)P.kv_ctx;
+      for (int t0 = a; t0 < b; t0 += ATT_CT) {
+        const int n = min(ATT_CT, b - t0);
+        if (!prod_reserve(C, it, (uint32_t)(2 * n * d * 2))) goto drain;
+        uint8_t* dst = C.ring + (size_t)(it % NSTAGE) * STAGE_BYTES;
+        for (int i = lane; i < n; i += 32) {
+          bulk_g2s(dst + (size_t)i * pitch, P.kv_k + (head + t0 + i) * d, (uint32_t)(d * 2), &C.ms->full[it % NSTAGE], pol);
+          bulk_g2s(dst + (size_t)(ATT_CT + i) * pitch, P.kv_v + (head + t0 + i) * d, (uint32_t)(d * 2),
+                   &C.ms->full[it % NSTAGE], pol);
+        }
+        __syncwarp();
+        ++it;
+      }
+    }
+  }
+drain:
+  // Wait (bounded) for every bulk copy this CTA issued, so none is in flight
+  // when the CTA exits, whether it finished or aborted.
+  if (lane == 0) {
+    for (int s = 0; s < NSTAGE; ++s) {
+      if (it <= (uint32_t)s) continue;
+      const uint32_t last = it - 1 - ((it - 1 - s) % NSTAGE);
+      const uint32_t par = (last / NSTAGE) & 1;
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(&C.ms->full[s], par)) {
+        if (globaltimer() - t0 > (uint64_t)P.timeout_ns) break;
+      }
+    }
+  }
+  __syncwarp();
+}
+
+// ---------------------------------------------------------------------------
+// activation producer warp
+// ---------------------------------------------------------------------------
+// Walks the same task list.  For each GEMV task it waits for the task's
+// dependency (acquire), then streams the activation slice of every chunk
+// (M rows x the chunk's columns) into the x ring with bulk copies, so the
+// consumers never wait on a global-memory round trip inside a task.
+__device__ bool xprod_wait_counter(const Ctx& C, int idx, uint32_t target) {
+  const Launch& P = *C.P;
+  const int lane = threadIdx.x & 31;
+  int ok = 1;
+  if (lane == 0) {
+    const uint32_t* p = P.ctr + idx;
+    uint64_t t0 = 0;
+    uint32_t spins = 0;
+    while ((int)(ld_acquire(p) - target) < 0) {
+      if (C.ms->abort) { ok = 0; break; }
+      __nanosleep(64);
+      if (++spins >= 16) {
+        spins = 0;
+        if (global_abort(P)) { C.ms->abort = 1; ok = 0; break; }
+        uint64_t now = globaltimer();
+        if (t0 == 0) t0 = now;
+        else if (now - t0 > (uint64_t)P.timeout_ns * 2) {
+          raise_error(P, C.ms, DERR_TIMEOUT, 0x30000 | idx);
+          ok = 0;
+          break;
+        }
+      }
+    }
+    // later bulk (async-proxy) reads must observe the generic-proxy writes
+    // that the acquire made visible
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  return ok != 0;
+}
+
+__device__ bool xprod_reserve(const Ctx& C, uint32_t ix, uint32_t bytes) {
+  const int lane = threadIdx.x & 31;
+  int ok = 1;
+  if (lane == 0) {
+    const int s = ix % XSLOTS;
+    if (ix >= (uint32_t)XSLOTS) {
+      const uint32_t par = ((ix / XSLOTS) + 1) & 1;
+      uint64_t t0 = 0;
+      uint32_t spins = 0;
+      while (!mbar_try_wait(&C.ms->xempty[s], par)) {
+        if (++spins >= 64) {
+          spins = 0;
+          if (C.ms->abort || global_abort(*C.P)) { ok = 0; break; }
+          uint64_t now = globaltimer();
+          if (t0 == 0) t0 = now;
+          else if (now - t0 > (uint64_t)C.P->timeout_ns * 2) {
+            raise_error(*C.P, C.ms, DERR_TIMEOUT, 0x40000 | s);
+            ok = 0;
+            break;
+          }
+        }
+      }
+    }
+    if (ok) mbar_arrive_expect_tx(&C.ms->xfull[s], bytes);
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  return ok != 0;
+}
+
+__device__ void xproducer(const Ctx& C) {
+  const Launch& P = *C.P;
+  const Model& md = *C.md;
+  const int lane = threadIdx.x & 31;
+  const int M = P.M;
+  const uint64_t pol = policy_evict_last();
+  uint32_t ix = 0;
+  const int beg = P.task_off[blockIdx.x], end = P.task_off[blockIdx.x + 1];
+  if (P.stall_ctr >= 0) return;
+  for (int ti = beg; ti < end; ++ti) {
+    const Task t = P.tasks[ti];
+    if (t.type != T_GEMV) continue;
+    const Mat& m = md.mats[t.mat];
+    const int tb = m.fp8 ? TILE_FP8 : TILE_BF16;
+    ChunkIt ci;
+    if (!ci.init(t.rt0, t.rt1, m.KT, tb, 0, x_cap(t, M))) continue;
+    if (t.wait_ctr >= 0 && !xprod_wait_counter(C, t.wait_ctr, (uint32_t)t.wait_tgt)) goto drain;
+    do {
+      const int es = x_esize(t);
+      const int rb = x_rowbytes(t, ci.nc);
+      const uint32_t rowdata = (uint32_t)(ci.nc * 16 * es);
+      if (!xprod_reserve(C, ix, (uint32_t)M * rowdata)) goto drain;
+      uint8_t* dst = C.xring + (size_t)(ix % XSLOTS) * XSLOT_BYTES;
+      if (lane < M) {
+        const uint8_t* src;
+        if (t.in_kind == IN_EMB_NORM) {
+          src = reinterpret_cast<const uint8_t*>(md.embed + (size_t)__ldg(P.tokens + lane) * md.H + ci.c0 * 16);
+        } else {
+          const int b = t.in_kind == IN_X_NORM ? (int)B_X : (int)t.in_buf;
+          src = reinterpret_cast<const uint8_t*>(P.buf[b] + (size_t)lane * P.ld[b] + ci.c0 * 16);
+        }
+        bulk_g2s(dst + (size_t)lane * rb, src, rowdata, &C.ms->xfull[ix % XSLOTS], pol);
+      }
+      __syncwarp();
+      ++ix;
+    } while (ci.next());
+  }
+drain:
+  if (lane == 0) {
+    for (int s = 0; s < XSLOTS; ++s) {
+      if (ix <= (uint32_t)s) continue;
+      const uint32_t last = ix - 1 - ((ix - 1 - s) % XSLOTS);
+      const uint32_t par = (last / XSLOTS) & 1;
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(&C.ms->xfull[s], par)) {
+        if (globaltimer() - t0 > (uint64_t)P.timeout_ns) break;
+      }
+    }
+  }
+  __syncwarp();
+}
+
+// ---------------------------------------------------------------------------
+// consumer helpers
+// ---------------------------------------------------------------------------
+// Wait for ring slot `it` to be filled.  On an abort the wait ends without
+// the data; callers keep walking their task list (so every consumer thread
+// passes the same barriers) and the outputs of the step are discarded.
+__device__ void wait_full(const Ctx& C, uint32_t it) {
+  const int s = it % NSTAGE;
+  const uint32_t par = (it / NSTAGE) & 1;
+  uint32_t spins = 0;
+  uint64_t t0 = 0;
+  const bool tr = C.P->trace && threadIdx.x == 0;
+  const long long c0 = tr ? clock64() : 0;
+  if (tr) C.ms->tr_chunks++;
+  while (!mbar_try_wait(&C.ms->full[s], par)) {
+    if (++spins >= 64) {
+      spins = 0;
+      if (C.ms->abort) return;
+      uint64_t now = globaltimer();
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > (uint64_t)C.P->timeout_ns * 2) {
+        raise_error(*C.P, C.ms, DERR_TIMEOUT, 0x20000 | s);
+        return;
+      }
+    }
+  }
+  if (tr) C.ms->tr_wf += clock64() - c0;
+}
+
+__device__ __forceinline__ void release_stage(const Ctx& C, uint32_t it) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(&C.ms->empty[it % NSTAGE]);
+}
+
+// Thread 0 decides, every consumer thread gets the same answer (a barrier
+// on each side of the read keeps the flag slot free for the next use).
+__device__ __forceinline__ int broadcast_from0(const Ctx& C, int v) {
+  if (threadIdx.x == 0) C.ms->flag = v;
+  bar_consumers();
+  const int r = C.ms->flag;
+  bar_consumers();
+  return r;
+}
+
+// Wait until counter `idx` reaches `target` (thread 0 polls with acquire).
+// Ends early, without the dependency, when the step is being aborted.
+__device__ void wait_counter(const Ctx& C, int idx, uint32_t target) {
+  const Launch& P = *C.P;
+  if (threadIdx.x == 0) {
+    const uint32_t* p = P.ctr + idx;
+    uint64_t t0 = 0;
+    uint32_t spins = 0;
+    while ((int)(ld_acquire(p) - target) < 0) {
+      if (C.ms->abort) break;
+      __nanosleep(64);
+      if (++spins >= 16) {
+        spins = 0;
+        if (global_abort(P)) { C.ms->abort = 1; break; }
+        uint64_t now = globaltimer();
+        if (t0 == 0) t0 = now;
+        else if (now - t0 > (uint64_t)P.timeout_ns) {
+          raise_error(P, C.ms, DERR_TIMEOUT, idx);
+          break;
+        }
+      }
+    }
+  }
+  bar_consumers();
+}
+
+__device__ __forceinline__ void signal_counter(const Ctx& C, int idx) {
+  bar_consumers();
+  if (threadIdx.x == 0 && !C.ms->abort) {
+    __threadfence();
+    red_release_add(C.P->ctr + idx, 1u);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// GEMV task: out rows [rt0, rt1) of W (16-row tiles) times M activation rows
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
+
+__device__ void wait_x(const Ctx& C, uint32_t ix) {
+  const int s = ix % XSLOTS;
+  const uint32_t par = (ix / XSLOTS) & 1;
+  uint32_t spins = 0;
+  uint64_t t0 = 0;
+  const bool tr = C.P->trace && threadIdx.x == 0;
+  const long long c0 = tr ? clock64() : 0;
+  while (!mbar_try_wait(&C.ms->xfull[s], par)) {
+    if (++spins >= 64) {
+      spins = 0;
+      if (C.ms->abort) return;
+      uint64_t now = globaltimer();
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > (uint64_t)C.P->timeout_ns * 2) {
+        raise_error(*C.P, C.ms, DERR_TIMEOUT, 0x50000 | s);
+        return;
+      }
+    }
+  }
+  if (tr) C.ms->tr_wx += clock64() - c0;
+}
+
+__device__ void gemv_task(const Ctx& C, const Task& t, uint32_t& it, uint32_t& ix) {
+  const Launch& P = *C.P;
+  const Model& md = *C.md;
+  const Mat& m = md.mats[t.mat];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, tq = lane & 3;
+  const int M = P.M;
+  const int tb = m.fp8 ? TILE_FP8 : TILE_BF16;
+  const bool emb = t.in_kind == IN_EMB_NORM;
+  const bool has_gain = t.in_kind != IN_BUF;
+
+  // ---- prologue: RMSNorm scale per activation row (fixed-order reductions) ----
+  if (t.in_kind == IN_X_NORM) {
+    if (warp < M) {
+      const float* src = P.ss_part + (size_t)t.ss_src * C.ncta * MAXM;
+      float ss = 0.f;
+      for (int c = lane; c < C.ncta; c += 32) ss += __ldcg(src + c * MAXM + warp);
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if (lane == 0) C.ms->scale[warp] = rsqrtf(ss / (float)md.H + md.eps);
+    }
+  } else if (emb) {
+    if (warp < M) {
+      const uint16_t* e = md.embed + (size_t)__ldg(P.tokens + warp) * md.H;
+      float ss = 0.f;
+      for (int k = lane * 2; k < md.H; k += 64) {
+        uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(e + k));
+        float a = bf16lo(u), b = bf16hi(u);
+        ss += a * a + b * b;
+      }
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if (lane == 0) C.ms->scale[warp] = rsqrtf(ss / (float)md.H + md.eps);
+    }
+  }
+  bar_consumers();
+  const float sc = (g < M && has_gain) ? C.ms->scale[g] : 1.0f;
+
+  float acc[RMAX][4];
+  float ss_acc[2] = {0.f, 0.f};
+  float am_v[2] = {-INFINITY, -INFINITY};
+  int am_i[2] = {0x7fffffff, 0x7fffffff};
+#pragma unroll
+  for (int r = 0; r < RMAX; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
+
+  ChunkIt ci;
+  bool have = ci.init(t.rt0, t.rt1, m.KT, tb, 0, x_cap(t, M));
+  float* red = reinterpret_cast<float*>(C.att);
+  while (have) {
+    wait_x(C, ix);
+    wait_full(C, it);
+    const uint8_t* stage = C.ring + (size_t)(it % NSTAGE) * STAGE_BYTES;
+    const uint8_t* xs = C.xring + (size_t)(ix % XSLOTS) * XSLOT_BYTES + (size_t)g * x_rowbytes(t, ci.nc);
+    const uint8_t* gs = stage + ci.bytes();
+    // activation fragments (hi/lo) of this warp's col tiles j = warp + 8 i
+    uint32_t bh[CPW][2], bl[CPW][2];
+#pragma unroll
+    for (int i = 0; i < CPW; ++i) {
+      const int j = warp + NCW * i;
+      float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+      if (j < ci.nc && g < M) {
+        if (emb) {
+          const uint32_t a = lds32(xs + (j * 16 + 2 * tq) * 2);
+          const uint32_t b = lds32(xs + (j * 16 + 2 * tq + 8) * 2);
+          y0 = bf16lo(a);
+          y1 = bf16hi(a);
+          y2 = bf16lo(b);
+          y3 = bf16hi(b);
+        } else {
+          const uint2 a = lds64(xs + (j * 16 + 2 * tq) * 4);
+          const uint2 b = lds64(xs + (j * 16 + 2 * tq + 8) * 4);
+          y0 = __uint_as_float(a.x);
+          y1 = __uint_as_float(a.y);
+          y2 = __uint_as_float(b.x);
+          y3 = __uint_as_float(b.y);
+        }
+        if (has_gain) {
+          const uint32_t g01 = lds32(gs + (j * 16 + 2 * tq) * 2);
+          const uint32_t g89 = lds32(gs + (j * 16 + 2 * tq + 8) * 2);
+          y0 = y0 * sc * bf16lo(g01);
+          y1 = y1 * sc * bf16hi(g01);
+          y2 = y2 * sc * bf16lo(g89);
+          y3 = y3 * sc * bf16hi(g89);
+        }
+      }
+      if (!m.fp8) {
+        split_bf16(y0, y1, bh[i][0], bl[i][0]);
+        split_bf16(y2, y3, bh[i][1], bl[i][1]);
+      } else {
+        split_f16(y0, y1, bh[i][0], bl[i][0]);
+        split_f16(y2, y3, bh[i][1], bl[i][1]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < CPW; ++i) {
+      const int j = warp + NCW * i;
+      if (j < ci.nc) {
+        if (!m.fp8) {
+          // all A fragments first, then the hi sweep, then the lo sweep:
+          // RMAX independent accumulator chains keep the tensor pipe busy
+          uint4 a[RMAX];
+#pragma unroll
+          for (int r = 0; r < RMAX; ++r)
+            if (r < ci.nr) a[r] = lds128(stage + ((size_t)r * ci.nc + j) * TILE_BF16 + lane * 16);
+#pragma unroll
+          for (int r = 0; r < RMAX; ++r)
+            if (r < ci.nr) mma_bf16(acc[r], a[r], bh[i][0], bh[i][1]);
+#pragma unroll
+          for (int r = 0; r < RMAX; ++r)
+            if (r < ci.nr) mma_bf16(acc[r], a[r], bl[i][0], bl[i][1]);
+        } else {
+          const int c = ci.c0 + j;
+          uint2 a8[RMAX];
+#pragma unroll
+          for (int r = 0; r < RMAX; ++r)
+            if (r < ci.nr) a8[r] = lds64(stage + ((size_t)r * ci.nc + j) * TILE_FP8 + lane * 8);
+#pragma unroll
+          for (int r = 0; r < RMAX; ++r) {
+            if (r < ci.nr) {
+              const uint4 a = fp8_frag_to_f16(a8[r]);
+              float tmp[4] = {0.f, 0.f, 0.f, 0.f};
+              mma_f16(tmp, a, bh[i][0], bh[i][1]);
+              mma_f16(tmp, a, bl[i][0], bl[i][1]);
+              const int rt = ci.g0 + r;
+              float s_top, s_bot;
+              if (m.gu) {
+                const int rb = rt >> 4;
+                s_top = __ldg(m.scales + rb * m.nbc + (c >> 3));
+                s_bot = __ldg(m.scales + (size_t)m.nbr * m.nbc + rb * m.nbc + (c >> 3));
+              } else {
+                s_top = s_bot = __ldg(m.scales + (rt >> 3) * m.nbc + (c >> 3));
+              }
+              acc[r][0] += s_top * tmp[0];
+              acc[r][1] += s_top * tmp[1];
+              acc[r][2] += s_bot * tmp[2];
+              acc[r][3] += s_bot * tmp[3];
+            }
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(&C.ms->empty[it % NSTAGE]);
+      mbar_arrive(&C.ms->xempty[ix % XSLOTS]);
+    }
+    ++it;
+    ++ix;
+
+    if (ci.group_done()) {
+      // ---- cross-warp reduction and epilogue for row tiles [g0, g0 + nr) ----
+#pragma unroll
+      for (int r = 0; r < RMAX; ++r)
+        if (r < ci.nr)
+          *reinterpret_cast<float4*>(red + ((warp * RMAX + r) * 32 + lane) * 4) =
+              make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+      bar_consumers();
+      {
+        const int r = tid >> 5, l = lane;
+        if (r < ci.nr) {
+          float v[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int w = 0; w < NCW; ++w) {
+            float4 q = *reinterpret_cast<const float4*>(red + ((w * RMAX + r) * 32 + l) * 4);
+            v[0] += q.x;
+            v[1] += q.y;
+            v[2] += q.z;
+            v[3] += q.w;
+          }
+          const int rt = ci.g0 + r;
+          const int row0 = rt * 16 + (l >> 2), row1 = row0 + 8;
+          const int m0 = 2 * (l & 3), m1 = m0 + 1;
+          if (t.epi == EPI_STORE) {
+            float* out = P.buf[t.out_buf];
+            const int ld = P.ld[t.out_buf];
+            if (row0 < m.rows) {
+              if (m0 < M) out[(size_t)m0 * ld + row0] = v[0];
+              if (m1 < M) out[(size_t)m1 * ld + row0] = v[1];
+            }
+            if (row1 < m.rows) {
+              if (m0 < M) out[(size_t)m0 * ld + row1] = v[2];
+              if (m1 < M) out[(size_t)m1 * ld + row1] = v[3];
+            }
+          } else if (t.epi == EPI_RESID) {
+            float* x = P.buf[B_X];
+            const int ld = P.ld[B_X];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int row = (q < 2) ? row0 : row1;
+              const int mm = (q & 1) ? m1 : m0;
+              if (row < m.rows && mm < M) {
+                float base;
+                if (t.resid_emb) {
+                  const uint16_t* e = md.embed + (size_t)__ldg(P.tokens + mm) * md.H;
+                  base = __uint_as_float((uint32_t)__ldg(e + row) << 16);
+                } else {
+                  base = __ldcg(x + (size_t)mm * ld + row);
+                }
+                const float nv = base + v[q];
+                x[(size_t)mm * ld + row] = nv;
+                ss_acc[q & 1] += nv * nv;
+              }
+            }
+          } else if (t.epi == EPI_SWIGLU) {
+            float* h = P.buf[t.out_buf];
+            const int ld = P.ld[t.out_buf];
+            const int i = rt * 8 + (l >> 2);
+            if (i * 2 < m.rows) {
+              if (m0 < M) h[(size_t)m0 * ld + i] = silu_f(v[0]) * v[2];
+              if (m1 < M) h[(size_t)m1 * ld + i] = silu_f(v[1]) * v[3];
+            }
+          } else if (t.epi == EPI_LOGITS) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int row = (q < 2) ? row0 : row1;
+              const int mm = (q & 1) ? m1 : m0;
+              if (row < m.rows && mm < M) {
+                if (P.logits) P.logits[(size_t)mm * md.V + row] = v[q];
+                const int k = q & 1;
+                if (v[q] > am_v[k] || (v[q] == am_v[k] && row < am_i[k])) {
+                  am_v[k] = v[q];
+                  am_i[k] = row;
+                }
+              }
+            }
+          }
+        }
+      }
+      bar_consumers();
+#pragma unroll
+      for (int r = 0; r < RMAX; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
+    }
+    have = ci.next();
+  }
+
+  // ---- task-level partials: sum of squares (RESID) or argmax (LOGITS) ----
+  if (t.epi == EPI_RESID || t.epi == EPI_LOGITS) {
+    float* f2 = reinterpret_cast<float*>(C.att);
+    int* i2 = reinterpret_cast<int*>(C.att + NCT * 2 * sizeof(float));
+    if (t.epi == EPI_RESID) {
+      f2[tid * 2 + 0] = ss_acc[0];
+      f2[tid * 2 + 1] = ss_acc[1];
+    } else {
+      f2[tid * 2 + 0] = am_v[0];
+      f2[tid * 2 + 1] = am_v[1];
+      i2[tid * 2 + 0] = am_i[0];
+      i2[tid * 2 + 1] = am_i[1];
+    }
+    bar_consumers();
+    if (tid < MAXM) {
+      const int mm = tid, tsel = mm >> 1, k = mm & 1;
+      if (t.epi == EPI_RESID) {
+        float s = 0.f;
+        for (int th = tsel; th < NCT; th += 4) s += f2[th * 2 + k];
+        P.ss_part[((size_t)t.ss_dst * C.ncta + blockIdx.x) * MAXM + mm] = s;
+      } else {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+        for (int th = tsel; th < NCT; th += 4) {
+          const float v = f2[th * 2 + k];
+          const int ix = i2[th * 2 + k];
+          if (v > bv || (v == bv && ix < bi)) {
+            bv = v;
+            bi = ix;
+          }
+        }
+        P.am_val[(size_t)blockIdx.x * MAXM + mm] = bv;
+        P.am_idx[(size_t)blockIdx.x * MAXM + mm] = bi;
+      }
+    }
+  }
+}
+
+// Last CTA to finish the LM head reduces the per-CTA argmax partials and,
+// for a verify step, the greedy acceptance.
+__device__ void lm_finish(const Ctx& C) {
+  const Launch& P = *C.P;
+  bar_consumers();
+  int last = 0;
+  if (threadIdx.x == 0 && !C.ms->abort) {
+    __threadfence();
+    const uint32_t old = atom_add_acqrel(P.ctr + P.ctr_lm, 1u);
+    last = (old == (uint32_t)C.ncta - 1) ? 1 : 0;
+  }
+  if (!broadcast_from0(C, last)) return;
+  {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp < P.M) {
+      const int mm = warp;
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+      for (int c = lane; c < C.ncta; c += 32) {
+        const float v = __ldcg(P.am_val + (size_t)c * MAXM + mm);
+        const int ix = __ldcg(P.am_idx + (size_t)c * MAXM + mm);
+        if (v > bv || (v == bv && ix < bi)) {
+          bv = v;
+          bi = ix;
+        }
+      }
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      if (lane == 0) {
+        P.argmax[mm] = bi;
+        C.ms->scale[mm] = __int_as_float(bi);
+      }
+    }
+  }
+  bar_consumers();
+  if (threadIdx.x == 0 && P.accepted) {
+    // tokens[0] = anchor, tokens[1..Q-1] = proposals; argmax[j] = greedy after position j
+    int a = 0;
+    while (a + 1 < P.Q && __ldg(P.tokens + a + 1) == __float_as_int(C.ms->scale[a])) ++a;
+    P.accepted[0] = a;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// GQA attention item: split-KV flash decoding with mma.sync
+// ---------------------------------------------------------------------------
+// Shared layout inside the attention scratch:
+//   Q fragments (hi, lo): [mt][d/16][32 lanes][16 B]
+//   P fragments (hi, lo): [mt][ATT_CT/16][32 lanes][16 B]
+//   smax: [2][NCW][48] fp32
+__device__ __forceinline__ int frag_off(int r, int k, int KTn) {
+  // byte offset of element (row r, col k) in an A-fragment tile array [mt][KTn][32][8 x 2B]
+  const int mi = r >> 4, rr = r & 15, kt = k >> 4, kk = k & 15;
+  const int ln = (rr & 7) * 4 + ((kk & 7) >> 1);
+  const int e = (kk & 1) + 2 * (rr >> 3) + 4 * (kk >> 3);
+  return (((mi * KTn + kt) * 32 + ln) * 8 + e) * 2;
+}
+
+struct AttState {
+  float o[3][2][4];   // [mt][n-tile of this warp][frag]
+  float M[3][2];      // running max (log2 units) of rows g, g+8 of each m-tile
+  float L[3][2];      // lane-partial running sums
+};
+
+// Process one chunk of n_valid cache positions whose K and V rows are in
+// shared memory (row pitch = 2d + 16 bytes).  causal: position i is visible
+// to query row r iff i <= r / gh.
+__device__ void att_chunk(const Ctx& C, AttState& st, const uint8_t* Ks, const uint8_t* Vs, int n_valid, bool causal,
+                          int gh, int mt, int d, int par) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, tq = lane & 3;
+  const int pitch = att_pitch(d);
+  const int KTq = d / 16;
+  uint8_t* qhi = C.att;
+  uint8_t* qlo = qhi + mt * KTq * 512;
+  uint8_t* phi = qlo + mt * KTq * 512;
+  uint8_t* plo = phi + mt * (ATT_CT / 16) * 512;
+  float* smax = reinterpret_cast<float*>(plo + mt * (ATT_CT / 16) * 512);
+
+  // ---- scores for positions [8 warp, 8 warp + 8) ----
+  float sacc[3][4];
+#pragma unroll
+  for (int mi = 0; mi < 3; ++mi) sacc[mi][0] = sacc[mi][1] = sacc[mi][2] = sacc[mi][3] = 0.f;
+  const int n0 = warp * 8;
+  if (n0 < n_valid) {
+    const uint8_t* krow = Ks + (size_t)(n0 + g) * pitch + tq * 4;
+    for (int ks = 0; ks < KTq; ++ks) {
+      const uint32_t b0 = lds32(krow + ks * 32);
+      const uint32_t b1 = lds32(krow + ks * 32 + 16);
+#pragma unroll
+      for (int mi = 0; mi < 3; ++mi) {
+        if (mi < mt) {
+          const uint4 ah = lds128(qhi + ((mi * KTq + ks) * 32 + lane) * 16);
+          const uint4 al = lds128(qlo + ((mi * KTq + ks) * 32 + lane) * 16);
+          mma_bf16(sacc[mi], ah, b0, b1);
+          mma_bf16(sacc[mi], al, b0, b1);
+        }
+      }
+    }
+  }
+  // masking and per-row max over this warp's 8 positions
+  const int p0 = n0 + 2 * tq, p1 = p0 + 1;
+  float* smx = smax + par * NCW * 48;
+#pragma unroll
+  for (int mi = 0; mi < 3; ++mi) {
+    if (mi < mt) {
+      const int rA = mi * 16 + g, rB = rA + 8;
+      const bool vA0 = p0 < n_valid && (!causal || p0 <= rA / gh);
+      const bool vA1 = p1 < n_valid && (!causal || p1 <= rA / gh);
+      const bool vB0 = p0 < n_valid && (!causal || p0 <= rB / gh);
+      const bool vB1 = p1 < n_valid && (!causal || p1 <= rB / gh);
+      if (!vA0) sacc[mi][0] = -INFINITY;
+      if (!vA1) sacc[mi][1] = -INFINITY;
+      if (!vB0) sacc[mi][2] = -INFINITY;
+      if (!vB1) sacc[mi][3] = -INFINITY;
+      float mA = fmaxf(sacc[mi][0], sacc[mi][1]), mB = fmaxf(sacc[mi][2], sacc[mi][3]);
+      mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 1));
+      mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 2));
+      mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 1));
+      mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 2));
+      if (tq == 0) {
+        smx[warp * 48 + rA] = mA;
+        smx[warp * 48 + rB] = mB;
+      }
+    }
+  }
+  bar_consumers();
+  // ---- online softmax update; P fragments written in A layout ----
+  const int kt = warp >> 1;
+  const int regA = (warp & 1) ? 2 : 0;  // u32 slot of row g within the lane's 16 bytes
+#pragma unroll
+  for (int mi = 0; mi < 3; ++mi) {
+    if (mi < mt) {
+      const int rA = mi * 16 + g, rB = rA + 8;
+      float cm[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int w = 0; w < NCW; ++w) {
+        cm[0] = fmaxf(cm[0], smx[w * 48 + rA]);
+        cm[1] = fmaxf(cm[1], smx[w * 48 + rB]);
+      }
+      float pv[4];
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const float mnew = fmaxf(st.M[mi][h2], cm[h2]);
+        const float corr = (mnew == -INFINITY) ? 1.f : exp2f(st.M[mi][h2] - mnew);
+        const float msafe = (mnew == -INFINITY) ? 0.f : mnew;
+        st.M[mi][h2] = mnew;
+        pv[2 * h2 + 0] = exp2f(sacc[mi][2 * h2 + 0] - msafe);
+        pv[2 * h2 + 1] = exp2f(sacc[mi][2 * h2 + 1] - msafe);
+        st.L[mi][h2] = st.L[mi][h2] * corr + pv[2 * h2 + 0] + pv[2 * h2 + 1];
+#pragma unroll
+        for (int jn = 0; jn < 2; ++jn) {
+          st.o[mi][jn][2 * h2 + 0] *= corr;
+          st.o[mi][jn][2 * h2 + 1] *= corr;
+        }
+      }
+      uint32_t hA, lA, hB, lB;
+      split_bf16(pv[0], pv[1], hA, lA);
+      split_bf16(pv[2], pv[3], hB, lB);
+      uint32_t* ph = reinterpret_cast<uint32_t*>(phi + ((mi * (ATT_CT / 16) + kt) * 32 + lane) * 16);
+      uint32_t* pl = reinterpret_cast<uint32_t*>(plo + ((mi * (ATT_CT / 16) + kt) * 32 + lane) * 16);
+      ph[regA] = hA;
+      ph[regA + 1] = hB;
+      pl[regA] = lA;
+      pl[regA + 1] = lB;
+    }
+  }
+  bar_consumers();
+  // ---- O += P V ; this warp owns dim tiles (8 dims each) ----
+  const int ntile = d / 8;
+  const int per_w = ntile / NCW;  // 2 for d = 128, 1 for d = 64
+  for (int ks = 0; ks < ATT_CT / 16; ++ks) {
+    if (ks * 16 >= n_valid) break;
+    const int pk = ks * 16 + 2 * tq;
+#pragma unroll
+    for (int jn = 0; jn < 2; ++jn) {
+      if (jn < per_w) {
+        const int dim = (warp * per_w + jn) * 8 + g;
+        const uint8_t* vc = Vs + dim * 2;
+        const uint32_t v0 = pk < n_valid ? lds16(vc + (size_t)pk * pitch) : 0u;
+        const uint32_t v1 = pk + 1 < n_valid ? lds16(vc + (size_t)(pk + 1) * pitch) : 0u;
+        const uint32_t v8 = pk + 8 < n_valid ? lds16(vc + (size_t)(pk + 8) * pitch) : 0u;
+        const uint32_t v9 = pk + 9 < n_valid ? lds16(vc + (size_t)(pk + 9) * pitch) : 0u;
+        const uint32_t b0 = v0 | (v1 << 16), b1 = v8 | (v9 << 16);
+#pragma unroll
+        for (int mi = 0; mi < 3; ++mi) {
+          if (mi < mt) {
+            const uint4 ah = lds128(phi + ((mi * (ATT_CT / 16) + ks) * 32 + lane) * 16);
+            const uint4 al = lds128(plo + ((mi * (ATT_CT / 16) + ks) * 32 + lane) * 16);
+            mma_bf16(st.o[mi][jn], ah, b0, b1);
+            mma_bf16(st.o[mi][jn], al, b0, b1);
+          }
+        }
+      }
+    }
+  }
+}
+
+__device__ void attn_task(const Ctx& C, const Task& t, uint32_t& it) {
+  const Launch& P = *C.P;
+  const Model& md = *C.md;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, tq = lane & 3;
+  const Item itm = decode_item(t.rt0, P.n_pairs, P.n_items);
+  const int s = itm.pair / md.Hkv, kvh = itm.pair % md.Hkv;
+  const int d = md.d, pitch = att_pitch(d), KTq = d / 16;
+  const int gh = md.Hq / md.Hkv, Q = P.Q, nr = Q * gh, mt = (nr + 15) >> 4;
+  const int T0 = seq_pos0(P, s);
+  const int a = (int)(((int64_t)itm.j * T0) / itm.ns), b = (int)(((int64_t)(itm.j + 1) * T0) / itm.ns);
+  const bool last = itm.j == itm.ns - 1;
+  const float qscale = rsqrtf((float)d) * 1.4426950408889634f;
+  const float* qkv = P.buf[B_QKV];
+  const int ldq = P.ld[B_QKV];
+  const float2* rope = md.rope;
+  const int half = d / 2;
+
+  // ---- stage Q (RoPE, scaled to log2 units) as bf16 hi/lo A fragments ----
+  uint8_t* qhi = C.att;
+  uint8_t* qlo = qhi + mt * KTq * 512;
+  for (int e = tid; e < mt * 16 * half; e += NCT) {
+    const int r = e / half, i = e % half;
+    float x0 = 0.f, x1 = 0.f;
+    if (r < nr) {
+      const int qi = r / gh, hh = r % gh;
+      const int mrow = s * Q + qi;
+      const int pos = T0 + qi;
+      const float* q = qkv + (size_t)mrow * ldq + (size_t)(kvh * gh + hh) * d;
+      const float a0 = __ldcg(q + i), a1 = __ldcg(q + i + half);
+      const float2 cs = __ldg(rope + (size_t)pos * half + i);
+      x0 = (a0 * cs.x - a1 * cs.y) * qscale;
+      x1 = (a0 * cs.y + a1 * cs.x) * qscale;
+    }
+    __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
+    __nv_bfloat16 l0 = __float2bfloat16_rn(x0 - __bfloat162float(h0));
+    __nv_bfloat16 l1 = __float2bfloat16_rn(x1 - __bfloat162float(h1));
+    *reinterpret_cast<__nv_bfloat16*>(qhi + frag_off(r, i, KTq)) = h0;
+    *reinterpret_cast<__nv_bfloat16*>(qhi + frag_off(r, i + half, KTq)) = h1;
+    *reinterpret_cast<__nv_bfloat16*>(qlo + frag_off(r, i, KTq)) = l0;
+    *reinterpret_cast<__nv_bfloat16*>(qlo + frag_off(r, i + half, KTq)) = l1;
+  }
+  // ---- the step's own new positions: RoPE(k), bf16, append to the cache ----
+  uint8_t* nk = C.newkv;
+  uint8_t* nv = C.newkv + 16 * pitch;
+  if (last) {
+    const size_t head = (((size_t)t.layer * P.kv_seqs + s) * md.Hkv + kvh) * (size_t)P.kv_ctx;
+    for (int e = tid; e < 16 * half; e += NCT) {
+      const int qi = e / half, i = e % half;
+      __nv_bfloat16 k0 = __float2bfloat16_rn(0.f), k1 = k0, v0 = k0, v1 = k0;
+      if (qi < Q) {
+        const int mrow = s * Q + qi, pos = T0 + qi;
+        const float* kr = qkv + (size_t)mrow * ldq + (size_t)(md.Hq + kvh) * d;
+        const float* vr = qkv + (size_t)mrow * ldq + (size_t)(md.Hq + md.Hkv + kvh) * d;
+        const float a0 = __ldcg(kr + i), a1 = __ldcg(kr + i + half);
+        const float2 cs = __ldg(rope + (size_t)pos * half + i);
+        k0 = __float2bfloat16_rn(a0 * cs.x - a1 * cs.y);
+        k1 = __float2bfloat16_rn(a0 * cs.y + a1 * cs.x);
+        v0 = __float2bfloat16_rn(__ldcg(vr + i));
+        v1 = __float2bfloat16_rn(__ldcg(vr + i + half));
+        __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(P.kv_k) + (head + pos) * d;
+        __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(P.kv_v) + (head + pos) * d;
+        kc[i] = k0;
+        kc[i + half] = k1;
+        vc[i] = v0;
+        vc[i + half] = v1;
+      }
+      *reinterpret_cast<__nv_bfloat16*>(nk + qi * pitch + i * 2) = k0;
+      *reinterpret_cast<__nv_bfloat16*>(nk + qi * pitch + (i + half) * 2) = k1;
+      *reinterpret_cast<__nv_bfloat16*>(nv + qi * pitch + i * 2) = v0;
+      *reinterpret_cast<__nv_bfloat16*>(nv + qi * pitch + (i + half) * 2) = v1;
+    }
+  }
+  bar_consumers();
+
+  AttState st;
+#pragma unroll
+  for (int mi = 0; mi < 3; ++mi) {
+    st.M[mi][0] = st.M[mi][1] = -INFINITY;
+    st.L[mi][0] = st.L[mi][1] = 0.f;
+#pragma unroll
+    for (int jn = 0; jn < 2; ++jn) st.o[mi][jn][0] = st.o[mi][jn][1] = st.o[mi][jn][2] = st.o[mi][jn][3] = 0.f;
+  }
+  int par = 0;
+  for (int t0 = a; t0 < b; t0 += ATT_CT) {
+    const int n = min(ATT_CT, b - t0);
+    wait_full(C, it);
+    const uint8_t* stage = C.ring + (size_t)(it % NSTAGE) * STAGE_BYTES;
+    att_chunk(C, st, stage, stage + (size_t)ATT_CT * pitch, n, false, gh, mt, d, par);
+    par ^= 1;
+    bar_consumers();  // every warp is done with the stage
+    release_stage(C, it);
+    ++it;
+  }
+  if (last) {
+    att_chunk(C, st, nk, nv, Q, true, gh, mt, d, par);
+    par ^= 1;
+  }
+  bar_consumers();
+
+  // ---- write the item's partial (M, L, O) per query row ----
+  float* smx = reinterpret_cast<float*>(C.att + 2 * mt * KTq * 512 + 2 * mt * (ATT_CT / 16) * 512);
+#pragma unroll
+  for (int mi = 0; mi < 3; ++mi) {
+    if (mi < mt) {
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        float l = st.L[mi][h2];
+        l += __shfl_xor_sync(0xffffffffu, l, 1);
+        l += __shfl_xor_sync(0xffffffffu, l, 2);
+        if (tq == 0) smx[warp * 48 + mi * 16 + g + 8 * h2] = l;
+      }
+    }
+  }
+  bar_consumers();
+  const int rows_max = P.att_rows_max;
+  float* part = P.att_part + (size_t)t.rt0 * rows_max * (d + 2);
+  if (tid < nr) {
+    float l = 0.f;
+    for (int w = 0; w < NCW; ++w) l += smx[w * 48 + tid];
+    part[(size_t)tid * (d + 2) + 1] = l;
+  }
+  if (warp == 0 && tq == 0) {
+#pragma unroll
+    for (int mi = 0; mi < 3; ++mi)
+      if (mi < mt) {
+        if (mi * 16 + g < nr) part[(size_t)(mi * 16 + g) * (d + 2)] = st.M[mi][0];
+        if (mi * 16 + g + 8 < nr) part[(size_t)(mi * 16 + g + 8) * (d + 2)] = st.M[mi][1];
+      }
+  }
+  {
+    const int per_w = (d / 8) / NCW;
+#pragma unroll
+    for (int mi = 0; mi < 3; ++mi) {
+      if (mi < mt) {
+#pragma unroll
+        for (int jn = 0; jn < 2; ++jn) {
+          if (jn < per_w) {
+            const int dim = (warp * per_w + jn) * 8 + 2 * tq;
+            const int rA = mi * 16 + g, rB = rA + 8;
+            if (rA < nr) {
+              part[(size_t)rA * (d + 2) + 2 + dim] = st.o[mi][jn][0];
+              part[(size_t)rA * (d + 2) + 3 + dim] = st.o[mi][jn][1];
+            }
+            if (rB < nr) {
+              part[(size_t)rB * (d + 2) + 2 + dim] = st.o[mi][jn][2];
+              part[(size_t)rB * (d + 2) + 3 + dim] = st.o[mi][jn][3];
+            }
+          }
+        }
+      }
+    }
+  }
+
+  // ---- the last item of this (sequence, kv head) combines all splits ----
+  bar_consumers();
+  int lastc = 0;
+  if (tid == 0 && !C.ms->abort) {
+    __threadfence();
+    const int pc = P.ctr_pair_base + t.layer * P.n_pairs + itm.pair;
+    const uint32_t old = atom_add_acqrel(P.ctr + pc, 1u);
+    lastc = (old == (uint32_t)itm.ns - 1) ? 1 : 0;
+  }
+  if (broadcast_from0(C, lastc)) {
+    float* out = P.buf[B_ATTN];
+    const int ldo = P.ld[B_ATTN];
+    // per (row, split) weight exp2(m_j - m*) / L*, one warp per row
+    float* wsh = reinterpret_cast<float*>(C.att);
+    const int ns = itm.ns;
+    for (int r = warp; r < nr; r += NCW) {
+      float mj[5], lj[5];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < 5; ++q) {
+        const int jj = lane + 32 * q;
+        mj[q] = -INFINITY;
+        lj[q] = 0.f;
+        if (jj < ns) {
+          const float* pp = P.att_part + ((size_t)(itm.first + jj) * rows_max + r) * (d + 2);
+          mj[q] = __ldcg(pp);
+          lj[q] = __ldcg(pp + 1);
+        }
+        mx = fmaxf(mx, mj[q]);
+      }
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      float den = 0.f, w[5];
+#pragma unroll
+      for (int q = 0; q < 5; ++q) {
+        w[q] = (mj[q] == -INFINITY) ? 0.f : exp2f(mj[q] - mx);
+        den += w[q] * lj[q];
+      }
+      for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+#pragma unroll
+      for (int q = 0; q < 5; ++q) {
+        const int jj = lane + 32 * q;
+        if (jj < ns) wsh[r * 160 + jj] = w[q] / den;
+      }
+    }
+    bar_consumers();
+    for (int e = tid; e < nr * d; e += NCT) {
+      const int r = e / d, k = e % d;
+      const float* wr = wsh + r * 160;
+      float num = 0.f;
+#pragma unroll 8
+      for (int jj = 0; jj < ns; ++jj)
+        num += wr[jj] * __ldcg(P.att_part + ((size_t)(itm.first + jj) * rows_max + r) * (d + 2) + 2 + k);
+      const int qi = r / gh, hh = r % gh;
+      out[(size_t)(s * Q + qi) * ldo + (size_t)(kvh * gh + hh) * d + k] = num;
+    }
+    bar_consumers();
+    if (tid == 0 && !C.ms->abort) {
+      __threadfence();
+      red_release_add(P.ctr + t.layer * P.ctr_layer_stride + C_ATTN, 1u);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// consumer warps
+// ---------------------------------------------------------------------------
+__device__ void consumer(const Ctx& C) {
+  const Launch& P = *C.P;
+  uint32_t it = 0, ix = 0;
+  if (P.stall_ctr >= 0) {
+    // test hook: a dependency that nothing signals
+    wait_counter(C, P.stall_ctr, 1u);
+    return;
+  }
+  const int beg = P.task_off[blockIdx.x], end = P.task_off[blockIdx.x + 1];
+  for (int ti = beg; ti < end; ++ti) {
+    const Task t = P.tasks[ti];
+    const bool tr = P.trace && (ti - beg) < P.trace_cap && threadIdx.x == 0;
+    uint64_t tb = 0, td = 0;
+    if (tr) {
+      tb = globaltimer();
+      C.ms->tr_wf = C.ms->tr_wx = C.ms->tr_bytes = 0;
+      C.ms->tr_chunks = 0;
+    }
+    if (t.wait_ctr >= 0) wait_counter(C, t.wait_ctr, (uint32_t)t.wait_tgt);
+    if (tr) td = globaltimer();
+    if (t.type == T_GEMV) {
+      gemv_task(C, t, it, ix);
+    } else if (t.type == T_ATTN) {
+      attn_task(C, t, it);
+    }
+    if (t.type == T_GEMV && t.epi == EPI_LOGITS) lm_finish(C);
+    else if (t.sig_ctr >= 0) signal_counter(C, t.sig_ctr);
+    if (tr) {
+      int64_t* rec = P.trace + ((size_t)blockIdx.x * P.trace_cap + (ti - beg)) * 8;
+      rec[0] = (int64_t)tb;
+      rec[1] = (int64_t)td;
+      rec[2] = (int64_t)globaltimer();
+      rec[3] = C.ms->tr_wf;
+      rec[4] = C.ms->tr_wx;
+      rec[5] = C.ms->tr_chunks;
+      rec[6] = (int64_t)t.layer;
+      rec[7] = (int64_t)t.type * 16 + t.epi;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// the kernel
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(NTHREADS, 1) mk_step_kernel(const __grid_constant__ Launch P) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  Ctx C;
+  C.P = &P;
+  C.md = P.model;
+  C.ring = smem;
+  C.xring = smem + (size_t)NSTAGE * STAGE_BYTES;
+  C.att = C.xring + (size_t)XSLOTS * XSLOT_BYTES;
+  C.newkv = C.att + ATT_BYTES;
+  C.ms = reinterpret_cast<Misc*>(C.newkv + NEWKV_BYTES);
+  C.ncta = gridDim.x;
+  const int tid = threadIdx.x;
+
+  // ---- input validation (every CTA checks, so all return together) ----
+  int bad = 0;
+  if (tid < P.M) {
+    const int tok = __ldg(P.tokens + tid);
+    if (tok < 0 || tok >= C.md->V) bad = 1;
+  }
+  if (tid < P.S) {
+    const int p0 = seq_pos0(P, tid);
+    if (p0 < 0 || p0 + P.Q > P.kv_ctx || p0 + P.Q > C.md->rope_ctx) bad = 1;
+  }
+  if (__syncthreads_or(bad)) {
+    if (tid == 0 && blockIdx.x == 0) {
+      atomicCAS(P.status, 0, DERR_BOUNDS);
+      atomicExch(P.status + 1, 1);
+    }
+    return;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(&C.ms->full[s], 1);
+      mbar_init(&C.ms->empty[s], NCW);
+    }
+    for (int s = 0; s < XSLOTS; ++s) {
+      mbar_init(&C.ms->xfull[s], 1);
+      mbar_init(&C.ms->xempty[s], NCW);
+    }
+    C.ms->abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  if ((tid >> 5) == WARP_WP) producer(C);
+  else if ((tid >> 5) == WARP_XP) xproducer(C);
+  else consumer(C);
+  __syncthreads();
+
+  // ---- teardown: the last CTA out zeroes every counter for the next launch ----
+  if (tid == 0) {
+    int last = 0;
+    if (!global_abort(P)) {
+      __threadfence();
+      const uint32_t old = atom_add_acqrel(P.ctr + P.ctr_done, 1u);
+      last = (old == (uint32_t)C.ncta - 1);
+    }
+    C.ms->flag = last;
+  }
+  __syncthreads();
+  if (C.ms->flag) {
+    for (int i = tid; i < P.n_ctr; i += NTHREADS) P.ctr[i] = 0u;
+    __threadfence();
+  }
+}
+
+}  // namespace mk

@@ -1,0 +1,98 @@
+"""Task trace of the decode megakernel (the in-kernel %globaltimer records
+written when mk_set_trace is enabled) and its summary: per phase, the time
+CTAs spend waiting on dependencies, on weight tiles and on activation slices,
+and the SM idle fraction between tasks.
+
+    python -m persistent_decode_megakernel_sm_b200.trace --config dense27b --batch 1
+"""
+from __future__ import annotations
+
+import argparse
+import collections
+import json
+import os
+import sys
+
+import numpy as np
+
+TYPE_NAMES = {1: "gemv", 2: "attn"}
+EPI_NAMES = {0: "store", 1: "resid", 2: "swiglu", 3: "logits"}
+
+
+def record(model, kv, tokens, positions, logits, argmax, cap: int = 512):
+    import torch
+    ctas, _, _ = model.launch_info()
+    buf = torch.zeros((ctas, cap, 8), dtype=torch.int64, device=tokens.device)
+    model.set_trace(buf, cap)
+    model.decode_step(tokens, positions, kv, logits, argmax)
+    torch.cuda.synchronize()
+    model.set_trace(None, 0)
+    return buf.cpu().numpy()
+
+
+def summarize(tr: np.ndarray, sm_clock_mhz: float = 1965.0) -> dict:
+    """tr: [ctas][cap][8] = t_begin, t_dep, t_end (ns), wait_full, wait_x (cycles),
+    chunks, layer, type*16+epi."""
+    valid = tr[:, :, 2] > 0
+    t0 = tr[:, :, 0][valid].min()
+    t1 = tr[:, :, 2][valid].max()
+    phases = collections.defaultdict(lambda: dict(n=0, dep_us=0.0, run_us=0.0, wf_us=0.0, wx_us=0.0, chunks=0))
+    busy = 0.0
+    for c in range(tr.shape[0]):
+        for k in range(tr.shape[1]):
+            if not valid[c, k]:
+                continue
+            tb, td, te, wf, wx, ch, layer, te16 = tr[c, k]
+            name = TYPE_NAMES.get(int(te16) // 16, "?") + ("/" + EPI_NAMES[int(te16) % 16] if int(te16) // 16 == 1 else "")
+            p = phases[name]
+            p["n"] += 1
+            p["dep_us"] += (td - tb) / 1e3
+            p["run_us"] += (te - td) / 1e3
+            p["wf_us"] += wf / sm_clock_mhz
+            p["wx_us"] += wx / sm_clock_mhz
+            p["chunks"] += int(ch)
+            busy += (te - td) / 1e3 - wf / sm_clock_mhz - wx / sm_clock_mhz
+    ctas = tr.shape[0]
+    step_us = (t1 - t0) / 1e3
+    out = {"step_us": step_us, "ctas": ctas, "phases": {}}
+    for name, p in sorted(phases.items()):
+        out["phases"][name] = {k: (v / ctas if k.endswith("_us") else v) for k, v in p.items()}
+        out["phases"][name]["per_cta_us_note"] = "times summed over the CTA's tasks, averaged over CTAs"
+    out["compute_fraction"] = busy / ctas / step_us
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--config", default="dense27b")
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--out", default=None)
+    a = ap.parse_args()
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import torch
+    import synth
+    from persistent_decode_megakernel_sm_b200 import Megakernel
+    mc = synth.preset(a.config)
+    m = Megakernel(mc, 0)
+    m.init_random(mc.seed, mc.w_sigma, mc.router_sigma, mc.gain_sigma, mc.fp8_block_base)
+    kv = m.kv_cache(8, mc.max_ctx)
+    kv.fill_random(synth.SEED_KV, mc.kv_sigma, mc.context)
+    B = a.batch
+    tok = torch.arange(B, dtype=torch.int32, device="cuda:0") + 7
+    lg = torch.empty((B, mc.vocab), dtype=torch.float32, device="cuda:0")
+    am = torch.empty(B, dtype=torch.int32, device="cuda:0")
+    for i in range(a.steps):
+        pos = torch.full((B,), mc.context + i, dtype=torch.int32, device="cuda:0")
+        m.decode_step(tok, pos, kv, lg, am)
+    pos = torch.full((B,), mc.context + a.steps, dtype=torch.int32, device="cuda:0")
+    tr = record(m, kv, tok, pos, lg, am)
+    assert m.sync_status() == 0
+    s = summarize(tr)
+    if a.out:
+        np.save(a.out, tr)
+    print(json.dumps(s, indent=1))
+
+
+if __name__ == "__main__":
+    main()
