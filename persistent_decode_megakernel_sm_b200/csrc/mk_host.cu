@@ -310,6 +310,7 @@ static mk_status add_mat(mk_handle* h, int rows, int cols, int fp8, int gu, cons
 static bool desc_ok(const mk_model_desc* d, std::string& why) {
   if (!d) { why = "null descriptor"; return false; }
   if (d->layers < 1 || d->hidden < 16 || d->hidden % 16) { why = "hidden must be a positive multiple of 16"; return false; }
+  if (d->hidden * 2 > GAIN_BYTES) { why = "hidden must be <= 6144"; return false; }
   if (d->vocab < 2) { why = "vocab < 2"; return false; }
   if (d->max_batch < 1 || d->max_batch > MAXM) { why = "max_batch must be in [1, 8]"; return false; }
   if (d->max_ctx < 2) { why = "max_ctx < 2"; return false; }

@@ -13,21 +13,34 @@ constexpr int WARP_WP = NCW;                 // weight producer warp
 constexpr int WARP_XP = NCW + 1;             // activation producer warp
 constexpr int NTHREADS = (NCW + 2) * 32;
 constexpr int NCT = NCW * 32;                // consumer threads
-constexpr int STAGE_BYTES = 34816;           // one ring stage (= 2 x 64 rows x 272 B)
-constexpr int TILE_CAP = 32768;              // weight tile bytes per GEMV chunk (gains follow)
-constexpr int NSTAGE = 4;                    // weight ring depth
-constexpr int XSLOTS = 4;                    // activation ring depth
-constexpr int XSLOT_BYTES = 8192;            // one activation slice: M rows x (cols + pad)
+// Ring shape (tunable at build time).
+#ifndef MK_TILE_CAP
+#define MK_TILE_CAP 65536
+#endif
+#ifndef MK_NSTAGE
+#define MK_NSTAGE 2
+#endif
+#ifndef MK_PREFETCH
+#define MK_PREFETCH 0
+#endif
+constexpr int TILE_CAP = MK_TILE_CAP;        // weight tile bytes per GEMV chunk (gains follow)
+constexpr int STAGE_BYTES = (TILE_CAP + 1024 > 34816) ? TILE_CAP + 1024 : 34816;  // >= one attention chunk
+constexpr int NSTAGE = MK_NSTAGE;            // weight ring depth
+constexpr int PREFETCH_CHUNKS = MK_PREFETCH; // L2 lookahead beyond the ring, in chunks
+constexpr int XSLOTS = 2;                    // activation ring depth
+constexpr int XSLOT_BYTES = 16384;           // one activation slice: M rows x (cols + pad)
 constexpr int XROW_PAD = 32;                 // bytes between activation rows (bank spread)
 constexpr int ATT_BYTES = 40960;             // GEMV reduction / attention scratch
 constexpr int NEWKV_BYTES = 8704;            // K/V rows of the step's own new positions
 constexpr int MISC_BYTES = 4096;
+constexpr int GAIN_BYTES = 12288;            // the task's RMSNorm gain vector (hidden <= 6144)
 constexpr int SMEM_BYTES =
-    NSTAGE * STAGE_BYTES + XSLOTS * XSLOT_BYTES + ATT_BYTES + NEWKV_BYTES + MISC_BYTES;
+    NSTAGE * STAGE_BYTES + XSLOTS * XSLOT_BYTES + ATT_BYTES + NEWKV_BYTES + MISC_BYTES + GAIN_BYTES;
 constexpr int RMAX = 8;                      // row tiles per chunk
-constexpr int CPW = 4;                       // col tiles per warp per chunk
+constexpr int CPW = 8;                       // col tiles per warp per chunk
 constexpr int MAXM = 8;                      // activation rows per step (S * Q)
 constexpr int ATT_CT = 64;                   // cache positions per attention chunk
+constexpr int TRACE_FIELDS = 16;             // int64 per traced task
 constexpr int TILE_BF16 = 512;               // 16x16 bf16 tile in A-fragment order
 constexpr int TILE_FP8 = 256;                // 16x16 e4m3 tile in A-fragment order
 

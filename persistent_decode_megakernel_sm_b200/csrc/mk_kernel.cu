@@ -183,6 +183,7 @@ struct Misc {
   int pad[2];
   // per-task trace accumulators (consumer thread 0)
   long long tr_wf, tr_wx, tr_bytes;
+  long long tr_frag, tr_mma, tr_epi, tr_rel;
   int tr_chunks;
 };
 
@@ -194,6 +195,7 @@ struct Ctx {
   uint8_t* xring;
   uint8_t* att;
   uint8_t* newkv;
+  uint16_t* gain;
   int ncta;
 };
 
@@ -211,7 +213,7 @@ __device__ void raise_error(const Launch& P, Misc* ms, int code, int detail) {
 // ---------------------------------------------------------------------------
 struct ChunkIt {
   int rt1, KT, tb, gsz, xcap;
-  int g0, nr, KC, c0, nc;
+  int g0, nr, KC, WC, c0, nc;
   __device__ __forceinline__ void set_group() {
     nr = min(RMAX, rt1 - g0);
     if (gsz > 0) {
@@ -219,6 +221,7 @@ struct ChunkIt {
       nr = min(nr, nb - g0);
     }
     KC = min(min(KT, TILE_CAP / (nr * tb)), min(NCW * CPW, xcap));
+    WC = (xcap / KC) * KC;  // activation window: a whole number of chunks
   }
   // xcap: most col tiles whose activation slice (M rows) fits one x slot
   __device__ __forceinline__ bool init(int rt0_, int rt1_, int KT_, int tb_, int gsz_, int xcap_) {
@@ -247,6 +250,11 @@ struct ChunkIt {
   }
   __device__ __forceinline__ bool group_done() const { return c0 + KC >= KT; }
   __device__ __forceinline__ uint32_t bytes() const { return (uint32_t)(nr * nc * tb); }
+  // activation windows
+  __device__ __forceinline__ int w0() const { return (c0 / WC) * WC; }
+  __device__ __forceinline__ int wn() const { return min(WC, KT - w0()); }
+  __device__ __forceinline__ bool win_first() const { return c0 % WC == 0; }
+  __device__ __forceinline__ bool win_last() const { return c0 + KC >= KT || (c0 + KC) % WC == 0; }
 };
 
 // Activation element size and the x-slot column cap of a GEMV task.
@@ -254,7 +262,8 @@ __device__ __forceinline__ int x_esize(const Task& t) { return t.in_kind == IN_E
 __device__ __forceinline__ int x_cap(const Task& t, int M) {
   return (XSLOT_BYTES / M - XROW_PAD) / (16 * x_esize(t));
 }
-__device__ __forceinline__ int x_rowbytes(const Task& t, int nc) { return nc * 16 * x_esize(t) + XROW_PAD; }
+// row stride of an activation window in the x slot
+__device__ __forceinline__ int x_rowbytes(const Task& t, int wc) { return wc * 16 * x_esize(t) + XROW_PAD; }
 __device__ __forceinline__ const uint16_t* task_gain(const Model& md, const Task& t) {
   if (t.in_kind == IN_BUF) return nullptr;
   const Layer* ly = md.layers + t.layer;
@@ -286,23 +295,25 @@ __device__ __forceinline__ int seq_pos0(const Launch& P, int s) {
   return P.positions ? __ldg(P.positions + s) : P.pos_const;
 }
 
-__device__ __forceinline__ int att_pitch(int d) { return d * 2 + 16; }
+__device__ __forceinline__ int att_pitch(int d) { return d * 2; }
 
 // ---------------------------------------------------------------------------
 // producer warp
 // ---------------------------------------------------------------------------
 // Reserve ring slot `it` for `bytes` (lane 0 waits for the consumers to free
 // it, then arms the full barrier).  Returns false on abort.
-__device__ bool prod_reserve(const Ctx& C, uint32_t it, uint32_t bytes) {
+__device__ bool prod_reserve(const Ctx& C, uint32_t it, uint32_t bytes, long long& blocked) {
   const int lane = threadIdx.x & 31;
   int ok = 1;
   if (lane == 0) {
     const int s = it % NSTAGE;
+    const long long c0 = clock64();
     if (it >= (uint32_t)NSTAGE) {
       const uint32_t par = ((it / NSTAGE) + 1) & 1;
       uint64_t t0 = 0;
       uint32_t spins = 0;
       while (!mbar_try_wait(&C.ms->empty[s], par)) {
+        __nanosleep(64);
         if (++spins >= 64) {
           spins = 0;
           if (C.ms->abort || global_abort(*C.P)) { ok = 0; break; }
@@ -316,10 +327,106 @@ __device__ bool prod_reserve(const Ctx& C, uint32_t it, uint32_t bytes) {
         }
       }
     }
+    blocked += clock64() - c0;
     if (ok) mbar_arrive_expect_tx(&C.ms->full[s], bytes);
   }
   ok = __shfl_sync(0xffffffffu, ok, 0);
   return ok != 0;
+}
+
+// One unit of streamed data, in the order the consumers take it.
+struct Chunk {
+  int kind;  // 1: GEMV tiles (+ gain slice), 2: attention K/V rows
+  const uint8_t* w;
+  int KT, tb, g0, nr, c0, nc;
+  const uint16_t* gain;
+  const uint16_t* kb;
+  const uint16_t* vb;
+  int n, d;
+};
+
+// Walks a CTA's task list and yields its chunks in consumption order (the
+// same enumeration the consumers use).  Two instances run in the producer:
+// one issues ring loads, the other runs ahead and prefetches into L2.
+struct ChunkStream {
+  int ti, end, state;
+  ChunkIt ci;
+  const uint8_t* w;
+  int KT, tb;
+  const uint16_t* gain;
+  const uint16_t* kb;
+  const uint16_t* vb;
+  int t0, b, d;
+  __device__ void init(int beg, int end_) {
+    ti = beg;
+    end = end_;
+    state = 0;
+  }
+  __device__ bool next(const Launch& P, const Model& md, Chunk& c) {
+    while (true) {
+      if (state == 1) {
+        c.kind = 1;
+        c.w = w;
+        c.KT = KT;
+        c.tb = tb;
+        c.g0 = ci.g0;
+        c.nr = ci.nr;
+        c.c0 = ci.c0;
+        c.nc = ci.nc;
+        c.gain = gain;
+        if (!ci.next()) state = 0;
+        return true;
+      }
+      if (state == 2) {
+        if (t0 < b) {
+          c.kind = 2;
+          c.kb = kb + (size_t)t0 * d;
+          c.vb = vb + (size_t)t0 * d;
+          c.n = min(ATT_CT, b - t0);
+          c.d = d;
+          t0 += ATT_CT;
+          return true;
+        }
+        state = 0;
+      }
+      if (ti >= end) return false;
+      const Task t = P.tasks[ti++];
+      if (t.type == T_GEMV) {
+        const Mat& m = md.mats[t.mat];
+        tb = m.fp8 ? TILE_FP8 : TILE_BF16;
+        w = m.w;
+        KT = m.KT;
+        gain = task_gain(md, t);
+        if (ci.init(t.rt0, t.rt1, m.KT, tb, 0, x_cap(t, P.M))) state = 1;
+      } else if (t.type == T_ATTN) {
+        const Item itm = decode_item(t.rt0, P.n_pairs, P.n_items);
+        const int s = itm.pair / md.Hkv, g = itm.pair % md.Hkv;
+        const int T0 = seq_pos0(P, s);
+        t0 = (int)(((int64_t)itm.j * T0) / itm.ns);
+        b = (int)(((int64_t)(itm.j + 1) * T0) / itm.ns);
+        d = md.d;
+        const size_t head = (((size_t)t.layer * P.kv_seqs + s) * md.Hkv + g) * (size_t)P.kv_ctx;
+        kb = P.kv_k + head * d;
+        vb = P.kv_v + head * d;
+        state = 2;
+      }
+    }
+  }
+};
+
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+
+__device__ __forceinline__ void prefetch_chunk(const Chunk& c, int lane) {
+  if (c.kind == 1) {
+    if (lane < c.nr)
+      prefetch_l2(c.w + ((size_t)(c.g0 + lane) * c.KT + c.c0) * c.tb, (uint32_t)(c.nc * c.tb));
+  } else if (c.kind == 2) {
+    if (lane == 0) prefetch_l2(c.kb, (uint32_t)(c.n * c.d * 2));
+    if (lane == 1) prefetch_l2(c.vb, (uint32_t)(c.n * c.d * 2));
+  }
 }
 
 __device__ void producer(const Ctx& C) {
@@ -329,51 +436,50 @@ __device__ void producer(const Ctx& C) {
   const uint64_t pol = policy_evict_first();
   uint32_t it = 0;
   const int beg = P.task_off[blockIdx.x], end = P.task_off[blockIdx.x + 1];
-  for (int ti = beg; ti < end; ++ti) {
-    const Task t = P.tasks[ti];
-    if (t.type == T_GEMV) {
-      const Mat& m = md.mats[t.mat];
-      const int tb = m.fp8 ? TILE_FP8 : TILE_BF16;
-      const uint16_t* gain = task_gain(md, t);
-      ChunkIt ci;
-      if (ci.init(t.rt0, t.rt1, m.KT, tb, 0, x_cap(t, P.M))) {
-        do {
-          const uint32_t gbytes = gain ? (uint32_t)(ci.nc * 32) : 0u;
-          if (!prod_reserve(C, it, ci.bytes() + gbytes)) goto drain;
-          uint8_t* dst = C.ring + (size_t)(it % NSTAGE) * STAGE_BYTES;
-          if (lane < ci.nr) {
-            const uint8_t* src = m.w + ((size_t)(ci.g0 + lane) * m.KT + ci.c0) * tb;
-            bulk_g2s(dst + (size_t)lane * ci.nc * tb, src, (uint32_t)(ci.nc * tb), &C.ms->full[it % NSTAGE], pol);
-          } else if (lane == 31 && gain) {
-            // the norm gain slice of these columns follows the tiles
-            bulk_g2s(dst + ci.bytes(), gain + ci.c0 * 16, gbytes, &C.ms->full[it % NSTAGE], pol);
-          }
-          __syncwarp();
-          ++it;
-        } while (ci.next());
+  long long blocked = 0;
+  const uint64_t t_first = globaltimer();
+  ChunkStream is, ps;
+  is.init(beg, end);
+  ps.init(beg, end);
+  Chunk c, pc;
+  bool pf_live = true;
+  for (int k = 0; k < NSTAGE + PREFETCH_CHUNKS && pf_live; ++k) {
+    pf_live = ps.next(P, md, pc);
+    if (pf_live && k >= NSTAGE) prefetch_chunk(pc, lane);
+  }
+  while (is.next(P, md, c)) {
+    uint8_t* dst = C.ring + (size_t)(it % NSTAGE) * STAGE_BYTES;
+    uint64_t* bar = &C.ms->full[it % NSTAGE];
+    if (c.kind == 1) {
+      const uint32_t tbytes = (uint32_t)(c.nr * c.nc * c.tb);
+      if (!prod_reserve(C, it, tbytes, blocked)) goto drain;
+      if (lane < c.nr) {
+        const uint8_t* src = c.w + ((size_t)(c.g0 + lane) * c.KT + c.c0) * c.tb;
+        bulk_g2s(dst + (size_t)lane * c.nc * c.tb, src, (uint32_t)(c.nc * c.tb), bar, pol);
       }
-    } else if (t.type == T_ATTN) {
-      const Item itm = decode_item(t.rt0, P.n_pairs, P.n_items);
-      const int s = itm.pair / md.Hkv, g = itm.pair % md.Hkv;
-      const int T0 = seq_pos0(P, s);
-      const int a = (int)(((int64_t)itm.j * T0) / itm.ns), b = (int)(((int64_t)(itm.j + 1) * T0) / itm.ns);
-      const int d = md.d, pitch = att_pitch(d);
-      const size_t head = (((size_t)t.layer * P.kv_seqs + s) * md.Hkv + g) * (size_t)P.kv_ctx;
-      for (int t0 = a; t0 < b; t0 += ATT_CT) {
-        const int n = min(ATT_CT, b - t0);
-        if (!prod_reserve(C, it, (uint32_t)(2 * n * d * 2))) goto drain;
-        uint8_t* dst = C.ring + (size_t)(it % NSTAGE) * STAGE_BYTES;
-        for (int i = lane; i < n; i += 32) {
-          bulk_g2s(dst + (size_t)i * pitch, P.kv_k + (head + t0 + i) * d, (uint32_t)(d * 2), &C.ms->full[it % NSTAGE], pol);
-          bulk_g2s(dst + (size_t)(ATT_CT + i) * pitch, P.kv_v + (head + t0 + i) * d, (uint32_t)(d * 2),
-                   &C.ms->full[it % NSTAGE], pol);
-        }
-        __syncwarp();
-        ++it;
-      }
+    } else {
+      // the cache rows of this chunk are contiguous: one copy for K, one for V
+      const int pitch = att_pitch(c.d);
+      const uint32_t rb = (uint32_t)(c.n * c.d * 2);
+      if (!prod_reserve(C, it, 2 * rb, blocked)) goto drain;
+      if (lane == 0) bulk_g2s(dst, c.kb, rb, bar, pol);
+      if (lane == 1) bulk_g2s(dst + (size_t)ATT_CT * pitch, c.vb, rb, bar, pol);
+    }
+    __syncwarp();
+    ++it;
+    if (pf_live) {
+      pf_live = ps.next(P, md, pc);
+      if (pf_live) prefetch_chunk(pc, lane);
     }
   }
 drain:
+  if (lane == 0 && P.trace && P.trace_cap > 0) {
+    int64_t* rec = P.trace + (size_t)blockIdx.x * P.trace_cap * TRACE_FIELDS;
+    rec[12] = blocked;
+    rec[13] = it;
+    rec[14] = (int64_t)t_first;
+    rec[15] = (int64_t)globaltimer();
+  }
   // Wait (bounded) for every bulk copy this CTA issued, so none is in flight
   // when the CTA exits, whether it finished or aborted.
   if (lane == 0) {
@@ -438,6 +544,7 @@ __device__ bool xprod_reserve(const Ctx& C, uint32_t ix, uint32_t bytes) {
       uint64_t t0 = 0;
       uint32_t spins = 0;
       while (!mbar_try_wait(&C.ms->xempty[s], par)) {
+        __nanosleep(64);
         if (++spins >= 64) {
           spins = 0;
           if (C.ms->abort || global_abort(*C.P)) { ok = 0; break; }
@@ -475,9 +582,10 @@ __device__ void xproducer(const Ctx& C) {
     if (!ci.init(t.rt0, t.rt1, m.KT, tb, 0, x_cap(t, M))) continue;
     if (t.wait_ctr >= 0 && !xprod_wait_counter(C, t.wait_ctr, (uint32_t)t.wait_tgt)) goto drain;
     do {
+      if (!ci.win_first()) continue;
       const int es = x_esize(t);
-      const int rb = x_rowbytes(t, ci.nc);
-      const uint32_t rowdata = (uint32_t)(ci.nc * 16 * es);
+      const int rb = x_rowbytes(t, ci.WC);
+      const uint32_t rowdata = (uint32_t)(ci.wn() * 16 * es);
       if (!xprod_reserve(C, ix, (uint32_t)M * rowdata)) goto drain;
       uint8_t* dst = C.xring + (size_t)(ix % XSLOTS) * XSLOT_BYTES;
       if (lane < M) {
@@ -614,10 +722,12 @@ __device__ void wait_x(const Ctx& C, uint32_t ix) {
   if (tr) C.ms->tr_wx += clock64() - c0;
 }
 
-__device__ void gemv_task(const Ctx& C, const Task& t, uint32_t& it, uint32_t& ix) {
+__device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix) {
   const Launch& P = *C.P;
   const Model& md = *C.md;
-  const Mat& m = md.mats[t.mat];
+  // Copies in registers: the barrier asm below clobbers "memory", which would
+  // otherwise force a reload of every struct field on every chunk.
+  const Mat m = md.mats[t.mat];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, tq = lane & 3;
   const int M = P.M;
@@ -647,6 +757,13 @@ __device__ void gemv_task(const Ctx& C, const Task& t, uint32_t& it, uint32_t& i
       if (lane == 0) C.ms->scale[warp] = rsqrtf(ss / (float)md.H + md.eps);
     }
   }
+  if (has_gain) {
+    // the task's gain vector (read-only weights) staged once in shared memory
+    const uint16_t* gsrc = task_gain(md, t);
+    const int nw = md.H / 8;
+    for (int i = tid; i < nw; i += NCT)
+      reinterpret_cast<uint4*>(C.gain)[i] = __ldg(reinterpret_cast<const uint4*>(gsrc) + i);
+  }
   bar_consumers();
   const float sc = (g < M && has_gain) ? C.ms->scale[g] : 1.0f;
 
@@ -660,69 +777,67 @@ __device__ void gemv_task(const Ctx& C, const Task& t, uint32_t& it, uint32_t& i
   ChunkIt ci;
   bool have = ci.init(t.rt0, t.rt1, m.KT, tb, 0, x_cap(t, M));
   float* red = reinterpret_cast<float*>(C.att);
+  const int es = emb ? 2 : 4;
+  const uint16_t* gainp = task_gain(md, t);
+  const bool trc = P.trace && tid == 0;
+  long long tc0 = 0;
   while (have) {
-    wait_x(C, ix);
+    if (ci.win_first()) wait_x(C, ix);
     wait_full(C, it);
     const uint8_t* stage = C.ring + (size_t)(it % NSTAGE) * STAGE_BYTES;
-    const uint8_t* xs = C.xring + (size_t)(ix % XSLOTS) * XSLOT_BYTES + (size_t)g * x_rowbytes(t, ci.nc);
-    const uint8_t* gs = stage + ci.bytes();
-    // activation fragments (hi/lo) of this warp's col tiles j = warp + 8 i
-    uint32_t bh[CPW][2], bl[CPW][2];
-#pragma unroll
-    for (int i = 0; i < CPW; ++i) {
-      const int j = warp + NCW * i;
-      float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
-      if (j < ci.nc && g < M) {
-        if (emb) {
-          const uint32_t a = lds32(xs + (j * 16 + 2 * tq) * 2);
-          const uint32_t b = lds32(xs + (j * 16 + 2 * tq + 8) * 2);
-          y0 = bf16lo(a);
-          y1 = bf16hi(a);
-          y2 = bf16lo(b);
-          y3 = bf16hi(b);
-        } else {
-          const uint2 a = lds64(xs + (j * 16 + 2 * tq) * 4);
-          const uint2 b = lds64(xs + (j * 16 + 2 * tq + 8) * 4);
-          y0 = __uint_as_float(a.x);
-          y1 = __uint_as_float(a.y);
-          y2 = __uint_as_float(b.x);
-          y3 = __uint_as_float(b.y);
-        }
-        if (has_gain) {
-          const uint32_t g01 = lds32(gs + (j * 16 + 2 * tq) * 2);
-          const uint32_t g89 = lds32(gs + (j * 16 + 2 * tq + 8) * 2);
-          y0 = y0 * sc * bf16lo(g01);
-          y1 = y1 * sc * bf16hi(g01);
-          y2 = y2 * sc * bf16lo(g89);
-          y3 = y3 * sc * bf16hi(g89);
-        }
-      }
-      if (!m.fp8) {
-        split_bf16(y0, y1, bh[i][0], bl[i][0]);
-        split_bf16(y2, y3, bh[i][1], bl[i][1]);
-      } else {
-        split_f16(y0, y1, bh[i][0], bl[i][0]);
-        split_f16(y2, y3, bh[i][1], bl[i][1]);
-      }
-    }
+    const uint8_t* xs = C.xring + (size_t)(ix % XSLOTS) * XSLOT_BYTES + (size_t)g * x_rowbytes(t, ci.WC) +
+                        (size_t)(ci.c0 - ci.w0()) * 16 * es;
+    if (trc) tc0 = clock64();
+    // one col tile at a time: its activation fragment (hi/lo), then all of
+    // its row tiles (RMAX independent accumulator chains)
 #pragma unroll
     for (int i = 0; i < CPW; ++i) {
       const int j = warp + NCW * i;
       if (j < ci.nc) {
+        float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+        if (g < M) {
+          if (emb) {
+            const uint32_t a = lds32(xs + (j * 16 + 2 * tq) * 2);
+            const uint32_t b = lds32(xs + (j * 16 + 2 * tq + 8) * 2);
+            y0 = bf16lo(a);
+            y1 = bf16hi(a);
+            y2 = bf16lo(b);
+            y3 = bf16hi(b);
+          } else {
+            const uint2 a = lds64(xs + (j * 16 + 2 * tq) * 4);
+            const uint2 b = lds64(xs + (j * 16 + 2 * tq + 8) * 4);
+            y0 = __uint_as_float(a.x);
+            y1 = __uint_as_float(a.y);
+            y2 = __uint_as_float(b.x);
+            y3 = __uint_as_float(b.y);
+          }
+          if (has_gain) {
+            const int col = (ci.c0 + j) * 16 + 2 * tq;
+            const uint32_t g01 = lds32(C.gain + col);
+            const uint32_t g89 = lds32(C.gain + col + 8);
+            y0 = y0 * sc * bf16lo(g01);
+            y1 = y1 * sc * bf16hi(g01);
+            y2 = y2 * sc * bf16lo(g89);
+            y3 = y3 * sc * bf16hi(g89);
+          }
+        }
+        uint32_t bh0, bl0, bh1, bl1;
         if (!m.fp8) {
-          // all A fragments first, then the hi sweep, then the lo sweep:
-          // RMAX independent accumulator chains keep the tensor pipe busy
+          split_bf16(y0, y1, bh0, bl0);
+          split_bf16(y2, y3, bh1, bl1);
           uint4 a[RMAX];
 #pragma unroll
           for (int r = 0; r < RMAX; ++r)
             if (r < ci.nr) a[r] = lds128(stage + ((size_t)r * ci.nc + j) * TILE_BF16 + lane * 16);
 #pragma unroll
           for (int r = 0; r < RMAX; ++r)
-            if (r < ci.nr) mma_bf16(acc[r], a[r], bh[i][0], bh[i][1]);
+            if (r < ci.nr) mma_bf16(acc[r], a[r], bh0, bh1);
 #pragma unroll
           for (int r = 0; r < RMAX; ++r)
-            if (r < ci.nr) mma_bf16(acc[r], a[r], bl[i][0], bl[i][1]);
+            if (r < ci.nr) mma_bf16(acc[r], a[r], bl0, bl1);
         } else {
+          split_f16(y0, y1, bh0, bl0);
+          split_f16(y2, y3, bh1, bl1);
           const int c = ci.c0 + j;
           uint2 a8[RMAX];
 #pragma unroll
@@ -733,8 +848,8 @@ __device__ void gemv_task(const Ctx& C, const Task& t, uint32_t& it, uint32_t& i
             if (r < ci.nr) {
               const uint4 a = fp8_frag_to_f16(a8[r]);
               float tmp[4] = {0.f, 0.f, 0.f, 0.f};
-              mma_f16(tmp, a, bh[i][0], bh[i][1]);
-              mma_f16(tmp, a, bl[i][0], bl[i][1]);
+              mma_f16(tmp, a, bh0, bh1);
+              mma_f16(tmp, a, bl0, bl1);
               const int rt = ci.g0 + r;
               float s_top, s_bot;
               if (m.gu) {
@@ -753,13 +868,29 @@ __device__ void gemv_task(const Ctx& C, const Task& t, uint32_t& it, uint32_t& i
         }
       }
     }
+    if (trc) {
+      // make the mma results part of the measured region
+      float sink = 0.f;
+#pragma unroll
+      for (int r = 0; r < RMAX; ++r) sink += acc[r][0];
+      if (sink == 12345.678f) C.ms->flag = 0;
+      const long long t1 = clock64();
+      C.ms->tr_mma += t1 - tc0;
+      tc0 = t1;
+    }
     __syncwarp();
+    const bool xlast = ci.win_last();
     if (lane == 0) {
       mbar_arrive(&C.ms->empty[it % NSTAGE]);
-      mbar_arrive(&C.ms->xempty[ix % XSLOTS]);
+      if (xlast) mbar_arrive(&C.ms->xempty[ix % XSLOTS]);
     }
     ++it;
-    ++ix;
+    if (xlast) ++ix;
+    if (trc) {
+      const long long t1 = clock64();
+      C.ms->tr_rel += t1 - tc0;
+      tc0 = t1;
+    }
 
     if (ci.group_done()) {
       // ---- cross-warp reduction and epilogue for row tiles [g0, g0 + nr) ----
@@ -843,6 +974,7 @@ __device__ void gemv_task(const Ctx& C, const Task& t, uint32_t& it, uint32_t& i
       bar_consumers();
 #pragma unroll
       for (int r = 0; r < RMAX; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
+      if (trc) C.ms->tr_epi += clock64() - tc0;
     }
     have = ci.next();
   }
@@ -1089,7 +1221,7 @@ __device__ void att_chunk(const Ctx& C, AttState& st, const uint8_t* Ks, const u
   }
 }
 
-__device__ void attn_task(const Ctx& C, const Task& t, uint32_t& it) {
+__device__ void attn_task(const Ctx& C, const Task t, uint32_t& it) {
   const Launch& P = *C.P;
   const Model& md = *C.md;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1325,6 +1457,7 @@ __device__ void consumer(const Ctx& C) {
     if (tr) {
       tb = globaltimer();
       C.ms->tr_wf = C.ms->tr_wx = C.ms->tr_bytes = 0;
+      C.ms->tr_frag = C.ms->tr_mma = C.ms->tr_epi = C.ms->tr_rel = 0;
       C.ms->tr_chunks = 0;
     }
     if (t.wait_ctr >= 0) wait_counter(C, t.wait_ctr, (uint32_t)t.wait_tgt);
@@ -1337,7 +1470,7 @@ __device__ void consumer(const Ctx& C) {
     if (t.type == T_GEMV && t.epi == EPI_LOGITS) lm_finish(C);
     else if (t.sig_ctr >= 0) signal_counter(C, t.sig_ctr);
     if (tr) {
-      int64_t* rec = P.trace + ((size_t)blockIdx.x * P.trace_cap + (ti - beg)) * 8;
+      int64_t* rec = P.trace + ((size_t)blockIdx.x * P.trace_cap + (ti - beg)) * TRACE_FIELDS;
       rec[0] = (int64_t)tb;
       rec[1] = (int64_t)td;
       rec[2] = (int64_t)globaltimer();
@@ -1346,6 +1479,10 @@ __device__ void consumer(const Ctx& C) {
       rec[5] = C.ms->tr_chunks;
       rec[6] = (int64_t)t.layer;
       rec[7] = (int64_t)t.type * 16 + t.epi;
+      rec[8] = C.ms->tr_frag;
+      rec[9] = C.ms->tr_mma;
+      rec[10] = C.ms->tr_epi;
+      rec[11] = C.ms->tr_rel;
     }
   }
 }
@@ -1363,6 +1500,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) mk_step_kernel(const __grid_const
   C.att = C.xring + (size_t)XSLOTS * XSLOT_BYTES;
   C.newkv = C.att + ATT_BYTES;
   C.ms = reinterpret_cast<Misc*>(C.newkv + NEWKV_BYTES);
+  C.gain = reinterpret_cast<uint16_t*>(C.newkv + NEWKV_BYTES + MISC_BYTES);
   C.ncta = gridDim.x;
   const int tid = threadIdx.x;
 

@@ -16,13 +16,14 @@ import sys
 import numpy as np
 
 TYPE_NAMES = {1: "gemv", 2: "attn"}
+FIELDS = 16
 EPI_NAMES = {0: "store", 1: "resid", 2: "swiglu", 3: "logits"}
 
 
 def record(model, kv, tokens, positions, logits, argmax, cap: int = 512):
     import torch
     ctas, _, _ = model.launch_info()
-    buf = torch.zeros((ctas, cap, 8), dtype=torch.int64, device=tokens.device)
+    buf = torch.zeros((ctas, cap, FIELDS), dtype=torch.int64, device=tokens.device)
     model.set_trace(buf, cap)
     model.decode_step(tokens, positions, kv, logits, argmax)
     torch.cuda.synchronize()
@@ -31,18 +32,22 @@ def record(model, kv, tokens, positions, logits, argmax, cap: int = 512):
 
 
 def summarize(tr: np.ndarray, sm_clock_mhz: float = 1965.0) -> dict:
-    """tr: [ctas][cap][8] = t_begin, t_dep, t_end (ns), wait_full, wait_x (cycles),
-    chunks, layer, type*16+epi."""
+    """tr: [ctas][cap][16] = t_begin, t_dep, t_end (ns), wait_full, wait_x (cycles),
+    chunks, layer, type*16+epi, then cycles in fragment prep, mma, epilogue,
+    release (consumer thread 0); record 0 also carries the producer's cycles
+    blocked on a full ring, chunks issued, first and last issue time."""
     valid = tr[:, :, 2] > 0
     t0 = tr[:, :, 0][valid].min()
     t1 = tr[:, :, 2][valid].max()
-    phases = collections.defaultdict(lambda: dict(n=0, dep_us=0.0, run_us=0.0, wf_us=0.0, wx_us=0.0, chunks=0))
+    phases = collections.defaultdict(lambda: dict(n=0, dep_us=0.0, run_us=0.0, wf_us=0.0, wx_us=0.0, chunks=0,
+                                                  frag_us=0.0, mma_us=0.0, epi_us=0.0, rel_us=0.0))
     busy = 0.0
     for c in range(tr.shape[0]):
         for k in range(tr.shape[1]):
             if not valid[c, k]:
                 continue
-            tb, td, te, wf, wx, ch, layer, te16 = tr[c, k]
+            tb, td, te, wf, wx, ch, layer, te16 = tr[c, k, :8]
+            fr, mm, ep, rl = tr[c, k, 8:12]
             name = TYPE_NAMES.get(int(te16) // 16, "?") + ("/" + EPI_NAMES[int(te16) % 16] if int(te16) // 16 == 1 else "")
             p = phases[name]
             p["n"] += 1
@@ -51,6 +56,10 @@ def summarize(tr: np.ndarray, sm_clock_mhz: float = 1965.0) -> dict:
             p["wf_us"] += wf / sm_clock_mhz
             p["wx_us"] += wx / sm_clock_mhz
             p["chunks"] += int(ch)
+            p["frag_us"] += fr / sm_clock_mhz
+            p["mma_us"] += mm / sm_clock_mhz
+            p["epi_us"] += ep / sm_clock_mhz
+            p["rel_us"] += rl / sm_clock_mhz
             busy += (te - td) / 1e3 - wf / sm_clock_mhz - wx / sm_clock_mhz
     ctas = tr.shape[0]
     step_us = (t1 - t0) / 1e3
@@ -59,6 +68,9 @@ def summarize(tr: np.ndarray, sm_clock_mhz: float = 1965.0) -> dict:
         out["phases"][name] = {k: (v / ctas if k.endswith("_us") else v) for k, v in p.items()}
         out["phases"][name]["per_cta_us_note"] = "times summed over the CTA's tasks, averaged over CTAs"
     out["compute_fraction"] = busy / ctas / step_us
+    out["producer_blocked_us_per_cta"] = float(tr[:, 0, 12].mean()) / sm_clock_mhz
+    out["producer_chunks_per_cta"] = float(tr[:, 0, 13].mean())
+    out["producer_span_us"] = float((tr[:, 0, 15] - tr[:, 0, 14]).mean()) / 1e3
     return out
 
 
