@@ -28,19 +28,17 @@ constexpr int STAGE_BYTES = (TILE_CAP + 1024 > 34816) ? TILE_CAP + 1024 : 34816;
 constexpr int NSTAGE = MK_NSTAGE;            // weight ring depth
 constexpr int PREFETCH_CHUNKS = MK_PREFETCH; // L2 lookahead beyond the ring, in chunks
 constexpr int XSLOTS = 2;                    // activation ring depth
-constexpr int XSLOT_BYTES = 16384;           // one activation slice: M rows x (cols + pad)
+constexpr int XSLOT_BYTES = 22528;           // one activation window: M rows x (cols + pad)
 constexpr int XROW_PAD = 32;                 // bytes between activation rows (bank spread)
 constexpr int ATT_BYTES = 40960;             // GEMV reduction / attention scratch
 constexpr int NEWKV_BYTES = 8704;            // K/V rows of the step's own new positions
 constexpr int MISC_BYTES = 4096;
-constexpr int GAIN_BYTES = 12288;            // the task's RMSNorm gain vector (hidden <= 6144)
-constexpr int SMEM_BYTES =
-    NSTAGE * STAGE_BYTES + XSLOTS * XSLOT_BYTES + ATT_BYTES + NEWKV_BYTES + MISC_BYTES + GAIN_BYTES;
+constexpr int SMEM_BYTES = NSTAGE * STAGE_BYTES + XSLOTS * XSLOT_BYTES + ATT_BYTES + NEWKV_BYTES + MISC_BYTES;
 constexpr int RMAX = 8;                      // row tiles per chunk
 constexpr int CPW = 8;                       // col tiles per warp per chunk
 constexpr int MAXM = 8;                      // activation rows per step (S * Q)
 constexpr int ATT_CT = 64;                   // cache positions per attention chunk
-constexpr int TRACE_FIELDS = 16;             // int64 per traced task
+constexpr int TRACE_FIELDS = 20;             // int64 per traced task
 constexpr int TILE_BF16 = 512;               // 16x16 bf16 tile in A-fragment order
 constexpr int TILE_FP8 = 256;                // 16x16 e4m3 tile in A-fragment order
 
@@ -53,6 +51,7 @@ enum TaskType : int16_t {
   T_MOE_GU = 3,    // routed expert gate/up tiles (data dependent)
   T_MOE_DOWN = 4,  // down projection over shared + selected experts
   T_TOPK = 5,      // (unused placeholder)
+  T_EMBED = 6,     // x[m][c0:c1) = embedding rows of the step's tokens (+ RMS partial sums)
 };
 
 enum InKind : int16_t {

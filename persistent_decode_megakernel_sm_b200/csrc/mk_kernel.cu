@@ -175,7 +175,8 @@ __device__ __forceinline__ uint4 fp8_frag_to_f16(uint2 v) {
 struct Misc {
   uint64_t full[NSTAGE];
   uint64_t empty[NSTAGE];
-  uint64_t xfull[XSLOTS];
+  uint64_t xfull[XSLOTS];   // activation slice landed (bulk copy)
+  uint64_t xready[XSLOTS];  // ... and converted to mma fragments
   uint64_t xempty[XSLOTS];
   float scale[MAXM];
   volatile int abort;
@@ -183,7 +184,7 @@ struct Misc {
   int pad[2];
   // per-task trace accumulators (consumer thread 0)
   long long tr_wf, tr_wx, tr_bytes;
-  long long tr_frag, tr_mma, tr_epi, tr_rel;
+  long long tr_frag, tr_mma, tr_epi, tr_rel, tr_loop, tr_pre, tr_post, tr_sig;
   int tr_chunks;
 };
 
@@ -195,7 +196,6 @@ struct Ctx {
   uint8_t* xring;
   uint8_t* att;
   uint8_t* newkv;
-  uint16_t* gain;
   int ncta;
 };
 
@@ -213,7 +213,7 @@ __device__ void raise_error(const Launch& P, Misc* ms, int code, int detail) {
 // ---------------------------------------------------------------------------
 struct ChunkIt {
   int rt1, KT, tb, gsz, xcap;
-  int g0, nr, KC, WC, c0, nc;
+  int g0, nr, KC, WC, c0, nc, wb;  // wb: first col tile of the current activation window
   __device__ __forceinline__ void set_group() {
     nr = min(RMAX, rt1 - g0);
     if (gsz > 0) {
@@ -234,6 +234,7 @@ struct ChunkIt {
     if (g0 >= rt1) return false;
     set_group();
     c0 = 0;
+    wb = 0;
     nc = min(KC, KT);
     return true;
   }
@@ -244,21 +245,24 @@ struct ChunkIt {
       if (g0 >= rt1) return false;
       set_group();
       c0 = 0;
+      wb = 0;
+    } else if (c0 - wb >= WC) {
+      wb = c0;
     }
     nc = min(KC, KT - c0);
     return true;
   }
   __device__ __forceinline__ bool group_done() const { return c0 + KC >= KT; }
   __device__ __forceinline__ uint32_t bytes() const { return (uint32_t)(nr * nc * tb); }
-  // activation windows
-  __device__ __forceinline__ int w0() const { return (c0 / WC) * WC; }
-  __device__ __forceinline__ int wn() const { return min(WC, KT - w0()); }
-  __device__ __forceinline__ bool win_first() const { return c0 % WC == 0; }
-  __device__ __forceinline__ bool win_last() const { return c0 + KC >= KT || (c0 + KC) % WC == 0; }
+  // activation windows (no division: tracked incrementally)
+  __device__ __forceinline__ int w0() const { return wb; }
+  __device__ __forceinline__ int wn() const { return min(WC, KT - wb); }
+  __device__ __forceinline__ bool win_first() const { return c0 == wb; }
+  __device__ __forceinline__ bool win_last() const { return c0 + KC >= KT || c0 + KC - wb >= WC; }
 };
 
 // Activation element size and the x-slot column cap of a GEMV task.
-__device__ __forceinline__ int x_esize(const Task& t) { return t.in_kind == IN_EMB_NORM ? 2 : 4; }
+__device__ __forceinline__ int x_esize(const Task& t) { return 4; }
 __device__ __forceinline__ int x_cap(const Task& t, int M) {
   return (XSLOT_BYTES / M - XROW_PAD) / (16 * x_esize(t));
 }
@@ -438,6 +442,7 @@ __device__ void producer(const Ctx& C) {
   const int beg = P.task_off[blockIdx.x], end = P.task_off[blockIdx.x + 1];
   long long blocked = 0;
   const uint64_t t_first = globaltimer();
+  const long long c_first = clock64();
   ChunkStream is, ps;
   is.init(beg, end);
   ps.init(beg, end);
@@ -479,6 +484,11 @@ drain:
     rec[13] = it;
     rec[14] = (int64_t)t_first;
     rec[15] = (int64_t)globaltimer();
+    if (P.trace_cap > 1) {
+      // effective SM clock over the producer's lifetime: cycles and ns
+      rec[TRACE_FIELDS + 12] = clock64() - c_first;
+      rec[TRACE_FIELDS + 13] = (int64_t)(globaltimer() - t_first);
+    }
   }
   // Wait (bounded) for every bulk copy this CTA issued, so none is in flight
   // when the CTA exits, whether it finished or aborted.
@@ -581,24 +591,93 @@ __device__ void xproducer(const Ctx& C) {
     ChunkIt ci;
     if (!ci.init(t.rt0, t.rt1, m.KT, tb, 0, x_cap(t, M))) continue;
     if (t.wait_ctr >= 0 && !xprod_wait_counter(C, t.wait_ctr, (uint32_t)t.wait_tgt)) goto drain;
+    // RMSNorm scale of every activation row (fixed-order reduction of the
+    // per-CTA sums of squares) and the norm gain of this task
+    float scale[MAXM];
+    const bool has_gain = t.in_kind == IN_X_NORM;
+    const uint16_t* gain = task_gain(md, t);
+#pragma unroll
+    for (int mm = 0; mm < MAXM; ++mm) {
+      scale[mm] = 1.f;
+      if (has_gain && mm < M) {
+        const float* src = P.ss_part + (size_t)t.ss_src * gridDim.x * MAXM;
+        float ss = 0.f;
+        for (int c = lane; c < (int)gridDim.x; c += 32) ss += __ldcg(src + c * MAXM + mm);
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        scale[mm] = rsqrtf(ss / (float)md.H + md.eps);
+      }
+    }
     do {
       if (!ci.win_first()) continue;
-      const int es = x_esize(t);
       const int rb = x_rowbytes(t, ci.WC);
-      const uint32_t rowdata = (uint32_t)(ci.wn() * 16 * es);
+      const int wn = ci.wn(), w0 = ci.w0();
+      const uint32_t rowdata = (uint32_t)(wn * 64);
+      const int sl = ix % XSLOTS;
       if (!xprod_reserve(C, ix, (uint32_t)M * rowdata)) goto drain;
-      uint8_t* dst = C.xring + (size_t)(ix % XSLOTS) * XSLOT_BYTES;
+      uint8_t* dst = C.xring + (size_t)sl * XSLOT_BYTES;
       if (lane < M) {
-        const uint8_t* src;
-        if (t.in_kind == IN_EMB_NORM) {
-          src = reinterpret_cast<const uint8_t*>(md.embed + (size_t)__ldg(P.tokens + lane) * md.H + ci.c0 * 16);
-        } else {
-          const int b = t.in_kind == IN_X_NORM ? (int)B_X : (int)t.in_buf;
-          src = reinterpret_cast<const uint8_t*>(P.buf[b] + (size_t)lane * P.ld[b] + ci.c0 * 16);
+        const int b = t.in_kind == IN_X_NORM ? (int)B_X : (int)t.in_buf;
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(P.buf[b] + (size_t)lane * P.ld[b] + ci.c0 * 16);
+        bulk_g2s(dst + (size_t)lane * rb, src, rowdata, &C.ms->xfull[sl], pol);
+      }
+      // wait for this warp's own copy, then convert the window in place into
+      // ready mma B fragments: col tile jj of row m (16 fp32, 64 B) becomes,
+      // for each quad lane tq, 16 B = {hi(k 2tq,2tq+1), hi(k 2tq+8,2tq+9),
+      // lo(..), lo(..)} of x * rms_scale * gain (bf16 split; f16 for fp8 weights)
+      {
+        const uint32_t par = (ix / XSLOTS) & 1;
+        const uint64_t t0 = globaltimer();
+        bool landed = true;
+        while (!mbar_try_wait(&C.ms->xfull[sl], par)) {
+          if (C.ms->abort || globaltimer() - t0 > (uint64_t)P.timeout_ns * 2) { landed = false; break; }
         }
-        bulk_g2s(dst + (size_t)lane * rb, src, rowdata, &C.ms->xfull[ix % XSLOTS], pol);
+        if (!__all_sync(0xffffffffu, landed)) {
+          if (lane == 0 && !C.ms->abort) raise_error(P, C.ms, DERR_TIMEOUT, 0x60000 | sl);
+          goto drain;
+        }
+      }
+      for (int e = lane; e < M * wn; e += 32) {
+        const int mm = e / wn, jj = e - mm * wn;
+        float4* p4 = reinterpret_cast<float4*>(dst + (size_t)mm * rb + (size_t)jj * 64);
+        float v[16];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 f = p4[q];
+          v[4 * q] = f.x;
+          v[4 * q + 1] = f.y;
+          v[4 * q + 2] = f.z;
+          v[4 * q + 3] = f.w;
+        }
+        if (has_gain) {
+          float s = 1.f;
+#pragma unroll
+          for (int q = 0; q < MAXM; ++q) if (q == mm) s = scale[q];
+          const uint4* gp = reinterpret_cast<const uint4*>(gain + (size_t)(w0 + jj) * 16);
+          const uint4 ga = __ldg(gp), gb = __ldg(gp + 1);
+          const uint32_t gw[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            v[2 * q] = v[2 * q] * s * bf16lo(gw[q]);
+            v[2 * q + 1] = v[2 * q + 1] * s * bf16hi(gw[q]);
+          }
+        }
+        uint4 o[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (!m.fp8) {
+            split_bf16(v[2 * q], v[2 * q + 1], o[q].x, o[q].z);
+            split_bf16(v[2 * q + 8], v[2 * q + 9], o[q].y, o[q].w);
+          } else {
+            split_f16(v[2 * q], v[2 * q + 1], o[q].x, o[q].z);
+            split_f16(v[2 * q + 8], v[2 * q + 9], o[q].y, o[q].w);
+          }
+        }
+        uint4* o4 = reinterpret_cast<uint4*>(p4);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) o4[q] = o[q];
       }
       __syncwarp();
+      if (lane == 0) mbar_arrive(&C.ms->xready[sl]);
       ++ix;
     } while (ci.next());
   }
@@ -623,26 +702,31 @@ drain:
 // Wait for ring slot `it` to be filled.  On an abort the wait ends without
 // the data; callers keep walking their task list (so every consumer thread
 // passes the same barriers) and the outputs of the step are discarded.
-__device__ void wait_full(const Ctx& C, uint32_t it) {
+__device__ __forceinline__ void wait_full(const Ctx& C, uint32_t it) {
   const int s = it % NSTAGE;
   const uint32_t par = (it / NSTAGE) & 1;
-  uint32_t spins = 0;
-  uint64_t t0 = 0;
   const bool tr = C.P->trace && threadIdx.x == 0;
   const long long c0 = tr ? clock64() : 0;
   if (tr) C.ms->tr_chunks++;
-  while (!mbar_try_wait(&C.ms->full[s], par)) {
-    if (++spins >= 64) {
-      spins = 0;
-      if (C.ms->abort) return;
-      uint64_t now = globaltimer();
-      if (t0 == 0) t0 = now;
-      else if (now - t0 > (uint64_t)C.P->timeout_ns * 2) {
-        raise_error(*C.P, C.ms, DERR_TIMEOUT, 0x20000 | s);
-        return;
+  if ((threadIdx.x & 31) == 0) {
+    uint32_t spins = 0;
+    uint64_t t0 = 0;
+    while (!mbar_try_wait(&C.ms->full[s], par)) {
+      if (++spins >= 64) {
+        spins = 0;
+        if (C.ms->abort) break;
+        uint64_t now = globaltimer();
+        if (t0 == 0) t0 = now;
+        else if (now - t0 > (uint64_t)C.P->timeout_ns * 2) {
+          raise_error(*C.P, C.ms, DERR_TIMEOUT, 0x20000 | s);
+          break;
+        }
       }
     }
   }
+  __syncwarp();
+  // the other lanes observe the completed phase (async-proxy writes visible)
+  if (!C.ms->abort) while (!mbar_try_wait(&C.ms->full[s], par)) {}
   if (tr) C.ms->tr_wf += clock64() - c0;
 }
 
@@ -700,179 +784,109 @@ __device__ __forceinline__ void signal_counter(const Ctx& C, int idx) {
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
 
-__device__ void wait_x(const Ctx& C, uint32_t ix) {
+__device__ __forceinline__ void wait_x(const Ctx& C, uint32_t ix) {
   const int s = ix % XSLOTS;
   const uint32_t par = (ix / XSLOTS) & 1;
-  uint32_t spins = 0;
-  uint64_t t0 = 0;
   const bool tr = C.P->trace && threadIdx.x == 0;
   const long long c0 = tr ? clock64() : 0;
-  while (!mbar_try_wait(&C.ms->xfull[s], par)) {
-    if (++spins >= 64) {
-      spins = 0;
-      if (C.ms->abort) return;
-      uint64_t now = globaltimer();
-      if (t0 == 0) t0 = now;
-      else if (now - t0 > (uint64_t)C.P->timeout_ns * 2) {
-        raise_error(*C.P, C.ms, DERR_TIMEOUT, 0x50000 | s);
-        return;
+  if ((threadIdx.x & 31) == 0) {
+    uint32_t spins = 0;
+    uint64_t t0 = 0;
+    while (!mbar_try_wait(&C.ms->xready[s], par)) {
+      if (++spins >= 64) {
+        spins = 0;
+        if (C.ms->abort) break;
+        uint64_t now = globaltimer();
+        if (t0 == 0) t0 = now;
+        else if (now - t0 > (uint64_t)C.P->timeout_ns * 2) {
+          raise_error(*C.P, C.ms, DERR_TIMEOUT, 0x50000 | s);
+          break;
+        }
       }
     }
   }
+  __syncwarp();
+  if (!C.ms->abort) while (!mbar_try_wait(&C.ms->xready[s], par)) {}
   if (tr) C.ms->tr_wx += clock64() - c0;
 }
 
-__device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix) {
-  const Launch& P = *C.P;
-  const Model& md = *C.md;
-  // Copies in registers: the barrier asm below clobbers "memory", which would
-  // otherwise force a reload of every struct field on every chunk.
-  const Mat m = md.mats[t.mat];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, tq = lane & 3;
-  const int M = P.M;
-  const int tb = m.fp8 ? TILE_FP8 : TILE_BF16;
-  const bool emb = t.in_kind == IN_EMB_NORM;
-  const bool has_gain = t.in_kind != IN_BUF;
+// Per-lane constants of a GEMV task.
+struct GemvLane {
+  int warp, lane, g, tq, M, rowbytes;
+  bool has_gain, trc;
+};
 
-  // ---- prologue: RMSNorm scale per activation row (fixed-order reductions) ----
-  if (t.in_kind == IN_X_NORM) {
-    if (warp < M) {
-      const float* src = P.ss_part + (size_t)t.ss_src * C.ncta * MAXM;
-      float ss = 0.f;
-      for (int c = lane; c < C.ncta; c += 32) ss += __ldcg(src + c * MAXM + warp);
-      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      if (lane == 0) C.ms->scale[warp] = rsqrtf(ss / (float)md.H + md.eps);
-    }
-  } else if (emb) {
-    if (warp < M) {
-      const uint16_t* e = md.embed + (size_t)__ldg(P.tokens + warp) * md.H;
-      float ss = 0.f;
-      for (int k = lane * 2; k < md.H; k += 64) {
-        uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(e + k));
-        float a = bf16lo(u), b = bf16hi(u);
-        ss += a * a + b * b;
-      }
-      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      if (lane == 0) C.ms->scale[warp] = rsqrtf(ss / (float)md.H + md.eps);
-    }
-  }
-  if (has_gain) {
-    // the task's gain vector (read-only weights) staged once in shared memory
-    const uint16_t* gsrc = task_gain(md, t);
-    const int nw = md.H / 8;
-    for (int i = tid; i < nw; i += NCT)
-      reinterpret_cast<uint4*>(C.gain)[i] = __ldg(reinterpret_cast<const uint4*>(gsrc) + i);
-  }
-  bar_consumers();
-  const float sc = (g < M && has_gain) ? C.ms->scale[g] : 1.0f;
-
-  float acc[RMAX][4];
-  float ss_acc[2] = {0.f, 0.f};
-  float am_v[2] = {-INFINITY, -INFINITY};
-  int am_i[2] = {0x7fffffff, 0x7fffffff};
+// All chunks of one row group [g0, g0 + NR): each warp takes col tiles
+// j = warp + 8 i of every chunk, builds the activation fragment (hi/lo) of
+// each and runs NR independent accumulator chains; the per-warp partial sums
+// are left in `red` for the cross-warp reduction.
+template <int NR, bool FP8>
+__device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& mr, const GemvLane& Lr, uint32_t& itr,
+                                        uint32_t& ixr, float* red) {
+  // register copies (the arguments live in the caller's frame)
+  const Ctx C = Cr;
+  const Mat m = mr;
+  const GemvLane L = Lr;
+  ChunkIt ci = cir;
+  uint32_t it = itr, ix = ixr;
+  float acc[NR][4];
 #pragma unroll
-  for (int r = 0; r < RMAX; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
-
-  ChunkIt ci;
-  bool have = ci.init(t.rt0, t.rt1, m.KT, tb, 0, x_cap(t, M));
-  float* red = reinterpret_cast<float*>(C.att);
-  const int es = emb ? 2 : 4;
-  const uint16_t* gainp = task_gain(md, t);
-  const bool trc = P.trace && tid == 0;
-  long long tc0 = 0;
-  while (have) {
-    if (ci.win_first()) wait_x(C, ix);
+  for (int r = 0; r < NR; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
+  const int lane = L.lane, g = L.g, tq = L.tq;
+  const bool xok = g < L.M;  // activation rows beyond M are zero
+  long long tc0 = 0, tl0 = L.trc ? clock64() : 0;
+  while (true) {
+    const uint8_t* slot = C.xring + (size_t)(ix % XSLOTS) * XSLOT_BYTES;
+    if (ci.win_first()) wait_x(C, ix);  // the window arrives converted
     wait_full(C, it);
     const uint8_t* stage = C.ring + (size_t)(it % NSTAGE) * STAGE_BYTES;
-    const uint8_t* xs = C.xring + (size_t)(ix % XSLOTS) * XSLOT_BYTES + (size_t)g * x_rowbytes(t, ci.WC) +
-                        (size_t)(ci.c0 - ci.w0()) * 16 * es;
-    if (trc) tc0 = clock64();
-    // one col tile at a time: its activation fragment (hi/lo), then all of
-    // its row tiles (RMAX independent accumulator chains)
+    const uint8_t* xs = slot + (size_t)g * L.rowbytes + (size_t)(ci.c0 - ci.w0()) * 64 + tq * 16;
+    const int nc = ci.nc;
+    if (L.trc) tc0 = clock64();
+    // kept rolled: the instruction working set of the whole kernel must stay
+    // small (one CTA executes every phase of every layer)
+#pragma unroll 1
+    for (int j = L.warp; j < nc; j += NCW) {
+      const uint4 xf = xok ? lds128(xs + j * 64) : make_uint4(0u, 0u, 0u, 0u);
+      if (!FP8) {
+        uint4 a[NR];
 #pragma unroll
-    for (int i = 0; i < CPW; ++i) {
-      const int j = warp + NCW * i;
-      if (j < ci.nc) {
-        float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
-        if (g < M) {
-          if (emb) {
-            const uint32_t a = lds32(xs + (j * 16 + 2 * tq) * 2);
-            const uint32_t b = lds32(xs + (j * 16 + 2 * tq + 8) * 2);
-            y0 = bf16lo(a);
-            y1 = bf16hi(a);
-            y2 = bf16lo(b);
-            y3 = bf16hi(b);
+        for (int r = 0; r < NR; ++r) a[r] = lds128(stage + ((size_t)r * nc + j) * TILE_BF16 + lane * 16);
+#pragma unroll
+        for (int r = 0; r < NR; ++r) mma_bf16(acc[r], a[r], xf.x, xf.y);
+#pragma unroll
+        for (int r = 0; r < NR; ++r) mma_bf16(acc[r], a[r], xf.z, xf.w);
+      } else {
+        const int c = ci.c0 + j;
+        uint2 a8[NR];
+#pragma unroll
+        for (int r = 0; r < NR; ++r) a8[r] = lds64(stage + ((size_t)r * nc + j) * TILE_FP8 + lane * 8);
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+          const uint4 af = fp8_frag_to_f16(a8[r]);
+          float tmp[4] = {0.f, 0.f, 0.f, 0.f};
+          mma_f16(tmp, af, xf.x, xf.y);
+          mma_f16(tmp, af, xf.z, xf.w);
+          const int rt = ci.g0 + r;
+          float s_top, s_bot;
+          if (m.gu) {
+            const int rb = rt >> 4;
+            s_top = __ldg(m.scales + rb * m.nbc + (c >> 3));
+            s_bot = __ldg(m.scales + (size_t)m.nbr * m.nbc + rb * m.nbc + (c >> 3));
           } else {
-            const uint2 a = lds64(xs + (j * 16 + 2 * tq) * 4);
-            const uint2 b = lds64(xs + (j * 16 + 2 * tq + 8) * 4);
-            y0 = __uint_as_float(a.x);
-            y1 = __uint_as_float(a.y);
-            y2 = __uint_as_float(b.x);
-            y3 = __uint_as_float(b.y);
+            s_top = s_bot = __ldg(m.scales + (rt >> 3) * m.nbc + (c >> 3));
           }
-          if (has_gain) {
-            const int col = (ci.c0 + j) * 16 + 2 * tq;
-            const uint32_t g01 = lds32(C.gain + col);
-            const uint32_t g89 = lds32(C.gain + col + 8);
-            y0 = y0 * sc * bf16lo(g01);
-            y1 = y1 * sc * bf16hi(g01);
-            y2 = y2 * sc * bf16lo(g89);
-            y3 = y3 * sc * bf16hi(g89);
-          }
-        }
-        uint32_t bh0, bl0, bh1, bl1;
-        if (!m.fp8) {
-          split_bf16(y0, y1, bh0, bl0);
-          split_bf16(y2, y3, bh1, bl1);
-          uint4 a[RMAX];
-#pragma unroll
-          for (int r = 0; r < RMAX; ++r)
-            if (r < ci.nr) a[r] = lds128(stage + ((size_t)r * ci.nc + j) * TILE_BF16 + lane * 16);
-#pragma unroll
-          for (int r = 0; r < RMAX; ++r)
-            if (r < ci.nr) mma_bf16(acc[r], a[r], bh0, bh1);
-#pragma unroll
-          for (int r = 0; r < RMAX; ++r)
-            if (r < ci.nr) mma_bf16(acc[r], a[r], bl0, bl1);
-        } else {
-          split_f16(y0, y1, bh0, bl0);
-          split_f16(y2, y3, bh1, bl1);
-          const int c = ci.c0 + j;
-          uint2 a8[RMAX];
-#pragma unroll
-          for (int r = 0; r < RMAX; ++r)
-            if (r < ci.nr) a8[r] = lds64(stage + ((size_t)r * ci.nc + j) * TILE_FP8 + lane * 8);
-#pragma unroll
-          for (int r = 0; r < RMAX; ++r) {
-            if (r < ci.nr) {
-              const uint4 a = fp8_frag_to_f16(a8[r]);
-              float tmp[4] = {0.f, 0.f, 0.f, 0.f};
-              mma_f16(tmp, a, bh0, bh1);
-              mma_f16(tmp, a, bl0, bl1);
-              const int rt = ci.g0 + r;
-              float s_top, s_bot;
-              if (m.gu) {
-                const int rb = rt >> 4;
-                s_top = __ldg(m.scales + rb * m.nbc + (c >> 3));
-                s_bot = __ldg(m.scales + (size_t)m.nbr * m.nbc + rb * m.nbc + (c >> 3));
-              } else {
-                s_top = s_bot = __ldg(m.scales + (rt >> 3) * m.nbc + (c >> 3));
-              }
-              acc[r][0] += s_top * tmp[0];
-              acc[r][1] += s_top * tmp[1];
-              acc[r][2] += s_bot * tmp[2];
-              acc[r][3] += s_bot * tmp[3];
-            }
-          }
+          acc[r][0] += s_top * tmp[0];
+          acc[r][1] += s_top * tmp[1];
+          acc[r][2] += s_bot * tmp[2];
+          acc[r][3] += s_bot * tmp[3];
         }
       }
     }
-    if (trc) {
-      // make the mma results part of the measured region
+    if (L.trc) {
       float sink = 0.f;
 #pragma unroll
-      for (int r = 0; r < RMAX; ++r) sink += acc[r][0];
+      for (int r = 0; r < NR; ++r) sink += acc[r][0];
       if (sink == 12345.678f) C.ms->flag = 0;
       const long long t1 = clock64();
       C.ms->tr_mma += t1 - tc0;
@@ -886,19 +900,81 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
     }
     ++it;
     if (xlast) ++ix;
-    if (trc) {
-      const long long t1 = clock64();
-      C.ms->tr_rel += t1 - tc0;
-      tc0 = t1;
-    }
-
-    if (ci.group_done()) {
-      // ---- cross-warp reduction and epilogue for row tiles [g0, g0 + nr) ----
+    if (L.trc) C.ms->tr_rel += clock64() - tc0;
+    if (ci.group_done()) break;
+    ci.next();
+  }
+  if (L.trc) C.ms->tr_loop += clock64() - tl0;
 #pragma unroll
-      for (int r = 0; r < RMAX; ++r)
-        if (r < ci.nr)
-          *reinterpret_cast<float4*>(red + ((warp * RMAX + r) * 32 + lane) * 4) =
-              make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+  for (int r = 0; r < NR; ++r)
+    *reinterpret_cast<float4*>(red + ((L.warp * RMAX + r) * 32 + lane) * 4) =
+        make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+  cir = ci;
+  itr = it;
+  ixr = ix;
+}
+
+__device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix) {
+  const Launch& P = *C.P;
+  const long long tpre = (P.trace && threadIdx.x == 0) ? clock64() : 0;
+  const Model& md = *C.md;
+  // Copies in registers: the barrier asm below clobbers "memory", which would
+  // otherwise force a reload of every struct field on every chunk.
+  const Mat m = md.mats[t.mat];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, tq = lane & 3;
+  const int M = P.M;
+  const int tb = m.fp8 ? TILE_FP8 : TILE_BF16;
+  const bool has_gain = t.in_kind != IN_BUF;
+
+  float ss_acc[2] = {0.f, 0.f};
+  float am_v[2] = {-INFINITY, -INFINITY};
+  int am_i[2] = {0x7fffffff, 0x7fffffff};
+
+  ChunkIt ci;
+  bool have = ci.init(t.rt0, t.rt1, m.KT, tb, 0, x_cap(t, M));
+  float* red = reinterpret_cast<float*>(C.att);
+  GemvLane L;
+  L.warp = warp;
+  L.lane = lane;
+  L.g = g;
+  L.tq = tq;
+  L.M = M;
+  L.has_gain = has_gain;
+  L.rowbytes = 0;
+  L.trc = P.trace && tid == 0;
+  if (L.trc) C.ms->tr_pre += clock64() - tpre;
+  while (have) {
+    L.rowbytes = x_rowbytes(t, ci.WC);
+    // one instance per row-tile count: every loop below is fully static
+    // one instance per row-tile count: every loop over rows is static
+    if (!m.fp8) {
+      switch (ci.nr) {
+        case 1: gemv_group<1, false>(C, ci, m, L, it, ix, red); break;
+        case 2: gemv_group<2, false>(C, ci, m, L, it, ix, red); break;
+        case 3: gemv_group<3, false>(C, ci, m, L, it, ix, red); break;
+        case 4: gemv_group<4, false>(C, ci, m, L, it, ix, red); break;
+        case 5: gemv_group<5, false>(C, ci, m, L, it, ix, red); break;
+        case 6: gemv_group<6, false>(C, ci, m, L, it, ix, red); break;
+        case 7: gemv_group<7, false>(C, ci, m, L, it, ix, red); break;
+        default: gemv_group<8, false>(C, ci, m, L, it, ix, red); break;
+      }
+    } else {
+      switch (ci.nr) {
+        case 1: gemv_group<1, true>(C, ci, m, L, it, ix, red); break;
+        case 2: gemv_group<2, true>(C, ci, m, L, it, ix, red); break;
+        case 3: gemv_group<3, true>(C, ci, m, L, it, ix, red); break;
+        case 4: gemv_group<4, true>(C, ci, m, L, it, ix, red); break;
+        case 5: gemv_group<5, true>(C, ci, m, L, it, ix, red); break;
+        case 6: gemv_group<6, true>(C, ci, m, L, it, ix, red); break;
+        case 7: gemv_group<7, true>(C, ci, m, L, it, ix, red); break;
+        default: gemv_group<8, true>(C, ci, m, L, it, ix, red); break;
+      }
+    }
+    const bool trc = L.trc;
+    long long tc0 = trc ? clock64() : 0;
+    {
+      // ---- cross-warp reduction and epilogue for row tiles [g0, g0 + nr) ----
       bar_consumers();
       {
         const int r = tid >> 5, l = lane;
@@ -934,13 +1010,7 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
               const int row = (q < 2) ? row0 : row1;
               const int mm = (q & 1) ? m1 : m0;
               if (row < m.rows && mm < M) {
-                float base;
-                if (t.resid_emb) {
-                  const uint16_t* e = md.embed + (size_t)__ldg(P.tokens + mm) * md.H;
-                  base = __uint_as_float((uint32_t)__ldg(e + row) << 16);
-                } else {
-                  base = __ldcg(x + (size_t)mm * ld + row);
-                }
+                const float base = __ldcg(x + (size_t)mm * ld + row);
                 const float nv = base + v[q];
                 x[(size_t)mm * ld + row] = nv;
                 ss_acc[q & 1] += nv * nv;
@@ -972,13 +1042,12 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
         }
       }
       bar_consumers();
-#pragma unroll
-      for (int r = 0; r < RMAX; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
       if (trc) C.ms->tr_epi += clock64() - tc0;
     }
     have = ci.next();
   }
 
+  const long long tpost = L.trc ? clock64() : 0;
   // ---- task-level partials: sum of squares (RESID) or argmax (LOGITS) ----
   if (t.epi == EPI_RESID || t.epi == EPI_LOGITS) {
     float* f2 = reinterpret_cast<float*>(C.att);
@@ -1014,6 +1083,41 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
         P.am_idx[(size_t)blockIdx.x * MAXM + mm] = bi;
       }
     }
+  }
+  if (L.trc) C.ms->tr_post += clock64() - tpost;
+}
+
+// Embedding gather: this CTA's column slice [c0, c1) of x[m] = E[token_m],
+// widened exactly to fp32, and its per-row sums of squares for the first
+// RMSNorm (fixed-order reduction).
+__device__ void embed_task(const Ctx& C, const Task t) {
+  const Launch& P = *C.P;
+  const Model& md = *C.md;
+  const int tid = threadIdx.x, M = P.M;
+  float* x = P.buf[B_X];
+  const int ld = P.ld[B_X];
+  float part[MAXM];
+#pragma unroll
+  for (int mm = 0; mm < MAXM; ++mm) part[mm] = 0.f;
+  for (int k = t.rt0 + tid; k < t.rt1; k += NCT) {
+#pragma unroll
+    for (int mm = 0; mm < MAXM; ++mm) {
+      if (mm < M) {
+        const uint16_t* e = md.embed + (size_t)__ldg(P.tokens + mm) * md.H;
+        const float v = __uint_as_float((uint32_t)__ldg(e + k) << 16);
+        x[(size_t)mm * ld + k] = v;
+        part[mm] += v * v;
+      }
+    }
+  }
+  float* red = reinterpret_cast<float*>(C.att);
+#pragma unroll
+  for (int mm = 0; mm < MAXM; ++mm) red[tid * MAXM + mm] = part[mm];
+  bar_consumers();
+  if (tid < M) {
+    float s2 = 0.f;
+    for (int th = 0; th < NCT; ++th) s2 += red[th * MAXM + tid];
+    P.ss_part[((size_t)t.ss_dst * C.ncta + blockIdx.x) * MAXM + tid] = s2;
   }
 }
 
@@ -1458,6 +1562,7 @@ __device__ void consumer(const Ctx& C) {
       tb = globaltimer();
       C.ms->tr_wf = C.ms->tr_wx = C.ms->tr_bytes = 0;
       C.ms->tr_frag = C.ms->tr_mma = C.ms->tr_epi = C.ms->tr_rel = 0;
+      C.ms->tr_loop = C.ms->tr_pre = C.ms->tr_post = C.ms->tr_sig = 0;
       C.ms->tr_chunks = 0;
     }
     if (t.wait_ctr >= 0) wait_counter(C, t.wait_ctr, (uint32_t)t.wait_tgt);
@@ -1466,9 +1571,13 @@ __device__ void consumer(const Ctx& C) {
       gemv_task(C, t, it, ix);
     } else if (t.type == T_ATTN) {
       attn_task(C, t, it);
+    } else if (t.type == T_EMBED) {
+      embed_task(C, t);
     }
+    const long long tsg = tr ? clock64() : 0;
     if (t.type == T_GEMV && t.epi == EPI_LOGITS) lm_finish(C);
     else if (t.sig_ctr >= 0) signal_counter(C, t.sig_ctr);
+    if (tr) C.ms->tr_sig += clock64() - tsg;
     if (tr) {
       int64_t* rec = P.trace + ((size_t)blockIdx.x * P.trace_cap + (ti - beg)) * TRACE_FIELDS;
       rec[0] = (int64_t)tb;
@@ -1483,6 +1592,10 @@ __device__ void consumer(const Ctx& C) {
       rec[9] = C.ms->tr_mma;
       rec[10] = C.ms->tr_epi;
       rec[11] = C.ms->tr_rel;
+      rec[16] = C.ms->tr_loop;
+      rec[17] = C.ms->tr_pre;
+      rec[18] = C.ms->tr_post;
+      rec[19] = C.ms->tr_sig;
     }
   }
 }
@@ -1500,7 +1613,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) mk_step_kernel(const __grid_const
   C.att = C.xring + (size_t)XSLOTS * XSLOT_BYTES;
   C.newkv = C.att + ATT_BYTES;
   C.ms = reinterpret_cast<Misc*>(C.newkv + NEWKV_BYTES);
-  C.gain = reinterpret_cast<uint16_t*>(C.newkv + NEWKV_BYTES + MISC_BYTES);
   C.ncta = gridDim.x;
   const int tid = threadIdx.x;
 
@@ -1528,6 +1640,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) mk_step_kernel(const __grid_const
     }
     for (int s = 0; s < XSLOTS; ++s) {
       mbar_init(&C.ms->xfull[s], 1);
+      mbar_init(&C.ms->xready[s], 1);
       mbar_init(&C.ms->xempty[s], NCW);
     }
     C.ms->abort = 0;

@@ -16,7 +16,7 @@ import sys
 import numpy as np
 
 TYPE_NAMES = {1: "gemv", 2: "attn"}
-FIELDS = 16
+FIELDS = 20
 EPI_NAMES = {0: "store", 1: "resid", 2: "swiglu", 3: "logits"}
 
 
@@ -31,16 +31,22 @@ def record(model, kv, tokens, positions, logits, argmax, cap: int = 512):
     return buf.cpu().numpy()
 
 
-def summarize(tr: np.ndarray, sm_clock_mhz: float = 1965.0) -> dict:
+def summarize(tr: np.ndarray, sm_clock_mhz: float = 0.0) -> dict:
     """tr: [ctas][cap][16] = t_begin, t_dep, t_end (ns), wait_full, wait_x (cycles),
     chunks, layer, type*16+epi, then cycles in fragment prep, mma, epilogue,
     release (consumer thread 0); record 0 also carries the producer's cycles
     blocked on a full ring, chunks issued, first and last issue time."""
+    if sm_clock_mhz <= 0:
+        # measured: SM cycles / ns over each producer's lifetime (record 1)
+        cyc, ns = tr[:, 1, 12].astype(np.float64), tr[:, 1, 13].astype(np.float64)
+        ok = ns > 0
+        sm_clock_mhz = float(np.median(cyc[ok] / ns[ok]) * 1e3) if ok.any() else 1965.0
     valid = tr[:, :, 2] > 0
     t0 = tr[:, :, 0][valid].min()
     t1 = tr[:, :, 2][valid].max()
     phases = collections.defaultdict(lambda: dict(n=0, dep_us=0.0, run_us=0.0, wf_us=0.0, wx_us=0.0, chunks=0,
-                                                  frag_us=0.0, mma_us=0.0, epi_us=0.0, rel_us=0.0))
+                                                  frag_us=0.0, mma_us=0.0, epi_us=0.0, rel_us=0.0,
+                                                  loop_us=0.0, pre_us=0.0, post_us=0.0, sig_us=0.0))
     busy = 0.0
     for c in range(tr.shape[0]):
         for k in range(tr.shape[1]):
@@ -48,6 +54,7 @@ def summarize(tr: np.ndarray, sm_clock_mhz: float = 1965.0) -> dict:
                 continue
             tb, td, te, wf, wx, ch, layer, te16 = tr[c, k, :8]
             fr, mm, ep, rl = tr[c, k, 8:12]
+            lo, pr, po, sg = tr[c, k, 16:20]
             name = TYPE_NAMES.get(int(te16) // 16, "?") + ("/" + EPI_NAMES[int(te16) % 16] if int(te16) // 16 == 1 else "")
             p = phases[name]
             p["n"] += 1
@@ -60,10 +67,14 @@ def summarize(tr: np.ndarray, sm_clock_mhz: float = 1965.0) -> dict:
             p["mma_us"] += mm / sm_clock_mhz
             p["epi_us"] += ep / sm_clock_mhz
             p["rel_us"] += rl / sm_clock_mhz
+            p["loop_us"] += lo / sm_clock_mhz
+            p["pre_us"] += pr / sm_clock_mhz
+            p["post_us"] += po / sm_clock_mhz
+            p["sig_us"] += sg / sm_clock_mhz
             busy += (te - td) / 1e3 - wf / sm_clock_mhz - wx / sm_clock_mhz
     ctas = tr.shape[0]
     step_us = (t1 - t0) / 1e3
-    out = {"step_us": step_us, "ctas": ctas, "phases": {}}
+    out = {"step_us": step_us, "ctas": ctas, "sm_clock_mhz": sm_clock_mhz, "phases": {}}
     for name, p in sorted(phases.items()):
         out["phases"][name] = {k: (v / ctas if k.endswith("_us") else v) for k, v in p.items()}
         out["phases"][name]["per_cta_us_note"] = "times summed over the CTA's tasks, averaged over CTAs"
