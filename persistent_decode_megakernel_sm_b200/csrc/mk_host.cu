@@ -276,7 +276,8 @@ static mk_status dalloc(mk_handle* h, void** p, size_t bytes) {
 
 static int cdiv(int a, int b) { return (a + b - 1) / b; }
 
-static mk_status add_mat(mk_handle* h, int rows, int cols, int fp8, int gu, const MatMap& mp, int* out_idx) {
+static mk_status add_mat(mk_handle* h, int rows, int cols, int fp8, int gu, const MatMap& mp, int* out_idx,
+                         int ne = 1) {
   MatHost mh{};
   mh.m.rows = rows;
   mh.m.cols = cols;
@@ -284,9 +285,12 @@ static mk_status add_mat(mk_handle* h, int rows, int cols, int fp8, int gu, cons
   mh.m.KT = cdiv(cols, 16);
   mh.m.fp8 = fp8;
   mh.m.gu = gu;
+  mh.m.ne = ne;
   mh.map = mp;
   const size_t tb = fp8 ? TILE_FP8 : TILE_BF16;
-  mh.bytes = (size_t)mh.m.RT * mh.m.KT * tb;
+  const size_t one = (size_t)mh.m.RT * mh.m.KT * tb;
+  mh.m.estride = (int64_t)one;
+  mh.bytes = one * ne;
   void* p = nullptr;
   mk_status s = dalloc(h, &p, mh.bytes);
   if (s != MK_OK) return s;
@@ -296,7 +300,9 @@ static mk_status add_mat(mk_handle* h, int rows, int cols, int fp8, int gu, cons
     const int lrows = gu ? rows / 2 : rows;
     mh.m.nbr = cdiv(lrows, 128);
     mh.m.nbc = cdiv(cols, 128);
-    const size_t sb = (size_t)(gu ? 2 : 1) * mh.m.nbr * mh.m.nbc * sizeof(float);
+    const size_t per = (size_t)(gu ? 2 : 1) * mh.m.nbr * mh.m.nbc;
+    mh.m.sstride = (int64_t)per;
+    const size_t sb = per * ne * sizeof(float);
     s = dalloc(h, &p, sb);
     if (s != MK_OK) return s;
     mh.m.scales = reinterpret_cast<const float*>(p);
@@ -320,9 +326,16 @@ static bool desc_ok(const mk_model_desc* d, std::string& why) {
   if (d->n_routed == 0) {
     if (d->ffn < 8 || d->ffn % 8) { why = "ffn must be a positive multiple of 8"; return false; }
   } else {
-    why = "mixture-of-experts layers are not supported by this build";
-    return false;
+    if (d->n_routed > 256 || d->top_k < 1 || d->top_k > 8 || d->top_k > d->n_routed) {
+      why = "MoE needs 1 <= top_k <= min(8, n_routed) and n_routed <= 256";
+      return false;
+    }
+    if (d->expert_ffn < 16 || d->expert_ffn % 16 || d->n_shared < 0 || d->n_shared > 8) {
+      why = "expert_ffn must be a positive multiple of 16, n_shared in [0, 8]";
+      return false;
+    }
   }
+  if (d->expert_fp8 && d->n_routed == 0) { why = "fp8 weights are supported for experts only"; return false; }
   return true;
 }
 
@@ -375,18 +388,54 @@ mk_status mk_create(const mk_model_desc* desc, int device, mk_handle** out) {
       mp.kindA = SYN_WO;
       mp.lcolsA = Hq * hd;
       TRY(add_mat(h, H, Hq * hd, 0, 0, mp, &ly.m_o));
-      mp = MatMap{};
-      mp.layer = l;
-      mp.type = MAP_GU;
-      mp.kindA = SYN_WGATE;
-      mp.kindB = SYN_WUP;
-      mp.lcolsA = mp.lcolsB = H;
-      TRY(add_mat(h, 2 * d.ffn, H, 0, 1, mp, &ly.m_gu));
-      mp = MatMap{};
-      mp.layer = l;
-      mp.kindA = SYN_WDOWN;
-      mp.lcolsA = d.ffn;
-      TRY(add_mat(h, H, d.ffn, 0, 0, mp, &ly.m_down));
+      ly.m_gu = ly.m_down = ly.m_router = ly.m_shgu = ly.m_shdown = ly.m_exgu = ly.m_exdown = -1;
+      if (d.n_routed == 0) {
+        mp = MatMap{};
+        mp.layer = l;
+        mp.type = MAP_GU;
+        mp.kindA = SYN_WGATE;
+        mp.kindB = SYN_WUP;
+        mp.lcolsA = mp.lcolsB = H;
+        TRY(add_mat(h, 2 * d.ffn, H, 0, 1, mp, &ly.m_gu));
+        mp = MatMap{};
+        mp.layer = l;
+        mp.kindA = SYN_WDOWN;
+        mp.lcolsA = d.ffn;
+        TRY(add_mat(h, H, d.ffn, 0, 0, mp, &ly.m_down));
+      } else {
+        const int Ie = d.expert_ffn, E = d.n_routed, NS = d.n_shared, f8 = d.expert_fp8 ? 1 : 0;
+        mp = MatMap{};
+        mp.layer = l;
+        mp.kindA = SYN_ROUTER;
+        mp.lcolsA = H;
+        TRY(add_mat(h, E, H, 0, 0, mp, &ly.m_router));
+        if (NS > 0) {
+          mp = MatMap{};
+          mp.layer = l;
+          mp.type = MAP_GU;
+          mp.kindA = SYN_SH_GATE;
+          mp.kindB = SYN_SH_UP;
+          mp.lcolsA = mp.lcolsB = H;
+          TRY(add_mat(h, 2 * Ie, H, f8, 1, mp, &ly.m_shgu, NS));
+          mp = MatMap{};
+          mp.layer = l;
+          mp.kindA = SYN_SH_DOWN;
+          mp.lcolsA = Ie;
+          TRY(add_mat(h, H, Ie, f8, 0, mp, &ly.m_shdown, NS));
+        }
+        mp = MatMap{};
+        mp.layer = l;
+        mp.type = MAP_GU;
+        mp.kindA = SYN_EX_GATE;
+        mp.kindB = SYN_EX_UP;
+        mp.lcolsA = mp.lcolsB = H;
+        TRY(add_mat(h, 2 * Ie, H, f8, 1, mp, &ly.m_exgu, E));
+        mp = MatMap{};
+        mp.layer = l;
+        mp.kindA = SYN_EX_DOWN;
+        mp.lcolsA = Ie;
+        TRY(add_mat(h, H, Ie, f8, 0, mp, &ly.m_exdown, E));
+      }
     }
     {
       MatMap mp{};
@@ -446,10 +495,15 @@ mk_status mk_create(const mk_model_desc* desc, int device, mk_handle** out) {
     }
     // ---- scratch ----
     const int MB = MAXM;
-    const int widths[NBUF] = {H, (Hq + 2 * G) * hd, Hq * hd, std::max(d.ffn, 8), 64};
+    // B_H: dense [M][ffn]; MoE [slot][M][expert_ffn] with slots = shared + the most
+    // distinct routed experts one step can select
+    const int hw = d.n_routed ? d.expert_ffn : d.ffn;
+    const int hslots = d.n_routed ? d.n_shared + std::min(d.n_routed, MAXM * d.top_k) : 1;
+    const int widths[NBUF] = {H, (Hq + 2 * G) * hd, Hq * hd, std::max(hw, 8), std::max(d.n_routed, 4)};
     for (int b = 0; b < NBUF; ++b) {
       h->ld[b] = (widths[b] + 3) & ~3;
-      TRY(dalloc(h, (void**)&h->buf[b], (size_t)MB * h->ld[b] * sizeof(float)));
+      const size_t rows = (b == B_H) ? (size_t)hslots * MB : (size_t)MB;
+      TRY(dalloc(h, (void**)&h->buf[b], rows * h->ld[b] * sizeof(float)));
     }
     TRY(dalloc(h, (void**)&h->ss_part, (size_t)2 * h->ncta * MAXM * sizeof(float)));
     TRY(dalloc(h, (void**)&h->am_val, (size_t)h->ncta * MAXM * sizeof(float)));
@@ -515,15 +569,31 @@ mk_status mk_launch_info(mk_handle* h, int32_t* ctas, int32_t* smem_bytes, int32
 // ---------------------------------------------------------------------------
 // weights
 // ---------------------------------------------------------------------------
-static void launch_fill(const MatHost& mh, uint64_t seed, float sigA, float sigB) {
-  const uint64_t kA = syn_key(seed, syn_stream((uint32_t)mh.map.kindA, (uint32_t)mh.map.layer, (uint32_t)mh.map.expert));
-  const uint64_t kB = syn_key(seed, syn_stream((uint32_t)mh.map.kindB, (uint32_t)mh.map.layer, (uint32_t)mh.map.expert));
-  const float sA = mh.m.fp8 ? syn_normal_scale(16.0) : syn_normal_scale(sigA);
-  const float sB = mh.m.fp8 ? syn_normal_scale(16.0) : syn_normal_scale(sigB);
+static void launch_fill(const MatHost& mh, uint64_t seed, float sigA, float sigB, float fp8_base) {
   const int64_t n = (int64_t)mh.m.RT * mh.m.KT * 32;
   const int blocks = (int)std::min<int64_t>((n + 255) / 256, 148 * 16);
-  fill_tiles_kernel<<<blocks, 256>>>(const_cast<uint8_t*>(mh.m.w), mh.m.RT, mh.m.KT, mh.m.rows, mh.m.cols, mh.m.fp8,
-                                     mh.map, kA, kB, sA, sB);
+  for (int e = 0; e < mh.m.ne; ++e) {
+    MatMap mp = mh.map;
+    if (mh.m.ne > 1 || mp.kindA == SYN_EX_GATE || mp.kindA == SYN_EX_DOWN || mp.kindA == SYN_SH_GATE ||
+        mp.kindA == SYN_SH_DOWN)
+      mp.expert = e;
+    const uint64_t kA = syn_key(seed, syn_stream((uint32_t)mp.kindA, (uint32_t)mp.layer, (uint32_t)mp.expert));
+    const uint64_t kB = syn_key(seed, syn_stream((uint32_t)mp.kindB, (uint32_t)mp.layer, (uint32_t)mp.expert));
+    const float sA = mh.m.fp8 ? syn_normal_scale(16.0) : syn_normal_scale(sigA);
+    const float sB = mh.m.fp8 ? syn_normal_scale(16.0) : syn_normal_scale(sigB);
+    uint8_t* w = const_cast<uint8_t*>(mh.m.w) + (size_t)e * mh.m.estride;
+    fill_tiles_kernel<<<blocks, 256>>>(w, mh.m.RT, mh.m.KT, mh.m.rows, mh.m.cols, mh.m.fp8, mp, kA, kB, sA, sB);
+    if (mh.m.fp8) {
+      const int64_t per = (int64_t)mh.m.nbr * mh.m.nbc;
+      float* sc = const_cast<float*>(mh.m.scales) + (size_t)e * mh.m.sstride;
+      const uint64_t sk = syn_key(seed, syn_stream(SYN_FP8_SCALE, (uint32_t)mp.layer, ((uint32_t)mp.kindA << 12) | (uint32_t)mp.expert));
+      fill_scales_kernel<<<64, 256>>>(sc, per, sk, fp8_base);
+      if (mh.m.gu) {
+        const uint64_t sk2 = syn_key(seed, syn_stream(SYN_FP8_SCALE, (uint32_t)mp.layer, ((uint32_t)mp.kindB << 12) | (uint32_t)mp.expert));
+        fill_scales_kernel<<<64, 256>>>(sc + per, per, sk2, fp8_base);
+      }
+    }
+  }
 }
 
 static void launch_fill_vec(uint16_t* dst, int64_t n, uint64_t key, float sc, int gain) {
@@ -548,7 +618,7 @@ mk_status mk_init_random(mk_handle* h, const mk_synth_params* p) {
   }
   for (auto& mh : h->mats) {
     const float sig = (mh.map.kindA == SYN_ROUTER) ? p->router_sigma : p->w_sigma;
-    launch_fill(mh, seed, sig, p->w_sigma);
+    launch_fill(mh, seed, sig, p->w_sigma, p->fp8_block_base);
   }
   CK(cudaGetLastError());
   CK(cudaDeviceSynchronize());
@@ -559,7 +629,13 @@ mk_status mk_init_random(mk_handle* h, const mk_synth_params* p) {
 static int find_mat(mk_handle* h, int kind, int layer, int expert, int* which) {
   for (size_t i = 0; i < h->mats.size(); ++i) {
     const MatMap& mp = h->mats[i].map;
-    if (mp.layer != layer || mp.expert != expert) continue;
+    if (mp.layer != layer) continue;
+    if (h->mats[i].m.ne > 1 || kind == SYN_EX_GATE || kind == SYN_EX_UP || kind == SYN_EX_DOWN ||
+        kind == SYN_SH_GATE || kind == SYN_SH_UP || kind == SYN_SH_DOWN) {
+      if (expert < 0 || expert >= h->mats[i].m.ne) continue;
+    } else if (mp.expert != expert) {
+      continue;
+    }
     if (mp.kindA == kind) { *which = 0; return (int)i; }
     if ((mp.type == MAP_GU || mp.type == MAP_CONCAT) && mp.kindB == kind) { *which = 1; return (int)i; }
   }
@@ -610,15 +686,15 @@ mk_status mk_load_weights(mk_handle* h, const mk_tensor_src* ts, int n) {
     }
     const int64_t nthr = (int64_t)mh.m.RT * mh.m.KT * 32;
     const int blocks = (int)std::min<int64_t>((nthr + 255) / 256, 148 * 16);
-    retile_kernel<<<blocks, 256>>>(const_cast<uint8_t*>(mh.m.w), mh.m.RT, mh.m.KT, mh.m.rows, mh.m.cols, mh.m.fp8,
-                                   mh.map, which, src, lcols);
+    retile_kernel<<<blocks, 256>>>(const_cast<uint8_t*>(mh.m.w) + (size_t)(mh.m.ne > 1 || t.expert > 0 ? t.expert : 0) * mh.m.estride,
+                                   mh.m.RT, mh.m.KT, mh.m.rows, mh.m.cols, mh.m.fp8, mh.map, which, src, lcols);
     cudaError_t e = cudaDeviceSynchronize();
     if (staging) cudaFree(staging);
     if (e != cudaSuccess) return fail(h, MK_ERR_CUDA, std::string("retile: ") + cudaGetErrorString(e));
     if (mh.m.fp8) {
       if (!t.scales) return fail(h, MK_ERR_INVALID, "fp8 tensor without scales");
       const size_t sn = (size_t)mh.m.nbr * mh.m.nbc;
-      float* dst = const_cast<float*>(mh.m.scales) + (mh.m.gu && which ? sn : 0);
+      float* dst = const_cast<float*>(mh.m.scales) + (size_t)t.expert * mh.m.sstride + (mh.m.gu && which ? sn : 0);
       CK(cudaMemcpy(dst, t.scales, sn * sizeof(float), kind));
     }
   }
@@ -790,24 +866,72 @@ static mk_status get_plan(mk_handle* h, int S, int Q, Plan** out) {
         per[c].push_back(t);
       }
     }
-    // gate/up + SwiGLU
-    {
-      auto rr = split_rows(h->mats[ly.m_gu].m.RT, ncta, rot);
+    if (d.n_routed == 0) {
+      // gate/up + SwiGLU
+      {
+        auto rr = split_rows(h->mats[ly.m_gu].m.RT, ncta, rot);
+        for (int c = 0; c < ncta; ++c) {
+          Task t = gemv(l, ly.m_gu, rr[c].first, rr[c].second, IN_X_NORM, 0, EPI_SWIGLU, B_H, 1, C(l, C_O), ncta,
+                        C(l, C_GU));
+          t.ss_src = 0;
+          per[c].push_back(t);
+        }
+      }
+      // down projection + residual
+      {
+        auto rr = split_rows(h->mats[ly.m_down].m.RT, ncta, rot);
+        for (int c = 0; c < ncta; ++c) {
+          Task t = gemv(l, ly.m_down, rr[c].first, rr[c].second, IN_BUF, B_H, EPI_RESID, 0, 0, C(l, C_GU), ncta,
+                        C(l, C_DOWN));
+          t.ss_dst = 1;
+          per[c].push_back(t);
+        }
+      }
+    } else {
+      // Phase order of one MoE layer: router -> shared expert -> routed experts
+      // -> down projection over all of them.  The shared expert's weights are
+      // streamed while the router's choice is being made; only the routed
+      // experts' (and the down) tiles wait for it.
+      {
+        auto rr = split_rows(h->mats[ly.m_router].m.RT, ncta, rot);
+        for (int c = 0; c < ncta; ++c) {
+          Task t = gemv(l, ly.m_router, rr[c].first, rr[c].second, IN_X_NORM, 0, EPI_STORE, B_RLOG, 1, C(l, C_O),
+                        ncta, C(l, C_ROUTER));
+          t.ss_src = 0;
+          per[c].push_back(t);
+        }
+      }
+      if (d.n_shared > 0) {
+        const MatHost& sh = h->mats[ly.m_shgu];
+        auto rr = split_rows(sh.m.RT * sh.m.ne, ncta, rot);
+        for (int c = 0; c < ncta; ++c) {
+          Task t = gemv(l, ly.m_shgu, rr[c].first, rr[c].second, IN_X_NORM, 0, EPI_SWIGLU_MOE, B_H, 1, C(l, C_O),
+                        ncta, C(l, C_GU));
+          t.type = T_MOE_GU;
+          t.moe = 1;
+          t.ss_src = 0;
+          per[c].push_back(t);
+        }
+      }
       for (int c = 0; c < ncta; ++c) {
-        Task t = gemv(l, ly.m_gu, rr[c].first, rr[c].second, IN_X_NORM, 0, EPI_SWIGLU, B_H, 1, C(l, C_O), ncta,
-                      C(l, C_GU));
+        // rows decided on the device from the router's union of experts
+        Task t = gemv(l, ly.m_exgu, 0, 0, IN_X_NORM, 0, EPI_SWIGLU_MOE, B_H, 1, C(l, C_ROUTER), ncta, C(l, C_GU));
+        t.type = T_MOE_GU;
+        t.moe = 2;
         t.ss_src = 0;
         per[c].push_back(t);
       }
-    }
-    // down projection + residual
-    {
-      auto rr = split_rows(h->mats[ly.m_down].m.RT, ncta, rot);
-      for (int c = 0; c < ncta; ++c) {
-        Task t = gemv(l, ly.m_down, rr[c].first, rr[c].second, IN_BUF, B_H, EPI_RESID, 0, 0, C(l, C_GU), ncta,
-                      C(l, C_DOWN));
-        t.ss_dst = 1;
-        per[c].push_back(t);
+      {
+        auto rr = split_rows(h->mats[ly.m_exdown].m.RT, ncta, rot);
+        const int ngu = (d.n_shared > 0 ? 2 : 1) * ncta;
+        for (int c = 0; c < ncta; ++c) {
+          Task t = gemv(l, ly.m_exdown, rr[c].first, rr[c].second, IN_BUF, B_H, EPI_RESID, 0, 0, C(l, C_GU), ngu,
+                        C(l, C_DOWN));
+          t.type = T_MOE_DOWN;
+          t.mat2 = ly.m_shdown;
+          t.ss_dst = 1;
+          per[c].push_back(t);
+        }
       }
     }
   }

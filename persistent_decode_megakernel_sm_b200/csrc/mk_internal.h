@@ -20,13 +20,9 @@ constexpr int NCT = NCW * 32;                // consumer threads
 #ifndef MK_NSTAGE
 #define MK_NSTAGE 2
 #endif
-#ifndef MK_PREFETCH
-#define MK_PREFETCH 0
-#endif
 constexpr int TILE_CAP = MK_TILE_CAP;        // weight tile bytes per GEMV chunk (gains follow)
 constexpr int STAGE_BYTES = (TILE_CAP + 1024 > 34816) ? TILE_CAP + 1024 : 34816;  // >= one attention chunk
 constexpr int NSTAGE = MK_NSTAGE;            // weight ring depth
-constexpr int PREFETCH_CHUNKS = MK_PREFETCH; // L2 lookahead beyond the ring, in chunks
 constexpr int XSLOTS = 2;                    // activation ring depth
 constexpr int XSLOT_BYTES = 22528;           // one activation window: M rows x (cols + pad)
 constexpr int XROW_PAD = 32;                 // bytes between activation rows (bank spread)
@@ -48,8 +44,8 @@ constexpr int TILE_FP8 = 256;                // 16x16 e4m3 tile in A-fragment or
 enum TaskType : int16_t {
   T_GEMV = 1,      // out rows [rt0, rt1) of a matrix
   T_ATTN = 2,      // one split-KV attention item (GQA)
-  T_MOE_GU = 3,    // routed expert gate/up tiles (data dependent)
-  T_MOE_DOWN = 4,  // down projection over shared + selected experts
+  T_MOE_GU = 3,    // expert gate/up row tiles (shared: static; routed: union of the router's picks)
+  T_MOE_DOWN = 4,  // down projection, K = shared + selected experts' hidden units
   T_TOPK = 5,      // (unused placeholder)
   T_EMBED = 6,     // x[m][c0:c1) = embedding rows of the step's tokens (+ RMS partial sums)
 };
@@ -61,10 +57,11 @@ enum InKind : int16_t {
 };
 
 enum Epi : int16_t {
-  EPI_STORE = 0,   // out[m][row] = v
-  EPI_RESID = 1,   // x[m][row] = base + v, base = x or the embedding (layer 0)
-  EPI_SWIGLU = 2,  // tile rows 0..7 gate, 8..15 up: h[m][i] = silu(g) u
-  EPI_LOGITS = 3,  // logits + per-CTA argmax partial
+  EPI_STORE = 0,       // out[m][row] = v
+  EPI_RESID = 1,       // x[m][row] += v (+ per-CTA sums of squares)
+  EPI_SWIGLU = 2,      // tile rows 0..7 gate, 8..15 up: h[m][i] = silu(g) u
+  EPI_LOGITS = 3,      // logits + per-CTA argmax partial
+  EPI_SWIGLU_MOE = 4,  // expert slot s: h[s][m][i] = w(s, m) silu(g) u
 };
 
 enum BufId : int16_t {
@@ -75,31 +72,36 @@ struct Task {
   int16_t type, layer;
   int16_t in_kind, epi;
   int16_t in_buf, out_buf;
-  int16_t resid_emb, gain;   // resid base = embedding; gain: 0 attn, 1 ffn, 2 final
+  int16_t moe, gain;         // moe: 1 shared experts, 2 routed experts; gain: 0 attn, 1 ffn, 2 final
   int32_t mat;               // matrix table index
   int32_t rt0, rt1;          // row tiles (GEMV) / item index (ATTN)
   int32_t wait_ctr, wait_tgt;
   int32_t sig_ctr;           // counter incremented when the task is done (-1: none)
   int32_t ss_src;            // IN_X_NORM: which partial-sum array (0: after O, 1: after down)
   int32_t ss_dst;            // EPI_RESID: partial-sum array written
+  int32_t mat2;              // T_MOE_DOWN: the shared experts' down matrix
 };
 
 // ---------------------------------------------------------------------------
 // device-resident model description
 // ---------------------------------------------------------------------------
 struct Mat {
-  const uint8_t* w;          // tiles [RT][KT][tile]
-  const float* scales;       // fp8: [nbr][nbc] (GU: [2][nbr][nbc], gate then up)
-  int32_t rows, cols, RT, KT;
+  const uint8_t* w;          // tiles [RT][KT][tile] (expert arrays: [ne][RT][KT][tile])
+  const float* scales;       // fp8: [nbr][nbc] (GU: [2][nbr][nbc], gate then up), per expert
+  int32_t rows, cols, RT, KT;  // of one expert
   int32_t fp8;
   int32_t nbr, nbc;
   int32_t gu;                // rows interleaved gate/up by 8
+  int32_t ne;                // experts in the array (1 for a plain matrix)
+  int64_t estride;           // bytes between experts' tiles
+  int64_t sstride;           // floats between experts' scales
 };
 
 struct Layer {
   const uint16_t* attn_norm;
   const uint16_t* ffn_norm;
   int32_t m_qkv, m_o, m_gu, m_down;
+  int32_t m_router, m_shgu, m_shdown, m_exgu, m_exdown;  // MoE (-1 when dense)
 };
 
 struct Model {

@@ -182,11 +182,17 @@ struct Misc {
   volatile int abort;
   int flag;
   int pad[2];
+  // MoE routing tables, one per role (each role computes its own copy)
+  int rt_u[3];
+  int16_t rt_ex[3][64];
+  float rt_w[64][MAXM];      // consumers: weight of (union slot, row)
   // per-task trace accumulators (consumer thread 0)
   long long tr_wf, tr_wx, tr_bytes;
   long long tr_frag, tr_mma, tr_epi, tr_rel, tr_loop, tr_pre, tr_post, tr_sig;
   int tr_chunks;
 };
+
+static_assert(sizeof(Misc) <= MISC_BYTES, "Misc must fit its shared-memory region");
 
 struct Ctx {
   const Launch* P;
@@ -302,6 +308,202 @@ __device__ __forceinline__ int seq_pos0(const Launch& P, int s) {
 __device__ __forceinline__ int att_pitch(int d) { return d * 2; }
 
 // ---------------------------------------------------------------------------
+// MoE routing: softmax over the router logits of each activation row, top-k by
+// logit (ties to the lower expert index), weights renormalised over the k
+// picks; the union of the picked experts in ascending expert order.  One
+// warp; every role that needs the result computes it itself from the same
+// logits with the same code, so all roles agree.
+// ---------------------------------------------------------------------------
+enum RouteRole { RR_CONS = 0, RR_PROD = 1, RR_XPROD = 2 };
+
+__device__ int moe_route(const Launch& P, const Model& md, int layer, Misc* ms, int role, bool want_w, bool trace) {
+  const int lane = threadIdx.x & 31;
+  const int E = md.E, K = md.K, M = P.M;
+  const float* rl = P.buf[B_RLOG];
+  const int ld = P.ld[B_RLOG];
+  uint32_t ubits = 0;  // bit q: expert lane + 32 q picked by some row
+  int selE[MAXM];
+  float selW[MAXM];
+#pragma unroll
+  for (int mm = 0; mm < MAXM; ++mm) {
+    selE[mm] = -1;
+    selW[mm] = 0.f;
+    if (mm < M) {
+      float v[8];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int e = lane + 32 * q;
+        v[q] = e < E ? __ldcg(rl + (size_t)mm * ld + e) : -INFINITY;
+        mx = fmaxf(mx, v[q]);
+      }
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      float sum = 0.f;
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (lane + 32 * q < E) sum += expf(v[q] - mx);
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      float psum = 0.f, my_p = 0.f;
+      int my_e = -1;
+      for (int j = 0; j < K; ++j) {
+        float bv = -INFINITY;
+        int be = 0x7fffffff;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int e = lane + 32 * q;
+          if (e < E && (v[q] > bv || (v[q] == bv && e < be))) {
+            bv = v[q];
+            be = e;
+          }
+        }
+        for (int o = 16; o > 0; o >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+          const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+          if (ov > bv || (ov == bv && oe < be)) {
+            bv = ov;
+            be = oe;
+          }
+        }
+        const float pj = expf(bv - mx) / sum;
+        psum += pj;
+        if (lane == j) {
+          my_e = be;
+          my_p = pj;
+        }
+        if ((be & 31) == lane) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            if (q == (be >> 5)) v[q] = -INFINITY;
+          ubits |= 1u << (be >> 5);
+        }
+      }
+      selE[mm] = my_e;
+      selW[mm] = my_p / psum;
+    }
+  }
+  // union in ascending expert order
+  int U = 0;
+  int16_t* ex = ms->rt_ex[role];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const uint32_t b = __ballot_sync(0xffffffffu, (ubits >> q) & 1u);
+    if ((ubits >> q) & 1u) ex[U + __popc(b & ((1u << lane) - 1u))] = (int16_t)(lane + 32 * q);
+    U += __popc(b);
+  }
+  if (lane == 0) ms->rt_u[role] = U;
+  __syncwarp();
+  if (want_w) {
+    for (int i = lane; i < 64 * MAXM; i += 32) ms->rt_w[i / MAXM][i % MAXM] = 0.f;
+    __syncwarp();
+#pragma unroll
+    for (int mm = 0; mm < MAXM; ++mm) {
+      if (mm < M && lane < K) {
+        int slot = 0;
+        while (slot < U && ex[slot] != selE[mm]) ++slot;
+        ms->rt_w[slot][mm] = selW[mm];
+        if (trace && P.router_idx) {
+          P.router_idx[((size_t)layer * M + mm) * K + lane] = selE[mm];
+          P.router_w[((size_t)layer * M + mm) * K + lane] = selW[mm];
+        }
+      }
+    }
+    __syncwarp();
+  }
+  return U;
+}
+
+// The pieces of a GEMV-like task: row groups (<= RMAX row tiles, not crossing
+// an expert boundary for virtual expert rows) x K segments (one per expert for
+// the MoE down projection).
+struct Pieces {
+  int rt1, gsz, nseg;
+  int g0, nr, seg;
+  __device__ __forceinline__ void set_nr() {
+    nr = min(RMAX, rt1 - g0);
+    if (gsz > 0) nr = min(nr, (g0 / gsz + 1) * gsz - g0);
+  }
+  __device__ __forceinline__ bool init(int rt0_, int rt1_, int gsz_, int nseg_) {
+    rt1 = rt1_;
+    gsz = gsz_;
+    nseg = nseg_;
+    g0 = rt0_;
+    seg = 0;
+    if (g0 >= rt1 || nseg <= 0) return false;
+    set_nr();
+    return true;
+  }
+  __device__ __forceinline__ bool next() {
+    if (++seg < nseg) return true;
+    seg = 0;
+    g0 += nr;
+    if (g0 >= rt1) return false;
+    set_nr();
+    return true;
+  }
+};
+
+// Matrix base, local row tile and activation source of the current piece.
+struct PieceSrc {
+  const uint8_t* w;
+  const float* scales;
+  int lg0;    // first row tile inside the piece's matrix
+  int xbuf;   // activation buffer
+  int xrow0;  // first activation row in it (expert slot * MAXM for the MoE down projection)
+};
+
+__device__ __forceinline__ PieceSrc piece_src(const Model& md, const Task& t, const Mat& m, const Mat& m2,
+                                              const int16_t* ex, const Pieces& pc) {
+  PieceSrc r;
+  r.lg0 = pc.g0;
+  r.xrow0 = 0;
+  r.xbuf = t.in_kind == IN_X_NORM ? (int)B_X : (int)t.in_buf;
+  r.w = m.w;
+  r.scales = m.scales;
+  if (t.type == T_MOE_GU) {
+    const int slot = pc.g0 / m.RT;
+    const int e = t.moe == 1 ? slot : ex[slot];
+    r.w = m.w + (size_t)e * m.estride;
+    r.scales = m.scales ? m.scales + (size_t)e * m.sstride : nullptr;
+    r.lg0 = pc.g0 - slot * m.RT;
+  } else if (t.type == T_MOE_DOWN) {
+    const int ns = md.NS;
+    const Mat& mm = pc.seg < ns ? m2 : m;
+    const int e = pc.seg < ns ? pc.seg : ex[pc.seg - ns];
+    r.w = mm.w + (size_t)e * mm.estride;
+    r.scales = mm.scales ? mm.scales + (size_t)e * mm.sstride : nullptr;
+    r.xbuf = B_H;
+    r.xrow0 = pc.seg * MAXM;
+  }
+  return r;
+}
+
+// Row range, expert-group size and K-segment count of a GEMV-like task.
+__device__ __forceinline__ void task_rows(const Model& md, const Task& t, const Mat& m, int U, int& rt0, int& rt1,
+                                          int& gsz, int& nseg) {
+  rt0 = t.rt0;
+  rt1 = t.rt1;
+  gsz = 0;
+  nseg = 1;
+  if (t.type == T_MOE_GU) {
+    gsz = m.RT;
+    if (t.moe == 2) {
+      const int T = U * m.RT;
+      rt0 = (int)(((int64_t)blockIdx.x * T) / gridDim.x);
+      rt1 = (int)(((int64_t)(blockIdx.x + 1) * T) / gridDim.x);
+    }
+  } else if (t.type == T_MOE_DOWN) {
+    nseg = md.NS + U;
+  }
+}
+
+__device__ __forceinline__ bool task_needs_route(const Task& t) {
+  return (t.type == T_MOE_GU && t.moe == 2) || t.type == T_MOE_DOWN;
+}
+__device__ __forceinline__ bool gemv_like(const Task& t) {
+  return t.type == T_GEMV || t.type == T_MOE_GU || t.type == T_MOE_DOWN;
+}
+
+// ---------------------------------------------------------------------------
 // producer warp
 // ---------------------------------------------------------------------------
 // Reserve ring slot `it` for `bytes` (lane 0 waits for the consumers to free
@@ -338,26 +540,59 @@ __device__ bool prod_reserve(const Ctx& C, uint32_t it, uint32_t bytes, long lon
   return ok != 0;
 }
 
+// Bounded wait of one warp on a dependency counter (lane 0 polls with
+// acquire); later bulk (async-proxy) reads must observe the generic-proxy
+// writes the acquire made visible, hence the proxy fence.
+__device__ bool warp_wait_counter(const Ctx& C, int idx, uint32_t target, int code) {
+  const Launch& P = *C.P;
+  const int lane = threadIdx.x & 31;
+  int ok = 1;
+  if (lane == 0) {
+    const uint32_t* p = P.ctr + idx;
+    uint64_t t0 = 0;
+    uint32_t spins = 0;
+    while ((int)(ld_acquire(p) - target) < 0) {
+      if (C.ms->abort) { ok = 0; break; }
+      __nanosleep(64);
+      if (++spins >= 16) {
+        spins = 0;
+        if (global_abort(P)) { C.ms->abort = 1; ok = 0; break; }
+        uint64_t now = globaltimer();
+        if (t0 == 0) t0 = now;
+        else if (now - t0 > (uint64_t)P.timeout_ns * 2) {
+          raise_error(P, C.ms, DERR_TIMEOUT, code | idx);
+          ok = 0;
+          break;
+        }
+      }
+    }
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  return ok != 0;
+}
+
 // One unit of streamed data, in the order the consumers take it.
 struct Chunk {
-  int kind;  // 1: GEMV tiles (+ gain slice), 2: attention K/V rows
+  int kind;  // 1: GEMV tiles, 2: attention K/V rows
   const uint8_t* w;
   int KT, tb, g0, nr, c0, nc;
-  const uint16_t* gain;
   const uint16_t* kb;
   const uint16_t* vb;
   int n, d;
 };
 
 // Walks a CTA's task list and yields its chunks in consumption order (the
-// same enumeration the consumers use).  Two instances run in the producer:
-// one issues ring loads, the other runs ahead and prefetches into L2.
+// enumeration the consumers use).  Routed-expert tasks first wait for the
+// router's counter: their tiles are the only ones that depend on activations.
 struct ChunkStream {
-  int ti, end, state;
+  int ti, end, state;  // state 0: next task, 1: GEMV-like pieces, 2: attention
+  Task t;
+  Mat m, m2;
+  Pieces pc;
   ChunkIt ci;
-  const uint8_t* w;
-  int KT, tb;
-  const uint16_t* gain;
+  PieceSrc src;
+  int tb, xcap;
   const uint16_t* kb;
   const uint16_t* vb;
   int t0, b, d;
@@ -366,20 +601,29 @@ struct ChunkStream {
     end = end_;
     state = 0;
   }
-  __device__ bool next(const Launch& P, const Model& md, Chunk& c) {
+  // returns 1 with a chunk, 0 at the end of the list, -1 on abort
+  __device__ int next(const Ctx& C, Chunk& c) {
+    const Launch& P = *C.P;
+    const Model& md = *C.md;
     while (true) {
       if (state == 1) {
         c.kind = 1;
-        c.w = w;
-        c.KT = KT;
+        c.w = src.w;
+        c.KT = m.KT;
         c.tb = tb;
         c.g0 = ci.g0;
         c.nr = ci.nr;
         c.c0 = ci.c0;
         c.nc = ci.nc;
-        c.gain = gain;
-        if (!ci.next()) state = 0;
-        return true;
+        if (!ci.next()) {
+          if (!pc.next()) {
+            state = 0;
+          } else {
+            src = piece_src(md, t, m, m2, C.ms->rt_ex[RR_PROD], pc);
+            ci.init(src.lg0, src.lg0 + pc.nr, m.KT, tb, 0, xcap);
+          }
+        }
+        return 1;
       }
       if (state == 2) {
         if (t0 < b) {
@@ -389,19 +633,29 @@ struct ChunkStream {
           c.n = min(ATT_CT, b - t0);
           c.d = d;
           t0 += ATT_CT;
-          return true;
+          return 1;
         }
         state = 0;
       }
-      if (ti >= end) return false;
-      const Task t = P.tasks[ti++];
-      if (t.type == T_GEMV) {
-        const Mat& m = md.mats[t.mat];
+      if (ti >= end) return 0;
+      t = P.tasks[ti++];
+      if (gemv_like(t)) {
+        m = md.mats[t.mat];
+        m2 = (t.type == T_MOE_DOWN && t.mat2 >= 0) ? md.mats[t.mat2] : m;
         tb = m.fp8 ? TILE_FP8 : TILE_BF16;
-        w = m.w;
-        KT = m.KT;
-        gain = task_gain(md, t);
-        if (ci.init(t.rt0, t.rt1, m.KT, tb, 0, x_cap(t, P.M))) state = 1;
+        xcap = x_cap(t, P.M);
+        int U = 0;
+        if (task_needs_route(t)) {
+          if (!warp_wait_counter(C, t.layer * P.ctr_layer_stride + C_ROUTER, (uint32_t)gridDim.x, 0x70000)) return -1;
+          U = moe_route(P, md, t.layer, C.ms, RR_PROD, false, false);
+        }
+        int rt0, rt1, gsz, nseg;
+        task_rows(md, t, m, U, rt0, rt1, gsz, nseg);
+        if (pc.init(rt0, rt1, gsz, nseg)) {
+          src = piece_src(md, t, m, m2, C.ms->rt_ex[RR_PROD], pc);
+          ci.init(src.lg0, src.lg0 + pc.nr, m.KT, tb, 0, xcap);
+          state = 1;
+        }
       } else if (t.type == T_ATTN) {
         const Item itm = decode_item(t.rt0, P.n_pairs, P.n_items);
         const int s = itm.pair / md.Hkv, g = itm.pair % md.Hkv;
@@ -418,24 +672,8 @@ struct ChunkStream {
   }
 };
 
-__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
-
-__device__ __forceinline__ void prefetch_chunk(const Chunk& c, int lane) {
-  if (c.kind == 1) {
-    if (lane < c.nr)
-      prefetch_l2(c.w + ((size_t)(c.g0 + lane) * c.KT + c.c0) * c.tb, (uint32_t)(c.nc * c.tb));
-  } else if (c.kind == 2) {
-    if (lane == 0) prefetch_l2(c.kb, (uint32_t)(c.n * c.d * 2));
-    if (lane == 1) prefetch_l2(c.vb, (uint32_t)(c.n * c.d * 2));
-  }
-}
-
 __device__ void producer(const Ctx& C) {
   const Launch& P = *C.P;
-  const Model& md = *C.md;
   const int lane = threadIdx.x & 31;
   const uint64_t pol = policy_evict_first();
   uint32_t it = 0;
@@ -443,24 +681,18 @@ __device__ void producer(const Ctx& C) {
   long long blocked = 0;
   const uint64_t t_first = globaltimer();
   const long long c_first = clock64();
-  ChunkStream is, ps;
+  ChunkStream is;
   is.init(beg, end);
-  ps.init(beg, end);
-  Chunk c, pc;
-  bool pf_live = true;
-  for (int k = 0; k < NSTAGE + PREFETCH_CHUNKS && pf_live; ++k) {
-    pf_live = ps.next(P, md, pc);
-    if (pf_live && k >= NSTAGE) prefetch_chunk(pc, lane);
-  }
-  while (is.next(P, md, c)) {
+  Chunk c;
+  while (is.next(C, c) > 0) {
     uint8_t* dst = C.ring + (size_t)(it % NSTAGE) * STAGE_BYTES;
     uint64_t* bar = &C.ms->full[it % NSTAGE];
     if (c.kind == 1) {
       const uint32_t tbytes = (uint32_t)(c.nr * c.nc * c.tb);
       if (!prod_reserve(C, it, tbytes, blocked)) goto drain;
       if (lane < c.nr) {
-        const uint8_t* src = c.w + ((size_t)(c.g0 + lane) * c.KT + c.c0) * c.tb;
-        bulk_g2s(dst + (size_t)lane * c.nc * c.tb, src, (uint32_t)(c.nc * c.tb), bar, pol);
+        const uint8_t* srcp = c.w + ((size_t)(c.g0 + lane) * c.KT + c.c0) * c.tb;
+        bulk_g2s(dst + (size_t)lane * c.nc * c.tb, srcp, (uint32_t)(c.nc * c.tb), bar, pol);
       }
     } else {
       // the cache rows of this chunk are contiguous: one copy for K, one for V
@@ -472,10 +704,6 @@ __device__ void producer(const Ctx& C) {
     }
     __syncwarp();
     ++it;
-    if (pf_live) {
-      pf_live = ps.next(P, md, pc);
-      if (pf_live) prefetch_chunk(pc, lane);
-    }
   }
 drain:
   if (lane == 0 && P.trace && P.trace_cap > 0) {
@@ -513,37 +741,6 @@ drain:
 // dependency (acquire), then streams the activation slice of every chunk
 // (M rows x the chunk's columns) into the x ring with bulk copies, so the
 // consumers never wait on a global-memory round trip inside a task.
-__device__ bool xprod_wait_counter(const Ctx& C, int idx, uint32_t target) {
-  const Launch& P = *C.P;
-  const int lane = threadIdx.x & 31;
-  int ok = 1;
-  if (lane == 0) {
-    const uint32_t* p = P.ctr + idx;
-    uint64_t t0 = 0;
-    uint32_t spins = 0;
-    while ((int)(ld_acquire(p) - target) < 0) {
-      if (C.ms->abort) { ok = 0; break; }
-      __nanosleep(64);
-      if (++spins >= 16) {
-        spins = 0;
-        if (global_abort(P)) { C.ms->abort = 1; ok = 0; break; }
-        uint64_t now = globaltimer();
-        if (t0 == 0) t0 = now;
-        else if (now - t0 > (uint64_t)P.timeout_ns * 2) {
-          raise_error(P, C.ms, DERR_TIMEOUT, 0x30000 | idx);
-          ok = 0;
-          break;
-        }
-      }
-    }
-    // later bulk (async-proxy) reads must observe the generic-proxy writes
-    // that the acquire made visible
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-  }
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  return ok != 0;
-}
-
 __device__ bool xprod_reserve(const Ctx& C, uint32_t ix, uint32_t bytes) {
   const int lane = threadIdx.x & 31;
   int ok = 1;
@@ -585,12 +782,18 @@ __device__ void xproducer(const Ctx& C) {
   if (P.stall_ctr >= 0) return;
   for (int ti = beg; ti < end; ++ti) {
     const Task t = P.tasks[ti];
-    if (t.type != T_GEMV) continue;
-    const Mat& m = md.mats[t.mat];
+    if (!gemv_like(t)) continue;
+    const Mat m = md.mats[t.mat];
+    const Mat m2 = (t.type == T_MOE_DOWN && t.mat2 >= 0) ? md.mats[t.mat2] : m;
     const int tb = m.fp8 ? TILE_FP8 : TILE_BF16;
-    ChunkIt ci;
-    if (!ci.init(t.rt0, t.rt1, m.KT, tb, 0, x_cap(t, M))) continue;
-    if (t.wait_ctr >= 0 && !xprod_wait_counter(C, t.wait_ctr, (uint32_t)t.wait_tgt)) goto drain;
+    const int xcap = x_cap(t, M);
+    if (t.wait_ctr >= 0 && !warp_wait_counter(C, t.wait_ctr, (uint32_t)t.wait_tgt, 0x30000)) goto drain;
+    int U = 0;
+    if (task_needs_route(t)) U = moe_route(P, md, t.layer, C.ms, RR_XPROD, false, false);
+    int rt0, rt1, gsz, nseg;
+    task_rows(md, t, m, U, rt0, rt1, gsz, nseg);
+    Pieces pc;
+    if (!pc.init(rt0, rt1, gsz, nseg)) continue;
     // RMSNorm scale of every activation row (fixed-order reduction of the
     // per-CTA sums of squares) and the norm gain of this task
     float scale[MAXM];
@@ -600,86 +803,92 @@ __device__ void xproducer(const Ctx& C) {
     for (int mm = 0; mm < MAXM; ++mm) {
       scale[mm] = 1.f;
       if (has_gain && mm < M) {
-        const float* src = P.ss_part + (size_t)t.ss_src * gridDim.x * MAXM;
+        const float* srcs = P.ss_part + (size_t)t.ss_src * gridDim.x * MAXM;
         float ss = 0.f;
-        for (int c = lane; c < (int)gridDim.x; c += 32) ss += __ldcg(src + c * MAXM + mm);
+        for (int c = lane; c < (int)gridDim.x; c += 32) ss += __ldcg(srcs + c * MAXM + mm);
         for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
         scale[mm] = rsqrtf(ss / (float)md.H + md.eps);
       }
     }
     do {
-      if (!ci.win_first()) continue;
-      const int rb = x_rowbytes(t, ci.WC);
-      const int wn = ci.wn(), w0 = ci.w0();
-      const uint32_t rowdata = (uint32_t)(wn * 64);
-      const int sl = ix % XSLOTS;
-      if (!xprod_reserve(C, ix, (uint32_t)M * rowdata)) goto drain;
-      uint8_t* dst = C.xring + (size_t)sl * XSLOT_BYTES;
-      if (lane < M) {
-        const int b = t.in_kind == IN_X_NORM ? (int)B_X : (int)t.in_buf;
-        const uint8_t* src = reinterpret_cast<const uint8_t*>(P.buf[b] + (size_t)lane * P.ld[b] + ci.c0 * 16);
-        bulk_g2s(dst + (size_t)lane * rb, src, rowdata, &C.ms->xfull[sl], pol);
-      }
-      // wait for this warp's own copy, then convert the window in place into
-      // ready mma B fragments: col tile jj of row m (16 fp32, 64 B) becomes,
-      // for each quad lane tq, 16 B = {hi(k 2tq,2tq+1), hi(k 2tq+8,2tq+9),
-      // lo(..), lo(..)} of x * rms_scale * gain (bf16 split; f16 for fp8 weights)
-      {
-        const uint32_t par = (ix / XSLOTS) & 1;
-        const uint64_t t0 = globaltimer();
-        bool landed = true;
-        while (!mbar_try_wait(&C.ms->xfull[sl], par)) {
-          if (C.ms->abort || globaltimer() - t0 > (uint64_t)P.timeout_ns * 2) { landed = false; break; }
+      const PieceSrc src = piece_src(md, t, m, m2, C.ms->rt_ex[RR_XPROD], pc);
+      ChunkIt ci;
+      ci.init(src.lg0, src.lg0 + pc.nr, m.KT, tb, 0, xcap);
+      do {
+        if (!ci.win_first()) continue;
+        const int rb = x_rowbytes(t, ci.WC);
+        const int wn = ci.wn(), w0 = ci.w0();
+        const uint32_t rowdata = (uint32_t)(wn * 64);
+        const int sl = ix % XSLOTS;
+        if (!xprod_reserve(C, ix, (uint32_t)M * rowdata)) goto drain;
+        uint8_t* dst = C.xring + (size_t)sl * XSLOT_BYTES;
+        if (lane < M) {
+          const uint8_t* xsrc = reinterpret_cast<const uint8_t*>(
+              P.buf[src.xbuf] + (size_t)(src.xrow0 + lane) * P.ld[src.xbuf] + ci.c0 * 16);
+          bulk_g2s(dst + (size_t)lane * rb, xsrc, rowdata, &C.ms->xfull[sl], pol);
         }
-        if (!__all_sync(0xffffffffu, landed)) {
-          if (lane == 0 && !C.ms->abort) raise_error(P, C.ms, DERR_TIMEOUT, 0x60000 | sl);
-          goto drain;
-        }
-      }
-      for (int e = lane; e < M * wn; e += 32) {
-        const int mm = e / wn, jj = e - mm * wn;
-        float4* p4 = reinterpret_cast<float4*>(dst + (size_t)mm * rb + (size_t)jj * 64);
-        float v[16];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4 f = p4[q];
-          v[4 * q] = f.x;
-          v[4 * q + 1] = f.y;
-          v[4 * q + 2] = f.z;
-          v[4 * q + 3] = f.w;
-        }
-        if (has_gain) {
-          float s = 1.f;
-#pragma unroll
-          for (int q = 0; q < MAXM; ++q) if (q == mm) s = scale[q];
-          const uint4* gp = reinterpret_cast<const uint4*>(gain + (size_t)(w0 + jj) * 16);
-          const uint4 ga = __ldg(gp), gb = __ldg(gp + 1);
-          const uint32_t gw[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            v[2 * q] = v[2 * q] * s * bf16lo(gw[q]);
-            v[2 * q + 1] = v[2 * q + 1] * s * bf16hi(gw[q]);
+        // wait for this warp's own copy, then convert the window in place into
+        // ready mma B fragments: col tile jj of row m (16 fp32, 64 B) becomes,
+        // for each quad lane tq, 16 B = {hi(k 2tq,2tq+1), hi(k 2tq+8,2tq+9),
+        // lo(..), lo(..)} of x * rms_scale * gain (bf16 split; f16 for fp8 weights)
+        {
+          const uint32_t par = (ix / XSLOTS) & 1;
+          const uint64_t t0 = globaltimer();
+          bool landed = true;
+          while (!mbar_try_wait(&C.ms->xfull[sl], par)) {
+            if (C.ms->abort || globaltimer() - t0 > (uint64_t)P.timeout_ns * 2) { landed = false; break; }
+          }
+          if (!__all_sync(0xffffffffu, landed)) {
+            if (lane == 0 && !C.ms->abort) raise_error(P, C.ms, DERR_TIMEOUT, 0x60000 | sl);
+            goto drain;
           }
         }
-        uint4 o[4];
+        for (int e = lane; e < M * wn; e += 32) {
+          const int mm = e / wn, jj = e - mm * wn;
+          float4* p4 = reinterpret_cast<float4*>(dst + (size_t)mm * rb + (size_t)jj * 64);
+          float v[16];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          if (!m.fp8) {
-            split_bf16(v[2 * q], v[2 * q + 1], o[q].x, o[q].z);
-            split_bf16(v[2 * q + 8], v[2 * q + 9], o[q].y, o[q].w);
-          } else {
-            split_f16(v[2 * q], v[2 * q + 1], o[q].x, o[q].z);
-            split_f16(v[2 * q + 8], v[2 * q + 9], o[q].y, o[q].w);
+          for (int q = 0; q < 4; ++q) {
+            const float4 f = p4[q];
+            v[4 * q] = f.x;
+            v[4 * q + 1] = f.y;
+            v[4 * q + 2] = f.z;
+            v[4 * q + 3] = f.w;
           }
-        }
-        uint4* o4 = reinterpret_cast<uint4*>(p4);
+          if (has_gain) {
+            float sc = 1.f;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) o4[q] = o[q];
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&C.ms->xready[sl]);
-      ++ix;
-    } while (ci.next());
+            for (int q = 0; q < MAXM; ++q)
+              if (q == mm) sc = scale[q];
+            const uint4* gp = reinterpret_cast<const uint4*>(gain + (size_t)(w0 + jj) * 16);
+            const uint4 ga = __ldg(gp), gb = __ldg(gp + 1);
+            const uint32_t gw[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              v[2 * q] = v[2 * q] * sc * bf16lo(gw[q]);
+              v[2 * q + 1] = v[2 * q + 1] * sc * bf16hi(gw[q]);
+            }
+          }
+          uint4 o[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (!m.fp8) {
+              split_bf16(v[2 * q], v[2 * q + 1], o[q].x, o[q].z);
+              split_bf16(v[2 * q + 8], v[2 * q + 9], o[q].y, o[q].w);
+            } else {
+              split_f16(v[2 * q], v[2 * q + 1], o[q].x, o[q].z);
+              split_f16(v[2 * q + 8], v[2 * q + 9], o[q].y, o[q].w);
+            }
+          }
+          uint4* o4 = reinterpret_cast<uint4*>(p4);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) o4[q] = o[q];
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&C.ms->xready[sl]);
+        ++ix;
+      } while (ci.next());
+    } while (pc.next());
   }
 drain:
   if (lane == 0) {
@@ -822,7 +1031,7 @@ struct GemvLane {
 // are left in `red` for the cross-warp reduction.
 template <int NR, bool FP8>
 __device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& mr, const GemvLane& Lr, uint32_t& itr,
-                                        uint32_t& ixr, float* red) {
+                                        uint32_t& ixr, float* red, bool accum) {
   // register copies (the arguments live in the caller's frame)
   const Ctx C = Cr;
   const Mat m = mr;
@@ -905,10 +1114,17 @@ __device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
     ci.next();
   }
   if (L.trc) C.ms->tr_loop += clock64() - tl0;
+  // per-warp partial sums (added to the previous K segments' when accum)
 #pragma unroll
-  for (int r = 0; r < NR; ++r)
-    *reinterpret_cast<float4*>(red + ((L.warp * RMAX + r) * 32 + lane) * 4) =
-        make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+  for (int r = 0; r < NR; ++r) {
+    float4* pr = reinterpret_cast<float4*>(red + ((L.warp * RMAX + r) * 32 + lane) * 4);
+    if (accum) {
+      const float4 q = *pr;
+      *pr = make_float4(q.x + acc[r][0], q.y + acc[r][1], q.z + acc[r][2], q.w + acc[r][3]);
+    } else {
+      *pr = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+    }
+  }
   cir = ci;
   itr = it;
   ixr = ix;
@@ -931,8 +1147,20 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
   float am_v[2] = {-INFINITY, -INFINITY};
   int am_i[2] = {0x7fffffff, 0x7fffffff};
 
-  ChunkIt ci;
-  bool have = ci.init(t.rt0, t.rt1, m.KT, tb, 0, x_cap(t, M));
+  // MoE: this task's rows / K segments follow the router's union of experts
+  int U = 0;
+  if (task_needs_route(t)) {
+    if (warp == 0)
+      moe_route(P, md, t.layer, C.ms, RR_CONS, t.type == T_MOE_GU, blockIdx.x == 0 && t.type == T_MOE_GU);
+    bar_consumers();
+    U = C.ms->rt_u[RR_CONS];
+  }
+  const Mat m2 = (t.type == T_MOE_DOWN && t.mat2 >= 0) ? md.mats[t.mat2] : m;
+  int rt0, rt1, gsz, nseg;
+  task_rows(md, t, m, U, rt0, rt1, gsz, nseg);
+  Pieces pc;
+  bool have = pc.init(rt0, rt1, gsz, nseg);
+  const int xcap = x_cap(t, M);
   float* red = reinterpret_cast<float*>(C.att);
   GemvLane L;
   L.warp = warp;
@@ -945,31 +1173,41 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
   L.trc = P.trace && tid == 0;
   if (L.trc) C.ms->tr_pre += clock64() - tpre;
   while (have) {
+    const PieceSrc src = piece_src(md, t, m, m2, C.ms->rt_ex[RR_CONS], pc);
+    ChunkIt ci;
+    ci.init(src.lg0, src.lg0 + pc.nr, m.KT, tb, 0, xcap);
     L.rowbytes = x_rowbytes(t, ci.WC);
-    // one instance per row-tile count: every loop below is fully static
+    Mat mg = (t.type == T_MOE_DOWN && pc.seg < md.NS) ? m2 : m;
+    mg.w = src.w;
+    mg.scales = src.scales;
+    const bool accum = pc.seg > 0;
     // one instance per row-tile count: every loop over rows is static
     if (!m.fp8) {
       switch (ci.nr) {
-        case 1: gemv_group<1, false>(C, ci, m, L, it, ix, red); break;
-        case 2: gemv_group<2, false>(C, ci, m, L, it, ix, red); break;
-        case 3: gemv_group<3, false>(C, ci, m, L, it, ix, red); break;
-        case 4: gemv_group<4, false>(C, ci, m, L, it, ix, red); break;
-        case 5: gemv_group<5, false>(C, ci, m, L, it, ix, red); break;
-        case 6: gemv_group<6, false>(C, ci, m, L, it, ix, red); break;
-        case 7: gemv_group<7, false>(C, ci, m, L, it, ix, red); break;
-        default: gemv_group<8, false>(C, ci, m, L, it, ix, red); break;
+        case 1: gemv_group<1, false>(C, ci, mg, L, it, ix, red, accum); break;
+        case 2: gemv_group<2, false>(C, ci, mg, L, it, ix, red, accum); break;
+        case 3: gemv_group<3, false>(C, ci, mg, L, it, ix, red, accum); break;
+        case 4: gemv_group<4, false>(C, ci, mg, L, it, ix, red, accum); break;
+        case 5: gemv_group<5, false>(C, ci, mg, L, it, ix, red, accum); break;
+        case 6: gemv_group<6, false>(C, ci, mg, L, it, ix, red, accum); break;
+        case 7: gemv_group<7, false>(C, ci, mg, L, it, ix, red, accum); break;
+        default: gemv_group<8, false>(C, ci, mg, L, it, ix, red, accum); break;
       }
     } else {
       switch (ci.nr) {
-        case 1: gemv_group<1, true>(C, ci, m, L, it, ix, red); break;
-        case 2: gemv_group<2, true>(C, ci, m, L, it, ix, red); break;
-        case 3: gemv_group<3, true>(C, ci, m, L, it, ix, red); break;
-        case 4: gemv_group<4, true>(C, ci, m, L, it, ix, red); break;
-        case 5: gemv_group<5, true>(C, ci, m, L, it, ix, red); break;
-        case 6: gemv_group<6, true>(C, ci, m, L, it, ix, red); break;
-        case 7: gemv_group<7, true>(C, ci, m, L, it, ix, red); break;
-        default: gemv_group<8, true>(C, ci, m, L, it, ix, red); break;
+        case 1: gemv_group<1, true>(C, ci, mg, L, it, ix, red, accum); break;
+        case 2: gemv_group<2, true>(C, ci, mg, L, it, ix, red, accum); break;
+        case 3: gemv_group<3, true>(C, ci, mg, L, it, ix, red, accum); break;
+        case 4: gemv_group<4, true>(C, ci, mg, L, it, ix, red, accum); break;
+        case 5: gemv_group<5, true>(C, ci, mg, L, it, ix, red, accum); break;
+        case 6: gemv_group<6, true>(C, ci, mg, L, it, ix, red, accum); break;
+        case 7: gemv_group<7, true>(C, ci, mg, L, it, ix, red, accum); break;
+        default: gemv_group<8, true>(C, ci, mg, L, it, ix, red, accum); break;
       }
+    }
+    if (pc.seg != pc.nseg - 1) {
+      have = pc.next();
+      continue;
     }
     const bool trc = L.trc;
     long long tc0 = trc ? clock64() : 0;
@@ -978,7 +1216,7 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
       bar_consumers();
       {
         const int r = tid >> 5, l = lane;
-        if (r < ci.nr) {
+        if (r < pc.nr) {
           float v[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int w = 0; w < NCW; ++w) {
@@ -988,7 +1226,7 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
             v[2] += q.z;
             v[3] += q.w;
           }
-          const int rt = ci.g0 + r;
+          const int rt = pc.g0 + r;
           const int row0 = rt * 16 + (l >> 2), row1 = row0 + 8;
           const int m0 = 2 * (l & 3), m1 = m0 + 1;
           if (t.epi == EPI_STORE) {
@@ -1015,6 +1253,19 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
                 x[(size_t)mm * ld + row] = nv;
                 ss_acc[q & 1] += nv * nv;
               }
+            }
+          } else if (t.epi == EPI_SWIGLU_MOE) {
+            // virtual row tile rt of expert slot rt / RTe (shared slots first)
+            const int slot = rt / m.RT;
+            const int hs = (t.moe == 1 ? 0 : md.NS) + slot;
+            const int i = (rt - slot * m.RT) * 8 + (l >> 2);
+            float* h = P.buf[B_H];
+            const int ld = P.ld[B_H];
+            if (i * 2 < m.rows) {
+              const float w0 = t.moe == 1 ? 1.f : C.ms->rt_w[slot][m0 < MAXM ? m0 : 0];
+              const float w1 = t.moe == 1 ? 1.f : C.ms->rt_w[slot][m1 < MAXM ? m1 : 0];
+              if (m0 < M) h[((size_t)hs * MAXM + m0) * ld + i] = w0 * silu_f(v[0]) * v[2];
+              if (m1 < M) h[((size_t)hs * MAXM + m1) * ld + i] = w1 * silu_f(v[1]) * v[3];
             }
           } else if (t.epi == EPI_SWIGLU) {
             float* h = P.buf[t.out_buf];
@@ -1044,7 +1295,7 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
       bar_consumers();
       if (trc) C.ms->tr_epi += clock64() - tc0;
     }
-    have = ci.next();
+    have = pc.next();
   }
 
   const long long tpost = L.trc ? clock64() : 0;
@@ -1567,7 +1818,7 @@ __device__ void consumer(const Ctx& C) {
     }
     if (t.wait_ctr >= 0) wait_counter(C, t.wait_ctr, (uint32_t)t.wait_tgt);
     if (tr) td = globaltimer();
-    if (t.type == T_GEMV) {
+    if (gemv_like(t)) {
       gemv_task(C, t, it, ix);
     } else if (t.type == T_ATTN) {
       attn_task(C, t, it);
