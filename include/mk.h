@@ -132,6 +132,38 @@ int64_t mk_kv_bytes(const mk_kv* kv);
 mk_status mk_decode_step(mk_handle* h, const int32_t* tokens, const int32_t* positions, int B,
                          mk_kv* kv, float* logits_out, int32_t* argmax_out, void* stream);
 
+/* Size of the static device array behind mk_decode_step_noalloc, in bytes.
+ * Every GPU that loads this library holds it until the process exits. */
+#define MK_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* mk_decode_step that allocates no device memory.  The pages this library
+ * follows have no counterpart; it is here for callers that cannot call
+ * cudaMalloc while they step the model: a process whose device memory is all
+ * owned by its own allocator (a framework's caching allocator, a serving
+ * engine that sizes its KV pool to fill the GPU), or a latency-critical loop
+ * that must not let cudaMalloc / cudaFree synchronise the device.
+ * (mk_decode_step allocates the device task list of a batch size the first
+ * time that size is used.)
+ *   Arguments, results and device-error reporting are those of
+ *   mk_decode_step (errors through mk_sync_status on the same handle).
+ *   The task list, activations, partial sums, split-KV partials and
+ *   inter-CTA counters live in one file-scope device array of
+ *   MK_NOALLOC_SCRATCH_BYTES, shared by every handle on the device and
+ *   keeping the last call's contents.  The counters must start at zero: each
+ *   call clears them on `stream` before its launch; nothing else needs it.
+ *   The task list is rebuilt on the host and copied in (from pageable host
+ *   memory, on `stream`) only when another handle or batch size used the
+ *   array last.
+ *   The first call on a device looks up the array's device address (a
+ *   one-time set-up); make that first call before any stream capture.
+ *   Calls that overlap on the GPU (other streams, other handles on the same
+ *   device, or mk_decode_step_noalloc from several host threads without
+ *   ordering their streams) race on the array: order them.
+ *   A model and batch size whose scratch exceeds MK_NOALLOC_SCRATCH_BYTES
+ *   are rejected with MK_ERR_INVALID (mk_last_error gives the bytes needed). */
+mk_status mk_decode_step_noalloc(mk_handle* h, const int32_t* tokens, const int32_t* positions, int B,
+                                 mk_kv* kv, float* logits_out, int32_t* argmax_out, void* stream);
+
 /* Speculative verify of one sequence (sequence 0 of the cache): tokens8 =
  * anchor followed by n_prop (<= 7) proposals, dev int32 [n_prop + 1], placed
  * at positions position .. position + n_prop, causal within the chunk.  K/V

@@ -7,7 +7,9 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <map>
+#include <mutex>
 #include <string>
 #include <utility>
 #include <vector>
@@ -241,6 +243,7 @@ struct mk_handle {
   int64_t timeout_ns = 1000000000LL;
   bool sticky = false;
   bool initialised = false;
+  uint64_t noalloc_id = 0;  // identity of this handle for mk_decode_step_noalloc's installed task list
   std::string err;
 };
 
@@ -808,12 +811,11 @@ static Task gemv(int layer, int mat, int rt0, int rt1, int in_kind, int in_buf, 
   return t;
 }
 
-static mk_status get_plan(mk_handle* h, int S, int Q, Plan** out) {
-  auto it = h->plans.find(PlanKey{S, Q});
-  if (it != h->plans.end()) {
-    *out = &it->second;
-    return MK_OK;
-  }
+// The task list of one step shape, built on the host: per-CTA task lists
+// flattened into `flat`, CTA c owning flat[off[c], off[c + 1]).
+static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>& flat, std::vector<int32_t>& off,
+                            int& n_items_out, int& n_pairs_out) {
+  (void)Q;
   const mk_model_desc& d = h->desc;
   const int ncta = h->ncta, L = d.layers;
   const int n_pairs = S * d.n_kv_heads;
@@ -945,13 +947,27 @@ static mk_status get_plan(mk_handle* h, int S, int Q, Plan** out) {
       per[c].push_back(t);
     }
   }
-  std::vector<Task> flat;
-  std::vector<int32_t> off(ncta + 1, 0);
+  flat.clear();
+  off.assign(ncta + 1, 0);
   for (int c = 0; c < ncta; ++c) {
     off[c] = (int32_t)flat.size();
     flat.insert(flat.end(), per[c].begin(), per[c].end());
   }
   off[ncta] = (int32_t)flat.size();
+  n_items_out = n_items;
+  n_pairs_out = n_pairs;
+}
+
+static mk_status get_plan(mk_handle* h, int S, int Q, Plan** out) {
+  auto it = h->plans.find(PlanKey{S, Q});
+  if (it != h->plans.end()) {
+    *out = &it->second;
+    return MK_OK;
+  }
+  std::vector<Task> flat;
+  std::vector<int32_t> off;
+  int n_items = 0, n_pairs = 0;
+  build_plan_host(h, S, Q, flat, off, n_items, n_pairs);
   Plan p;
   p.n_items = n_items;
   p.n_pairs = n_pairs;
@@ -1091,3 +1107,166 @@ mk_status mk_debug_inject_stall(mk_handle* h, int64_t timeout_ns) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// mk_decode_step_noalloc: the decode step with its scratch in a static array
+// ---------------------------------------------------------------------------
+// Who needs it: a caller that has handed its whole device-memory budget to its
+// own allocator (a framework's caching allocator, a serving engine that sizes
+// its KV pool to fill the GPU after warm-up) has nothing left for cudaMalloc,
+// and a caller that steps the model from a latency-critical loop cannot let a
+// cudaMalloc or cudaFree synchronise the device in the middle of it.
+// mk_decode_step itself allocates the device task list of a batch size on the
+// first call with that size; this variant keeps the task list and every
+// per-step scratch buffer (activations, per-CTA partial sums, split-KV
+// partials, inter-CTA counters) in the one array below instead.
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MK_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+struct NoallocDevice {
+  unsigned char* base = nullptr;  // device address of g_noalloc_scratch on this device
+  uint64_t plan_owner = 0;        // handle whose task list is in the array (0: none)
+  int plan_S = 0;                 // ... and its batch size
+  size_t plan_tasks = 0;
+  int plan_items = 0, plan_pairs = 0;
+};
+constexpr int NOALLOC_MAX_DEVICES = 64;
+std::mutex g_noalloc_mu;
+NoallocDevice g_noalloc_dev[NOALLOC_MAX_DEVICES];
+std::atomic<uint64_t> g_noalloc_next_id{1};
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+}  // namespace
+
+extern "C" mk_status mk_decode_step_noalloc(mk_handle* h, const int32_t* tokens, const int32_t* positions, int B,
+                                            mk_kv* kv, float* logits_out, int32_t* argmax_out, void* stream) {
+  if (!h) return MK_ERR_INVALID;
+  if (!tokens || !positions || !kv || !argmax_out) return fail(h, MK_ERR_INVALID, "null argument");
+  if (kv->h != h) return fail(h, MK_ERR_INVALID, "kv cache belongs to another model");
+  if (B < 1 || B > h->desc.max_batch || B > kv->max_seqs) return fail(h, MK_ERR_INVALID, "B out of range");
+  if (h->sticky) return fail(h, MK_ERR_STATE, "a previous device error is pending; call mk_reset");
+  if (!h->initialised) return fail(h, MK_ERR_STATE, "weights not initialised");
+  if (h->device < 0 || h->device >= NOALLOC_MAX_DEVICES) return fail(h, MK_ERR_INVALID, "device ordinal too large");
+  CK(cudaSetDevice(h->device));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const mk_model_desc& d = h->desc;
+
+  // The task list is rebuilt only when another handle or batch size used the
+  // array last; it is built on the host (no device memory involved).
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  NoallocDevice& nd = g_noalloc_dev[h->device];
+  if (!nd.base) {
+    // one-time set-up on this device (the device is current): the host-side
+    // name of the array is not a device address, so ask the runtime for it
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(h, MK_ERR_CUDA, std::string("cudaGetSymbolAddress of the static scratch: ") + cudaGetErrorString(e));
+    nd.base = static_cast<unsigned char*>(p);
+  }
+  if (h->noalloc_id == 0) h->noalloc_id = g_noalloc_next_id.fetch_add(1);
+
+  std::vector<Task> flat;
+  std::vector<int32_t> off;
+  const bool installed = nd.plan_owner == h->noalloc_id && nd.plan_S == B;
+  int n_items = nd.plan_items, n_pairs = nd.plan_pairs;
+  size_t n_tasks = nd.plan_tasks;
+  if (!installed) {
+    build_plan_host(h, B, 1, flat, off, n_items, n_pairs);
+    n_tasks = flat.size();
+  }
+
+  // carve the array: task list, offsets, activation buffers, partials, counters
+  const int hw_rows_h = d.n_routed ? d.n_shared + std::min(d.n_routed, MAXM * d.top_k) : 1;
+  size_t at = 0;
+  const size_t o_tasks = at;
+  at = align256(at + n_tasks * sizeof(Task));
+  const size_t o_off = at;
+  at = align256(at + (size_t)(h->ncta + 1) * sizeof(int32_t));
+  size_t o_buf[NBUF];
+  for (int b = 0; b < NBUF; ++b) {
+    o_buf[b] = at;
+    const size_t rows = (b == B_H) ? (size_t)hw_rows_h * MAXM : (size_t)MAXM;
+    at = align256(at + rows * h->ld[b] * sizeof(float));
+  }
+  const size_t o_ss = at;
+  at = align256(at + (size_t)2 * h->ncta * MAXM * sizeof(float));
+  const size_t o_amv = at;
+  at = align256(at + (size_t)h->ncta * MAXM * sizeof(float));
+  const size_t o_ami = at;
+  at = align256(at + (size_t)h->ncta * MAXM * sizeof(int32_t));
+  const size_t o_att = at;
+  at = align256(at + (size_t)n_items * h->att_rows_max * (d.head_dim + 2) * sizeof(float));
+  const size_t o_ctr = at;
+  at = align256(at + (size_t)h->n_ctr * sizeof(uint32_t));
+  if (at > (size_t)MK_NOALLOC_SCRATCH_BYTES)
+    return fail(h, MK_ERR_INVALID,
+                "mk_decode_step_noalloc: this model and batch need " + std::to_string(at) +
+                    " bytes of scratch; the static array holds " + std::to_string((size_t)MK_NOALLOC_SCRATCH_BYTES));
+  unsigned char* base = nd.base;
+
+  if (!installed) {
+    // pageable host source: the call returns once the source has been read
+    nd.plan_owner = 0;
+    CK(cudaMemcpyAsync(base + o_tasks, flat.data(), n_tasks * sizeof(Task), cudaMemcpyHostToDevice, st));
+    CK(cudaMemcpyAsync(base + o_off, off.data(), off.size() * sizeof(int32_t), cudaMemcpyHostToDevice, st));
+    nd.plan_owner = h->noalloc_id;
+    nd.plan_S = B;
+    nd.plan_tasks = n_tasks;
+    nd.plan_items = n_items;
+    nd.plan_pairs = n_pairs;
+  }
+  // The inter-CTA counters must start at zero.  A completed step leaves them
+  // zero, but one that stopped on a device error does not, and the array is
+  // shared by every handle on the device: clear them before every step.
+  // Nothing else needs clearing: every other region is written before it is read.
+  CK(cudaMemsetAsync(base + o_ctr, 0, (size_t)h->n_ctr * sizeof(uint32_t), st));
+
+  Launch P{};
+  P.model = h->d_model;
+  P.tasks = reinterpret_cast<const Task*>(base + o_tasks);
+  P.task_off = reinterpret_cast<const int32_t*>(base + o_off);
+  P.tokens = tokens;
+  P.positions = positions;
+  P.pos_const = 0;
+  P.S = B;
+  P.Q = 1;
+  P.M = B;
+  P.kv_k = kv->k;
+  P.kv_v = kv->v;
+  P.kv_seqs = kv->max_seqs;
+  P.kv_ctx = kv->max_ctx;
+  P.logits = logits_out;
+  P.argmax = argmax_out;
+  P.accepted = nullptr;
+  P.router_idx = h->trace_idx;
+  P.router_w = h->trace_w;
+  for (int b = 0; b < NBUF; ++b) {
+    P.buf[b] = reinterpret_cast<float*>(base + o_buf[b]);
+    P.ld[b] = h->ld[b];
+  }
+  P.ss_part = reinterpret_cast<float*>(base + o_ss);
+  P.am_val = reinterpret_cast<float*>(base + o_amv);
+  P.am_idx = reinterpret_cast<int32_t*>(base + o_ami);
+  P.att_part = reinterpret_cast<float*>(base + o_att);
+  P.att_rows_max = h->att_rows_max;
+  P.ctr = reinterpret_cast<uint32_t*>(base + o_ctr);
+  P.ctr_layer_stride = NCTR_LAYER;
+  P.ctr_pair_base = (d.layers + 1) * NCTR_LAYER;
+  P.ctr_lm = P.ctr_pair_base + d.layers * h->max_pairs;
+  P.ctr_done = P.ctr_lm + 1;
+  P.n_ctr = h->n_ctr;
+  P.status = h->status;  // device errors are read with mk_sync_status, as for mk_decode_step
+  P.timeout_ns = h->timeout_ns;
+  P.stall_ctr = -1;
+  P.n_items = n_items;
+  P.n_pairs = n_pairs;
+  P.trace = h->task_trace;
+  P.trace_cap = h->task_trace_cap;
+  void* args[] = {&P};
+  const cudaError_t e = cudaLaunchCooperativeKernel((const void*)mk_step_kernel, dim3(h->ncta), dim3(NTHREADS), args,
+                                                    SMEM_BYTES, st);
+  if (e != cudaSuccess) return fail(h, MK_ERR_CUDA, std::string("launch: ") + cudaGetErrorString(e));
+  return MK_OK;
+}

@@ -20,7 +20,7 @@ STATUS_NAMES = {0: "MK_OK", 1: "MK_ERR_INVALID", 2: "MK_ERR_OOM", 3: "MK_ERR_CUD
 
 # Every symbol include/mk.h declares.
 EXPORTS = ("mk_create", "mk_init_random", "mk_load_weights", "mk_kv_create", "mk_kv_fill_random", "mk_kv_copy_out",
-           "mk_kv_bytes", "mk_decode_step", "mk_verify", "mk_set_router_trace", "mk_set_trace", "mk_sync_status", "mk_reset",
+           "mk_kv_bytes", "mk_decode_step", "mk_decode_step_noalloc", "mk_verify", "mk_set_router_trace", "mk_set_trace", "mk_sync_status", "mk_reset",
            "mk_launch_info", "mk_weight_bytes", "mk_debug_inject_stall", "mk_last_error", "mk_kv_destroy",
            "mk_destroy")
 
@@ -65,6 +65,7 @@ def _load() -> ctypes.CDLL:
         "mk_kv_copy_out": ([vp, vp], st),
         "mk_kv_bytes": ([vp], i64),
         "mk_decode_step": ([vp, vp, vp, ctypes.c_int, vp, vp, vp, vp], st),
+        "mk_decode_step_noalloc": ([vp, vp, vp, ctypes.c_int, vp, vp, vp, vp], st),
         "mk_verify": ([vp, vp, ctypes.c_int, i32, vp, vp, vp, vp, vp], st),
         "mk_set_router_trace": ([vp, vp, vp], st),
         "mk_set_trace": ([vp, vp, i32], st),
@@ -152,6 +153,13 @@ def mk_kv_bytes(kv: int) -> int:
 def mk_decode_step(h: int, tokens, positions, B: int, kv: int, logits_out, argmax_out, stream=None) -> None:
     _check(h, lib.mk_decode_step(h, _ptr(tokens), _ptr(positions), B, kv, _ptr(logits_out), _ptr(argmax_out),
                                  _stream(stream)))
+
+
+def mk_decode_step_noalloc(h: int, tokens, positions, B: int, kv: int, logits_out, argmax_out, stream=None) -> None:
+    """mk_decode_step with every scratch buffer in the library's static
+    device array: no device allocation in the call (include/mk.h)."""
+    _check(h, lib.mk_decode_step_noalloc(h, _ptr(tokens), _ptr(positions), B, kv, _ptr(logits_out), _ptr(argmax_out),
+                                         _stream(stream)))
 
 
 def mk_verify(h: int, tokens8, n_prop: int, position: int, kv: int, logits_out, argmax_out, accepted_out,
