@@ -40,7 +40,12 @@ def parse():
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--config", default="dense27b")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--sweep", default="1,8", help="extra batch sizes timed for the by_batch table ('' = none)")
+    ap.add_argument("--sweep", default="1,2,4,8", help="batch sizes timed for the by_batch table ('' = none)")
+    ap.add_argument("--workloads", default="moe,mla_fp8,verify",
+                    help="other workloads of the study timed after the headline ('' = none)")
+    ap.add_argument("--verify-steps", type=int, default=256)
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="DRAM bytes per launch of the kernel from an ncu capture of this build (null if none)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=16)
     return ap.parse_args()
@@ -58,17 +63,47 @@ def measured_peaks():
 # ---------------------------------------------------------------------------
 # algorithmic bytes of one decode step (what the method must move)
 # ---------------------------------------------------------------------------
-def step_bytes(mc, B, positions, weight_bytes, write_logits=True):
-    """All streamed weights (the embedding table only for the B rows used),
-    the KV rows attended (positions 0..p per sequence, every layer), the KV
-    rows written and the logits written."""
-    embed_table = mc.vocab * mc.hidden * 2
-    w = weight_bytes - embed_table + B * mc.hidden * 2
-    kv_tok_layer = 2 * mc.n_kv_heads * mc.head_dim * 2
-    kv_read = sum(int(p) for p in positions) * kv_tok_layer * mc.layers   # prefix 0..p-1 read from HBM
-    kv_write = B * kv_tok_layer * mc.layers
-    logits = B * mc.vocab * 4 if write_logits else 0
-    return w + kv_read + kv_write + logits
+def _mat_bytes(rows, cols, fp8=False):
+    if not fp8:
+        return rows * cols * 2
+    return rows * cols + (-(-rows // 128)) * (-(-cols // 128)) * 4
+
+
+def expert_bytes(mc):
+    f8 = bool(mc.expert_fp8)
+    return 2 * _mat_bytes(mc.expert_ffn, mc.hidden, f8) + _mat_bytes(mc.hidden, mc.expert_ffn, f8)
+
+
+def step_bytes(mc, pos0, Q=1, unions=None, write_logits=True):
+    """Algorithmic bytes of one step: every weight the step needs (for MoE
+    layers the router, the shared experts and only the union of the routed
+    experts picked by the step's rows, `unions[l]`), B embedding rows, the
+    cached KV / latent rows attended (positions 0..p-1 of each sequence, read
+    once even in verify), the rows written and the logits written.
+    pos0: first position of each sequence; Q positions per sequence."""
+    H, L, V = mc.hidden, mc.layers, mc.vocab
+    Hq, d = mc.n_q_heads, mc.head_dim
+    M = len(pos0) * Q
+    total = _mat_bytes(V, H) + H * 2 + M * H * 2          # LM head, final norm, embedding rows
+    for l in range(L):
+        total += 2 * H * 2                                 # norm gains
+        if mc.mla:
+            R, dr = mc.kv_lora_rank, mc.rope_dim
+            total += (_mat_bytes(Hq * (d + dr) + R + dr, H) + _mat_bytes(Hq * R, d) + _mat_bytes(Hq * d, R)
+                      + _mat_bytes(H, Hq * d))
+        else:
+            total += _mat_bytes((Hq + 2 * mc.n_kv_heads) * d, H) + _mat_bytes(H, Hq * d)
+        if mc.n_routed == 0:
+            total += _mat_bytes(2 * mc.ffn, H) + _mat_bytes(H, mc.ffn)
+        else:
+            u = unions[l] if unions is not None else min(mc.n_routed, M * mc.top_k)
+            total += _mat_bytes(mc.n_routed, H) + (mc.n_shared + u) * expert_bytes(mc)
+    kvt = (mc.kv_lora_rank + mc.rope_dim) * 2 if mc.mla else 2 * mc.n_kv_heads * d * 2
+    total += sum(int(p) for p in pos0) * kvt * L           # cached rows read
+    total += M * kvt * L                                   # new rows written
+    if write_logits:
+        total += M * V * 4
+    return total
 
 
 # ---------------------------------------------------------------------------
@@ -119,26 +154,38 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = f"cuda:{local_rank}"
-    mc = synth.preset(args.config)
-    Bmax = max([args.batch] + [int(b) for b in args.sweep.split(",") if b])
-    model = Megakernel(mc, device=local_rank, max_batch=8)
-    model.init_random(mc.seed, mc.w_sigma, mc.router_sigma, mc.gain_sigma, mc.fp8_block_base)
-    kv = model.kv_cache(8, mc.max_ctx)
-    kv.fill_random(synth.SEED_KV, mc.kv_sigma, mc.context)
-    ctas, smem, threads = model.launch_info()
     stream = torch.cuda.current_stream()
+    peak, peak_kind = measured_peaks()
 
-    def time_batch(B, steps, warmup, clocks=False):
+    def load(config):
+        mc = synth.preset(config)
+        model = Megakernel(mc, device=local_rank, max_batch=8)
+        model.init_random(mc.seed, mc.w_sigma, mc.router_sigma, mc.gain_sigma, mc.fp8_block_base)
+        kv = model.kv_cache(8, mc.max_ctx)
+        kv.fill_random(synth.SEED_KV, mc.kv_sigma, mc.context)
+        return mc, model, kv
+
+    def router_unions(mc, idx):
+        a = idx.cpu().numpy()
+        return [len(set(a[l].reshape(-1).tolist())) for l in range(mc.layers)]
+
+    def decode_run(mc, model, kv, B, steps, warmup, clocks=False):
+        """Greedy decode of B sequences from the synthetic context: `warmup`
+        untimed steps, then `steps` steps timed with CUDA events on the
+        launching stream.  For MoE models the same steps are replayed
+        afterwards (same cache state, same tokens) with the router trace on,
+        to count the experts each timed step had to read."""
         total = warmup + steps
         assert mc.context + total <= mc.max_ctx
         pos = torch.tensor([[mc.context + i] * B for i in range(total)], dtype=torch.int32, device=dev)
         toks = torch.tensor(synth.tokens(synth.SEED_TOKENS, B, mc.vocab), dtype=torch.int32, device=dev)
-        am = [torch.zeros(B, dtype=torch.int32, device=dev) for _ in range(2)]
+        am = [torch.zeros(B, dtype=torch.int32, device=dev) for _ in range(total)]
         logits = torch.empty((B, mc.vocab), dtype=torch.float32, device=dev)
+        kv.fill_random(synth.SEED_KV, mc.kv_sigma, mc.context)
         cur = toks
         for i in range(warmup):
-            model.decode_step(cur, pos[i], kv, logits, am[i & 1], stream)
-            cur = am[i & 1]
+            model.decode_step(cur, pos[i], kv, logits, am[i], stream)
+            cur = am[i]
         torch.cuda.synchronize()
         assert model.sync_status() == 0, "device error during warm-up"
         if world > 1:
@@ -148,8 +195,8 @@ def run_ours(args, rank, world, local_rank):
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
         ev[0].record(stream)
         for i in range(steps):
-            model.decode_step(cur, pos[warmup + i], kv, logits, am[i & 1], stream)
-            cur = am[i & 1]
+            model.decode_step(cur, pos[warmup + i], kv, logits, am[warmup + i], stream)
+            cur = am[warmup + i]
             ev[i + 1].record(stream)
         torch.cuda.synchronize()
         clk = ck.stop() if ck else None
@@ -160,32 +207,102 @@ def run_ours(args, rank, world, local_rank):
             t = torch.tensor([ms], device=dev)
             torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
             ms = float(t.item())
-        positions = [mc.context + warmup] * B
-        return ms, per, clk, positions
+        unions = None
+        if mc.n_routed:
+            kv.fill_random(synth.SEED_KV, mc.kv_sigma, mc.context)
+            idx = torch.zeros((mc.layers, B, mc.top_k), dtype=torch.int32, device=dev)
+            w = torch.zeros((mc.layers, B, mc.top_k), dtype=torch.float32, device=dev)
+            unions = []
+            cur = toks
+            for i in range(total):
+                model.set_router_trace(idx, w)
+                model.decode_step(cur, pos[i], kv, logits, am[i], stream)
+                model.set_router_trace(None, None)
+                cur = am[i]
+                if i >= warmup:
+                    unions.append(router_unions(mc, idx))
+        nbytes = [step_bytes(mc, [mc.context + warmup + i] * B, 1, unions[i] if unions else None)
+                  for i in range(steps)]
+        mean_bytes = statistics.mean(nbytes)
+        launch_ms = statistics.mean(per)
+        gbs = mean_bytes / (launch_ms / 1e3) / 1e9
+        out = {"tokens_per_s": world * B * steps / (ms / 1e3), "ms_per_step": ms / steps,
+               "bytes_per_step": mean_bytes, "hbm_gbs": gbs, "frac_of_measured": gbs / peak, "frac_of_8tbs": gbs / 8000.0}
+        if unions:
+            out["routed_experts_per_layer_mean"] = statistics.mean(statistics.mean(u) for u in unions)
+        return out, ms, per, clk, mean_bytes
 
-    ms, per, clk, positions = time_batch(args.batch, args.steps, args.warmup, clocks=True)
+    def verify_run(mc, model, kv, steps, warmup):
+        """Speculative verify on one sequence: each step checks an anchor and
+        7 seeded uniform proposals at position P over the synthetic context;
+        the next anchor is the greedy token after the accepted prefix and P
+        advances by accepted + 1 (rewound to the context end when the cache
+        would overflow).  Device time per launch from CUDA events."""
+        def one_pass(record_unions):
+            kv.fill_random(synth.SEED_KV, mc.kv_sigma, mc.context)
+            anchor = int(synth.tokens(synth.SEED_TOKENS, 1, mc.vocab)[0])
+            P = mc.context
+            am = torch.zeros(8, dtype=torch.int32, device=dev)
+            acc = torch.zeros(1, dtype=torch.int32, device=dev)
+            idx = torch.zeros((mc.layers, 8, mc.top_k), dtype=torch.int32, device=dev)
+            w = torch.zeros((mc.layers, 8, mc.top_k), dtype=torch.float32, device=dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            times, accepted, unions, starts = [], [], [], []
+            for i in range(warmup + steps):
+                props = synth.proposals(synth.SEED_PROPOSALS, i, 7, mc.vocab)
+                toks = torch.tensor([anchor] + [int(x) for x in props], dtype=torch.int32, device=dev)
+                if record_unions:
+                    model.set_router_trace(idx, w)
+                e0.record(stream)
+                model.verify(toks, P, kv, None, am, acc, stream)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                if record_unions:
+                    model.set_router_trace(None, None)
+                a = int(acc.item())
+                if i >= warmup:
+                    times.append(e0.elapsed_time(e1))
+                    accepted.append(a)
+                    starts.append(P)
+                    if record_unions:
+                        unions.append(router_unions(mc, idx))
+                anchor = int(am[a].item())
+                P += a + 1
+                if P + 8 > mc.max_ctx:
+                    P = mc.context
+            assert model.sync_status() == 0
+            return times, accepted, unions, starts
+
+        times, accepted, _, starts = one_pass(False)
+        _, acc2, unions, _ = one_pass(True)
+        assert acc2 == accepted, "verify replay diverged"
+        nbytes = [step_bytes(mc, [starts[i]], 8, unions[i], write_logits=False) for i in range(steps)]
+        ms = statistics.mean(times)
+        gbs = statistics.mean(nbytes) / (ms / 1e3) / 1e9
+        hist = {}
+        for a in accepted:
+            hist[str(a)] = hist.get(str(a), 0) + 1
+        return {"verify_steps": steps, "ms_per_verify_step": ms, "accepted_hist": hist,
+                "emitted_tokens_per_s": sum(a + 1 for a in accepted) / (sum(times) / 1e3),
+                "bytes_per_step": statistics.mean(nbytes), "hbm_gbs": gbs, "frac_of_measured": gbs / peak,
+                "frac_of_8tbs": gbs / 8000.0,
+                "routed_experts_per_layer_mean": statistics.mean(statistics.mean(u) for u in unions),
+                "proposals": "seeded uniform over the vocabulary"}
+
+    # ---- the headline workload ----
+    mc, model, kv = load(args.config)
+    ctas, smem, threads = model.launch_info()
     B = args.batch
+    head, ms, per, clk, abytes = decode_run(mc, model, kv, B, args.steps, args.warmup, clocks=True)
     ms_step = ms / args.steps
-    value = world * B * args.steps / (ms / 1e3)
-    # roofline of the (only) kernel: algorithmic bytes / average launch time
-    mid_pos = [p + args.steps // 2 for p in positions]
-    abytes = step_bytes(mc, B, mid_pos, model.weight_bytes())
-    peak, peak_kind = measured_peaks()
+    value = head["tokens_per_s"]
     launch_ms = statistics.mean(per)
     achieved = abytes / (launch_ms / 1e3) / 1e9
 
-    by_batch = {}
+    by_batch = {str(B): head}
     for b in [int(x) for x in args.sweep.split(",") if x]:
-        if b == B:
-            by_batch[str(b)] = {"tokens_per_s": world * b / (ms_step / 1e3), "ms_per_step": ms_step,
-                                "hbm_gbs": achieved}
-            continue
-        kv.fill_random(synth.SEED_KV, mc.kv_sigma, mc.context)
-        msb, perb, _, posb = time_batch(b, max(8, args.steps // 4), 3)
-        stepb = msb / max(8, args.steps // 4)
-        bb = step_bytes(mc, b, [p + 4 for p in posb], model.weight_bytes())
-        by_batch[str(b)] = {"tokens_per_s": world * b / (stepb / 1e3), "ms_per_step": stepb,
-                            "hbm_gbs": bb / (statistics.mean(perb) / 1e3) / 1e9}
+        if b != B:
+            by_batch[str(b)] = decode_run(mc, model, kv, b, max(8, args.steps // 4), 3)[0]
 
     # ---- end to end through the public API with host buffers ----
     kv.fill_random(synth.SEED_KV, mc.kv_sigma, mc.context)
@@ -224,6 +341,21 @@ def run_ours(args, rank, world, local_rank):
            "d2h_bytes_per_step": B * 4}
     kv.close()
     model.close()
+
+    # ---- the other workloads of the study (one GPU each, rank-local) ----
+    workloads = {}
+    extra_steps = max(8, args.steps // 4)
+    for name in [w for w in args.workloads.split(",") if w]:
+        if name == "verify":
+            wmc, wm, wkv = load("moe")
+            workloads["verify_moe"] = verify_run(wmc, wm, wkv, args.verify_steps, 4)
+        else:
+            wmc, wm, wkv = load(name)
+            batches = (1, 2, 4, 8) if name == "moe" else (1, 8)
+            workloads[name] = {str(b): decode_run(wmc, wm, wkv, b, extra_steps, 3)[0] for b in batches}
+        wkv.close()
+        wm.close()
+
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -232,9 +364,10 @@ def run_ours(args, rank, world, local_rank):
                    "model": args.config, "global_batch": B * world, "seq_len": mc.context, "parallelism": f"dp{world}",
                    "l2": "inputs larger than L2 (44 GB weights), no flush"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_kind": peak_kind, "traffic": None,
+                     "peak_kind": peak_kind, "traffic": args.traffic,
                      "frac_of_8tbs": achieved / 8000.0, "algorithmic_bytes_per_launch": abytes},
         "by_batch": by_batch,
+        "workloads": workloads,
         "e2e": e2e,
         "gpu_launches": args.steps,
         "launch": {"ctas": ctas, "threads": threads, "smem_bytes": smem},

@@ -19,6 +19,7 @@
 #include "mk_internal.h"
 
 namespace mk {
+template <bool MLA>
 __global__ void mk_step_kernel(const __grid_constant__ Launch P);
 }
 
@@ -227,6 +228,7 @@ struct mk_handle {
   int32_t* am_idx = nullptr;
   float* att_part = nullptr;
   int att_rows_max = 0;
+  int att_dpart = 0;  // values per attention partial row (head_dim, or kv_lora_rank for latent attention)
   int n_items_max = 0;
   int max_pairs = 0;
   uint32_t* ctr = nullptr;
@@ -244,6 +246,7 @@ struct mk_handle {
   bool sticky = false;
   bool initialised = false;
   uint64_t noalloc_id = 0;  // identity of this handle for mk_decode_step_noalloc's installed task list
+  const void* kernel = nullptr;  // the step kernel instance of this model's attention family
   std::string err;
 };
 
@@ -322,10 +325,23 @@ static bool desc_ok(const mk_model_desc* d, std::string& why) {
   if (d->vocab < 2) { why = "vocab < 2"; return false; }
   if (d->max_batch < 1 || d->max_batch > MAXM) { why = "max_batch must be in [1, 8]"; return false; }
   if (d->max_ctx < 2) { why = "max_ctx < 2"; return false; }
-  if (d->kv_lora_rank > 0) { why = "latent attention is not supported by this build"; return false; }
-  if (d->head_dim != 64 && d->head_dim != 128) { why = "head_dim must be 64 or 128"; return false; }
-  if (d->n_kv_heads < 1 || d->n_q_heads % d->n_kv_heads) { why = "n_q_heads must be a multiple of n_kv_heads"; return false; }
-  if ((d->n_q_heads / d->n_kv_heads) * MAXM > 48) { why = "query heads per kv head must be <= 6"; return false; }
+  if (d->kv_lora_rank > 0) {
+    // latent attention: one item holds all heads of one query row (<= 2 m-tiles), the latent
+    // rows [c | k_rope] are moved as whole rows (16-byte multiples), each consumer warp owns
+    // kv_lora_rank / 8 latent dims (whole 8-dim tiles, at most 8 of them)
+    if (d->n_q_heads < 1 || d->n_q_heads > 32) { why = "latent attention needs 1 <= n_q_heads <= 32"; return false; }
+    if (d->kv_lora_rank % 64 || d->kv_lora_rank > 512) { why = "kv_lora_rank must be a multiple of 64, <= 512"; return false; }
+    if (d->rope_dim < 16 || d->rope_dim % 16) { why = "rope_dim must be a positive multiple of 16"; return false; }
+    if (d->head_dim < 16 || d->head_dim % 16) { why = "head_dim must be a positive multiple of 16"; return false; }
+    if (mla_smem_need(d->n_q_heads, d->kv_lora_rank, d->rope_dim) > MLA_SCRATCH_BYTES) {
+      why = "latent attention shapes exceed the shared-memory scratch";
+      return false;
+    }
+  } else {
+    if (d->head_dim != 64 && d->head_dim != 128) { why = "head_dim must be 64 or 128"; return false; }
+    if (d->n_kv_heads < 1 || d->n_q_heads % d->n_kv_heads) { why = "n_q_heads must be a multiple of n_kv_heads"; return false; }
+    if ((d->n_q_heads / d->n_kv_heads) * MAXM > 48) { why = "query heads per kv head must be <= 6"; return false; }
+  }
   if (d->n_routed == 0) {
     if (d->ffn < 8 || d->ffn % 8) { why = "ffn must be a positive multiple of 8"; return false; }
   } else {
@@ -366,6 +382,8 @@ mk_status mk_create(const mk_model_desc* desc, int device, mk_handle** out) {
     h->ncta = prop.multiProcessorCount;
     const mk_model_desc& d = *desc;
     const int L = d.layers, H = d.hidden, Hq = d.n_q_heads, G = d.n_kv_heads, hd = d.head_dim;
+    const bool mla = d.kv_lora_rank > 0;
+    const int R = d.kv_lora_rank, dr = d.rope_dim;
     // ---- weights ----
     TRY(dalloc(h, (void**)&h->embed, (size_t)d.vocab * H * 2));
     TRY(dalloc(h, (void**)&h->final_norm, (size_t)H * 2));
@@ -381,11 +399,38 @@ mk_status mk_create(const mk_model_desc* desc, int device, mk_handle** out) {
       ly.attn_norm = h->attn_norm[l];
       ly.ffn_norm = h->ffn_norm[l];
       MatMap mp{};
-      mp.layer = l;
-      mp.type = MAP_PLAIN;
-      mp.kindA = SYN_WQKV;
-      mp.lcolsA = H;
-      TRY(add_mat(h, (Hq + 2 * G) * hd, H, 0, 0, mp, &ly.m_qkv));
+      ly.m_ukt = ly.m_uv = -1;
+      if (!mla) {
+        mp.layer = l;
+        mp.type = MAP_PLAIN;
+        mp.kindA = SYN_WQKV;
+        mp.lcolsA = H;
+        TRY(add_mat(h, (Hq + 2 * G) * hd, H, 0, 0, mp, &ly.m_qkv));
+      } else {
+        // queries [nope | rope] per head, then the latent c and the shared rope key
+        mp.layer = l;
+        mp.type = MAP_CONCAT;
+        mp.kindA = SYN_MLA_WQ;
+        mp.kindB = SYN_MLA_WDKV;
+        mp.rowsA = Hq * (hd + dr);
+        mp.lcolsA = mp.lcolsB = H;
+        TRY(add_mat(h, Hq * (hd + dr) + R + dr, H, 0, 0, mp, &ly.m_qkv));
+        // W_uk transposed per head: row h * R + c reads W_uk[h * dn + i][c] over i
+        mp = MatMap{};
+        mp.layer = l;
+        mp.type = MAP_UKT;
+        mp.kindA = SYN_MLA_WUK;
+        mp.lcolsA = R;
+        mp.Hq = Hq;
+        mp.dn = hd;
+        mp.R = R;
+        TRY(add_mat(h, Hq * R, hd, 0, 0, mp, &ly.m_ukt));
+        mp = MatMap{};
+        mp.layer = l;
+        mp.kindA = SYN_MLA_WUV;
+        mp.lcolsA = R;
+        TRY(add_mat(h, Hq * hd, R, 0, 0, mp, &ly.m_uv));
+      }
       mp = MatMap{};
       mp.layer = l;
       mp.kindA = SYN_WO;
@@ -448,11 +493,12 @@ mk_status mk_create(const mk_model_desc* desc, int device, mk_handle** out) {
     }
     // ---- RoPE table, double precision angles rounded to fp32 ----
     {
-      const int half = hd / 2;
+      const int rd = mla ? dr : hd;  // rotary dims
+      const int half = rd / 2;
       std::vector<float2> tab((size_t)d.max_ctx * half);
       for (int p = 0; p < d.max_ctx; ++p)
         for (int i = 0; i < half; ++i) {
-          const double inv = pow((double)d.rope_theta, -2.0 * i / (double)hd);
+          const double inv = pow((double)d.rope_theta, -2.0 * i / (double)rd);
           const double ang = (double)p * inv;
           tab[(size_t)p * half + i] = make_float2((float)cos(ang), (float)sin(ang));
         }
@@ -502,7 +548,9 @@ mk_status mk_create(const mk_model_desc* desc, int device, mk_handle** out) {
     // distinct routed experts one step can select
     const int hw = d.n_routed ? d.expert_ffn : d.ffn;
     const int hslots = d.n_routed ? d.n_shared + std::min(d.n_routed, MAXM * d.top_k) : 1;
-    const int widths[NBUF] = {H, (Hq + 2 * G) * hd, Hq * hd, std::max(hw, 8), std::max(d.n_routed, 4)};
+    const int qkv_w = mla ? Hq * (hd + dr) + R + dr : (Hq + 2 * G) * hd;
+    const int lat_w = mla ? Hq * R : 4;
+    const int widths[NBUF] = {H, qkv_w, Hq * hd, std::max(hw, 8), std::max(d.n_routed, 4), lat_w, lat_w};
     for (int b = 0; b < NBUF; ++b) {
       h->ld[b] = (widths[b] + 3) & ~3;
       const size_t rows = (b == B_H) ? (size_t)hslots * MB : (size_t)MB;
@@ -511,10 +559,13 @@ mk_status mk_create(const mk_model_desc* desc, int device, mk_handle** out) {
     TRY(dalloc(h, (void**)&h->ss_part, (size_t)2 * h->ncta * MAXM * sizeof(float)));
     TRY(dalloc(h, (void**)&h->am_val, (size_t)h->ncta * MAXM * sizeof(float)));
     TRY(dalloc(h, (void**)&h->am_idx, (size_t)h->ncta * MAXM * sizeof(int32_t)));
-    h->max_pairs = d.max_batch * G;
+    // attention pairs: (sequence, kv head) for GQA, one query row for latent attention
+    h->max_pairs = mla ? d.max_batch : d.max_batch * G;
     h->n_items_max = std::max(h->ncta, h->max_pairs);
-    h->att_rows_max = MAXM * (Hq / G);
-    TRY(dalloc(h, (void**)&h->att_part, (size_t)h->n_items_max * h->att_rows_max * (hd + 2) * sizeof(float)));
+    h->att_rows_max = mla ? Hq : MAXM * (Hq / G);
+    h->att_dpart = mla ? R : hd;
+    TRY(dalloc(h, (void**)&h->att_part,
+               (size_t)h->n_items_max * h->att_rows_max * (h->att_dpart + 2) * sizeof(float)));
     h->n_ctr = (L + 1) * NCTR_LAYER + L * h->max_pairs + 2;
     TRY(dalloc(h, (void**)&h->ctr, (size_t)h->n_ctr * sizeof(uint32_t)));
     TRY(dalloc(h, (void**)&h->status, 4 * sizeof(int32_t)));
@@ -524,13 +575,14 @@ mk_status mk_create(const mk_model_desc* desc, int device, mk_handle** out) {
       s = MK_ERR_CUDA;
       goto fail_out;
     }
-    if (cudaFuncSetAttribute(mk_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess) {
+    h->kernel = d.kv_lora_rank > 0 ? (const void*)mk_step_kernel<true> : (const void*)mk_step_kernel<false>;
+    if (cudaFuncSetAttribute(h->kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess) {
       s = MK_ERR_CUDA;
       h->err = "cannot reserve dynamic shared memory";
       goto fail_out;
     }
     int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, mk_step_kernel, NTHREADS, SMEM_BYTES) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, h->kernel, NTHREADS, SMEM_BYTES) != cudaSuccess ||
         occ < 1) {
       s = MK_ERR_CUDA;
       h->err = "kernel does not fit one CTA per SM";
@@ -675,6 +727,10 @@ mk_status mk_load_weights(mk_handle* h, const mk_tensor_src* ts, int n) {
     int64_t lrows = mh.m.rows, lcols = mh.m.cols;
     if (mh.map.type == MAP_GU) lrows = mh.m.rows / 2;
     if (mh.map.type == MAP_CONCAT) lrows = which ? mh.m.rows - mh.map.rowsA : mh.map.rowsA;
+    if (mh.map.type == MAP_UKT) {  // the source is W_uk [Hq dn, R]; the tiles hold its per-head transpose
+      lrows = (int64_t)mh.map.Hq * mh.map.dn;
+      lcols = mh.map.R;
+    }
     if (t.rows != lrows || t.cols != lcols)
       return fail(h, MK_ERR_INVALID, "tensor " + std::to_string(i) + ": shape mismatch");
     const size_t eb = mh.m.fp8 ? 1 : 2;
@@ -719,6 +775,20 @@ mk_status mk_kv_create(mk_handle* h, int max_seqs, int max_ctx, mk_kv** out) {
   kv->h = h;
   kv->max_seqs = max_seqs;
   kv->max_ctx = max_ctx;
+  if (d.kv_lora_rank > 0) {
+    // latent rows [c | k_rope] per (layer, sequence, position); no separate values
+    const size_t n = (size_t)d.layers * max_seqs * max_ctx * (d.kv_lora_rank + d.rope_dim);
+    if (cudaMalloc(&kv->k, n * 2) != cudaSuccess) {
+      cudaGetLastError();
+      delete kv;
+      return fail(h, MK_ERR_OOM, "kv cache allocation failed");
+    }
+    kv->bytes = (int64_t)n * 2;
+    cudaMemset(kv->k, 0, n * 2);
+    CK(cudaDeviceSynchronize());
+    *out = kv;
+    return MK_OK;
+  }
   const size_t n = (size_t)d.layers * max_seqs * d.n_kv_heads * max_ctx * d.head_dim;
   if (cudaMalloc(&kv->k, n * 2) != cudaSuccess || cudaMalloc(&kv->v, n * 2) != cudaSuccess) {
     cudaGetLastError();
@@ -755,6 +825,14 @@ mk_status mk_kv_fill_random(mk_kv* kv, uint64_t seed, float sigma, int32_t lengt
   const mk_model_desc& d = h->desc;
   const int blocks = 148 * 16;
   const float sc = syn_normal_scale(sigma);
+  if (d.kv_lora_rank > 0) {
+    // latent rows: element i of (sequence s, position t) has index (s << 32) + t * W + i
+    fill_kv_kernel<<<blocks, 256>>>(kv->k, d.layers, kv->max_seqs, 1, kv->max_ctx, d.kv_lora_rank + d.rope_dim,
+                                    length, seed, SYN_KV_LAT, sc);
+    CK(cudaGetLastError());
+    CK(cudaDeviceSynchronize());
+    return MK_OK;
+  }
   fill_kv_kernel<<<blocks, 256>>>(kv->k, d.layers, kv->max_seqs, d.n_kv_heads, kv->max_ctx, d.head_dim, length, seed,
                                   SYN_KV_K, sc);
   fill_kv_kernel<<<blocks, 256>>>(kv->v, d.layers, kv->max_seqs, d.n_kv_heads, kv->max_ctx, d.head_dim, length, seed,
@@ -768,6 +846,10 @@ mk_status mk_kv_copy_out(mk_kv* kv, void* dst) {
   if (!kv || !dst) return MK_ERR_INVALID;
   mk_handle* h = kv->h;
   cudaSetDevice(h->device);
+  if (!kv->v) {  // latent cache: one array
+    CK(cudaMemcpy(dst, kv->k, (size_t)kv->bytes, cudaMemcpyDeviceToDevice));
+    return MK_OK;
+  }
   const size_t half = (size_t)kv->bytes / 2;
   CK(cudaMemcpy(dst, kv->k, half, cudaMemcpyDeviceToDevice));
   CK(cudaMemcpy(reinterpret_cast<uint8_t*>(dst) + half, kv->v, half, cudaMemcpyDeviceToDevice));
@@ -818,7 +900,8 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
   (void)Q;
   const mk_model_desc& d = h->desc;
   const int ncta = h->ncta, L = d.layers;
-  const int n_pairs = S * d.n_kv_heads;
+  const bool mla = d.kv_lora_rank > 0;
+  const int n_pairs = mla ? S * Q : S * d.n_kv_heads;
   const int n_items = std::max(n_pairs, ncta);
   auto C = [&](int l, int slot) { return l * NCTR_LAYER + slot; };
   std::vector<std::vector<Task>> per(ncta);
@@ -837,8 +920,66 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
   }
   for (int l = 0; l < L; ++l) {
     const Layer& ly = h->layers[l];
+    if (mla) {
+      // latent attention: [q | c | k_rope] = W h, absorbed queries per head,
+      // attention over the latent rows, per-head value up-projection, W_o
+      const int hd = d.head_dim, dr = d.rope_dim, R = d.kv_lora_rank;
+      auto rr = split_rows(h->mats[ly.m_qkv].m.RT, ncta, rot);
+      for (int c = 0; c < ncta; ++c) {
+        Task t = gemv(l, ly.m_qkv, rr[c].first, rr[c].second, IN_X_NORM, 0, EPI_STORE, B_QKV, 0,
+                      l == 0 ? C(L, C_QKV) : C(l - 1, C_DOWN), ncta, C(l, C_QKV));
+        t.ss_src = 1;
+        per[c].push_back(t);
+      }
+      rr = split_rows(h->mats[ly.m_ukt].m.RT, ncta, rot);
+      for (int c = 0; c < ncta; ++c) {
+        // head g's rows read q_nope of head g: columns g * (dn + dr) of the QKV output
+        Task t = gemv(l, ly.m_ukt, rr[c].first, rr[c].second, IN_BUF, B_QKV, EPI_STORE, B_QL, 0, C(l, C_QKV), ncta,
+                      C(l, C_UKT));
+        t.xg_rt = (int16_t)(R / 16);
+        t.xg_stride = hd + dr;
+        per[c].push_back(t);
+      }
+      for (int i = 0; i < n_items; ++i) {
+        // every item writes its partial (M, L, O) and counts itself done
+        Task t{};
+        t.type = T_MLA;
+        t.layer = (int16_t)l;
+        t.rt0 = i;
+        t.wait_ctr = C(l, C_UKT);
+        t.wait_tgt = ncta;
+        t.sig_ctr = C(l, C_ATTN);
+        per[i % ncta].push_back(t);
+      }
+      for (int c = 0; c < ncta; ++c) {
+        // the split combine, a slice per CTA
+        Task t{};
+        t.type = T_MLA_COMB;
+        t.layer = (int16_t)l;
+        t.wait_ctr = C(l, C_ATTN);
+        t.wait_tgt = n_items;
+        t.sig_ctr = C(l, C_COMB);
+        per[c].push_back(t);
+      }
+      rr = split_rows(h->mats[ly.m_uv].m.RT, ncta, rot);
+      for (int c = 0; c < ncta; ++c) {
+        // head g's rows read the attention output of head g: columns g * R
+        Task t = gemv(l, ly.m_uv, rr[c].first, rr[c].second, IN_BUF, B_OL, EPI_STORE, B_ATTN, 0, C(l, C_COMB),
+                      ncta, C(l, C_UV));
+        t.xg_rt = (int16_t)(hd / 16);
+        t.xg_stride = R;
+        per[c].push_back(t);
+      }
+      rr = split_rows(h->mats[ly.m_o].m.RT, ncta, rot);
+      for (int c = 0; c < ncta; ++c) {
+        Task t = gemv(l, ly.m_o, rr[c].first, rr[c].second, IN_BUF, B_ATTN, EPI_RESID, 0, 0, C(l, C_UV), ncta,
+                      C(l, C_O));
+        t.ss_dst = 0;
+        per[c].push_back(t);
+      }
+    }
     // QKV projection (layer 0 reads the embedding rows directly)
-    {
+    if (!mla) {
       auto rr = split_rows(h->mats[ly.m_qkv].m.RT, ncta, rot);
       for (int c = 0; c < ncta; ++c) {
         Task t = gemv(l, ly.m_qkv, rr[c].first, rr[c].second, IN_X_NORM, 0, EPI_STORE, B_QKV, 0,
@@ -848,7 +989,7 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
       }
     }
     // attention items
-    for (int i = 0; i < n_items; ++i) {
+    for (int i = 0; i < (mla ? 0 : n_items); ++i) {
       Task t{};
       t.type = T_ATTN;
       t.layer = (int16_t)l;
@@ -859,7 +1000,7 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
       per[i % ncta].push_back(t);
     }
     // output projection + residual
-    {
+    if (!mla) {
       auto rr = split_rows(h->mats[ly.m_o].m.RT, ncta, rot);
       for (int c = 0; c < ncta; ++c) {
         Task t = gemv(l, ly.m_o, rr[c].first, rr[c].second, IN_BUF, B_ATTN, EPI_RESID, 0, 0, C(l, C_ATTN), n_pairs,
@@ -1035,7 +1176,7 @@ static mk_status launch_step(mk_handle* h, mk_kv* kv, int S, int Q, const int32_
   P.trace_cap = h->task_trace_cap;
   h->stall_ns = 0;
   void* args[] = {&P};
-  cudaError_t e = cudaLaunchCooperativeKernel((const void*)mk_step_kernel, dim3(h->ncta), dim3(NTHREADS), args,
+  cudaError_t e = cudaLaunchCooperativeKernel(h->kernel, dim3(h->ncta), dim3(NTHREADS), args,
                                               SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(h, MK_ERR_CUDA, std::string("launch: ") + cudaGetErrorString(e));
   return MK_OK;
@@ -1197,7 +1338,7 @@ extern "C" mk_status mk_decode_step_noalloc(mk_handle* h, const int32_t* tokens,
   const size_t o_ami = at;
   at = align256(at + (size_t)h->ncta * MAXM * sizeof(int32_t));
   const size_t o_att = at;
-  at = align256(at + (size_t)n_items * h->att_rows_max * (d.head_dim + 2) * sizeof(float));
+  at = align256(at + (size_t)n_items * h->att_rows_max * (h->att_dpart + 2) * sizeof(float));
   const size_t o_ctr = at;
   at = align256(at + (size_t)h->n_ctr * sizeof(uint32_t));
   if (at > (size_t)MK_NOALLOC_SCRATCH_BYTES)
@@ -1265,7 +1406,7 @@ extern "C" mk_status mk_decode_step_noalloc(mk_handle* h, const int32_t* tokens,
   P.trace = h->task_trace;
   P.trace_cap = h->task_trace_cap;
   void* args[] = {&P};
-  const cudaError_t e = cudaLaunchCooperativeKernel((const void*)mk_step_kernel, dim3(h->ncta), dim3(NTHREADS), args,
+  const cudaError_t e = cudaLaunchCooperativeKernel(h->kernel, dim3(h->ncta), dim3(NTHREADS), args,
                                                     SMEM_BYTES, st);
   if (e != cudaSuccess) return fail(h, MK_ERR_CUDA, std::string("launch: ") + cudaGetErrorString(e));
   return MK_OK;

@@ -38,6 +38,42 @@ constexpr int TRACE_FIELDS = 20;             // int64 per traced task
 constexpr int TILE_BF16 = 512;               // 16x16 bf16 tile in A-fragment order
 constexpr int TILE_FP8 = 256;                // 16x16 e4m3 tile in A-fragment order
 
+// Latent attention (MLA) items use the activation ring, the attention scratch
+// and the new-KV rows as one contiguous shared-memory region: while a CTA runs
+// a latent-attention item its activation producer is parked on the next
+// task's dependency (the per-head value projection, which waits for every
+// attention item of the layer), so the activation ring is idle.
+constexpr int MLA_SCRATCH_BYTES = XSLOTS * XSLOT_BYTES + ATT_BYTES + NEWKV_BYTES;
+
+// One latent cache row [c (R) | k_rope (dr)] bf16 in shared memory, padded by
+// 16 bytes so that the 8 rows of an mma fragment load hit distinct banks.
+__host__ __device__ inline int mla_pitch(int R, int dr) { return (R + dr) * 2 + 16; }
+// Cache positions per streamed chunk (one ring stage, a multiple of 8, <= 64).
+__host__ __device__ inline int mla_ct(int R, int dr) {
+  int n = STAGE_BYTES / mla_pitch(R, dr);
+  n = n > 64 ? 64 : n;
+  return n & ~7;
+}
+// Byte offsets inside the latent-attention scratch: query A fragments (hi, lo
+// bf16 parts), probability A fragments for <= 64 positions (hi, lo), per-warp
+// row maxima (two parities), the step's own new latent rows (<= MAXM).
+struct MlaLayout {
+  int qhi, qlo, phi, plo, smax, newr, total;
+};
+__host__ __device__ inline MlaLayout mla_layout(int Hq, int R, int dr) {
+  const int mt = (Hq + 15) / 16, KW = (R + dr) / 16;
+  MlaLayout L;
+  L.qhi = 0;
+  L.qlo = mt * KW * 512;
+  L.phi = 2 * mt * KW * 512;
+  L.plo = L.phi + mt * 4 * 512;
+  L.smax = L.plo + mt * 4 * 512;
+  L.newr = L.smax + 2 * NCW * 32 * 4;
+  L.total = L.newr + MAXM * mla_pitch(R, dr);
+  return L;
+}
+__host__ __device__ inline int mla_smem_need(int Hq, int R, int dr) { return mla_layout(Hq, R, dr).total; }
+
 // ---------------------------------------------------------------------------
 // tasks
 // ---------------------------------------------------------------------------
@@ -48,6 +84,8 @@ enum TaskType : int16_t {
   T_MOE_DOWN = 4,  // down projection, K = shared + selected experts' hidden units
   T_TOPK = 5,      // (unused placeholder)
   T_EMBED = 6,     // x[m][c0:c1) = embedding rows of the step's tokens (+ RMS partial sums)
+  T_MLA = 7,       // one split-KV latent-attention item (one query row, all heads)
+  T_MLA_COMB = 8,  // this CTA's slice of the latent-attention split combine
 };
 
 enum InKind : int16_t {
@@ -65,7 +103,10 @@ enum Epi : int16_t {
 };
 
 enum BufId : int16_t {
-  B_X = 0, B_QKV = 1, B_ATTN = 2, B_H = 3, B_RLOG = 4, NBUF = 5
+  B_X = 0, B_QKV = 1, B_ATTN = 2, B_H = 3, B_RLOG = 4,
+  B_QL = 5,  // latent attention: query heads absorbed into the latent space [M][Hq * R]
+  B_OL = 6,  // latent attention: attention-weighted latent rows per head [M][Hq * R]
+  NBUF = 7
 };
 
 struct Task {
@@ -73,6 +114,8 @@ struct Task {
   int16_t in_kind, epi;
   int16_t in_buf, out_buf;
   int16_t moe, gain;         // moe: 1 shared experts, 2 routed experts; gain: 0 attn, 1 ffn, 2 final
+  int16_t xg_rt, pad16;      // > 0: rows come in groups of xg_rt row tiles (one per head), each reading
+  int32_t xg_stride;         //      its own activation columns, xg_stride floats further per group
   int32_t mat;               // matrix table index
   int32_t rt0, rt1;          // row tiles (GEMV) / item index (ATTN)
   int32_t wait_ctr, wait_tgt;
@@ -102,6 +145,7 @@ struct Layer {
   const uint16_t* ffn_norm;
   int32_t m_qkv, m_o, m_gu, m_down;
   int32_t m_router, m_shgu, m_shdown, m_exgu, m_exdown;  // MoE (-1 when dense)
+  int32_t m_ukt, m_uv;       // latent attention: per-head W_uk^T [Hq R, dn] and W_uv [Hq dv, R] (-1 otherwise)
 };
 
 struct Model {
@@ -112,7 +156,7 @@ struct Model {
   const uint16_t* embed;     // [V][H] row-major bf16
   const uint16_t* final_norm;
   int32_t m_lm;
-  const float2* rope;        // [max_ctx][d/2] (cos, sin)
+  const float2* rope;        // [max_ctx][rotary dims / 2] (cos, sin)
   int32_t rope_ctx;
   const Layer* layers;
   const Mat* mats;
@@ -161,7 +205,13 @@ struct Launch {
 };
 
 // counter slots inside one layer
-enum CtrSlot { C_QKV = 0, C_ATTN = 1, C_O = 2, C_GU = 3, C_DOWN = 4, C_ROUTER = 5, C_STALL = 6, NCTR_LAYER = 8 };
+enum CtrSlot {
+  C_QKV = 0, C_ATTN = 1, C_O = 2, C_GU = 3, C_DOWN = 4, C_ROUTER = 5, C_STALL = 6,
+  C_UKT = 7,  // latent attention: absorbed queries written
+  C_UV = 8,   // latent attention: per-head value up-projection written
+  C_COMB = 9, // latent attention: splits combined
+  NCTR_LAYER = 10
+};
 
 enum DevErr { DERR_NONE = 0, DERR_TIMEOUT = 4, DERR_BOUNDS = 5 };
 

@@ -179,6 +179,7 @@ struct Misc {
   uint64_t xready[XSLOTS];  // ... and converted to mma fragments
   uint64_t xempty[XSLOTS];
   float scale[MAXM];
+  float xscale[XSLOTS][MAXM];  // RMSNorm scale of the rows of the window in each activation slot
   volatile int abort;
   int flag;
   int pad[2];
@@ -284,6 +285,9 @@ __device__ __forceinline__ const uint16_t* task_gain(const Model& md, const Task
 struct Item {
   int pair, j, ns, first;
 };
+__device__ __forceinline__ int pair_first_item(int pair, int n_pairs, int n_items) {
+  return n_pairs >= n_items ? pair : (int)(((int64_t)pair * n_items + n_pairs - 1) / n_pairs);
+}
 __device__ __forceinline__ Item decode_item(int item, int n_pairs, int n_items) {
   Item it;
   if (n_pairs >= n_items) {
@@ -449,6 +453,7 @@ struct PieceSrc {
   int lg0;    // first row tile inside the piece's matrix
   int xbuf;   // activation buffer
   int xrow0;  // first activation row in it (expert slot * MAXM for the MoE down projection)
+  int xcol0;  // first activation column (per-head groups of the latent-attention projections)
 };
 
 __device__ __forceinline__ PieceSrc piece_src(const Model& md, const Task& t, const Mat& m, const Mat& m2,
@@ -456,6 +461,7 @@ __device__ __forceinline__ PieceSrc piece_src(const Model& md, const Task& t, co
   PieceSrc r;
   r.lg0 = pc.g0;
   r.xrow0 = 0;
+  r.xcol0 = t.xg_rt > 0 ? (pc.g0 / t.xg_rt) * t.xg_stride : 0;
   r.xbuf = t.in_kind == IN_X_NORM ? (int)B_X : (int)t.in_buf;
   r.w = m.w;
   r.scales = m.scales;
@@ -482,7 +488,7 @@ __device__ __forceinline__ void task_rows(const Model& md, const Task& t, const 
                                           int& gsz, int& nseg) {
   rt0 = t.rt0;
   rt1 = t.rt1;
-  gsz = 0;
+  gsz = t.xg_rt > 0 ? t.xg_rt : 0;
   nseg = 1;
   if (t.type == T_MOE_GU) {
     gsz = m.RT;
@@ -574,7 +580,7 @@ __device__ bool warp_wait_counter(const Ctx& C, int idx, uint32_t target, int co
 
 // One unit of streamed data, in the order the consumers take it.
 struct Chunk {
-  int kind;  // 1: GEMV tiles, 2: attention K/V rows
+  int kind;  // 1: GEMV tiles, 2: attention K/V rows, 3: latent cache rows (kb, n rows of d values)
   const uint8_t* w;
   int KT, tb, g0, nr, c0, nc;
   const uint16_t* kb;
@@ -585,8 +591,9 @@ struct Chunk {
 // Walks a CTA's task list and yields its chunks in consumption order (the
 // enumeration the consumers use).  Routed-expert tasks first wait for the
 // router's counter: their tiles are the only ones that depend on activations.
+template <bool MLA>
 struct ChunkStream {
-  int ti, end, state;  // state 0: next task, 1: GEMV-like pieces, 2: attention
+  int ti, end, state;  // state 0: next task, 1: GEMV-like pieces, 2: attention, 3: latent attention
   Task t;
   Mat m, m2;
   Pieces pc;
@@ -625,7 +632,7 @@ struct ChunkStream {
         }
         return 1;
       }
-      if (state == 2) {
+      if (!MLA && state == 2) {
         if (t0 < b) {
           c.kind = 2;
           c.kb = kb + (size_t)t0 * d;
@@ -633,6 +640,17 @@ struct ChunkStream {
           c.n = min(ATT_CT, b - t0);
           c.d = d;
           t0 += ATT_CT;
+          return 1;
+        }
+        state = 0;
+      }
+      if (MLA && state == 3) {
+        if (t0 < b) {
+          c.kind = 3;
+          c.kb = kb + (size_t)t0 * d;
+          c.n = min(mla_ct(md.R, md.dr), b - t0);
+          c.d = d;
+          t0 += mla_ct(md.R, md.dr);
           return 1;
         }
         state = 0;
@@ -656,7 +674,7 @@ struct ChunkStream {
           ci.init(src.lg0, src.lg0 + pc.nr, m.KT, tb, 0, xcap);
           state = 1;
         }
-      } else if (t.type == T_ATTN) {
+      } else if (!MLA && t.type == T_ATTN) {
         const Item itm = decode_item(t.rt0, P.n_pairs, P.n_items);
         const int s = itm.pair / md.Hkv, g = itm.pair % md.Hkv;
         const int T0 = seq_pos0(P, s);
@@ -667,11 +685,22 @@ struct ChunkStream {
         kb = P.kv_k + head * d;
         vb = P.kv_v + head * d;
         state = 2;
+      } else if (MLA && t.type == T_MLA) {
+        // cached positions [0, T0) of the query row's sequence, split like GQA
+        const Item itm = decode_item(t.rt0, P.n_pairs, P.n_items);
+        const int s = itm.pair / P.Q;
+        const int T0 = seq_pos0(P, s);
+        t0 = (int)(((int64_t)itm.j * T0) / itm.ns);
+        b = (int)(((int64_t)(itm.j + 1) * T0) / itm.ns);
+        d = md.R + md.dr;
+        kb = P.kv_k + ((size_t)t.layer * P.kv_seqs + s) * (size_t)P.kv_ctx * d;
+        state = 3;
       }
     }
   }
 };
 
+template <bool MLA>
 __device__ void producer(const Ctx& C) {
   const Launch& P = *C.P;
   const int lane = threadIdx.x & 31;
@@ -681,7 +710,7 @@ __device__ void producer(const Ctx& C) {
   long long blocked = 0;
   const uint64_t t_first = globaltimer();
   const long long c_first = clock64();
-  ChunkStream is;
+  ChunkStream<MLA> is;
   is.init(beg, end);
   Chunk c;
   while (is.next(C, c) > 0) {
@@ -694,6 +723,12 @@ __device__ void producer(const Ctx& C) {
         const uint8_t* srcp = c.w + ((size_t)(c.g0 + lane) * c.KT + c.c0) * c.tb;
         bulk_g2s(dst + (size_t)lane * c.nc * c.tb, srcp, (uint32_t)(c.nc * c.tb), bar, pol);
       }
+    } else if (MLA) {
+      // latent rows, one copy each into padded shared-memory rows
+      const int pitch = c.d * 2 + 16;
+      const uint32_t rb = (uint32_t)(c.d * 2);
+      if (!prod_reserve(C, it, rb * (uint32_t)c.n, blocked)) goto drain;
+      for (int r = lane; r < c.n; r += 32) bulk_g2s(dst + (size_t)r * pitch, c.kb + (size_t)r * c.d, rb, bar, pol);
     } else {
       // the cache rows of this chunk are contiguous: one copy for K, one for V
       const int pitch = att_pitch(c.d);
@@ -741,7 +776,66 @@ drain:
 // dependency (acquire), then streams the activation slice of every chunk
 // (M rows x the chunk's columns) into the x ring with bulk copies, so the
 // consumers never wait on a global-memory round trip inside a task.
-__device__ bool xprod_reserve(const Ctx& C, uint32_t ix, uint32_t bytes) {
+// Convert an activation window in place into ready mma B fragments: col tile
+// jj of row m (16 fp32, 64 B) becomes, for each quad lane tq, 16 B =
+// {hi(k 2tq,2tq+1), hi(k 2tq+8,2tq+9), lo(..), lo(..)} of x * rms_scale * gain
+// (bf16 split; f16 for fp8 weights).  Threads t0, t0 + nt, ... share the work.
+__device__ __forceinline__ void convert_window(uint8_t* dst, int rb, int M, int wn, int w0, bool has_gain,
+                                               const uint16_t* gain, const float* scale, bool f16, int t0, int nt) {
+  for (int e = t0; e < M * wn; e += nt) {
+    const int mm = e / wn, jj = e - mm * wn;
+    float4* p4 = reinterpret_cast<float4*>(dst + (size_t)mm * rb + (size_t)jj * 64);
+    float v[16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 f = p4[q];
+      v[4 * q] = f.x;
+      v[4 * q + 1] = f.y;
+      v[4 * q + 2] = f.z;
+      v[4 * q + 3] = f.w;
+    }
+    if (has_gain) {
+      const float sc = scale[mm];
+      const uint4* gp = reinterpret_cast<const uint4*>(gain + (size_t)(w0 + jj) * 16);
+      const uint4 ga = __ldg(gp), gb = __ldg(gp + 1);
+      const uint32_t gw[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        v[2 * q] = v[2 * q] * sc * bf16lo(gw[q]);
+        v[2 * q + 1] = v[2 * q + 1] * sc * bf16hi(gw[q]);
+      }
+    }
+    uint4 o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (!f16) {
+        split_bf16(v[2 * q], v[2 * q + 1], o[q].x, o[q].z);
+        split_bf16(v[2 * q + 8], v[2 * q + 9], o[q].y, o[q].w);
+      } else {
+        split_f16(v[2 * q], v[2 * q + 1], o[q].x, o[q].z);
+        split_f16(v[2 * q + 8], v[2 * q + 9], o[q].y, o[q].w);
+      }
+    }
+    uint4* o4 = reinterpret_cast<uint4*>(p4);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) o4[q] = o[q];
+  }
+  // the slot is written again by bulk copies (async proxy) once released
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Out of line for the consumers: keeps the GEMV inner loops small (one CTA
+// runs every phase of the step, so their instruction footprint matters).
+__device__ __noinline__ void convert_window_coop(uint8_t* dst, int rb, int M, int wn, int w0, bool has_gain,
+                                                 const uint16_t* gain, const float* scale, bool f16) {
+  convert_window(dst, rb, M, wn, w0, has_gain, gain, scale, f16, threadIdx.x, NCT);
+}
+
+// Windows of more than XCONV_M rows are converted by all consumer warps
+// together (a single warp would fall behind the tensor cores at M = 8).
+constexpr int XCONV_M = 0;
+
+__device__ bool xprod_reserve(const Ctx& C, uint32_t ix, uint32_t bytes, const float* scale) {
   const int lane = threadIdx.x & 31;
   int ok = 1;
   if (lane == 0) {
@@ -765,7 +859,11 @@ __device__ bool xprod_reserve(const Ctx& C, uint32_t ix, uint32_t bytes) {
         }
       }
     }
-    if (ok) mbar_arrive_expect_tx(&C.ms->xfull[s], bytes);
+    if (ok) {
+#pragma unroll
+      for (int q = 0; q < MAXM; ++q) C.ms->xscale[s][q] = scale[q];
+      mbar_arrive_expect_tx(&C.ms->xfull[s], bytes);  // release: the scales are visible with the phase
+    }
   }
   ok = __shfl_sync(0xffffffffu, ok, 0);
   return ok != 0;
@@ -820,17 +918,20 @@ __device__ void xproducer(const Ctx& C) {
         const int wn = ci.wn(), w0 = ci.w0();
         const uint32_t rowdata = (uint32_t)(wn * 64);
         const int sl = ix % XSLOTS;
-        if (!xprod_reserve(C, ix, (uint32_t)M * rowdata)) goto drain;
+        if (!xprod_reserve(C, ix, (uint32_t)M * rowdata, scale)) goto drain;
+        __syncwarp();
         uint8_t* dst = C.xring + (size_t)sl * XSLOT_BYTES;
         if (lane < M) {
           const uint8_t* xsrc = reinterpret_cast<const uint8_t*>(
-              P.buf[src.xbuf] + (size_t)(src.xrow0 + lane) * P.ld[src.xbuf] + ci.c0 * 16);
+              P.buf[src.xbuf] + (size_t)(src.xrow0 + lane) * P.ld[src.xbuf] + src.xcol0 + ci.c0 * 16);
           bulk_g2s(dst + (size_t)lane * rb, xsrc, rowdata, &C.ms->xfull[sl], pol);
         }
-        // wait for this warp's own copy, then convert the window in place into
-        // ready mma B fragments: col tile jj of row m (16 fp32, 64 B) becomes,
-        // for each quad lane tq, 16 B = {hi(k 2tq,2tq+1), hi(k 2tq+8,2tq+9),
-        // lo(..), lo(..)} of x * rms_scale * gain (bf16 split; f16 for fp8 weights)
+        if (M > XCONV_M) {
+          // the consumers convert this window themselves
+          ++ix;
+          continue;
+        }
+        // wait for this warp's own copy, then convert the window in place
         {
           const uint32_t par = (ix / XSLOTS) & 1;
           const uint64_t t0 = globaltimer();
@@ -843,47 +944,7 @@ __device__ void xproducer(const Ctx& C) {
             goto drain;
           }
         }
-        for (int e = lane; e < M * wn; e += 32) {
-          const int mm = e / wn, jj = e - mm * wn;
-          float4* p4 = reinterpret_cast<float4*>(dst + (size_t)mm * rb + (size_t)jj * 64);
-          float v[16];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float4 f = p4[q];
-            v[4 * q] = f.x;
-            v[4 * q + 1] = f.y;
-            v[4 * q + 2] = f.z;
-            v[4 * q + 3] = f.w;
-          }
-          if (has_gain) {
-            float sc = 1.f;
-#pragma unroll
-            for (int q = 0; q < MAXM; ++q)
-              if (q == mm) sc = scale[q];
-            const uint4* gp = reinterpret_cast<const uint4*>(gain + (size_t)(w0 + jj) * 16);
-            const uint4 ga = __ldg(gp), gb = __ldg(gp + 1);
-            const uint32_t gw[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              v[2 * q] = v[2 * q] * sc * bf16lo(gw[q]);
-              v[2 * q + 1] = v[2 * q + 1] * sc * bf16hi(gw[q]);
-            }
-          }
-          uint4 o[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if (!m.fp8) {
-              split_bf16(v[2 * q], v[2 * q + 1], o[q].x, o[q].z);
-              split_bf16(v[2 * q + 8], v[2 * q + 9], o[q].y, o[q].w);
-            } else {
-              split_f16(v[2 * q], v[2 * q + 1], o[q].x, o[q].z);
-              split_f16(v[2 * q + 8], v[2 * q + 9], o[q].y, o[q].w);
-            }
-          }
-          uint4* o4 = reinterpret_cast<uint4*>(p4);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) o4[q] = o[q];
-        }
+        convert_window(dst, rb, M, wn, w0, has_gain, gain, C.ms->xscale[sl], m.fp8 != 0, lane, 32);
         __syncwarp();
         if (lane == 0) mbar_arrive(&C.ms->xready[sl]);
         ++ix;
@@ -993,29 +1054,32 @@ __device__ __forceinline__ void signal_counter(const Ctx& C, int idx) {
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
 
-__device__ __forceinline__ void wait_x(const Ctx& C, uint32_t ix) {
+// Wait for activation slot `ix`: converted by the activation producer
+// (`landed` false), or only landed, for the consumers to convert (true).
+__device__ __forceinline__ void wait_x(const Ctx& C, uint32_t ix, bool landed = false) {
   const int s = ix % XSLOTS;
   const uint32_t par = (ix / XSLOTS) & 1;
+  uint64_t* bar = landed ? &C.ms->xfull[s] : &C.ms->xready[s];
   const bool tr = C.P->trace && threadIdx.x == 0;
   const long long c0 = tr ? clock64() : 0;
   if ((threadIdx.x & 31) == 0) {
     uint32_t spins = 0;
     uint64_t t0 = 0;
-    while (!mbar_try_wait(&C.ms->xready[s], par)) {
+    while (!mbar_try_wait(bar, par)) {
       if (++spins >= 64) {
         spins = 0;
         if (C.ms->abort) break;
         uint64_t now = globaltimer();
         if (t0 == 0) t0 = now;
         else if (now - t0 > (uint64_t)C.P->timeout_ns * 2) {
-          raise_error(*C.P, C.ms, DERR_TIMEOUT, 0x50000 | s);
+          raise_error(*C.P, C.ms, DERR_TIMEOUT, (landed ? 0x58000 : 0x50000) | s);
           break;
         }
       }
     }
   }
   __syncwarp();
-  if (!C.ms->abort) while (!mbar_try_wait(&C.ms->xready[s], par)) {}
+  if (!C.ms->abort) while (!mbar_try_wait(bar, par)) {}
   if (tr) C.ms->tr_wx += clock64() - c0;
 }
 
@@ -1023,6 +1087,8 @@ __device__ __forceinline__ void wait_x(const Ctx& C, uint32_t ix) {
 struct GemvLane {
   int warp, lane, g, tq, M, rowbytes;
   bool has_gain, trc;
+  bool coop;              // the consumers convert the activation windows (M > XCONV_M)
+  const uint16_t* gain;   // norm gain of the task's input
 };
 
 // All chunks of one row group [g0, g0 + NR): each warp takes col tiles
@@ -1046,7 +1112,18 @@ __device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
   long long tc0 = 0, tl0 = L.trc ? clock64() : 0;
   while (true) {
     const uint8_t* slot = C.xring + (size_t)(ix % XSLOTS) * XSLOT_BYTES;
-    if (ci.win_first()) wait_x(C, ix);  // the window arrives converted
+    if (ci.win_first()) {
+      if (!L.coop) {
+        wait_x(C, ix);  // the window arrives converted
+      } else {
+        wait_x(C, ix, true);
+        const long long tv0 = L.trc ? clock64() : 0;
+        convert_window_coop(const_cast<uint8_t*>(slot), L.rowbytes, L.M, ci.wn(), ci.w0(), L.has_gain, L.gain,
+                            C.ms->xscale[ix % XSLOTS], FP8);
+        bar_consumers();
+        if (L.trc) C.ms->tr_frag += clock64() - tv0;
+      }
+    }
     wait_full(C, it);
     const uint8_t* stage = C.ring + (size_t)(it % NSTAGE) * STAGE_BYTES;
     const uint8_t* xs = slot + (size_t)g * L.rowbytes + (size_t)(ci.c0 - ci.w0()) * 64 + tq * 16;
@@ -1171,6 +1248,8 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
   L.has_gain = has_gain;
   L.rowbytes = 0;
   L.trc = P.trace && tid == 0;
+  L.coop = M > XCONV_M;
+  L.gain = task_gain(md, t);
   if (L.trc) C.ms->tr_pre += clock64() - tpre;
   while (have) {
     const PieceSrc src = piece_src(md, t, m, m2, C.ms->rt_ex[RR_CONS], pc);
@@ -1576,11 +1655,13 @@ __device__ void att_chunk(const Ctx& C, AttState& st, const uint8_t* Ks, const u
   }
 }
 
-__device__ void attn_task(const Ctx& C, const Task t, uint32_t& it) {
+__device__ __noinline__ void attn_task(const Ctx& C, const Task t, uint32_t& it) {
   const Launch& P = *C.P;
   const Model& md = *C.md;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, tq = lane & 3;
+  const bool trc = P.trace && threadIdx.x == 0;
+  long long tA = trc ? clock64() : 0;
   const Item itm = decode_item(t.rt0, P.n_pairs, P.n_items);
   const int s = itm.pair / md.Hkv, kvh = itm.pair % md.Hkv;
   const int d = md.d, pitch = att_pitch(d), KTq = d / 16;
@@ -1650,6 +1731,11 @@ __device__ void attn_task(const Ctx& C, const Task t, uint32_t& it) {
     }
   }
   bar_consumers();
+  if (trc) {
+    const long long t1 = clock64();
+    C.ms->tr_pre += t1 - tA;
+    tA = t1;
+  }
 
   AttState st;
 #pragma unroll
@@ -1675,6 +1761,11 @@ __device__ void attn_task(const Ctx& C, const Task t, uint32_t& it) {
     par ^= 1;
   }
   bar_consumers();
+  if (trc) {
+    const long long t1 = clock64();
+    C.ms->tr_loop += t1 - tA;
+    tA = t1;
+  }
 
   // ---- write the item's partial (M, L, O) per query row ----
   float* smx = reinterpret_cast<float*>(C.att + 2 * mt * KTq * 512 + 2 * mt * (ATT_CT / 16) * 512);
@@ -1739,6 +1830,11 @@ __device__ void attn_task(const Ctx& C, const Task t, uint32_t& it) {
     const uint32_t old = atom_add_acqrel(P.ctr + pc, 1u);
     lastc = (old == (uint32_t)itm.ns - 1) ? 1 : 0;
   }
+  if (trc) {
+    const long long t1 = clock64();
+    C.ms->tr_post += t1 - tA;
+    tA = t1;
+  }
   if (broadcast_from0(C, lastc)) {
     float* out = P.buf[B_ATTN];
     const int ldo = P.ld[B_ATTN];
@@ -1790,12 +1886,416 @@ __device__ void attn_task(const Ctx& C, const Task t, uint32_t& it) {
       __threadfence();
       red_release_add(P.ctr + t.layer * P.ctr_layer_stride + C_ATTN, 1u);
     }
+    if (trc) C.ms->tr_epi += clock64() - tA;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// multi-head latent attention items (absorbed form)
+// ---------------------------------------------------------------------------
+// The cache holds per position the latent row [c (R) | k_rope (dr)], shared by
+// all heads.  With the key up-projection absorbed into the query
+// (q_abs,h = W_uk,h^T q_nope,h, computed by the preceding grouped GEMV), the
+// score of head h at position t is (q_abs,h . c_t + q_rope,h . k_rope,t) /
+// sqrt(dn + dr), and the head's value is W_uv,h applied to sum_t p_t c_t
+// (the following grouped GEMV).  So one item attends one query row over a
+// range of latent rows with all heads as the mma M dimension: multi-query
+// attention with 576-wide keys and 512-wide values.
+struct MlaState {
+  float o[2][8][4];  // [m-tile][latent-dim tile of this warp][frag]
+  float M[2][2];     // running max (log2 units) of rows g, g + 8 of each m-tile
+  float L[2][2];     // lane-partial running sums
+};
+
+__device__ __forceinline__ void mla_chunk(const Ctx& C, MlaState& st, const uint8_t* rows, int n_valid, int mt,
+                                          int KW, int NTW, int pitch, int par, const MlaLayout& lay) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, tq = lane & 3;
+  uint8_t* base = C.xring;
+  const uint8_t* qhi = base + lay.qhi;
+  const uint8_t* qlo = base + lay.qlo;
+  uint8_t* phi = base + lay.phi;
+  uint8_t* plo = base + lay.plo;
+  float* smx = reinterpret_cast<float*>(base + lay.smax) + par * NCW * 32;
+
+  // ---- scores of positions [8 warp, 8 warp + 8) over all KW k-steps ----
+  float sacc[2][4];
+#pragma unroll
+  for (int mi = 0; mi < 2; ++mi) sacc[mi][0] = sacc[mi][1] = sacc[mi][2] = sacc[mi][3] = 0.f;
+  const int n0 = warp * 8;
+  if (n0 < n_valid) {
+    const uint8_t* krow = rows + (size_t)(n0 + g) * pitch + tq * 4;
+#pragma unroll 2
+    for (int ks = 0; ks < KW; ++ks) {
+      const uint32_t b0 = lds32(krow + ks * 32);
+      const uint32_t b1 = lds32(krow + ks * 32 + 16);
+#pragma unroll
+      for (int mi = 0; mi < 2; ++mi) {
+        if (mi < mt) {
+          const uint4 ah = lds128(qhi + ((mi * KW + ks) * 32 + lane) * 16);
+          const uint4 al = lds128(qlo + ((mi * KW + ks) * 32 + lane) * 16);
+          mma_bf16(sacc[mi], ah, b0, b1);
+          mma_bf16(sacc[mi], al, b0, b1);
+        }
+      }
+    }
+  }
+  const int p0 = n0 + 2 * tq, p1 = p0 + 1;
+#pragma unroll
+  for (int mi = 0; mi < 2; ++mi) {
+    if (mi < mt) {
+      if (p0 >= n_valid) sacc[mi][0] = sacc[mi][2] = -INFINITY;
+      if (p1 >= n_valid) sacc[mi][1] = sacc[mi][3] = -INFINITY;
+      float mA = fmaxf(sacc[mi][0], sacc[mi][1]), mB = fmaxf(sacc[mi][2], sacc[mi][3]);
+      mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 1));
+      mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 2));
+      mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 1));
+      mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 2));
+      if (tq == 0) {
+        smx[warp * 32 + mi * 16 + g] = mA;
+        smx[warp * 32 + mi * 16 + g + 8] = mB;
+      }
+    }
+  }
+  bar_consumers();
+  // ---- online softmax; P written as A fragments (k-step warp / 2) ----
+  const int kt = warp >> 1;
+  const int regA = (warp & 1) ? 2 : 0;
+#pragma unroll
+  for (int mi = 0; mi < 2; ++mi) {
+    if (mi < mt) {
+      float cm[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int w = 0; w < NCW; ++w) {
+        cm[0] = fmaxf(cm[0], smx[w * 32 + mi * 16 + g]);
+        cm[1] = fmaxf(cm[1], smx[w * 32 + mi * 16 + g + 8]);
+      }
+      float pv[4];
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const float mnew = fmaxf(st.M[mi][h2], cm[h2]);
+        const float corr = (mnew == -INFINITY) ? 1.f : exp2f(st.M[mi][h2] - mnew);
+        const float msafe = (mnew == -INFINITY) ? 0.f : mnew;
+        st.M[mi][h2] = mnew;
+        pv[2 * h2 + 0] = exp2f(sacc[mi][2 * h2 + 0] - msafe);
+        pv[2 * h2 + 1] = exp2f(sacc[mi][2 * h2 + 1] - msafe);
+        st.L[mi][h2] = st.L[mi][h2] * corr + pv[2 * h2 + 0] + pv[2 * h2 + 1];
+#pragma unroll
+        for (int jn = 0; jn < 8; ++jn) {
+          st.o[mi][jn][2 * h2 + 0] *= corr;
+          st.o[mi][jn][2 * h2 + 1] *= corr;
+        }
+      }
+      uint32_t hA, lA, hB, lB;
+      split_bf16(pv[0], pv[1], hA, lA);
+      split_bf16(pv[2], pv[3], hB, lB);
+      uint32_t* ph = reinterpret_cast<uint32_t*>(phi + ((mi * 4 + kt) * 32 + lane) * 16);
+      uint32_t* pl = reinterpret_cast<uint32_t*>(plo + ((mi * 4 + kt) * 32 + lane) * 16);
+      ph[regA] = hA;
+      ph[regA + 1] = hB;
+      pl[regA] = lA;
+      pl[regA + 1] = lB;
+    }
+  }
+  bar_consumers();
+  // ---- O += P C over this warp's latent dims [8 NTW warp, 8 NTW (warp + 1)) ----
+  for (int ks = 0; ks < 4; ++ks) {
+    if (ks * 16 >= n_valid) break;
+    const int pk = ks * 16 + 2 * tq;
+    uint4 ah[2], al[2];
+#pragma unroll
+    for (int mi = 0; mi < 2; ++mi) {
+      if (mi < mt) {
+        ah[mi] = lds128(phi + ((mi * 4 + ks) * 32 + lane) * 16);
+        al[mi] = lds128(plo + ((mi * 4 + ks) * 32 + lane) * 16);
+      }
+    }
+#pragma unroll
+    for (int jn = 0; jn < 8; ++jn) {
+      if (jn < NTW) {
+        const uint8_t* vc = rows + ((warp * NTW + jn) * 8 + g) * 2;
+        const uint32_t v0 = pk < n_valid ? lds16(vc + (size_t)pk * pitch) : 0u;
+        const uint32_t v1 = pk + 1 < n_valid ? lds16(vc + (size_t)(pk + 1) * pitch) : 0u;
+        const uint32_t v8 = pk + 8 < n_valid ? lds16(vc + (size_t)(pk + 8) * pitch) : 0u;
+        const uint32_t v9 = pk + 9 < n_valid ? lds16(vc + (size_t)(pk + 9) * pitch) : 0u;
+        const uint32_t b0 = v0 | (v1 << 16), b1 = v8 | (v9 << 16);
+#pragma unroll
+        for (int mi = 0; mi < 2; ++mi) {
+          if (mi < mt) {
+            mma_bf16(st.o[mi][jn], ah[mi], b0, b1);
+            mma_bf16(st.o[mi][jn], al[mi], b0, b1);
+          }
+        }
+      }
+    }
+  }
+}
+
+__device__ __noinline__ void mla_task(const Ctx& C, const Task t, uint32_t& it) {
+  const Launch& P = *C.P;
+  const Model& md = *C.md;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, tq = lane & 3;
+  const bool trc = P.trace && threadIdx.x == 0;
+  long long tA = trc ? clock64() : 0;
+  const Item itm = decode_item(t.rt0, P.n_pairs, P.n_items);
+  const int mrow = itm.pair, Q = P.Q, s = mrow / Q, qi = mrow % Q;
+  const int Hq = md.Hq, R = md.R, dr = md.dr, dn = md.d, W = R + dr, KW = W / 16, mt = (Hq + 15) >> 4;
+  const int pitch = mla_pitch(R, dr), MCT = mla_ct(R, dr), NTW = R / 64;
+  const MlaLayout lay = mla_layout(Hq, R, dr);
+  const int T0 = seq_pos0(P, s);
+  const int a = (int)(((int64_t)itm.j * T0) / itm.ns), b = (int)(((int64_t)(itm.j + 1) * T0) / itm.ns);
+  const bool last = itm.j == itm.ns - 1;
+  const float qscale = rsqrtf((float)(dn + dr)) * 1.4426950408889634f;
+  const float* qkv = P.buf[B_QKV];
+  const int ldq = P.ld[B_QKV];
+  const float* qa = P.buf[B_QL];
+  const int lda = P.ld[B_QL];
+  const int QW = Hq * (dn + dr), half = dr / 2;
+  const float2* rope = md.rope;
+  uint8_t* base = C.xring;
+  uint8_t* qhi = base + lay.qhi;
+  uint8_t* qlo = base + lay.qlo;
+
+  // ---- queries: absorbed latent part, then the rotary part (RoPE at this row's
+  //      position), scaled to log2 units, as bf16 hi / lo A fragments ----
+  {
+    // 4 consecutive latent dims per thread and step, 4 steps in flight
+    const int R4 = R / 4, n4 = mt * 16 * R4;
+#pragma unroll 4
+    for (int e = tid; e < n4; e += NCT) {
+      const int r = e / R4, k = (e - r * R4) * 4;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < Hq) v = __ldcg(reinterpret_cast<const float4*>(qa + (size_t)mrow * lda + (size_t)r * R + k));
+      const float xs[4] = {v.x * qscale, v.y * qscale, v.z * qscale, v.w * qscale};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const __nv_bfloat16 h = __float2bfloat16_rn(xs[q]);
+        *reinterpret_cast<__nv_bfloat16*>(qhi + frag_off(r, k + q, KW)) = h;
+        *reinterpret_cast<__nv_bfloat16*>(qlo + frag_off(r, k + q, KW)) =
+            __float2bfloat16_rn(xs[q] - __bfloat162float(h));
+      }
+    }
+  }
+  const int pos = T0 + qi;
+  for (int e = tid; e < mt * 16 * half; e += NCT) {
+    const int r = e / half, i = e - r * half;
+    float x0 = 0.f, x1 = 0.f;
+    if (r < Hq) {
+      const float* q = qkv + (size_t)mrow * ldq + (size_t)r * (dn + dr) + dn;
+      const float a0 = __ldcg(q + i), a1 = __ldcg(q + i + half);
+      const float2 cs = __ldg(rope + (size_t)pos * half + i);
+      x0 = (a0 * cs.x - a1 * cs.y) * qscale;
+      x1 = (a0 * cs.y + a1 * cs.x) * qscale;
+    }
+    const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
+    *reinterpret_cast<__nv_bfloat16*>(qhi + frag_off(r, R + i, KW)) = h0;
+    *reinterpret_cast<__nv_bfloat16*>(qhi + frag_off(r, R + i + half, KW)) = h1;
+    *reinterpret_cast<__nv_bfloat16*>(qlo + frag_off(r, R + i, KW)) = __float2bfloat16_rn(x0 - __bfloat162float(h0));
+    *reinterpret_cast<__nv_bfloat16*>(qlo + frag_off(r, R + i + half, KW)) =
+        __float2bfloat16_rn(x1 - __bfloat162float(h1));
+  }
+  // ---- the step's own latent rows 0..qi of this sequence (RoPE on k_rope, bf16);
+  //      row qi is this query's position and is appended to the cache here ----
+  uint8_t* newr = base + lay.newr;
+  if (last) {
+    __nv_bfloat16* cache = reinterpret_cast<__nv_bfloat16*>(P.kv_k) +
+                           (((size_t)t.layer * P.kv_seqs + s) * (size_t)P.kv_ctx + pos) * W;
+    const int per = R + half;
+    for (int e = tid; e < (qi + 1) * per; e += NCT) {
+      const int j = e / per, k = e - j * per;
+      const float* src = qkv + (size_t)(s * Q + j) * ldq + QW;
+      __nv_bfloat16* row = reinterpret_cast<__nv_bfloat16*>(newr + (size_t)j * pitch);
+      if (k < R) {
+        const __nv_bfloat16 v = __float2bfloat16_rn(__ldcg(src + k));
+        row[k] = v;
+        if (j == qi) cache[k] = v;
+      } else {
+        const int i = k - R;
+        const float a0 = __ldcg(src + R + i), a1 = __ldcg(src + R + i + half);
+        const float2 cs = __ldg(rope + (size_t)(T0 + j) * half + i);
+        const __nv_bfloat16 k0 = __float2bfloat16_rn(a0 * cs.x - a1 * cs.y);
+        const __nv_bfloat16 k1 = __float2bfloat16_rn(a0 * cs.y + a1 * cs.x);
+        row[R + i] = k0;
+        row[R + i + half] = k1;
+        if (j == qi) {
+          cache[R + i] = k0;
+          cache[R + i + half] = k1;
+        }
+      }
+    }
+  }
+  bar_consumers();
+  if (trc) {
+    const long long t1 = clock64();
+    C.ms->tr_pre += t1 - tA;
+    tA = t1;
+  }
+
+  MlaState st;
+#pragma unroll
+  for (int mi = 0; mi < 2; ++mi) {
+    st.M[mi][0] = st.M[mi][1] = -INFINITY;
+    st.L[mi][0] = st.L[mi][1] = 0.f;
+#pragma unroll
+    for (int jn = 0; jn < 8; ++jn) st.o[mi][jn][0] = st.o[mi][jn][1] = st.o[mi][jn][2] = st.o[mi][jn][3] = 0.f;
+  }
+  int par = 0;
+  for (int t0 = a; t0 < b; t0 += MCT) {
+    const int n = min(MCT, b - t0);
+    wait_full(C, it);
+    const uint8_t* stage = C.ring + (size_t)(it % NSTAGE) * STAGE_BYTES;
+    mla_chunk(C, st, stage, n, mt, KW, NTW, pitch, par, lay);
+    par ^= 1;
+    bar_consumers();  // every warp is done with the stage
+    release_stage(C, it);
+    ++it;
+  }
+  if (last) {
+    mla_chunk(C, st, newr, qi + 1, mt, KW, NTW, pitch, par, lay);
+    par ^= 1;
+  }
+  bar_consumers();
+  if (trc) {
+    const long long t1 = clock64();
+    C.ms->tr_loop += t1 - tA;
+    tA = t1;
+  }
+
+  // ---- the item's partial (M, L, O) per head ----
+  float* smx = reinterpret_cast<float*>(base + lay.smax);
+#pragma unroll
+  for (int mi = 0; mi < 2; ++mi) {
+    if (mi < mt) {
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        float l = st.L[mi][h2];
+        l += __shfl_xor_sync(0xffffffffu, l, 1);
+        l += __shfl_xor_sync(0xffffffffu, l, 2);
+        if (tq == 0) smx[warp * 32 + mi * 16 + g + 8 * h2] = l;
+      }
+    }
+  }
+  bar_consumers();
+  const int rows_max = P.att_rows_max, dP = R + 2;
+  float* part = P.att_part + (size_t)t.rt0 * rows_max * dP;
+  if (tid < Hq) {
+    float l = 0.f;
+    for (int w = 0; w < NCW; ++w) l += smx[w * 32 + tid];
+    part[(size_t)tid * dP + 1] = l;
+  }
+  if (warp == 0 && tq == 0) {
+#pragma unroll
+    for (int mi = 0; mi < 2; ++mi)
+      if (mi < mt) {
+        if (mi * 16 + g < Hq) part[(size_t)(mi * 16 + g) * dP] = st.M[mi][0];
+        if (mi * 16 + g + 8 < Hq) part[(size_t)(mi * 16 + g + 8) * dP] = st.M[mi][1];
+      }
+  }
+#pragma unroll
+  for (int mi = 0; mi < 2; ++mi) {
+    if (mi < mt) {
+#pragma unroll
+      for (int jn = 0; jn < 8; ++jn) {
+        if (jn < NTW) {
+          const int dim = (warp * NTW + jn) * 8 + 2 * tq;
+          const int rA = mi * 16 + g, rB = rA + 8;
+          if (rA < Hq) {
+            part[(size_t)rA * dP + 2 + dim] = st.o[mi][jn][0];
+            part[(size_t)rA * dP + 3 + dim] = st.o[mi][jn][1];
+          }
+          if (rB < Hq) {
+            part[(size_t)rB * dP + 2 + dim] = st.o[mi][jn][2];
+            part[(size_t)rB * dP + 3 + dim] = st.o[mi][jn][3];
+          }
+        }
+      }
+    }
+  }
+  // this region is the activation ring, which bulk copies write again later
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  bar_consumers();
+  if (trc) {
+    const long long t1 = clock64();
+    C.ms->tr_post += t1 - tA;
+    tA = t1;
+  }
+
+  (void)trc;
+}
+
+// The split combine of every query row's latent attention, spread over all
+// CTAs: CTA c owns a contiguous slice of the outputs [pair][head][R] and
+// forms each as sum_j exp2(M_j - M*) O_j / sum_j exp2(M_j - M*) L_j over the
+// pair's splits j (fixed order).
+__device__ __noinline__ void mla_comb_task(const Ctx& C, const Task t) {
+  const Launch& P = *C.P;
+  const Model& md = *C.md;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int Hq = md.Hq, R = md.R, dP = R + 2, rows_max = P.att_rows_max;
+  const int64_t total = (int64_t)P.n_pairs * Hq * R;
+  const int64_t o0 = total * blockIdx.x / gridDim.x, o1 = total * (blockIdx.x + 1) / gridDim.x;
+  if (o0 >= o1) return;
+  float* out = P.buf[B_OL];
+  const int ldo = P.ld[B_OL];
+  float* wsh = reinterpret_cast<float*>(C.att);  // [row][160] split weights
+  const int row0 = (int)(o0 / R), row1 = (int)((o1 - 1) / R) + 1;
+  for (int rb = row0; rb < row1; rb += 64) {
+    const int re = min(row1, rb + 64);
+    const int64_t a = max(o0, (int64_t)rb * R), b = min(o1, (int64_t)re * R);
+    for (int rr = rb + warp; rr < re; rr += NCW) {
+      const int pair = rr / Hq, h = rr - pair * Hq;
+      const Item itm = decode_item(pair_first_item(pair, P.n_pairs, P.n_items), P.n_pairs, P.n_items);
+      const int ns = itm.ns;
+      float mj[5], lj[5];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < 5; ++q) {
+        const int jj = lane + 32 * q;
+        mj[q] = -INFINITY;
+        lj[q] = 0.f;
+        if (jj < ns) {
+          const float* pp = P.att_part + ((size_t)(itm.first + jj) * rows_max + h) * dP;
+          mj[q] = __ldcg(pp);
+          lj[q] = __ldcg(pp + 1);
+        }
+        mx = fmaxf(mx, mj[q]);
+      }
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      float den = 0.f, w[5];
+#pragma unroll
+      for (int q = 0; q < 5; ++q) {
+        w[q] = (mj[q] == -INFINITY) ? 0.f : exp2f(mj[q] - mx);
+        den += w[q] * lj[q];
+      }
+      for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+#pragma unroll
+      for (int q = 0; q < 5; ++q) {
+        const int jj = lane + 32 * q;
+        if (jj < ns) wsh[(rr - rb) * 160 + jj] = w[q] / den;
+      }
+    }
+    bar_consumers();
+    for (int64_t o = a + tid; o < b; o += NCT) {
+      const int rr = (int)(o / R), k = (int)(o - (int64_t)rr * R);
+      const int pair = rr / Hq, h = rr - pair * Hq;
+      const Item itm = decode_item(pair_first_item(pair, P.n_pairs, P.n_items), P.n_pairs, P.n_items);
+      const float* wr = wsh + (rr - rb) * 160;
+      const float* src = P.att_part + ((size_t)itm.first * rows_max + h) * dP + 2 + k;
+      const size_t js = (size_t)rows_max * dP;
+      float num = 0.f;
+#pragma unroll 16
+      for (int jj = 0; jj < itm.ns; ++jj) num += wr[jj] * __ldcg(src + jj * js);
+      out[(size_t)pair * ldo + (size_t)h * R + k] = num;
+    }
+    bar_consumers();
   }
 }
 
 // ---------------------------------------------------------------------------
 // consumer warps
 // ---------------------------------------------------------------------------
+template <bool MLA>
 __device__ void consumer(const Ctx& C) {
   const Launch& P = *C.P;
   uint32_t it = 0, ix = 0;
@@ -1820,8 +2320,12 @@ __device__ void consumer(const Ctx& C) {
     if (tr) td = globaltimer();
     if (gemv_like(t)) {
       gemv_task(C, t, it, ix);
-    } else if (t.type == T_ATTN) {
+    } else if (!MLA && t.type == T_ATTN) {
       attn_task(C, t, it);
+    } else if (MLA && t.type == T_MLA) {
+      mla_task(C, t, it);
+    } else if (MLA && t.type == T_MLA_COMB) {
+      mla_comb_task(C, t);
     } else if (t.type == T_EMBED) {
       embed_task(C, t);
     }
@@ -1854,6 +2358,10 @@ __device__ void consumer(const Ctx& C) {
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
+// One instance per attention family (GQA or latent): each kernel holds only
+// the code its models run, which keeps the instruction footprint of the
+// whole-step loop small.
+template <bool MLA>
 __global__ void __launch_bounds__(NTHREADS, 1) mk_step_kernel(const __grid_constant__ Launch P) {
   extern __shared__ __align__(128) uint8_t smem[];
   Ctx C;
@@ -1899,9 +2407,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) mk_step_kernel(const __grid_const
   }
   __syncthreads();
 
-  if ((tid >> 5) == WARP_WP) producer(C);
+  if ((tid >> 5) == WARP_WP) producer<MLA>(C);
   else if ((tid >> 5) == WARP_XP) xproducer(C);
-  else consumer(C);
+  else consumer<MLA>(C);
   __syncthreads();
 
   // ---- teardown: the last CTA out zeroes every counter for the next launch ----
@@ -1920,5 +2428,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) mk_step_kernel(const __grid_const
     __threadfence();
   }
 }
+
+template __global__ void mk_step_kernel<false>(const __grid_constant__ Launch P);
+template __global__ void mk_step_kernel<true>(const __grid_constant__ Launch P);
 
 }  // namespace mk

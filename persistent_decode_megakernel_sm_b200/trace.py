@@ -15,9 +15,9 @@ import sys
 
 import numpy as np
 
-TYPE_NAMES = {1: "gemv", 2: "attn"}
+TYPE_NAMES = {1: "gemv", 2: "attn", 3: "moe_gu", 4: "moe_down", 6: "embed", 7: "mla", 8: "mla_comb"}
 FIELDS = 20
-EPI_NAMES = {0: "store", 1: "resid", 2: "swiglu", 3: "logits"}
+EPI_NAMES = {0: "store", 1: "resid", 2: "swiglu", 3: "logits", 4: "swiglu_moe"}
 
 
 def record(model, kv, tokens, positions, logits, argmax, cap: int = 512):
@@ -55,7 +55,7 @@ def summarize(tr: np.ndarray, sm_clock_mhz: float = 0.0) -> dict:
             tb, td, te, wf, wx, ch, layer, te16 = tr[c, k, :8]
             fr, mm, ep, rl = tr[c, k, 8:12]
             lo, pr, po, sg = tr[c, k, 16:20]
-            name = TYPE_NAMES.get(int(te16) // 16, "?") + ("/" + EPI_NAMES[int(te16) % 16] if int(te16) // 16 == 1 else "")
+            name = TYPE_NAMES.get(int(te16) // 16, "?") + ("/" + EPI_NAMES[int(te16) % 16] if int(te16) // 16 in (1, 3) else "")
             p = phases[name]
             p["n"] += 1
             p["dep_us"] += (td - tb) / 1e3
