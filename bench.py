@@ -51,6 +51,28 @@ def parse():
     return ap.parse_args()
 
 
+def recorded_traffic(config: str, B: int):
+    """DRAM bytes per launch recorded from an ncu capture under profiles/,
+    valid only while the kernel sources are the ones it was taken on (the
+    summary carries their hash); None otherwise."""
+    import glob
+    import hashlib
+    import re
+    h = hashlib.sha256()
+    for f in ("mk_kernel.cu", "mk_host.cu", "mk_internal.h"):
+        with open(os.path.join(ROOT, "persistent_decode_megakernel_sm_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    sha = h.hexdigest()[:16]
+    pat = re.compile(r"traffic_bytes_per_launch: ([0-9.eE+]+); case: (\S+) B=(\d+) .*sources_sha256_16: (\w+)")
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        with open(path) as fh:
+            for line in fh:
+                m = pat.search(line)
+                if m and m.group(2) == config and int(m.group(3)) == B and m.group(4) == sha:
+                    return float(m.group(1))
+    return None
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -364,7 +386,8 @@ def run_ours(args, rank, world, local_rank):
                    "model": args.config, "global_batch": B * world, "seq_len": mc.context, "parallelism": f"dp{world}",
                    "l2": "inputs larger than L2 (44 GB weights), no flush"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_kind": peak_kind, "traffic": args.traffic,
+                     "peak_kind": peak_kind,
+                     "traffic": args.traffic if args.traffic is not None else recorded_traffic(args.config, B),
                      "frac_of_8tbs": achieved / 8000.0, "algorithmic_bytes_per_launch": abytes},
         "by_batch": by_batch,
         "workloads": workloads,
