@@ -1095,6 +1095,13 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
     flat.insert(flat.end(), per[c].begin(), per[c].end());
   }
   off[ncta] = (int32_t)flat.size();
+  // copies the kernel would otherwise load, dependently, at every task start
+  for (Task& t : flat) {
+    t.m = h->mats[t.mat].m;
+    t.gvec = nullptr;
+    if (t.in_kind == IN_X_NORM)
+      t.gvec = t.gain == 0 ? h->attn_norm[t.layer] : (t.gain == 1 ? h->ffn_norm[t.layer] : h->final_norm);
+  }
   n_items_out = n_items;
   n_pairs_out = n_pairs;
 }

@@ -109,6 +109,18 @@ enum BufId : int16_t {
   NBUF = 7
 };
 
+struct Mat {
+  const uint8_t* w;          // tiles [RT][KT][tile] (expert arrays: [ne][RT][KT][tile])
+  const float* scales;       // fp8: [nbr][nbc] (GU: [2][nbr][nbc], gate then up), per expert
+  int32_t rows, cols, RT, KT;  // of one expert
+  int32_t fp8;
+  int32_t nbr, nbc;
+  int32_t gu;                // rows interleaved gate/up by 8
+  int32_t ne;                // experts in the array (1 for a plain matrix)
+  int64_t estride;           // bytes between experts' tiles
+  int64_t sstride;           // floats between experts' scales
+};
+
 struct Task {
   int16_t type, layer;
   int16_t in_kind, epi;
@@ -123,22 +135,15 @@ struct Task {
   int32_t ss_src;            // IN_X_NORM: which partial-sum array (0: after O, 1: after down)
   int32_t ss_dst;            // EPI_RESID: partial-sum array written
   int32_t mat2;              // T_MOE_DOWN: the shared experts' down matrix
+  // Copies taken when the plan is built, so that starting a task needs no
+  // dependent global loads: the matrix descriptor and the input's norm gain.
+  Mat m;                     // mats[mat]
+  const uint16_t* gvec;      // the norm gain of an IN_X_NORM input (null otherwise)
 };
 
 // ---------------------------------------------------------------------------
 // device-resident model description
 // ---------------------------------------------------------------------------
-struct Mat {
-  const uint8_t* w;          // tiles [RT][KT][tile] (expert arrays: [ne][RT][KT][tile])
-  const float* scales;       // fp8: [nbr][nbc] (GU: [2][nbr][nbc], gate then up), per expert
-  int32_t rows, cols, RT, KT;  // of one expert
-  int32_t fp8;
-  int32_t nbr, nbc;
-  int32_t gu;                // rows interleaved gate/up by 8
-  int32_t ne;                // experts in the array (1 for a plain matrix)
-  int64_t estride;           // bytes between experts' tiles
-  int64_t sstride;           // floats between experts' scales
-};
 
 struct Layer {
   const uint16_t* attn_norm;

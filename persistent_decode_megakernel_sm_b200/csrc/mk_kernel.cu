@@ -65,6 +65,9 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
       : "memory");
 }
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
@@ -275,11 +278,6 @@ __device__ __forceinline__ int x_cap(const Task& t, int M) {
 }
 // row stride of an activation window in the x slot
 __device__ __forceinline__ int x_rowbytes(const Task& t, int wc) { return wc * 16 * x_esize(t) + XROW_PAD; }
-__device__ __forceinline__ const uint16_t* task_gain(const Model& md, const Task& t) {
-  if (t.in_kind == IN_BUF) return nullptr;
-  const Layer* ly = md.layers + t.layer;
-  return t.gain == 0 ? ly->attn_norm : (t.gain == 1 ? ly->ffn_norm : md.final_norm);
-}
 
 // Attention item -> (pair, split index, number of splits, first item of pair).
 struct Item {
@@ -658,7 +656,7 @@ struct ChunkStream {
       if (ti >= end) return 0;
       t = P.tasks[ti++];
       if (gemv_like(t)) {
-        m = md.mats[t.mat];
+        m = t.m;
         m2 = (t.type == T_MOE_DOWN && t.mat2 >= 0) ? md.mats[t.mat2] : m;
         tb = m.fp8 ? TILE_FP8 : TILE_BF16;
         xcap = x_cap(t, P.M);
@@ -835,7 +833,7 @@ __device__ __noinline__ void convert_window_coop(uint8_t* dst, int rb, int M, in
 // together (a single warp would fall behind the tensor cores at M = 8).
 constexpr int XCONV_M = 0;
 
-__device__ bool xprod_reserve(const Ctx& C, uint32_t ix, uint32_t bytes, const float* scale) {
+__device__ bool xprod_reserve(const Ctx& C, uint32_t ix, uint32_t bytes) {
   const int lane = threadIdx.x & 31;
   int ok = 1;
   if (lane == 0) {
@@ -859,11 +857,7 @@ __device__ bool xprod_reserve(const Ctx& C, uint32_t ix, uint32_t bytes, const f
         }
       }
     }
-    if (ok) {
-#pragma unroll
-      for (int q = 0; q < MAXM; ++q) C.ms->xscale[s][q] = scale[q];
-      mbar_arrive_expect_tx(&C.ms->xfull[s], bytes);  // release: the scales are visible with the phase
-    }
+    if (ok) mbar_arrive_expect_tx(&C.ms->xfull[s], bytes);
   }
   ok = __shfl_sync(0xffffffffu, ok, 0);
   return ok != 0;
@@ -881,7 +875,7 @@ __device__ void xproducer(const Ctx& C) {
   for (int ti = beg; ti < end; ++ti) {
     const Task t = P.tasks[ti];
     if (!gemv_like(t)) continue;
-    const Mat m = md.mats[t.mat];
+    const Mat m = t.m;
     const Mat m2 = (t.type == T_MOE_DOWN && t.mat2 >= 0) ? md.mats[t.mat2] : m;
     const int tb = m.fp8 ? TILE_FP8 : TILE_BF16;
     const int xcap = x_cap(t, M);
@@ -893,21 +887,14 @@ __device__ void xproducer(const Ctx& C) {
     Pieces pc;
     if (!pc.init(rt0, rt1, gsz, nseg)) continue;
     // RMSNorm scale of every activation row (fixed-order reduction of the
-    // per-CTA sums of squares) and the norm gain of this task
+    // per-CTA sums of squares), computed once the task's first activation
+    // copy is in flight, and the norm gain of this task
     float scale[MAXM];
     const bool has_gain = t.in_kind == IN_X_NORM;
-    const uint16_t* gain = task_gain(md, t);
+    bool have_scale = !has_gain;
+    const uint16_t* gain = t.gvec;
 #pragma unroll
-    for (int mm = 0; mm < MAXM; ++mm) {
-      scale[mm] = 1.f;
-      if (has_gain && mm < M) {
-        const float* srcs = P.ss_part + (size_t)t.ss_src * gridDim.x * MAXM;
-        float ss = 0.f;
-        for (int c = lane; c < (int)gridDim.x; c += 32) ss += __ldcg(srcs + c * MAXM + mm);
-        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        scale[mm] = rsqrtf(ss / (float)md.H + md.eps);
-      }
-    }
+    for (int mm = 0; mm < MAXM; ++mm) scale[mm] = 1.f;
     do {
       const PieceSrc src = piece_src(md, t, m, m2, C.ms->rt_ex[RR_XPROD], pc);
       ChunkIt ci;
@@ -918,14 +905,33 @@ __device__ void xproducer(const Ctx& C) {
         const int wn = ci.wn(), w0 = ci.w0();
         const uint32_t rowdata = (uint32_t)(wn * 64);
         const int sl = ix % XSLOTS;
-        if (!xprod_reserve(C, ix, (uint32_t)M * rowdata, scale)) goto drain;
-        __syncwarp();
+        if (!xprod_reserve(C, ix, (uint32_t)M * rowdata)) goto drain;
         uint8_t* dst = C.xring + (size_t)sl * XSLOT_BYTES;
         if (lane < M) {
           const uint8_t* xsrc = reinterpret_cast<const uint8_t*>(
               P.buf[src.xbuf] + (size_t)(src.xrow0 + lane) * P.ld[src.xbuf] + src.xcol0 + ci.c0 * 16);
           bulk_g2s(dst + (size_t)lane * rb, xsrc, rowdata, &C.ms->xfull[sl], pol);
         }
+        if (!have_scale) {
+#pragma unroll
+          for (int mm = 0; mm < MAXM; ++mm) {
+            if (mm < M) {
+              const float* srcs = P.ss_part + (size_t)t.ss_src * gridDim.x * MAXM;
+              float ss = 0.f;
+              for (int c = lane; c < (int)gridDim.x; c += 32) ss += __ldcg(srcs + c * MAXM + mm);
+              for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+              scale[mm] = rsqrtf(ss / (float)md.H + md.eps);
+            }
+          }
+          have_scale = true;
+        }
+        // the slot's second arrival publishes the rows' scales (release)
+        if (lane == 0) {
+#pragma unroll
+          for (int q = 0; q < MAXM; ++q) C.ms->xscale[sl][q] = scale[q];
+          mbar_arrive(&C.ms->xfull[sl]);
+        }
+        __syncwarp();
         if (M > XCONV_M) {
           // the consumers convert this window themselves
           ++ix;
@@ -1213,7 +1219,7 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
   const Model& md = *C.md;
   // Copies in registers: the barrier asm below clobbers "memory", which would
   // otherwise force a reload of every struct field on every chunk.
-  const Mat m = md.mats[t.mat];
+  const Mat m = t.m;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, tq = lane & 3;
   const int M = P.M;
@@ -1249,7 +1255,7 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
   L.rowbytes = 0;
   L.trc = P.trace && tid == 0;
   L.coop = M > XCONV_M;
-  L.gain = task_gain(md, t);
+  L.gain = t.gvec;
   if (L.trc) C.ms->tr_pre += clock64() - tpre;
   while (have) {
     const PieceSrc src = piece_src(md, t, m, m2, C.ms->rt_ex[RR_CONS], pc);
@@ -2307,6 +2313,17 @@ __device__ void consumer(const Ctx& C) {
   const int beg = P.task_off[blockIdx.x], end = P.task_off[blockIdx.x + 1];
   for (int ti = beg; ti < end; ++ti) {
     const Task t = P.tasks[ti];
+    // while this task waits and runs: the next task's record, and this
+    // task's norm gain (read while converting activation windows), into L1
+    if (ti + 1 < end && threadIdx.x < 3) {
+      const uintptr_t a = reinterpret_cast<uintptr_t>(P.tasks + ti + 1);
+      const uintptr_t line = (a & ~(uintptr_t)127) + threadIdx.x * 128;
+      if (line < a + sizeof(Task)) prefetch_l1(reinterpret_cast<const void*>(line));
+    }
+    if (t.gvec) {
+      const int lines = (C.md->H * 2 + 127) / 128;
+      for (int i = threadIdx.x; i < lines; i += NCT) prefetch_l1(reinterpret_cast<const char*>(t.gvec) + i * 128);
+    }
     const bool tr = P.trace && (ti - beg) < P.trace_cap && threadIdx.x == 0;
     uint64_t tb = 0, td = 0;
     if (tr) {
@@ -2398,7 +2415,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) mk_step_kernel(const __grid_const
       mbar_init(&C.ms->empty[s], NCW);
     }
     for (int s = 0; s < XSLOTS; ++s) {
-      mbar_init(&C.ms->xfull[s], 1);
+      mbar_init(&C.ms->xfull[s], 2);  // the copies' expect-tx arrival + the scales
       mbar_init(&C.ms->xready[s], 1);
       mbar_init(&C.ms->xempty[s], NCW);
     }
