@@ -1047,12 +1047,12 @@ __device__ void wait_counter(const Ctx& C, int idx, uint32_t target) {
   bar_consumers();
 }
 
+// The consumers' writes of the task precede thread 0's release through the
+// barrier (causality order is transitive; the release is cumulative), so the
+// release alone publishes them at gpu scope: no separate full fence.
 __device__ __forceinline__ void signal_counter(const Ctx& C, int idx) {
   bar_consumers();
-  if (threadIdx.x == 0 && !C.ms->abort) {
-    __threadfence();
-    red_release_add(C.P->ctr + idx, 1u);
-  }
+  if (threadIdx.x == 0 && !C.ms->abort) red_release_add(C.P->ctr + idx, 1u);
 }
 
 // ---------------------------------------------------------------------------
@@ -1464,7 +1464,6 @@ __device__ void lm_finish(const Ctx& C) {
   bar_consumers();
   int last = 0;
   if (threadIdx.x == 0 && !C.ms->abort) {
-    __threadfence();
     const uint32_t old = atom_add_acqrel(P.ctr + P.ctr_lm, 1u);
     last = (old == (uint32_t)C.ncta - 1) ? 1 : 0;
   }
@@ -1831,7 +1830,6 @@ __device__ __noinline__ void attn_task(const Ctx& C, const Task t, uint32_t& it)
   bar_consumers();
   int lastc = 0;
   if (tid == 0 && !C.ms->abort) {
-    __threadfence();
     const int pc = P.ctr_pair_base + t.layer * P.n_pairs + itm.pair;
     const uint32_t old = atom_add_acqrel(P.ctr + pc, 1u);
     lastc = (old == (uint32_t)itm.ns - 1) ? 1 : 0;
@@ -1889,7 +1887,6 @@ __device__ __noinline__ void attn_task(const Ctx& C, const Task t, uint32_t& it)
     }
     bar_consumers();
     if (tid == 0 && !C.ms->abort) {
-      __threadfence();
       red_release_add(P.ctr + t.layer * P.ctr_layer_stride + C_ATTN, 1u);
     }
     if (trc) C.ms->tr_epi += clock64() - tA;
