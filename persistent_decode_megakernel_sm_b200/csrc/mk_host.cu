@@ -565,7 +565,7 @@ mk_status mk_create(const mk_model_desc* desc, int device, mk_handle** out) {
     h->att_rows_max = mla ? Hq : MAXM * (Hq / G);
     h->att_dpart = mla ? R : hd;
     TRY(dalloc(h, (void**)&h->att_part,
-               (size_t)h->n_items_max * h->att_rows_max * (h->att_dpart + 2) * sizeof(float)));
+               (size_t)h->n_items_max * h->att_rows_max * (h->att_dpart + 4) * sizeof(float)));
     h->n_ctr = (L + 1) * NCTR_LAYER + L * h->max_pairs + 2;
     TRY(dalloc(h, (void**)&h->ctr, (size_t)h->n_ctr * sizeof(uint32_t)));
     TRY(dalloc(h, (void**)&h->status, 4 * sizeof(int32_t)));
@@ -1345,7 +1345,7 @@ extern "C" mk_status mk_decode_step_noalloc(mk_handle* h, const int32_t* tokens,
   const size_t o_ami = at;
   at = align256(at + (size_t)h->ncta * MAXM * sizeof(int32_t));
   const size_t o_att = at;
-  at = align256(at + (size_t)n_items * h->att_rows_max * (h->att_dpart + 2) * sizeof(float));
+  at = align256(at + (size_t)n_items * h->att_rows_max * (h->att_dpart + 4) * sizeof(float));
   const size_t o_ctr = at;
   at = align256(at + (size_t)h->n_ctr * sizeof(uint32_t));
   if (at > (size_t)MK_NOALLOC_SCRATCH_BYTES)

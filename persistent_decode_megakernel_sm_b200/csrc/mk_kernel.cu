@@ -1788,18 +1788,20 @@ __device__ __noinline__ void attn_task(const Ctx& C, const Task t, uint32_t& it)
   }
   bar_consumers();
   const int rows_max = P.att_rows_max;
-  float* part = P.att_part + (size_t)t.rt0 * rows_max * (d + 2);
+  // partial row: O (d values) | M | L | 2 pad  (16-byte rows for vector loads)
+  const int dP = d + 4;
+  float* part = P.att_part + (size_t)t.rt0 * rows_max * dP;
   if (tid < nr) {
     float l = 0.f;
     for (int w = 0; w < NCW; ++w) l += smx[w * 48 + tid];
-    part[(size_t)tid * (d + 2) + 1] = l;
+    part[(size_t)tid * dP + d + 1] = l;
   }
   if (warp == 0 && tq == 0) {
 #pragma unroll
     for (int mi = 0; mi < 3; ++mi)
       if (mi < mt) {
-        if (mi * 16 + g < nr) part[(size_t)(mi * 16 + g) * (d + 2)] = st.M[mi][0];
-        if (mi * 16 + g + 8 < nr) part[(size_t)(mi * 16 + g + 8) * (d + 2)] = st.M[mi][1];
+        if (mi * 16 + g < nr) part[(size_t)(mi * 16 + g) * dP + d] = st.M[mi][0];
+        if (mi * 16 + g + 8 < nr) part[(size_t)(mi * 16 + g + 8) * dP + d] = st.M[mi][1];
       }
   }
   {
@@ -1813,12 +1815,12 @@ __device__ __noinline__ void attn_task(const Ctx& C, const Task t, uint32_t& it)
             const int dim = (warp * per_w + jn) * 8 + 2 * tq;
             const int rA = mi * 16 + g, rB = rA + 8;
             if (rA < nr) {
-              part[(size_t)rA * (d + 2) + 2 + dim] = st.o[mi][jn][0];
-              part[(size_t)rA * (d + 2) + 3 + dim] = st.o[mi][jn][1];
+              part[(size_t)rA * dP + dim] = st.o[mi][jn][0];
+              part[(size_t)rA * dP + 1 + dim] = st.o[mi][jn][1];
             }
             if (rB < nr) {
-              part[(size_t)rB * (d + 2) + 2 + dim] = st.o[mi][jn][2];
-              part[(size_t)rB * (d + 2) + 3 + dim] = st.o[mi][jn][3];
+              part[(size_t)rB * dP + dim] = st.o[mi][jn][2];
+              part[(size_t)rB * dP + 1 + dim] = st.o[mi][jn][3];
             }
           }
         }
@@ -1854,7 +1856,7 @@ __device__ __noinline__ void attn_task(const Ctx& C, const Task t, uint32_t& it)
         mj[q] = -INFINITY;
         lj[q] = 0.f;
         if (jj < ns) {
-          const float* pp = P.att_part + ((size_t)(itm.first + jj) * rows_max + r) * (d + 2);
+          const float* pp = P.att_part + ((size_t)(itm.first + jj) * rows_max + r) * dP + d;
           mj[q] = __ldcg(pp);
           lj[q] = __ldcg(pp + 1);
         }
@@ -1875,15 +1877,25 @@ __device__ __noinline__ void attn_task(const Ctx& C, const Task t, uint32_t& it)
       }
     }
     bar_consumers();
-    for (int e = tid; e < nr * d; e += NCT) {
-      const int r = e / d, k = e % d;
+    // 4 consecutive dims per thread, the splits' loads 16 at a time in flight
+    const int d4 = d / 4;
+    for (int e = tid; e < nr * d4; e += NCT) {
+      const int r = e / d4, k = (e - r * d4) * 4;
       const float* wr = wsh + r * 160;
-      float num = 0.f;
-#pragma unroll 8
-      for (int jj = 0; jj < ns; ++jj)
-        num += wr[jj] * __ldcg(P.att_part + ((size_t)(itm.first + jj) * rows_max + r) * (d + 2) + 2 + k);
+      const float* src = P.att_part + ((size_t)itm.first * rows_max + r) * dP + k;
+      const size_t js = (size_t)rows_max * dP;
+      float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 16
+      for (int jj = 0; jj < ns; ++jj) {
+        const float w = wr[jj];
+        const float4 q = __ldcg(reinterpret_cast<const float4*>(src + jj * js));
+        num.x += w * q.x;
+        num.y += w * q.y;
+        num.z += w * q.z;
+        num.w += w * q.w;
+      }
       const int qi = r / gh, hh = r % gh;
-      out[(size_t)(s * Q + qi) * ldo + (size_t)(kvh * gh + hh) * d + k] = num;
+      *reinterpret_cast<float4*>(out + (size_t)(s * Q + qi) * ldo + (size_t)(kvh * gh + hh) * d + k) = num;
     }
     bar_consumers();
     if (tid == 0 && !C.ms->abort) {
@@ -2180,19 +2192,19 @@ __device__ __noinline__ void mla_task(const Ctx& C, const Task t, uint32_t& it) 
     }
   }
   bar_consumers();
-  const int rows_max = P.att_rows_max, dP = R + 2;
+  const int rows_max = P.att_rows_max, dP = R + 4;  // O (R) | M | L | 2 pad
   float* part = P.att_part + (size_t)t.rt0 * rows_max * dP;
   if (tid < Hq) {
     float l = 0.f;
     for (int w = 0; w < NCW; ++w) l += smx[w * 32 + tid];
-    part[(size_t)tid * dP + 1] = l;
+    part[(size_t)tid * dP + R + 1] = l;
   }
   if (warp == 0 && tq == 0) {
 #pragma unroll
     for (int mi = 0; mi < 2; ++mi)
       if (mi < mt) {
-        if (mi * 16 + g < Hq) part[(size_t)(mi * 16 + g) * dP] = st.M[mi][0];
-        if (mi * 16 + g + 8 < Hq) part[(size_t)(mi * 16 + g + 8) * dP] = st.M[mi][1];
+        if (mi * 16 + g < Hq) part[(size_t)(mi * 16 + g) * dP + R] = st.M[mi][0];
+        if (mi * 16 + g + 8 < Hq) part[(size_t)(mi * 16 + g + 8) * dP + R] = st.M[mi][1];
       }
   }
 #pragma unroll
@@ -2204,12 +2216,12 @@ __device__ __noinline__ void mla_task(const Ctx& C, const Task t, uint32_t& it) 
           const int dim = (warp * NTW + jn) * 8 + 2 * tq;
           const int rA = mi * 16 + g, rB = rA + 8;
           if (rA < Hq) {
-            part[(size_t)rA * dP + 2 + dim] = st.o[mi][jn][0];
-            part[(size_t)rA * dP + 3 + dim] = st.o[mi][jn][1];
+            part[(size_t)rA * dP + dim] = st.o[mi][jn][0];
+            part[(size_t)rA * dP + 1 + dim] = st.o[mi][jn][1];
           }
           if (rB < Hq) {
-            part[(size_t)rB * dP + 2 + dim] = st.o[mi][jn][2];
-            part[(size_t)rB * dP + 3 + dim] = st.o[mi][jn][3];
+            part[(size_t)rB * dP + dim] = st.o[mi][jn][2];
+            part[(size_t)rB * dP + 1 + dim] = st.o[mi][jn][3];
           }
         }
       }
@@ -2235,7 +2247,7 @@ __device__ __noinline__ void mla_comb_task(const Ctx& C, const Task t) {
   const Launch& P = *C.P;
   const Model& md = *C.md;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int Hq = md.Hq, R = md.R, dP = R + 2, rows_max = P.att_rows_max;
+  const int Hq = md.Hq, R = md.R, dP = R + 4, rows_max = P.att_rows_max;
   const int64_t total = (int64_t)P.n_pairs * Hq * R;
   const int64_t o0 = total * blockIdx.x / gridDim.x, o1 = total * (blockIdx.x + 1) / gridDim.x;
   if (o0 >= o1) return;
@@ -2258,7 +2270,7 @@ __device__ __noinline__ void mla_comb_task(const Ctx& C, const Task t) {
         mj[q] = -INFINITY;
         lj[q] = 0.f;
         if (jj < ns) {
-          const float* pp = P.att_part + ((size_t)(itm.first + jj) * rows_max + h) * dP;
+          const float* pp = P.att_part + ((size_t)(itm.first + jj) * rows_max + h) * dP + R;
           mj[q] = __ldcg(pp);
           lj[q] = __ldcg(pp + 1);
         }
@@ -2284,7 +2296,7 @@ __device__ __noinline__ void mla_comb_task(const Ctx& C, const Task t) {
       const int pair = rr / Hq, h = rr - pair * Hq;
       const Item itm = decode_item(pair_first_item(pair, P.n_pairs, P.n_items), P.n_pairs, P.n_items);
       const float* wr = wsh + (rr - rb) * 160;
-      const float* src = P.att_part + ((size_t)itm.first * rows_max + h) * dP + 2 + k;
+      const float* src = P.att_part + ((size_t)itm.first * rows_max + h) * dP + k;
       const size_t js = (size_t)rows_max * dP;
       float num = 0.f;
 #pragma unroll 16
