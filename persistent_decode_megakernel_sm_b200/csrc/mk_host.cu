@@ -19,7 +19,7 @@
 #include "mk_internal.h"
 
 namespace mk {
-template <bool MLA>
+template <bool MLA, bool MOE>
 __global__ void mk_step_kernel(const __grid_constant__ Launch P);
 }
 
@@ -246,7 +246,7 @@ struct mk_handle {
   bool sticky = false;
   bool initialised = false;
   uint64_t noalloc_id = 0;  // identity of this handle for mk_decode_step_noalloc's installed task list
-  const void* kernel = nullptr;  // the step kernel instance of this model's attention family
+  const void* kernel = nullptr;  // the step kernel instance of this model's family
   std::string err;
 };
 
@@ -575,7 +575,11 @@ mk_status mk_create(const mk_model_desc* desc, int device, mk_handle** out) {
       s = MK_ERR_CUDA;
       goto fail_out;
     }
-    h->kernel = d.kv_lora_rank > 0 ? (const void*)mk_step_kernel<true> : (const void*)mk_step_kernel<false>;
+    {
+      const bool mla = d.kv_lora_rank > 0, moe = d.n_routed > 0;
+      h->kernel = mla ? (moe ? (const void*)mk_step_kernel<true, true> : (const void*)mk_step_kernel<true, false>)
+                      : (moe ? (const void*)mk_step_kernel<false, true> : (const void*)mk_step_kernel<false, false>);
+    }
     if (cudaFuncSetAttribute(h->kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess) {
       s = MK_ERR_CUDA;
       h->err = "cannot reserve dynamic shared memory";

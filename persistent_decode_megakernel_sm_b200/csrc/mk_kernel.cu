@@ -188,10 +188,13 @@ struct Misc {
   int pad[2];
   // MoE routing tables, one per role (each role computes its own copy)
   int rt_u[3];
+  int route_layer;  // layer + 1 of the route the activation producer last published
   int16_t rt_ex[3][64];
+  int16_t rt_sel[3][MAXM * 8];  // each row's picks in top-k order, per role
+  float rt_selw[MAXM][8];       // consumers: their renormalised weights
   float rt_w[64][MAXM];      // consumers: weight of (union slot, row)
   // per-task trace accumulators (consumer thread 0)
-  long long tr_wf, tr_wx, tr_bytes;
+  long long tr_wf, tr_wx, tr_bytes, tr_route;
   long long tr_frag, tr_mma, tr_epi, tr_rel, tr_loop, tr_pre, tr_post, tr_sig;
   int tr_chunks;
 };
@@ -316,72 +319,69 @@ __device__ __forceinline__ int att_pitch(int d) { return d * 2; }
 // warp; every role that needs the result computes it itself from the same
 // logits with the same code, so all roles agree.
 // ---------------------------------------------------------------------------
-enum RouteRole { RR_CONS = 0, RR_PROD = 1, RR_XPROD = 2 };
+enum RouteRole { RR_CONS = 0, RR_PROD = 1, RR_XPROD = 2 };  // RR_XPROD's tables also serve the consumers
 
-__device__ int moe_route(const Launch& P, const Model& md, int layer, Misc* ms, int role, bool want_w, bool trace) {
+__device__ __noinline__ int moe_route(const Launch& P, const Model& md, int layer, Misc* ms, int role, bool want_w,
+                                      bool trace) {
+  // Compact on purpose (a runtime loop over rows, one out-of-line copy for
+  // the three roles): it runs once per layer, so its instruction fetch is
+  // cold every time and dominates its cost.
   const int lane = threadIdx.x & 31;
   const int E = md.E, K = md.K, M = P.M;
   const float* rl = P.buf[B_RLOG];
   const int ld = P.ld[B_RLOG];
+  int16_t* sel = ms->rt_sel[role];
   uint32_t ubits = 0;  // bit q: expert lane + 32 q picked by some row
-  int selE[MAXM];
-  float selW[MAXM];
+#pragma unroll 1
+  for (int mm = 0; mm < M; ++mm) {
+    float v[8];
+    float mx = -INFINITY;
 #pragma unroll
-  for (int mm = 0; mm < MAXM; ++mm) {
-    selE[mm] = -1;
-    selW[mm] = 0.f;
-    if (mm < M) {
-      float v[8];
-      float mx = -INFINITY;
+    for (int q = 0; q < 8; ++q) {
+      const int e = lane + 32 * q;
+      v[q] = e < E ? __ldcg(rl + (size_t)mm * ld + e) : -INFINITY;
+      mx = fmaxf(mx, v[q]);
+    }
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float sum = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) sum += expf(v[q] - mx);  // -inf lanes add 0
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    float psum = 0.f, my_p = 0.f;
+#pragma unroll 1
+    for (int j = 0; j < K; ++j) {
+      float bv = -INFINITY;
+      int be = 0x7fffffff;
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         const int e = lane + 32 * q;
-        v[q] = e < E ? __ldcg(rl + (size_t)mm * ld + e) : -INFINITY;
-        mx = fmaxf(mx, v[q]);
-      }
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      float sum = 0.f;
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        if (lane + 32 * q < E) sum += expf(v[q] - mx);
-      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      float psum = 0.f, my_p = 0.f;
-      int my_e = -1;
-      for (int j = 0; j < K; ++j) {
-        float bv = -INFINITY;
-        int be = 0x7fffffff;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int e = lane + 32 * q;
-          if (e < E && (v[q] > bv || (v[q] == bv && e < be))) {
-            bv = v[q];
-            be = e;
-          }
-        }
-        for (int o = 16; o > 0; o >>= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-          const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-          if (ov > bv || (ov == bv && oe < be)) {
-            bv = ov;
-            be = oe;
-          }
-        }
-        const float pj = expf(bv - mx) / sum;
-        psum += pj;
-        if (lane == j) {
-          my_e = be;
-          my_p = pj;
-        }
-        if ((be & 31) == lane) {
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            if (q == (be >> 5)) v[q] = -INFINITY;
-          ubits |= 1u << (be >> 5);
+        if (v[q] > bv || (v[q] == bv && e < be)) {
+          bv = v[q];
+          be = e;
         }
       }
-      selE[mm] = my_e;
-      selW[mm] = my_p / psum;
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        if (ov > bv || (ov == bv && oe < be)) {
+          bv = ov;
+          be = oe;
+        }
+      }
+      const float pj = expf(bv - mx) / sum;
+      psum += pj;
+      if (lane == j) {
+        sel[mm * 8 + j] = (int16_t)be;
+        my_p = pj;
+      }
+      if ((be & 31) == lane) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (q == (be >> 5)) v[q] = -INFINITY;
+        ubits |= 1u << (be >> 5);
+      }
     }
+    if (want_w && lane < K) ms->rt_selw[mm][lane] = my_p / psum;
   }
   // union in ascending expert order
   int U = 0;
@@ -397,16 +397,16 @@ __device__ int moe_route(const Launch& P, const Model& md, int layer, Misc* ms, 
   if (want_w) {
     for (int i = lane; i < 64 * MAXM; i += 32) ms->rt_w[i / MAXM][i % MAXM] = 0.f;
     __syncwarp();
-#pragma unroll
-    for (int mm = 0; mm < MAXM; ++mm) {
-      if (mm < M && lane < K) {
-        int slot = 0;
-        while (slot < U && ex[slot] != selE[mm]) ++slot;
-        ms->rt_w[slot][mm] = selW[mm];
-        if (trace && P.router_idx) {
-          P.router_idx[((size_t)layer * M + mm) * K + lane] = selE[mm];
-          P.router_w[((size_t)layer * M + mm) * K + lane] = selW[mm];
-        }
+    for (int i = lane; i < M * K; i += 32) {
+      const int mm = i / K, j = i - mm * K;
+      const int e = sel[mm * 8 + j];
+      const float w = ms->rt_selw[mm][j];
+      int slot = 0;
+      while (slot < U && ex[slot] != e) ++slot;
+      ms->rt_w[slot][mm] = w;
+      if (trace && P.router_idx) {
+        P.router_idx[((size_t)layer * M + mm) * K + j] = e;
+        P.router_w[((size_t)layer * M + mm) * K + j] = w;
       }
     }
     __syncwarp();
@@ -454,6 +454,7 @@ struct PieceSrc {
   int xcol0;  // first activation column (per-head groups of the latent-attention projections)
 };
 
+template <bool MOE>
 __device__ __forceinline__ PieceSrc piece_src(const Model& md, const Task& t, const Mat& m, const Mat& m2,
                                               const int16_t* ex, const Pieces& pc) {
   PieceSrc r;
@@ -463,13 +464,13 @@ __device__ __forceinline__ PieceSrc piece_src(const Model& md, const Task& t, co
   r.xbuf = t.in_kind == IN_X_NORM ? (int)B_X : (int)t.in_buf;
   r.w = m.w;
   r.scales = m.scales;
-  if (t.type == T_MOE_GU) {
+  if (MOE && t.type == T_MOE_GU) {
     const int slot = pc.g0 / m.RT;
     const int e = t.moe == 1 ? slot : ex[slot];
     r.w = m.w + (size_t)e * m.estride;
     r.scales = m.scales ? m.scales + (size_t)e * m.sstride : nullptr;
     r.lg0 = pc.g0 - slot * m.RT;
-  } else if (t.type == T_MOE_DOWN) {
+  } else if (MOE && t.type == T_MOE_DOWN) {
     const int ns = md.NS;
     const Mat& mm = pc.seg < ns ? m2 : m;
     const int e = pc.seg < ns ? pc.seg : ex[pc.seg - ns];
@@ -482,29 +483,32 @@ __device__ __forceinline__ PieceSrc piece_src(const Model& md, const Task& t, co
 }
 
 // Row range, expert-group size and K-segment count of a GEMV-like task.
+template <bool MOE>
 __device__ __forceinline__ void task_rows(const Model& md, const Task& t, const Mat& m, int U, int& rt0, int& rt1,
                                           int& gsz, int& nseg) {
   rt0 = t.rt0;
   rt1 = t.rt1;
   gsz = t.xg_rt > 0 ? t.xg_rt : 0;
   nseg = 1;
-  if (t.type == T_MOE_GU) {
+  if (MOE && t.type == T_MOE_GU) {
     gsz = m.RT;
     if (t.moe == 2) {
       const int T = U * m.RT;
       rt0 = (int)(((int64_t)blockIdx.x * T) / gridDim.x);
       rt1 = (int)(((int64_t)(blockIdx.x + 1) * T) / gridDim.x);
     }
-  } else if (t.type == T_MOE_DOWN) {
+  } else if (MOE && t.type == T_MOE_DOWN) {
     nseg = md.NS + U;
   }
 }
 
+template <bool MOE>
 __device__ __forceinline__ bool task_needs_route(const Task& t) {
-  return (t.type == T_MOE_GU && t.moe == 2) || t.type == T_MOE_DOWN;
+  return MOE && ((t.type == T_MOE_GU && t.moe == 2) || t.type == T_MOE_DOWN);
 }
+template <bool MOE>
 __device__ __forceinline__ bool gemv_like(const Task& t) {
-  return t.type == T_GEMV || t.type == T_MOE_GU || t.type == T_MOE_DOWN;
+  return t.type == T_GEMV || (MOE && (t.type == T_MOE_GU || t.type == T_MOE_DOWN));
 }
 
 // ---------------------------------------------------------------------------
@@ -589,7 +593,7 @@ struct Chunk {
 // Walks a CTA's task list and yields its chunks in consumption order (the
 // enumeration the consumers use).  Routed-expert tasks first wait for the
 // router's counter: their tiles are the only ones that depend on activations.
-template <bool MLA>
+template <bool MLA, bool MOE>
 struct ChunkStream {
   int ti, end, state;  // state 0: next task, 1: GEMV-like pieces, 2: attention, 3: latent attention
   Task t;
@@ -624,7 +628,7 @@ struct ChunkStream {
           if (!pc.next()) {
             state = 0;
           } else {
-            src = piece_src(md, t, m, m2, C.ms->rt_ex[RR_PROD], pc);
+            src = piece_src<MOE>(md, t, m, m2, C.ms->rt_ex[RR_PROD], pc);
             ci.init(src.lg0, src.lg0 + pc.nr, m.KT, tb, 0, xcap);
           }
         }
@@ -655,20 +659,20 @@ struct ChunkStream {
       }
       if (ti >= end) return 0;
       t = P.tasks[ti++];
-      if (gemv_like(t)) {
+      if (gemv_like<MOE>(t)) {
         m = t.m;
-        m2 = (t.type == T_MOE_DOWN && t.mat2 >= 0) ? md.mats[t.mat2] : m;
+        m2 = (MOE && t.type == T_MOE_DOWN && t.mat2 >= 0) ? md.mats[t.mat2] : m;
         tb = m.fp8 ? TILE_FP8 : TILE_BF16;
         xcap = x_cap(t, P.M);
         int U = 0;
-        if (task_needs_route(t)) {
+        if (task_needs_route<MOE>(t)) {
           if (!warp_wait_counter(C, t.layer * P.ctr_layer_stride + C_ROUTER, (uint32_t)gridDim.x, 0x70000)) return -1;
           U = moe_route(P, md, t.layer, C.ms, RR_PROD, false, false);
         }
         int rt0, rt1, gsz, nseg;
-        task_rows(md, t, m, U, rt0, rt1, gsz, nseg);
+        task_rows<MOE>(md, t, m, U, rt0, rt1, gsz, nseg);
         if (pc.init(rt0, rt1, gsz, nseg)) {
-          src = piece_src(md, t, m, m2, C.ms->rt_ex[RR_PROD], pc);
+          src = piece_src<MOE>(md, t, m, m2, C.ms->rt_ex[RR_PROD], pc);
           ci.init(src.lg0, src.lg0 + pc.nr, m.KT, tb, 0, xcap);
           state = 1;
         }
@@ -698,7 +702,7 @@ struct ChunkStream {
   }
 };
 
-template <bool MLA>
+template <bool MLA, bool MOE>
 __device__ void producer(const Ctx& C) {
   const Launch& P = *C.P;
   const int lane = threadIdx.x & 31;
@@ -708,7 +712,7 @@ __device__ void producer(const Ctx& C) {
   long long blocked = 0;
   const uint64_t t_first = globaltimer();
   const long long c_first = clock64();
-  ChunkStream<MLA> is;
+  ChunkStream<MLA, MOE> is;
   is.init(beg, end);
   Chunk c;
   while (is.next(C, c) > 0) {
@@ -863,6 +867,7 @@ __device__ bool xprod_reserve(const Ctx& C, uint32_t ix, uint32_t bytes) {
   return ok != 0;
 }
 
+template <bool MOE>
 __device__ void xproducer(const Ctx& C) {
   const Launch& P = *C.P;
   const Model& md = *C.md;
@@ -874,16 +879,29 @@ __device__ void xproducer(const Ctx& C) {
   if (P.stall_ctr >= 0) return;
   for (int ti = beg; ti < end; ++ti) {
     const Task t = P.tasks[ti];
-    if (!gemv_like(t)) continue;
+    if (!gemv_like<MOE>(t)) continue;
     const Mat m = t.m;
-    const Mat m2 = (t.type == T_MOE_DOWN && t.mat2 >= 0) ? md.mats[t.mat2] : m;
+    const Mat m2 = (MOE && t.type == T_MOE_DOWN && t.mat2 >= 0) ? md.mats[t.mat2] : m;
     const int tb = m.fp8 ? TILE_FP8 : TILE_BF16;
     const int xcap = x_cap(t, M);
     if (t.wait_ctr >= 0 && !warp_wait_counter(C, t.wait_ctr, (uint32_t)t.wait_tgt, 0x30000)) goto drain;
     int U = 0;
-    if (task_needs_route(t)) U = moe_route(P, md, t.layer, C.ms, RR_XPROD, false, false);
+    if (task_needs_route<MOE>(t)) {
+      if (t.type == T_MOE_GU) {
+        // the layer's route, with the routed weights, for this warp and for
+        // the consumers (published through shared memory)
+        U = moe_route(P, md, t.layer, C.ms, RR_XPROD, true, blockIdx.x == 0);
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence_block();
+          *reinterpret_cast<volatile int*>(&C.ms->route_layer) = t.layer + 1;
+        }
+      } else {
+        U = C.ms->rt_u[RR_XPROD];  // the down projection of the same layer: same route
+      }
+    }
     int rt0, rt1, gsz, nseg;
-    task_rows(md, t, m, U, rt0, rt1, gsz, nseg);
+    task_rows<MOE>(md, t, m, U, rt0, rt1, gsz, nseg);
     Pieces pc;
     if (!pc.init(rt0, rt1, gsz, nseg)) continue;
     // RMSNorm scale of every activation row (fixed-order reduction of the
@@ -896,7 +914,7 @@ __device__ void xproducer(const Ctx& C) {
 #pragma unroll
     for (int mm = 0; mm < MAXM; ++mm) scale[mm] = 1.f;
     do {
-      const PieceSrc src = piece_src(md, t, m, m2, C.ms->rt_ex[RR_XPROD], pc);
+      const PieceSrc src = piece_src<MOE>(md, t, m, m2, C.ms->rt_ex[RR_XPROD], pc);
       ChunkIt ci;
       ci.init(src.lg0, src.lg0 + pc.nr, m.KT, tb, 0, xcap);
       do {
@@ -1213,6 +1231,7 @@ __device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
   ixr = ix;
 }
 
+template <bool MOE>
 __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix) {
   const Launch& P = *C.P;
   const long long tpre = (P.trace && threadIdx.x == 0) ? clock64() : 0;
@@ -1232,15 +1251,28 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
 
   // MoE: this task's rows / K segments follow the router's union of experts
   int U = 0;
-  if (task_needs_route(t)) {
-    if (warp == 0)
-      moe_route(P, md, t.layer, C.ms, RR_CONS, t.type == T_MOE_GU, blockIdx.x == 0 && t.type == T_MOE_GU);
+  if (task_needs_route<MOE>(t)) {
+    // the activation producer publishes the layer's route (it waits on the
+    // router's counter anyway); the consumers only check that it is there
+    const long long tr0 = (P.trace && tid == 0) ? clock64() : 0;
+    if (tid == 0) {
+      const uint64_t t0 = globaltimer();
+      while (*reinterpret_cast<volatile int*>(&C.ms->route_layer) != t.layer + 1) {
+        if (C.ms->abort) break;
+        if (globaltimer() - t0 > (uint64_t)P.timeout_ns * 2) {
+          raise_error(P, C.ms, DERR_TIMEOUT, 0x80000 | t.layer);
+          break;
+        }
+      }
+      __threadfence_block();
+    }
+    if (P.trace && tid == 0) C.ms->tr_route += clock64() - tr0;
     bar_consumers();
-    U = C.ms->rt_u[RR_CONS];
+    U = C.ms->rt_u[RR_XPROD];
   }
-  const Mat m2 = (t.type == T_MOE_DOWN && t.mat2 >= 0) ? md.mats[t.mat2] : m;
+  const Mat m2 = (MOE && t.type == T_MOE_DOWN && t.mat2 >= 0) ? md.mats[t.mat2] : m;
   int rt0, rt1, gsz, nseg;
-  task_rows(md, t, m, U, rt0, rt1, gsz, nseg);
+  task_rows<MOE>(md, t, m, U, rt0, rt1, gsz, nseg);
   Pieces pc;
   bool have = pc.init(rt0, rt1, gsz, nseg);
   const int xcap = x_cap(t, M);
@@ -1258,11 +1290,11 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
   L.gain = t.gvec;
   if (L.trc) C.ms->tr_pre += clock64() - tpre;
   while (have) {
-    const PieceSrc src = piece_src(md, t, m, m2, C.ms->rt_ex[RR_CONS], pc);
+    const PieceSrc src = piece_src<MOE>(md, t, m, m2, C.ms->rt_ex[RR_XPROD], pc);
     ChunkIt ci;
     ci.init(src.lg0, src.lg0 + pc.nr, m.KT, tb, 0, xcap);
     L.rowbytes = x_rowbytes(t, ci.WC);
-    Mat mg = (t.type == T_MOE_DOWN && pc.seg < md.NS) ? m2 : m;
+    Mat mg = (MOE && t.type == T_MOE_DOWN && pc.seg < md.NS) ? m2 : m;
     mg.w = src.w;
     mg.scales = src.scales;
     const bool accum = pc.seg > 0;
@@ -1339,7 +1371,7 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
                 ss_acc[q & 1] += nv * nv;
               }
             }
-          } else if (t.epi == EPI_SWIGLU_MOE) {
+          } else if (MOE && t.epi == EPI_SWIGLU_MOE) {
             // virtual row tile rt of expert slot rt / RTe (shared slots first)
             const int slot = rt / m.RT;
             const int hs = (t.moe == 1 ? 0 : md.NS) + slot;
@@ -2310,7 +2342,7 @@ __device__ __noinline__ void mla_comb_task(const Ctx& C, const Task t) {
 // ---------------------------------------------------------------------------
 // consumer warps
 // ---------------------------------------------------------------------------
-template <bool MLA>
+template <bool MLA, bool MOE>
 __device__ void consumer(const Ctx& C) {
   const Launch& P = *C.P;
   uint32_t it = 0, ix = 0;
@@ -2340,12 +2372,13 @@ __device__ void consumer(const Ctx& C) {
       C.ms->tr_wf = C.ms->tr_wx = C.ms->tr_bytes = 0;
       C.ms->tr_frag = C.ms->tr_mma = C.ms->tr_epi = C.ms->tr_rel = 0;
       C.ms->tr_loop = C.ms->tr_pre = C.ms->tr_post = C.ms->tr_sig = 0;
+      C.ms->tr_route = 0;
       C.ms->tr_chunks = 0;
     }
     if (t.wait_ctr >= 0) wait_counter(C, t.wait_ctr, (uint32_t)t.wait_tgt);
     if (tr) td = globaltimer();
-    if (gemv_like(t)) {
-      gemv_task(C, t, it, ix);
+    if (gemv_like<MOE>(t)) {
+      gemv_task<MOE>(C, t, it, ix);
     } else if (!MLA && t.type == T_ATTN) {
       attn_task(C, t, it);
     } else if (MLA && t.type == T_MLA) {
@@ -2377,6 +2410,7 @@ __device__ void consumer(const Ctx& C) {
       rec[17] = C.ms->tr_pre;
       rec[18] = C.ms->tr_post;
       rec[19] = C.ms->tr_sig;
+      if (ti - beg >= 2) rec[12] = C.ms->tr_route;  // records 0 and 1 carry the producer's counters there
     }
   }
 }
@@ -2384,10 +2418,10 @@ __device__ void consumer(const Ctx& C) {
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
-// One instance per attention family (GQA or latent): each kernel holds only
+// One instance per model family (GQA or latent attention, dense or MoE FFN): each kernel holds only
 // the code its models run, which keeps the instruction footprint of the
 // whole-step loop small.
-template <bool MLA>
+template <bool MLA, bool MOE>
 __global__ void __launch_bounds__(NTHREADS, 1) mk_step_kernel(const __grid_constant__ Launch P) {
   extern __shared__ __align__(128) uint8_t smem[];
   Ctx C;
@@ -2429,13 +2463,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) mk_step_kernel(const __grid_const
       mbar_init(&C.ms->xempty[s], NCW);
     }
     C.ms->abort = 0;
+    C.ms->route_layer = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
 
-  if ((tid >> 5) == WARP_WP) producer<MLA>(C);
-  else if ((tid >> 5) == WARP_XP) xproducer(C);
-  else consumer<MLA>(C);
+  if ((tid >> 5) == WARP_WP) producer<MLA, MOE>(C);
+  else if ((tid >> 5) == WARP_XP) xproducer<MOE>(C);
+  else consumer<MLA, MOE>(C);
   __syncthreads();
 
   // ---- teardown: the last CTA out zeroes every counter for the next launch ----
@@ -2455,7 +2490,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) mk_step_kernel(const __grid_const
   }
 }
 
-template __global__ void mk_step_kernel<false>(const __grid_constant__ Launch P);
-template __global__ void mk_step_kernel<true>(const __grid_constant__ Launch P);
+template __global__ void mk_step_kernel<false, false>(const __grid_constant__ Launch P);
+template __global__ void mk_step_kernel<false, true>(const __grid_constant__ Launch P);
+template __global__ void mk_step_kernel<true, false>(const __grid_constant__ Launch P);
+template __global__ void mk_step_kernel<true, true>(const __grid_constant__ Launch P);
 
 }  // namespace mk
