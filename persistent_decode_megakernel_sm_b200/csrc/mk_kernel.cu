@@ -117,6 +117,15 @@ __device__ __forceinline__ uint32_t lds32(const void* p) {
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)));
   return v;
 }
+// Two 8x8 bf16 matrices, transposed: with rows = positions of a row-major
+// [position][dim] tile, thread (g, tq) receives the mma B fragment
+// {V[2tq][g], V[2tq+1][g]} of matrix 0 (rows 0-7) and of matrix 1 (rows 8-15).
+// Lanes 0-15 give the row addresses (16-byte aligned).
+__device__ __forceinline__ void ldsm_x2_trans(const void* row_addr, uint32_t& b0, uint32_t& b1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+               : "=r"(b0), "=r"(b1)
+               : "r"(smem_u32(row_addr)));
+}
 __device__ __forceinline__ uint32_t lds16(const void* p) {
   uint16_t v;
   asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(smem_u32(p)));
@@ -310,6 +319,9 @@ __device__ __forceinline__ int seq_pos0(const Launch& P, int s) {
   return P.positions ? __ldg(P.positions + s) : P.pos_const;
 }
 
+// K / V rows in shared memory, unpadded: a chunk's rows are contiguous in the
+// cache and arrive as one bulk copy each for K and V (per-row copies into
+// padded rows avoid bank conflicts but cost more in copy issue than they save).
 __device__ __forceinline__ int att_pitch(int d) { return d * 2; }
 
 // ---------------------------------------------------------------------------
@@ -1671,13 +1683,16 @@ __device__ void att_chunk(const Ctx& C, AttState& st, const uint8_t* Ks, const u
 #pragma unroll
     for (int jn = 0; jn < 2; ++jn) {
       if (jn < per_w) {
-        const int dim = (warp * per_w + jn) * 8 + g;
-        const uint8_t* vc = Vs + dim * 2;
-        const uint32_t v0 = pk < n_valid ? lds16(vc + (size_t)pk * pitch) : 0u;
-        const uint32_t v1 = pk + 1 < n_valid ? lds16(vc + (size_t)(pk + 1) * pitch) : 0u;
-        const uint32_t v8 = pk + 8 < n_valid ? lds16(vc + (size_t)(pk + 8) * pitch) : 0u;
-        const uint32_t v9 = pk + 9 < n_valid ? lds16(vc + (size_t)(pk + 9) * pitch) : 0u;
-        const uint32_t b0 = v0 | (v1 << 16), b1 = v8 | (v9 << 16);
+        // rows ks*16 .. ks*16+15 of this warp's 8 dims; rows past n_valid may
+        // hold anything (even NaN), so their values are zeroed, not just
+        // weighted by P = 0
+        const int dim0 = (warp * per_w + jn) * 8;
+        uint32_t b0, b1;
+        ldsm_x2_trans(Vs + (size_t)(ks * 16 + (lane & 15)) * pitch + dim0 * 2, b0, b1);
+        if (pk >= n_valid) b0 = 0u;
+        else if (pk + 1 >= n_valid) b0 &= 0xFFFFu;
+        if (pk + 8 >= n_valid) b1 = 0u;
+        else if (pk + 9 >= n_valid) b1 &= 0xFFFFu;
 #pragma unroll
         for (int mi = 0; mi < 3; ++mi) {
           if (mi < mt) {
