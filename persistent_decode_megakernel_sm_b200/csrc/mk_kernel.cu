@@ -1131,6 +1131,31 @@ struct GemvLane {
 // j = warp + 8 i of every chunk, builds the activation fragment (hi/lo) of
 // each and runs NR independent accumulator chains; the per-warp partial sums
 // are left in `red` for the cross-warp reduction.
+// acc += block scale * raw for col block cb of the rows of row tiles g0.. (raw
+// is cleared).  Gate / up interleaved tiles take the gate scale for rows
+// 0-7 and the up scale for rows 8-15 of each tile.
+template <int NR>
+__device__ __forceinline__ void fp8_apply_scales(const Mat& m, int g0, int cb, float (&raw)[NR][4],
+                                                 float (&acc)[NR][4]) {
+#pragma unroll
+  for (int r = 0; r < NR; ++r) {
+    const int rt = g0 + r;
+    float s_top, s_bot;
+    if (m.gu) {
+      const int rb = rt >> 4;
+      s_top = __ldg(m.scales + rb * m.nbc + cb);
+      s_bot = __ldg(m.scales + (size_t)m.nbr * m.nbc + rb * m.nbc + cb);
+    } else {
+      s_top = s_bot = __ldg(m.scales + (rt >> 3) * m.nbc + cb);
+    }
+    acc[r][0] += s_top * raw[r][0];
+    acc[r][1] += s_top * raw[r][1];
+    acc[r][2] += s_bot * raw[r][2];
+    acc[r][3] += s_bot * raw[r][3];
+    raw[r][0] = raw[r][1] = raw[r][2] = raw[r][3] = 0.f;
+  }
+}
+
 template <int NR, bool FP8>
 __device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& mr, const GemvLane& Lr, uint32_t& itr,
                                         uint32_t& ixr, float* red, bool accum) {
@@ -1167,10 +1192,10 @@ __device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
     if (L.trc) tc0 = clock64();
     // kept rolled: the instruction working set of the whole kernel must stay
     // small (one CTA executes every phase of every layer)
+    if (!FP8) {
 #pragma unroll 1
-    for (int j = L.warp; j < nc; j += NCW) {
-      const uint4 xf = xok ? lds128(xs + j * 64) : make_uint4(0u, 0u, 0u, 0u);
-      if (!FP8) {
+      for (int j = L.warp; j < nc; j += NCW) {
+        const uint4 xf = xok ? lds128(xs + j * 64) : make_uint4(0u, 0u, 0u, 0u);
         uint4 a[NR];
 #pragma unroll
         for (int r = 0; r < NR; ++r) a[r] = lds128(stage + ((size_t)r * nc + j) * TILE_BF16 + lane * 16);
@@ -1178,32 +1203,36 @@ __device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
         for (int r = 0; r < NR; ++r) mma_bf16(acc[r], a[r], xf.x, xf.y);
 #pragma unroll
         for (int r = 0; r < NR; ++r) mma_bf16(acc[r], a[r], xf.z, xf.w);
-      } else {
-        const int c = ci.c0 + j;
+      }
+    } else {
+      // fp8: each warp takes a contiguous run of the chunk's col tiles and
+      // sums raw products per 128-column scale block, applying the block's
+      // scale once per block rather than once per tile
+      const int per = (nc + NCW - 1) / NCW;
+      const int j0 = min(nc, L.warp * per), j1 = min(nc, j0 + per);
+      float raw[NR][4];
+#pragma unroll
+      for (int r = 0; r < NR; ++r) raw[r][0] = raw[r][1] = raw[r][2] = raw[r][3] = 0.f;
+      int cb = (ci.c0 + j0) >> 3;
+#pragma unroll 1
+      for (int j = j0; j < j1; ++j) {
+        const int cbj = (ci.c0 + j) >> 3;
+        if (cbj != cb) {
+          fp8_apply_scales<NR>(m, ci.g0, cb, raw, acc);
+          cb = cbj;
+        }
+        const uint4 xf = xok ? lds128(xs + j * 64) : make_uint4(0u, 0u, 0u, 0u);
         uint2 a8[NR];
 #pragma unroll
         for (int r = 0; r < NR; ++r) a8[r] = lds64(stage + ((size_t)r * nc + j) * TILE_FP8 + lane * 8);
 #pragma unroll
         for (int r = 0; r < NR; ++r) {
           const uint4 af = fp8_frag_to_f16(a8[r]);
-          float tmp[4] = {0.f, 0.f, 0.f, 0.f};
-          mma_f16(tmp, af, xf.x, xf.y);
-          mma_f16(tmp, af, xf.z, xf.w);
-          const int rt = ci.g0 + r;
-          float s_top, s_bot;
-          if (m.gu) {
-            const int rb = rt >> 4;
-            s_top = __ldg(m.scales + rb * m.nbc + (c >> 3));
-            s_bot = __ldg(m.scales + (size_t)m.nbr * m.nbc + rb * m.nbc + (c >> 3));
-          } else {
-            s_top = s_bot = __ldg(m.scales + (rt >> 3) * m.nbc + (c >> 3));
-          }
-          acc[r][0] += s_top * tmp[0];
-          acc[r][1] += s_top * tmp[1];
-          acc[r][2] += s_bot * tmp[2];
-          acc[r][3] += s_bot * tmp[3];
+          mma_f16(raw[r], af, xf.x, xf.y);
+          mma_f16(raw[r], af, xf.z, xf.w);
         }
       }
+      if (j0 < j1) fp8_apply_scales<NR>(m, ci.g0, cb, raw, acc);
     }
     if (L.trc) {
       float sink = 0.f;
