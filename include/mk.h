@@ -207,6 +207,8 @@ int64_t mk_weight_bytes(const mk_handle* h);
  * MK_ERR_DEVICE_TIMEOUT through mk_sync_status.  0 disables. */
 mk_status mk_debug_inject_stall(mk_handle* h, int64_t timeout_ns);
 
+/* The description of h's last failure; with h == NULL, why the calling
+ * thread's last mk_create failed. */
 const char* mk_last_error(const mk_handle* h);
 void mk_kv_destroy(mk_kv* kv);
 void mk_destroy(mk_handle* h);

@@ -19,8 +19,7 @@
 #include "mk_internal.h"
 
 namespace mk {
-template <bool MLA, bool MOE>
-__global__ void mk_step_kernel(const __grid_constant__ Launch P);
+const void* step_kernel_for(bool mla, bool moe);  // the kernel instance of a model family
 }
 
 using namespace mk;
@@ -258,6 +257,9 @@ struct mk_kv {
   int64_t bytes = 0;
 };
 
+// Why the calling thread's last mk_create failed (it returns no handle).
+static thread_local std::string g_create_error = "null handle";
+
 static mk_status fail(mk_handle* h, mk_status s, const std::string& msg) {
   if (h) h->err = msg;
   return s;
@@ -364,7 +366,10 @@ mk_status mk_create(const mk_model_desc* desc, int device, mk_handle** out) {
   if (!out) return MK_ERR_INVALID;
   *out = nullptr;
   std::string why;
-  if (!desc_ok(desc, why)) return MK_ERR_INVALID;
+  if (!desc_ok(desc, why)) {
+    g_create_error = "invalid model description: " + why;
+    return MK_ERR_INVALID;
+  }
   mk_handle* h = new mk_handle();
   h->desc = *desc;
   h->device = device;
@@ -575,21 +580,18 @@ mk_status mk_create(const mk_model_desc* desc, int device, mk_handle** out) {
       s = MK_ERR_CUDA;
       goto fail_out;
     }
-    {
-      const bool mla = d.kv_lora_rank > 0, moe = d.n_routed > 0;
-      h->kernel = mla ? (moe ? (const void*)mk_step_kernel<true, true> : (const void*)mk_step_kernel<true, false>)
-                      : (moe ? (const void*)mk_step_kernel<false, true> : (const void*)mk_step_kernel<false, false>);
-    }
+    h->kernel = step_kernel_for(d.kv_lora_rank > 0, d.n_routed > 0);
     if (cudaFuncSetAttribute(h->kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess) {
       s = MK_ERR_CUDA;
-      h->err = "cannot reserve dynamic shared memory";
+      h->err = std::string("cannot reserve dynamic shared memory: ") + cudaGetErrorString(cudaGetLastError());
       goto fail_out;
     }
     int occ = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, h->kernel, NTHREADS, SMEM_BYTES) != cudaSuccess ||
         occ < 1) {
       s = MK_ERR_CUDA;
-      h->err = "kernel does not fit one CTA per SM";
+      h->err = "kernel does not fit one CTA per SM (occupancy " + std::to_string(occ) + ", " +
+               cudaGetErrorString(cudaGetLastError()) + ")";
       goto fail_out;
     }
   }
@@ -597,6 +599,7 @@ mk_status mk_create(const mk_model_desc* desc, int device, mk_handle** out) {
   *out = h;
   return MK_OK;
 fail_out:
+  g_create_error = h->err.empty() ? std::string("mk_create failed (status ") + std::to_string((int)s) + ")" : h->err;
   for (void* p : h->allocs) cudaFree(p);
   delete h;
   return s;
@@ -614,7 +617,7 @@ void mk_destroy(mk_handle* h) {
   delete h;
 }
 
-const char* mk_last_error(const mk_handle* h) { return h ? h->err.c_str() : "null handle"; }
+const char* mk_last_error(const mk_handle* h) { return h ? h->err.c_str() : g_create_error.c_str(); }
 int64_t mk_weight_bytes(const mk_handle* h) { return h ? h->weight_bytes : 0; }
 
 mk_status mk_launch_info(mk_handle* h, int32_t* ctas, int32_t* smem_bytes, int32_t* threads) {

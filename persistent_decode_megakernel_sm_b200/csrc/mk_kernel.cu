@@ -1339,8 +1339,9 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
     mg.w = src.w;
     mg.scales = src.scales;
     const bool accum = pc.seg > 0;
-    // one instance per row-tile count: every loop over rows is static
-    if (!m.fp8) {
+    // one instance per row-tile count: every loop over rows is static (fp8
+    // weights exist only for experts, so only MoE kernels reach the fp8 ones)
+    if (!MOE || !m.fp8) {
       switch (ci.nr) {
         case 1: gemv_group<1, false>(C, ci, mg, L, it, ix, red, accum); break;
         case 2: gemv_group<2, false>(C, ci, mg, L, it, ix, red, accum); break;
@@ -2324,16 +2325,20 @@ __device__ __noinline__ void mla_comb_task(const Ctx& C, const Task t) {
   const Model& md = *C.md;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int Hq = md.Hq, R = md.R, dP = R + 4, rows_max = P.att_rows_max;
-  const int64_t total = (int64_t)P.n_pairs * Hq * R;
-  const int64_t o0 = total * blockIdx.x / gridDim.x, o1 = total * (blockIdx.x + 1) / gridDim.x;
-  if (o0 >= o1) return;
+  // slices of whole float4 groups (R is a multiple of 64, so a group never
+  // straddles two rows)
+  const int64_t total4 = (int64_t)P.n_pairs * Hq * (R / 4);
+  const int64_t q0 = total4 * blockIdx.x / gridDim.x, q1 = total4 * (blockIdx.x + 1) / gridDim.x;
+  if (q0 >= q1) return;
   float* out = P.buf[B_OL];
   const int ldo = P.ld[B_OL];
-  float* wsh = reinterpret_cast<float*>(C.att);  // [row][160] split weights
-  const int row0 = (int)(o0 / R), row1 = (int)((o1 - 1) / R) + 1;
-  for (int rb = row0; rb < row1; rb += 64) {
-    const int re = min(row1, rb + 64);
-    const int64_t a = max(o0, (int64_t)rb * R), b = min(o1, (int64_t)re * R);
+  float* wsh = reinterpret_cast<float*>(C.att);                  // [row][160] split weights
+  float4* red = reinterpret_cast<float4*>(C.att + 32 * 160 * 4);  // [split group][unit]
+  const int R4 = R / 4;
+  const int row0 = (int)(q0 / R4), row1 = (int)((q1 - 1) / R4) + 1;
+  for (int rb = row0; rb < row1; rb += 32) {
+    const int re = min(row1, rb + 32);
+    const int64_t a = max(q0, (int64_t)rb * R4), b = min(q1, (int64_t)re * R4);
     for (int rr = rb + warp; rr < re; rr += NCW) {
       const int pair = rr / Hq, h = rr - pair * Hq;
       const Item itm = decode_item(pair_first_item(pair, P.n_pairs, P.n_items), P.n_pairs, P.n_items);
@@ -2367,19 +2372,51 @@ __device__ __noinline__ void mla_comb_task(const Ctx& C, const Task t) {
       }
     }
     bar_consumers();
-    for (int64_t o = a + tid; o < b; o += NCT) {
-      const int rr = (int)(o / R), k = (int)(o - (int64_t)rr * R);
-      const int pair = rr / Hq, h = rr - pair * Hq;
-      const Item itm = decode_item(pair_first_item(pair, P.n_pairs, P.n_items), P.n_pairs, P.n_items);
-      const float* wr = wsh + (rr - rb) * 160;
-      const float* src = P.att_part + ((size_t)itm.first * rows_max + h) * dP + k;
-      const size_t js = (size_t)rows_max * dP;
-      float num = 0.f;
+    // units of 4 outputs; when there are fewer units than threads, the
+    // splits of each unit are shared by `sg_n` thread groups and the groups'
+    // sums added in group order
+    const int units = (int)(b - a);
+    const int sg_n = max(1, min(NCT / max(units, 1), 16));
+    for (int base = 0; base < units; base += NCT / sg_n) {
+      const int per = NCT / sg_n;
+      const int u = base + tid % per, sg = tid / per;
+      float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (u < units && sg < sg_n) {
+        const int64_t q = a + u;
+        const int rr = (int)(q / R4), k = (int)(q - (int64_t)rr * R4) * 4;
+        const int pair = rr / Hq, h = rr - pair * Hq;
+        const Item itm = decode_item(pair_first_item(pair, P.n_pairs, P.n_items), P.n_pairs, P.n_items);
+        const float* wr = wsh + (rr - rb) * 160;
+        const float* src = P.att_part + ((size_t)itm.first * rows_max + h) * dP + k;
+        const size_t js = (size_t)rows_max * dP;
 #pragma unroll 16
-      for (int jj = 0; jj < itm.ns; ++jj) num += wr[jj] * __ldcg(src + jj * js);
-      out[(size_t)pair * ldo + (size_t)h * R + k] = num;
+        for (int jj = sg; jj < itm.ns; jj += sg_n) {
+          const float wv = wr[jj];
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(src + jj * js));
+          num.x += wv * v.x;
+          num.y += wv * v.y;
+          num.z += wv * v.z;
+          num.w += wv * v.w;
+        }
+      }
+      if (sg < sg_n) red[sg * per + tid % per] = num;
+      bar_consumers();
+      if (tid < per && base + tid < units) {
+        float4 tot = red[tid];
+        for (int g2 = 1; g2 < sg_n; ++g2) {
+          const float4 v = red[g2 * per + tid];
+          tot.x += v.x;
+          tot.y += v.y;
+          tot.z += v.z;
+          tot.w += v.w;
+        }
+        const int64_t q = a + base + tid;
+        const int rr = (int)(q / R4), k = (int)(q - (int64_t)rr * R4) * 4;
+        const int pair = rr / Hq, h = rr - pair * Hq;
+        *reinterpret_cast<float4*>(out + (size_t)pair * ldo + (size_t)h * R + k) = tot;
+      }
+      bar_consumers();
     }
-    bar_consumers();
   }
 }
 
@@ -2465,6 +2502,8 @@ __device__ void consumer(const Ctx& C) {
 // One instance per model family (GQA or latent attention, dense or MoE FFN): each kernel holds only
 // the code its models run, which keeps the instruction footprint of the
 // whole-step loop small.
+// 10 warps put 3 warps on two of the SM's four register-file partitions
+// (16K registers each), so a thread gets at most 168 registers.
 template <bool MLA, bool MOE>
 __global__ void __launch_bounds__(NTHREADS, 1) mk_step_kernel(const __grid_constant__ Launch P) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -2534,9 +2573,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) mk_step_kernel(const __grid_const
   }
 }
 
-template __global__ void mk_step_kernel<false, false>(const __grid_constant__ Launch P);
-template __global__ void mk_step_kernel<false, true>(const __grid_constant__ Launch P);
-template __global__ void mk_step_kernel<true, false>(const __grid_constant__ Launch P);
-template __global__ void mk_step_kernel<true, true>(const __grid_constant__ Launch P);
+// The host code (another translation unit) takes the kernel instances from here.
+const void* step_kernel_for(bool mla, bool moe) {
+  return mla ? (moe ? (const void*)mk_step_kernel<true, true> : (const void*)mk_step_kernel<true, false>)
+             : (moe ? (const void*)mk_step_kernel<false, true> : (const void*)mk_step_kernel<false, false>);
+}
 
 }  // namespace mk

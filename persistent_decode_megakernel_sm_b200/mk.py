@@ -107,7 +107,7 @@ def _stream(s) -> Optional[int]:
 
 def _check(h, code: int):
     if code != MK_OK:
-        msg = lib.mk_last_error(h).decode() if h else ""
+        msg = lib.mk_last_error(h).decode()  # with h = None: why mk_create failed
         raise MkError(code, msg)
 
 
