@@ -1594,150 +1594,113 @@ __device__ __forceinline__ int frag_off(int r, int k, int KTn) {
   return (((mi * KTn + kt) * 32 + ln) * 8 + e) * 2;
 }
 
-struct AttState {
-  float o[3][2][4];   // [mt][n-tile of this warp][frag]
-  float M[3][2];      // running max (log2 units) of rows g, g+8 of each m-tile
-  float L[3][2];      // lane-partial running sums
+// Each consumer warp owns 16 positions of every 64-position chunk (position
+// group w & 3) and half of the head dims (w >> 2), and runs its own online
+// softmax: scores go from the QK accumulators straight into the PV A
+// fragments, with no barrier inside a chunk.  The four position groups of
+// each dim half are merged once per item.
+template <int MT, int NTD>  // MT: 16-row tiles of query rows; NTD: 8-dim tiles of this warp's half
+struct WarpAtt {
+  float o[MT][NTD][4];
+  float M[MT][2];  // running max (log2 units) of rows g, g + 8 of each row tile
+  float L[MT][2];  // lane-partial running sums
 };
 
-// Process one chunk of n_valid cache positions whose K and V rows are in
-// shared memory (row pitch = 2d + 16 bytes).  causal: position i is visible
-// to query row r iff i <= r / gh.
-__device__ void att_chunk(const Ctx& C, AttState& st, const uint8_t* Ks, const uint8_t* Vs, int n_valid, bool causal,
-                          int gh, int mt, int d, int par) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, tq = lane & 3;
-  const int pitch = att_pitch(d);
-  const int KTq = d / 16;
-  uint8_t* qhi = C.att;
-  uint8_t* qlo = qhi + mt * KTq * 512;
-  uint8_t* phi = qlo + mt * KTq * 512;
-  uint8_t* plo = phi + mt * (ATT_CT / 16) * 512;
-  float* smax = reinterpret_cast<float*>(plo + mt * (ATT_CT / 16) * 512);
-
-  // ---- scores for positions [8 warp, 8 warp + 8) ----
-  float sacc[3][4];
+template <int MT, int NTD>
+__device__ __forceinline__ void warp_att_chunk(WarpAtt<MT, NTD>& st, const uint8_t* qhi, const uint8_t* qlo,
+                                               const uint8_t* Ks, const uint8_t* Vs, int pitch, int KTq, int n_valid,
+                                               bool causal, int gh, int p0, int dim0) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+  if (p0 >= n_valid) return;
+  // ---- scores of positions p0 .. p0 + 15 (two 8-position n-tiles) ----
+  float sc[MT][2][4];
 #pragma unroll
-  for (int mi = 0; mi < 3; ++mi) sacc[mi][0] = sacc[mi][1] = sacc[mi][2] = sacc[mi][3] = 0.f;
-  const int n0 = warp * 8;
-  if (n0 < n_valid) {
-    const uint8_t* krow = Ks + (size_t)(n0 + g) * pitch + tq * 4;
-    for (int ks = 0; ks < KTq; ++ks) {
-      const uint32_t b0 = lds32(krow + ks * 32);
-      const uint32_t b1 = lds32(krow + ks * 32 + 16);
+  for (int mi = 0; mi < MT; ++mi)
 #pragma unroll
-      for (int mi = 0; mi < 3; ++mi) {
-        if (mi < mt) {
-          const uint4 ah = lds128(qhi + ((mi * KTq + ks) * 32 + lane) * 16);
-          const uint4 al = lds128(qlo + ((mi * KTq + ks) * 32 + lane) * 16);
-          mma_bf16(sacc[mi], ah, b0, b1);
-          mma_bf16(sacc[mi], al, b0, b1);
-        }
-      }
+    for (int nt = 0; nt < 2; ++nt) sc[mi][nt][0] = sc[mi][nt][1] = sc[mi][nt][2] = sc[mi][nt][3] = 0.f;
+  const uint8_t* k0 = Ks + (size_t)(p0 + g) * pitch + tq * 4;
+  const uint8_t* k1 = k0 + (size_t)8 * pitch;
+#pragma unroll 2
+  for (int ks = 0; ks < KTq; ++ks) {
+    const uint32_t b00 = lds32(k0 + ks * 32), b01 = lds32(k0 + ks * 32 + 16);
+    const uint32_t b10 = lds32(k1 + ks * 32), b11 = lds32(k1 + ks * 32 + 16);
+#pragma unroll
+    for (int mi = 0; mi < MT; ++mi) {
+      const uint4 ah = lds128(qhi + ((mi * KTq + ks) * 32 + lane) * 16);
+      const uint4 al = lds128(qlo + ((mi * KTq + ks) * 32 + lane) * 16);
+      mma_bf16(sc[mi][0], ah, b00, b01);
+      mma_bf16(sc[mi][0], al, b00, b01);
+      mma_bf16(sc[mi][1], ah, b10, b11);
+      mma_bf16(sc[mi][1], al, b10, b11);
     }
   }
-  // masking and per-row max over this warp's 8 positions
-  const int p0 = n0 + 2 * tq, p1 = p0 + 1;
-  float* smx = smax + par * NCW * 48;
+  // ---- masking, online softmax, P as A fragments (bf16 hi / lo) ----
+  uint4 ph[MT], pl[MT];
 #pragma unroll
-  for (int mi = 0; mi < 3; ++mi) {
-    if (mi < mt) {
-      const int rA = mi * 16 + g, rB = rA + 8;
-      const bool vA0 = p0 < n_valid && (!causal || p0 <= rA / gh);
-      const bool vA1 = p1 < n_valid && (!causal || p1 <= rA / gh);
-      const bool vB0 = p0 < n_valid && (!causal || p0 <= rB / gh);
-      const bool vB1 = p1 < n_valid && (!causal || p1 <= rB / gh);
-      if (!vA0) sacc[mi][0] = -INFINITY;
-      if (!vA1) sacc[mi][1] = -INFINITY;
-      if (!vB0) sacc[mi][2] = -INFINITY;
-      if (!vB1) sacc[mi][3] = -INFINITY;
-      float mA = fmaxf(sacc[mi][0], sacc[mi][1]), mB = fmaxf(sacc[mi][2], sacc[mi][3]);
-      mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 1));
-      mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 2));
-      mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 1));
-      mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 2));
-      if (tq == 0) {
-        smx[warp * 48 + rA] = mA;
-        smx[warp * 48 + rB] = mB;
+  for (int mi = 0; mi < MT; ++mi) {
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const int row = mi * 16 + g + 8 * h2;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int pos = p0 + nt * 8 + 2 * tq + e;
+          float& v = sc[mi][nt][2 * h2 + e];
+          if (pos >= n_valid || (causal && pos > row / gh)) v = -INFINITY;
+          mx = fmaxf(mx, v);
+        }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float mnew = fmaxf(st.M[mi][h2], mx);
+      const float corr = (mnew == -INFINITY) ? 1.f : exp2f(st.M[mi][h2] - mnew);
+      const float msafe = (mnew == -INFINITY) ? 0.f : mnew;
+      st.M[mi][h2] = mnew;
+      float ls = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float& v = sc[mi][nt][2 * h2 + e];
+          v = exp2f(v - msafe);
+          ls += v;
+        }
+      st.L[mi][h2] = st.L[mi][h2] * corr + ls;
+#pragma unroll
+      for (int nt = 0; nt < NTD; ++nt) {
+        st.o[mi][nt][2 * h2 + 0] *= corr;
+        st.o[mi][nt][2 * h2 + 1] *= corr;
       }
     }
+    // A fragment of P (16 rows x 16 positions): a0 rows g / k 2tq.., a1 rows g+8,
+    // a2 rows g / k 8+2tq.., a3 rows g+8 / k 8+2tq..
+    split_bf16(sc[mi][0][0], sc[mi][0][1], ph[mi].x, pl[mi].x);
+    split_bf16(sc[mi][0][2], sc[mi][0][3], ph[mi].y, pl[mi].y);
+    split_bf16(sc[mi][1][0], sc[mi][1][1], ph[mi].z, pl[mi].z);
+    split_bf16(sc[mi][1][2], sc[mi][1][3], ph[mi].w, pl[mi].w);
   }
-  bar_consumers();
-  // ---- online softmax update; P fragments written in A layout ----
-  const int kt = warp >> 1;
-  const int regA = (warp & 1) ? 2 : 0;  // u32 slot of row g within the lane's 16 bytes
+  // ---- O += P V over this warp's dims; rows past n_valid of V are zeroed ----
+  const int pk = p0 + 2 * tq;
+  const uint8_t* vrow = Vs + (size_t)(p0 + (lane & 15)) * pitch + (size_t)dim0 * 2;
 #pragma unroll
-  for (int mi = 0; mi < 3; ++mi) {
-    if (mi < mt) {
-      const int rA = mi * 16 + g, rB = rA + 8;
-      float cm[2] = {-INFINITY, -INFINITY};
+  for (int nt = 0; nt < NTD; ++nt) {
+    uint32_t b0, b1;
+    ldsm_x2_trans(vrow + nt * 16, b0, b1);
+    if (pk >= n_valid) b0 = 0u;
+    else if (pk + 1 >= n_valid) b0 &= 0xFFFFu;
+    if (pk + 8 >= n_valid) b1 = 0u;
+    else if (pk + 9 >= n_valid) b1 &= 0xFFFFu;
 #pragma unroll
-      for (int w = 0; w < NCW; ++w) {
-        cm[0] = fmaxf(cm[0], smx[w * 48 + rA]);
-        cm[1] = fmaxf(cm[1], smx[w * 48 + rB]);
-      }
-      float pv[4];
-#pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        const float mnew = fmaxf(st.M[mi][h2], cm[h2]);
-        const float corr = (mnew == -INFINITY) ? 1.f : exp2f(st.M[mi][h2] - mnew);
-        const float msafe = (mnew == -INFINITY) ? 0.f : mnew;
-        st.M[mi][h2] = mnew;
-        pv[2 * h2 + 0] = exp2f(sacc[mi][2 * h2 + 0] - msafe);
-        pv[2 * h2 + 1] = exp2f(sacc[mi][2 * h2 + 1] - msafe);
-        st.L[mi][h2] = st.L[mi][h2] * corr + pv[2 * h2 + 0] + pv[2 * h2 + 1];
-#pragma unroll
-        for (int jn = 0; jn < 2; ++jn) {
-          st.o[mi][jn][2 * h2 + 0] *= corr;
-          st.o[mi][jn][2 * h2 + 1] *= corr;
-        }
-      }
-      uint32_t hA, lA, hB, lB;
-      split_bf16(pv[0], pv[1], hA, lA);
-      split_bf16(pv[2], pv[3], hB, lB);
-      uint32_t* ph = reinterpret_cast<uint32_t*>(phi + ((mi * (ATT_CT / 16) + kt) * 32 + lane) * 16);
-      uint32_t* pl = reinterpret_cast<uint32_t*>(plo + ((mi * (ATT_CT / 16) + kt) * 32 + lane) * 16);
-      ph[regA] = hA;
-      ph[regA + 1] = hB;
-      pl[regA] = lA;
-      pl[regA + 1] = lB;
-    }
-  }
-  bar_consumers();
-  // ---- O += P V ; this warp owns dim tiles (8 dims each) ----
-  const int ntile = d / 8;
-  const int per_w = ntile / NCW;  // 2 for d = 128, 1 for d = 64
-  for (int ks = 0; ks < ATT_CT / 16; ++ks) {
-    if (ks * 16 >= n_valid) break;
-    const int pk = ks * 16 + 2 * tq;
-#pragma unroll
-    for (int jn = 0; jn < 2; ++jn) {
-      if (jn < per_w) {
-        // rows ks*16 .. ks*16+15 of this warp's 8 dims; rows past n_valid may
-        // hold anything (even NaN), so their values are zeroed, not just
-        // weighted by P = 0
-        const int dim0 = (warp * per_w + jn) * 8;
-        uint32_t b0, b1;
-        ldsm_x2_trans(Vs + (size_t)(ks * 16 + (lane & 15)) * pitch + dim0 * 2, b0, b1);
-        if (pk >= n_valid) b0 = 0u;
-        else if (pk + 1 >= n_valid) b0 &= 0xFFFFu;
-        if (pk + 8 >= n_valid) b1 = 0u;
-        else if (pk + 9 >= n_valid) b1 &= 0xFFFFu;
-#pragma unroll
-        for (int mi = 0; mi < 3; ++mi) {
-          if (mi < mt) {
-            const uint4 ah = lds128(phi + ((mi * (ATT_CT / 16) + ks) * 32 + lane) * 16);
-            const uint4 al = lds128(plo + ((mi * (ATT_CT / 16) + ks) * 32 + lane) * 16);
-            mma_bf16(st.o[mi][jn], ah, b0, b1);
-            mma_bf16(st.o[mi][jn], al, b0, b1);
-          }
-        }
-      }
+    for (int mi = 0; mi < MT; ++mi) {
+      mma_bf16(st.o[mi][nt], ph[mi], b0, b1);
+      mma_bf16(st.o[mi][nt], pl[mi], b0, b1);
     }
   }
 }
 
-__device__ __noinline__ void attn_task(const Ctx& C, const Task t, uint32_t& it) {
+template <int MT, int NTD>
+__device__ void attn_item(const Ctx& C, const Task t, uint32_t& it) {
   const Launch& P = *C.P;
   const Model& md = *C.md;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1747,7 +1710,7 @@ __device__ __noinline__ void attn_task(const Ctx& C, const Task t, uint32_t& it)
   const Item itm = decode_item(t.rt0, P.n_pairs, P.n_items);
   const int s = itm.pair / md.Hkv, kvh = itm.pair % md.Hkv;
   const int d = md.d, pitch = att_pitch(d), KTq = d / 16;
-  const int gh = md.Hq / md.Hkv, Q = P.Q, nr = Q * gh, mt = (nr + 15) >> 4;
+  const int gh = md.Hq / md.Hkv, Q = P.Q, nr = Q * gh, mt = MT;
   const int T0 = seq_pos0(P, s);
   const int a = (int)(((int64_t)itm.j * T0) / itm.ns), b = (int)(((int64_t)(itm.j + 1) * T0) / itm.ns);
   const bool last = itm.j == itm.ns - 1;
@@ -1819,94 +1782,104 @@ __device__ __noinline__ void attn_task(const Ctx& C, const Task t, uint32_t& it)
     tA = t1;
   }
 
-  AttState st;
+  WarpAtt<MT, NTD> st;
 #pragma unroll
-  for (int mi = 0; mi < 3; ++mi) {
+  for (int mi = 0; mi < MT; ++mi) {
     st.M[mi][0] = st.M[mi][1] = -INFINITY;
     st.L[mi][0] = st.L[mi][1] = 0.f;
 #pragma unroll
-    for (int jn = 0; jn < 2; ++jn) st.o[mi][jn][0] = st.o[mi][jn][1] = st.o[mi][jn][2] = st.o[mi][jn][3] = 0.f;
+    for (int nt = 0; nt < NTD; ++nt) st.o[mi][nt][0] = st.o[mi][nt][1] = st.o[mi][nt][2] = st.o[mi][nt][3] = 0.f;
   }
-  int par = 0;
+  const int pg = warp & 3, dh = warp >> 2;
+  const int p0 = pg * 16, dim0 = dh * half;
   for (int t0 = a; t0 < b; t0 += ATT_CT) {
     const int n = min(ATT_CT, b - t0);
     wait_full(C, it);
     const uint8_t* stage = C.ring + (size_t)(it % NSTAGE) * STAGE_BYTES;
-    att_chunk(C, st, stage, stage + (size_t)ATT_CT * pitch, n, false, gh, mt, d, par);
-    par ^= 1;
-    bar_consumers();  // every warp is done with the stage
-    release_stage(C, it);
+    warp_att_chunk<MT, NTD>(st, qhi, qlo, stage, stage + (size_t)ATT_CT * pitch, pitch, KTq, n, false, gh, p0, dim0);
+    release_stage(C, it);  // per warp: the ring's empty barrier counts the consumer warps
     ++it;
   }
-  if (last) {
-    att_chunk(C, st, nk, nv, Q, true, gh, mt, d, par);
-    par ^= 1;
-  }
-  bar_consumers();
+  if (last) warp_att_chunk<MT, NTD>(st, qhi, qlo, nk, nv, pitch, KTq, Q, true, gh, p0, dim0);
+  bar_consumers();  // every warp is done with the query fragments: the scratch is reused below
   if (trc) {
     const long long t1 = clock64();
     C.ms->tr_loop += t1 - tA;
     tA = t1;
   }
 
-  // ---- write the item's partial (M, L, O) per query row ----
-  float* smx = reinterpret_cast<float*>(C.att + 2 * mt * KTq * 512 + 2 * mt * (ATT_CT / 16) * 512);
-#pragma unroll
-  for (int mi = 0; mi < 3; ++mi) {
-    if (mi < mt) {
-#pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        float l = st.L[mi][h2];
-        l += __shfl_xor_sync(0xffffffffu, l, 1);
-        l += __shfl_xor_sync(0xffffffffu, l, 2);
-        if (tq == 0) smx[warp * 48 + mi * 16 + g + 8 * h2] = l;
-      }
-    }
-  }
-  bar_consumers();
+  // ---- merge the four position groups of each dim half, one row tile at a
+  //      time, into the item's partial (O | M | L per query row) ----
   const int rows_max = P.att_rows_max;
-  // partial row: O (d values) | M | L | 2 pad  (16-byte rows for vector loads)
   const int dP = d + 4;
   float* part = P.att_part + (size_t)t.rt0 * rows_max * dP;
-  if (tid < nr) {
-    float l = 0.f;
-    for (int w = 0; w < NCW; ++w) l += smx[w * 48 + tid];
-    part[(size_t)tid * dP + d + 1] = l;
-  }
-  if (warp == 0 && tq == 0) {
+  float* Ow = reinterpret_cast<float*>(C.att);              // [warp][16 rows][half]
+  float* Mw = Ow + NCW * 16 * half;                           // [warp][16]
+  float* Lw = Mw + NCW * 16;                                  // [warp][16]
 #pragma unroll
-    for (int mi = 0; mi < 3; ++mi)
-      if (mi < mt) {
-        if (mi * 16 + g < nr) part[(size_t)(mi * 16 + g) * dP + d] = st.M[mi][0];
-        if (mi * 16 + g + 8 < nr) part[(size_t)(mi * 16 + g + 8) * dP + d] = st.M[mi][1];
+  for (int mi = 0; mi < MT; ++mi) {
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      float l = st.L[mi][h2];
+      l += __shfl_xor_sync(0xffffffffu, l, 1);
+      l += __shfl_xor_sync(0xffffffffu, l, 2);
+      if (tq == 0) {
+        Mw[warp * 16 + g + 8 * h2] = st.M[mi][h2];
+        Lw[warp * 16 + g + 8 * h2] = l;
       }
-  }
-  {
-    const int per_w = (d / 8) / NCW;
+    }
 #pragma unroll
-    for (int mi = 0; mi < 3; ++mi) {
-      if (mi < mt) {
+    for (int nt = 0; nt < NTD; ++nt) {
+      float* o0 = Ow + ((size_t)warp * 16 + g) * half + nt * 8 + 2 * tq;
+      o0[0] = st.o[mi][nt][0];
+      o0[1] = st.o[mi][nt][1];
+      o0[8 * half] = st.o[mi][nt][2];
+      o0[8 * half + 1] = st.o[mi][nt][3];
+    }
+    bar_consumers();
+    // thread -> (row, 8 consecutive dims)
+    for (int e = tid; e < 16 * (d / 8); e += NCT) {
+      const int r = e / (d / 8), k0 = (e - r * (d / 8)) * 8;
+      const int row = mi * 16 + r;
+      const int dhk = k0 / half, kl = k0 - dhk * half;
+      float mx = -INFINITY;
 #pragma unroll
-        for (int jn = 0; jn < 2; ++jn) {
-          if (jn < per_w) {
-            const int dim = (warp * per_w + jn) * 8 + 2 * tq;
-            const int rA = mi * 16 + g, rB = rA + 8;
-            if (rA < nr) {
-              part[(size_t)rA * dP + dim] = st.o[mi][jn][0];
-              part[(size_t)rA * dP + 1 + dim] = st.o[mi][jn][1];
-            }
-            if (rB < nr) {
-              part[(size_t)rB * dP + dim] = st.o[mi][jn][2];
-              part[(size_t)rB * dP + 1 + dim] = st.o[mi][jn][3];
-            }
-          }
+      for (int q = 0; q < 4; ++q) mx = fmaxf(mx, Mw[(dhk * 4 + q) * 16 + r]);
+      float wq[4], lsum = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float mq = Mw[(dhk * 4 + q) * 16 + r];
+        wq[q] = (mq == -INFINITY) ? 0.f : exp2f(mq - mx);
+        lsum += wq[q] * Lw[(dhk * 4 + q) * 16 + r];
+      }
+      float acc8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc8[i] = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float* src = Ow + ((size_t)(dhk * 4 + q) * 16 + r) * half + kl;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc8[i] += wq[q] * src[i];
+      }
+      if (row < nr) {
+        float* dst = part + (size_t)row * dP;
+        *reinterpret_cast<float4*>(dst + k0) = make_float4(acc8[0], acc8[1], acc8[2], acc8[3]);
+        *reinterpret_cast<float4*>(dst + k0 + 4) = make_float4(acc8[4], acc8[5], acc8[6], acc8[7]);
+        if (k0 == 0) {
+          dst[d] = mx;
+          dst[d + 1] = lsum;
         }
       }
     }
+    bar_consumers();
+  }
+  if (trc) {
+    const long long t1 = clock64();
+    C.ms->tr_post += t1 - tA;
+    tA = t1;
   }
 
   // ---- the last item of this (sequence, kv head) combines all splits ----
-  bar_consumers();
   int lastc = 0;
   if (tid == 0 && !C.ms->abort) {
     const int pc = P.ctr_pair_base + t.layer * P.n_pairs + itm.pair;
@@ -1979,6 +1952,22 @@ __device__ __noinline__ void attn_task(const Ctx& C, const Task t, uint32_t& it)
       red_release_add(P.ctr + t.layer * P.ctr_layer_stride + C_ATTN, 1u);
     }
     if (trc) C.ms->tr_epi += clock64() - tA;
+  }
+}
+
+
+__device__ __noinline__ void attn_task(const Ctx& C, const Task t, uint32_t& it) {
+  const Model& md = *C.md;
+  const int nr = C.P->Q * (md.Hq / md.Hkv);
+  const int mt = (nr + 15) >> 4;
+  if (md.d == 128) {
+    if (mt == 1) attn_item<1, 8>(C, t, it);
+    else if (mt == 2) attn_item<2, 8>(C, t, it);
+    else attn_item<3, 8>(C, t, it);
+  } else {
+    if (mt == 1) attn_item<1, 4>(C, t, it);
+    else if (mt == 2) attn_item<2, 4>(C, t, it);
+    else attn_item<3, 4>(C, t, it);
   }
 }
 
