@@ -166,6 +166,32 @@ __device__ __forceinline__ void split_f16(float a, float b, uint32_t& hi, uint32
   hi = *reinterpret_cast<uint32_t*>(&h);
   lo = *reinterpret_cast<uint32_t*>(&l);
 }
+
+// Activation buffers that feed only GEMVs and no other phase (the attention
+// output, the SwiGLU hidden units, the latent attention output) are written
+// by their producers directly in the GEMV's B-operand layout: per 16-value
+// col tile 64 bytes = for each quad lane tq, {hi(k 2tq, 2tq+1), hi(k 2tq+8,
+// 2tq+9), lo(..), lo(..)} (bf16 split, or f16 for fp8 weights), so that the
+// consuming GEMV copies them in and skips the conversion.
+__device__ __forceinline__ bool frag_buf(int b) { return b == B_ATTN || b == B_H || b == B_OL; }
+__device__ __forceinline__ void st_frag(float* row, int k, float v, bool f16) {
+  uint8_t* p = reinterpret_cast<uint8_t*>(row) + (size_t)(k >> 4) * 64 + ((k & 7) >> 1) * 16 + ((k >> 3) & 1) * 4 +
+               (k & 1) * 2;
+  uint16_t hb, lb;
+  if (!f16) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    const __nv_bfloat16 l = __float2bfloat16_rn(v - __bfloat162float(h));
+    hb = *reinterpret_cast<const uint16_t*>(&h);
+    lb = *reinterpret_cast<const uint16_t*>(&l);
+  } else {
+    const __half h = __float2half_rn(v);
+    const __half l = __float2half_rn(v - __half2float(h));
+    hb = *reinterpret_cast<const uint16_t*>(&h);
+    lb = *reinterpret_cast<const uint16_t*>(&l);
+  }
+  *reinterpret_cast<uint16_t*>(p) = hb;
+  *reinterpret_cast<uint16_t*>(p + 8) = lb;
+}
 __device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 __device__ __forceinline__ uint32_t fp8x2_to_f16x2(uint32_t two) {
@@ -962,8 +988,8 @@ __device__ void xproducer(const Ctx& C) {
           mbar_arrive(&C.ms->xfull[sl]);
         }
         __syncwarp();
-        if (M > XCONV_M) {
-          // the consumers convert this window themselves
+        if (M > XCONV_M || (t.in_kind != IN_X_NORM && frag_buf(t.in_buf))) {
+          // the consumers convert this window themselves, or it needs no conversion
           ++ix;
           continue;
         }
@@ -1124,6 +1150,7 @@ struct GemvLane {
   int warp, lane, g, tq, M, rowbytes;
   bool has_gain, trc;
   bool coop;              // the consumers convert the activation windows (M > XCONV_M)
+  bool conv;              // the windows need converting (false: the input buffer holds fragments)
   const uint16_t* gain;   // norm gain of the task's input
 };
 
@@ -1174,7 +1201,9 @@ __device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
   while (true) {
     const uint8_t* slot = C.xring + (size_t)(ix % XSLOTS) * XSLOT_BYTES;
     if (ci.win_first()) {
-      if (!L.coop) {
+      if (!L.conv) {
+        wait_x(C, ix, true);  // the window arrives in fragment layout: nothing to do
+      } else if (!L.coop) {
         wait_x(C, ix);  // the window arrives converted
       } else {
         wait_x(C, ix, true);
@@ -1328,6 +1357,7 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
   L.rowbytes = 0;
   L.trc = P.trace && tid == 0;
   L.coop = M > XCONV_M;
+  L.conv = t.in_kind == IN_X_NORM || !frag_buf(t.in_buf);
   L.gain = t.gvec;
   if (L.trc) C.ms->tr_pre += clock64() - tpre;
   while (have) {
@@ -1391,13 +1421,24 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
           if (t.epi == EPI_STORE) {
             float* out = P.buf[t.out_buf];
             const int ld = P.ld[t.out_buf];
-            if (row0 < m.rows) {
-              if (m0 < M) out[(size_t)m0 * ld + row0] = v[0];
-              if (m1 < M) out[(size_t)m1 * ld + row0] = v[1];
-            }
-            if (row1 < m.rows) {
-              if (m0 < M) out[(size_t)m0 * ld + row1] = v[2];
-              if (m1 < M) out[(size_t)m1 * ld + row1] = v[3];
+            if (frag_buf(t.out_buf)) {  // feeds the next GEMV only (bf16 weights)
+              if (row0 < m.rows) {
+                if (m0 < M) st_frag(out + (size_t)m0 * ld, row0, v[0], false);
+                if (m1 < M) st_frag(out + (size_t)m1 * ld, row0, v[1], false);
+              }
+              if (row1 < m.rows) {
+                if (m0 < M) st_frag(out + (size_t)m0 * ld, row1, v[2], false);
+                if (m1 < M) st_frag(out + (size_t)m1 * ld, row1, v[3], false);
+              }
+            } else {
+              if (row0 < m.rows) {
+                if (m0 < M) out[(size_t)m0 * ld + row0] = v[0];
+                if (m1 < M) out[(size_t)m1 * ld + row0] = v[1];
+              }
+              if (row1 < m.rows) {
+                if (m0 < M) out[(size_t)m0 * ld + row1] = v[2];
+                if (m1 < M) out[(size_t)m1 * ld + row1] = v[3];
+              }
             }
           } else if (t.epi == EPI_RESID) {
             float* x = P.buf[B_X];
@@ -1423,16 +1464,16 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
             if (i * 2 < m.rows) {
               const float w0 = t.moe == 1 ? 1.f : C.ms->rt_w[slot][m0 < MAXM ? m0 : 0];
               const float w1 = t.moe == 1 ? 1.f : C.ms->rt_w[slot][m1 < MAXM ? m1 : 0];
-              if (m0 < M) h[((size_t)hs * MAXM + m0) * ld + i] = w0 * silu_f(v[0]) * v[2];
-              if (m1 < M) h[((size_t)hs * MAXM + m1) * ld + i] = w1 * silu_f(v[1]) * v[3];
+              if (m0 < M) st_frag(h + ((size_t)hs * MAXM + m0) * ld, i, w0 * silu_f(v[0]) * v[2], md.fp8 != 0);
+              if (m1 < M) st_frag(h + ((size_t)hs * MAXM + m1) * ld, i, w1 * silu_f(v[1]) * v[3], md.fp8 != 0);
             }
           } else if (t.epi == EPI_SWIGLU) {
             float* h = P.buf[t.out_buf];
             const int ld = P.ld[t.out_buf];
             const int i = rt * 8 + (l >> 2);
             if (i * 2 < m.rows) {
-              if (m0 < M) h[(size_t)m0 * ld + i] = silu_f(v[0]) * v[2];
-              if (m1 < M) h[(size_t)m1 * ld + i] = silu_f(v[1]) * v[3];
+              if (m0 < M) st_frag(h + (size_t)m0 * ld, i, silu_f(v[0]) * v[2], false);
+              if (m1 < M) st_frag(h + (size_t)m1 * ld, i, silu_f(v[1]) * v[3], false);
             }
           } else if (t.epi == EPI_LOGITS) {
 #pragma unroll
@@ -1945,7 +1986,12 @@ __device__ void attn_item(const Ctx& C, const Task t, uint32_t& it) {
         num.w += w * q.w;
       }
       const int qi = r / gh, hh = r % gh;
-      *reinterpret_cast<float4*>(out + (size_t)(s * Q + qi) * ldo + (size_t)(kvh * gh + hh) * d + k) = num;
+      float* orow = out + (size_t)(s * Q + qi) * ldo;
+      const int kc = (kvh * gh + hh) * d + k;
+      st_frag(orow, kc, num.x, false);
+      st_frag(orow, kc + 1, num.y, false);
+      st_frag(orow, kc + 2, num.z, false);
+      st_frag(orow, kc + 3, num.w, false);
     }
     bar_consumers();
     if (tid == 0 && !C.ms->abort) {
@@ -2402,7 +2448,11 @@ __device__ __noinline__ void mla_comb_task(const Ctx& C, const Task t) {
         const int64_t q = a + base + tid;
         const int rr = (int)(q / R4), k = (int)(q - (int64_t)rr * R4) * 4;
         const int pair = rr / Hq, h = rr - pair * Hq;
-        *reinterpret_cast<float4*>(out + (size_t)pair * ldo + (size_t)h * R + k) = tot;
+        float* orow = out + (size_t)pair * ldo;
+        st_frag(orow, h * R + k, tot.x, false);
+        st_frag(orow, h * R + k + 1, tot.y, false);
+        st_frag(orow, h * R + k + 2, tot.z, false);
+        st_frag(orow, h * R + k + 3, tot.w, false);
       }
       bar_consumers();
     }
