@@ -555,7 +555,8 @@ mk_status mk_create(const mk_model_desc* desc, int device, mk_handle** out) {
     const int hslots = d.n_routed ? d.n_shared + std::min(d.n_routed, MAXM * d.top_k) : 1;
     const int qkv_w = mla ? Hq * (hd + dr) + R + dr : (Hq + 2 * G) * hd;
     const int lat_w = mla ? Hq * R : 4;
-    const int widths[NBUF] = {H, qkv_w, Hq * hd, std::max(hw, 8), std::max(d.n_routed, 4), lat_w, lat_w};
+    const int xf16_w = (d.n_routed && d.expert_fp8) ? H : 4;
+    const int widths[NBUF] = {H, qkv_w, Hq * hd, std::max(hw, 8), std::max(d.n_routed, 4), lat_w, lat_w, H, xf16_w};
     for (int b = 0; b < NBUF; ++b) {
       h->ld[b] = (widths[b] + 3) & ~3;
       const size_t rows = (b == B_H) ? (size_t)hslots * MB : (size_t)MB;
@@ -1108,6 +1109,19 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
     t.gvec = nullptr;
     if (t.in_kind == IN_X_NORM)
       t.gvec = t.gain == 0 ? h->attn_norm[t.layer] : (t.gain == 1 ? h->ffn_norm[t.layer] : h->final_norm);
+    // producers of x write x * (the gain of the norm that reads it next) as GEMV fragments
+    t.gnext = nullptr;
+    t.xf16 = 0;
+    if (t.type == T_EMBED) {
+      t.gnext = h->attn_norm[0];
+    } else if (t.epi == EPI_RESID) {
+      if (t.ss_dst == 0) {  // after attention: the FFN (router, shared and routed experts)
+        t.gnext = h->ffn_norm[t.layer];
+        t.xf16 = (d.n_routed && d.expert_fp8) ? 1 : 0;
+      } else {  // after the FFN: the next layer's attention, or the final norm
+        t.gnext = t.layer + 1 < L ? h->attn_norm[t.layer + 1] : h->final_norm;
+      }
+    }
   }
   n_items_out = n_items;
   n_pairs_out = n_pairs;

@@ -106,7 +106,9 @@ enum BufId : int16_t {
   B_X = 0, B_QKV = 1, B_ATTN = 2, B_H = 3, B_RLOG = 4,
   B_QL = 5,  // latent attention: query heads absorbed into the latent space [M][Hq * R]
   B_OL = 6,  // latent attention: attention-weighted latent rows per head [M][Hq * R]
-  NBUF = 7
+  B_XF = 7,   // x * (the next norm's gain) in the GEMV's B-fragment layout, bf16 hi / lo
+  B_XF16 = 8, // the same as f16 hi / lo, for fp8 expert weights
+  NBUF = 9
 };
 
 struct Mat {
@@ -139,6 +141,8 @@ struct Task {
   // dependent global loads: the matrix descriptor and the input's norm gain.
   Mat m;                     // mats[mat]
   const uint16_t* gvec;      // the norm gain of an IN_X_NORM input (null otherwise)
+  const uint16_t* gnext;     // EPI_RESID / T_EMBED: the gain of the norm that reads the new x
+  int32_t xf16;              // ... and whether an f16 fragment copy is written too (fp8 experts read it)
 };
 
 // ---------------------------------------------------------------------------

@@ -218,6 +218,7 @@ struct Misc {
   uint64_t xempty[XSLOTS];
   float scale[MAXM];
   float xscale[XSLOTS][MAXM];  // RMSNorm scale of the rows of the window in each activation slot
+  float gscale[MAXM];          // ... of the row group the consumers are on
   volatile int abort;
   int flag;
   int pad[2];
@@ -499,7 +500,8 @@ __device__ __forceinline__ PieceSrc piece_src(const Model& md, const Task& t, co
   r.lg0 = pc.g0;
   r.xrow0 = 0;
   r.xcol0 = t.xg_rt > 0 ? (pc.g0 / t.xg_rt) * t.xg_stride : 0;
-  r.xbuf = t.in_kind == IN_X_NORM ? (int)B_X : (int)t.in_buf;
+  // normed inputs: the fragment copy of x * gain (the RMS scale is applied after the GEMV)
+  r.xbuf = t.in_kind == IN_X_NORM ? (m.fp8 ? (int)B_XF16 : (int)B_XF) : (int)t.in_buf;
   r.w = m.w;
   r.scales = m.scales;
   if (MOE && t.type == T_MOE_GU) {
@@ -988,7 +990,7 @@ __device__ void xproducer(const Ctx& C) {
           mbar_arrive(&C.ms->xfull[sl]);
         }
         __syncwarp();
-        if (M > XCONV_M || (t.in_kind != IN_X_NORM && frag_buf(t.in_buf))) {
+        if (M > XCONV_M || t.in_kind == IN_X_NORM || frag_buf(t.in_buf)) {
           // the consumers convert this window themselves, or it needs no conversion
           ++ix;
           continue;
@@ -1203,6 +1205,9 @@ __device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
     if (ci.win_first()) {
       if (!L.conv) {
         wait_x(C, ix, true);  // the window arrives in fragment layout: nothing to do
+        // normed input: the rows' RMS scales, applied to the group's sums
+        if (L.has_gain && ci.c0 == 0 && L.warp == 0 && lane < MAXM)
+          C.ms->gscale[lane] = C.ms->xscale[ix % XSLOTS][lane];
       } else if (!L.coop) {
         wait_x(C, ix);  // the window arrives converted
       } else {
@@ -1357,7 +1362,7 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
   L.rowbytes = 0;
   L.trc = P.trace && tid == 0;
   L.coop = M > XCONV_M;
-  L.conv = t.in_kind == IN_X_NORM || !frag_buf(t.in_buf);
+  L.conv = t.in_kind != IN_X_NORM && !frag_buf(t.in_buf);
   L.gain = t.gvec;
   if (L.trc) C.ms->tr_pre += clock64() - tpre;
   while (have) {
@@ -1418,6 +1423,13 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
           const int rt = pc.g0 + r;
           const int row0 = rt * 16 + (l >> 2), row1 = row0 + 8;
           const int m0 = 2 * (l & 3), m1 = m0 + 1;
+          if (has_gain) {  // RMSNorm, a per-row scale, applied to the GEMV's sums
+            const float s0 = C.ms->gscale[m0], s1 = C.ms->gscale[m1];
+            v[0] *= s0;
+            v[1] *= s1;
+            v[2] *= s0;
+            v[3] *= s1;
+          }
           if (t.epi == EPI_STORE) {
             float* out = P.buf[t.out_buf];
             const int ld = P.ld[t.out_buf];
@@ -1452,6 +1464,9 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
                 const float nv = base + v[q];
                 x[(size_t)mm * ld + row] = nv;
                 ss_acc[q & 1] += nv * nv;
+                const float gx = nv * __uint_as_float((uint32_t)__ldg(t.gnext + row) << 16);
+                st_frag(P.buf[B_XF] + (size_t)mm * P.ld[B_XF], row, gx, false);
+                if (t.xf16) st_frag(P.buf[B_XF16] + (size_t)mm * P.ld[B_XF16], row, gx, true);
               }
             }
           } else if (MOE && t.epi == EPI_SWIGLU_MOE) {
@@ -1558,6 +1573,8 @@ __device__ void embed_task(const Ctx& C, const Task t) {
         const float v = __uint_as_float((uint32_t)__ldg(e + k) << 16);
         x[(size_t)mm * ld + k] = v;
         part[mm] += v * v;
+        st_frag(P.buf[B_XF] + (size_t)mm * P.ld[B_XF], k, v * __uint_as_float((uint32_t)__ldg(t.gnext + k) << 16),
+                false);
       }
     }
   }
@@ -2474,16 +2491,16 @@ __device__ void consumer(const Ctx& C) {
   const int beg = P.task_off[blockIdx.x], end = P.task_off[blockIdx.x + 1];
   for (int ti = beg; ti < end; ++ti) {
     const Task t = P.tasks[ti];
-    // while this task waits and runs: the next task's record, and this
-    // task's norm gain (read while converting activation windows), into L1
+    // while this task waits and runs: the next task's record into L1, and
+    // the gain that this task's x updates are multiplied by for the next norm
     if (ti + 1 < end && threadIdx.x < 3) {
       const uintptr_t a = reinterpret_cast<uintptr_t>(P.tasks + ti + 1);
       const uintptr_t line = (a & ~(uintptr_t)127) + threadIdx.x * 128;
       if (line < a + sizeof(Task)) prefetch_l1(reinterpret_cast<const void*>(line));
     }
-    if (t.gvec) {
+    if (t.gnext) {
       const int lines = (C.md->H * 2 + 127) / 128;
-      for (int i = threadIdx.x; i < lines; i += NCT) prefetch_l1(reinterpret_cast<const char*>(t.gvec) + i * 128);
+      for (int i = threadIdx.x; i < lines; i += NCT) prefetch_l1(reinterpret_cast<const char*>(t.gnext) + i * 128);
     }
     const bool tr = P.trace && (ti - beg) < P.trace_cap && threadIdx.x == 0;
     uint64_t tb = 0, td = 0;
