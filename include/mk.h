@@ -107,16 +107,19 @@ mk_status mk_load_weights(mk_handle* h, const mk_tensor_src* tensors, int n);
 
 /* A KV cache for up to `max_seqs` sequences of `max_ctx` positions, owned by
  * the library, zero-filled.  Layout (device, bf16): GQA keys and values
- * [layers][max_seqs][n_kv_heads][max_ctx][head_dim] each; MLA latent
- * [layers][max_seqs][max_ctx][kv_lora_rank + rope_dim]. */
+ * [layers][max_seqs][n_kv_heads][max_ctx][head_dim] each, with the 16-byte
+ * groups of each row permuted by the position (group c at c ^ (pos & 7), so
+ * that the kernel's shared-memory reads are free of bank conflicts); MLA
+ * latent [layers][max_seqs][max_ctx][kv_lora_rank + rope_dim]. */
 mk_status mk_kv_create(mk_handle* h, int max_seqs, int max_ctx, mk_kv** out);
 
 /* Fill positions [0, length) of every sequence with seeded bf16 values
  * ~ N(0, sigma^2) (a synthetic pre-filled context).  Synchronous. */
 mk_status mk_kv_fill_random(mk_kv* kv, uint64_t seed, float sigma, int32_t length);
 
-/* Copy the whole cache, in the layout above, into caller device memory of
- * mk_kv_bytes() bytes (keys first, then values, for GQA).  Synchronous. */
+/* Copy the whole cache into caller device memory of mk_kv_bytes() bytes, in
+ * logical order (rows not permuted; keys first, then values, for GQA).
+ * Synchronous. */
 mk_status mk_kv_copy_out(mk_kv* kv, void* dst_dev);
 int64_t mk_kv_bytes(const mk_kv* kv);
 

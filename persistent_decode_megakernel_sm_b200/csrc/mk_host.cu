@@ -165,7 +165,7 @@ __global__ void fill_scales_kernel(float* dst, int64_t n, uint64_t key, float ba
 // Synthetic KV context: sequence s, kv head g, position t, element i of
 // layer l has index ((s * G + g) << 32) + t * d + i in stream (KV_K|KV_V, l).
 __global__ void fill_kv_kernel(uint16_t* dst, int L, int S, int G, int Tmax, int d, int T, uint64_t seed, int kind,
-                               float sc) {
+                               float sc, int permuted) {
   const int64_t n = (int64_t)L * S * G * T * d;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     const int e = (int)(i % d);
@@ -178,7 +178,19 @@ __global__ void fill_kv_kernel(uint16_t* dst, int L, int S, int G, int Tmax, int
     const int l = (int)(r / S);
     const uint64_t key = syn_key(seed, syn_stream((uint32_t)kind, (uint32_t)l, 0));
     const uint64_t idx = ((uint64_t)(s * G + g) << 32) + (uint64_t)t * d + e;
-    dst[((((int64_t)l * S + s) * G + g) * Tmax + t) * d + e] = syn_bf16_normal(key, idx, sc);
+    dst[((((int64_t)l * S + s) * G + g) * Tmax + t) * d + (permuted ? kv_swz(t, e) : e)] = syn_bf16_normal(key, idx, sc);
+  }
+}
+
+// Copy GQA K or V rows out of the cache in logical order (undo the in-row
+// permutation of the 16-byte groups).
+__global__ void unpermute_kv_kernel(uint16_t* dst, const uint16_t* src, int64_t rows, int Tmax, int d) {
+  const int64_t n = rows * d;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / d;
+    const int e = (int)(i - r * d);
+    const int t = (int)(r % Tmax);
+    dst[i] = src[r * d + kv_swz(t, e)];
   }
 }
 
@@ -836,15 +848,15 @@ mk_status mk_kv_fill_random(mk_kv* kv, uint64_t seed, float sigma, int32_t lengt
   if (d.kv_lora_rank > 0) {
     // latent rows: element i of (sequence s, position t) has index (s << 32) + t * W + i
     fill_kv_kernel<<<blocks, 256>>>(kv->k, d.layers, kv->max_seqs, 1, kv->max_ctx, d.kv_lora_rank + d.rope_dim,
-                                    length, seed, SYN_KV_LAT, sc);
+                                    length, seed, SYN_KV_LAT, sc, 0);
     CK(cudaGetLastError());
     CK(cudaDeviceSynchronize());
     return MK_OK;
   }
   fill_kv_kernel<<<blocks, 256>>>(kv->k, d.layers, kv->max_seqs, d.n_kv_heads, kv->max_ctx, d.head_dim, length, seed,
-                                  SYN_KV_K, sc);
+                                  SYN_KV_K, sc, 1);
   fill_kv_kernel<<<blocks, 256>>>(kv->v, d.layers, kv->max_seqs, d.n_kv_heads, kv->max_ctx, d.head_dim, length, seed,
-                                  SYN_KV_V, sc);
+                                  SYN_KV_V, sc, 1);
   CK(cudaGetLastError());
   CK(cudaDeviceSynchronize());
   return MK_OK;
@@ -859,8 +871,13 @@ mk_status mk_kv_copy_out(mk_kv* kv, void* dst) {
     return MK_OK;
   }
   const size_t half = (size_t)kv->bytes / 2;
-  CK(cudaMemcpy(dst, kv->k, half, cudaMemcpyDeviceToDevice));
-  CK(cudaMemcpy(reinterpret_cast<uint8_t*>(dst) + half, kv->v, half, cudaMemcpyDeviceToDevice));
+  const int d = h->desc.head_dim;
+  const int64_t rows = (int64_t)(half / 2) / d;
+  unpermute_kv_kernel<<<148 * 16, 256>>>(reinterpret_cast<uint16_t*>(dst), kv->k, rows, kv->max_ctx, d);
+  unpermute_kv_kernel<<<148 * 16, 256>>>(reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(dst) + half), kv->v,
+                                         rows, kv->max_ctx, d);
+  CK(cudaGetLastError());
+  CK(cudaDeviceSynchronize());
   return MK_OK;
 }
 

@@ -33,10 +33,18 @@ constexpr int SMEM_BYTES = NSTAGE * STAGE_BYTES + XSLOTS * XSLOT_BYTES + ATT_BYT
 constexpr int RMAX = 8;                      // row tiles per chunk
 constexpr int CPW = 8;                       // col tiles per warp per chunk
 constexpr int MAXM = 8;                      // activation rows per step (S * Q)
-constexpr int ATT_CT = 64;                   // cache positions per attention chunk
+constexpr int ATT_CT = 128;                  // cache positions per attention chunk (K and V fill one stage)
+static_assert(2 * ATT_CT * 128 * 2 <= STAGE_BYTES, "a K/V chunk of head_dim 128 fills at most one stage");
 constexpr int TRACE_FIELDS = 20;             // int64 per traced task
 constexpr int TILE_BF16 = 512;               // 16x16 bf16 tile in A-fragment order
 constexpr int TILE_FP8 = 256;                // 16x16 e4m3 tile in A-fragment order
+
+// GQA K / V rows (head_dim bf16 values) are stored with their 16-byte groups
+// permuted by the position: group c of the row at position pos sits at
+// group c ^ (pos & 7).  A chunk of consecutive rows, copied to shared memory
+// as one block, then spreads any 8 consecutive rows' accesses to one group
+// over all banks.  Element index of dim e of the row at position pos:
+__host__ __device__ inline int kv_swz(int pos, int e) { return (((e >> 3) ^ (pos & 7)) << 3) | (e & 7); }
 
 // Latent attention (MLA) items use the activation ring, the attention scratch
 // and the new-KV rows as one contiguous shared-memory region: while a CTA runs

@@ -1642,7 +1642,7 @@ __device__ void lm_finish(const Ctx& C) {
 // ---------------------------------------------------------------------------
 // Shared layout inside the attention scratch:
 //   Q fragments (hi, lo): [mt][d/16][32 lanes][16 B]
-//   P fragments (hi, lo): [mt][ATT_CT/16][32 lanes][16 B]
+//   P fragments (hi, lo): [mt][64/16][32 lanes][16 B]
 //   smax: [2][NCW][48] fp32
 __device__ __forceinline__ int frag_off(int r, int k, int KTn) {
   // byte offset of element (row r, col k) in an A-fragment tile array [mt][KTn][32][8 x 2B]
@@ -1667,7 +1667,7 @@ struct WarpAtt {
 template <int MT, int NTD>
 __device__ __forceinline__ void warp_att_chunk(WarpAtt<MT, NTD>& st, const uint8_t* qhi, const uint8_t* qlo,
                                                const uint8_t* Ks, const uint8_t* Vs, int pitch, int KTq, int n_valid,
-                                               bool causal, int gh, int p0, int dim0) {
+                                               bool causal, int gh, int p0, int dim0, int base) {
   const int lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
   if (p0 >= n_valid) return;
   // ---- scores of positions p0 .. p0 + 15 (two 8-position n-tiles) ----
@@ -1676,12 +1676,15 @@ __device__ __forceinline__ void warp_att_chunk(WarpAtt<MT, NTD>& st, const uint8
   for (int mi = 0; mi < MT; ++mi)
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) sc[mi][nt][0] = sc[mi][nt][1] = sc[mi][nt][2] = sc[mi][nt][3] = 0.f;
+  // rows p0 + g and p0 + 8 + g share the permutation key (base + p0 + g) & 7
+  const int key = (base + p0 + g) & 7;
   const uint8_t* k0 = Ks + (size_t)(p0 + g) * pitch + tq * 4;
   const uint8_t* k1 = k0 + (size_t)8 * pitch;
 #pragma unroll 2
   for (int ks = 0; ks < KTq; ++ks) {
-    const uint32_t b00 = lds32(k0 + ks * 32), b01 = lds32(k0 + ks * 32 + 16);
-    const uint32_t b10 = lds32(k1 + ks * 32), b11 = lds32(k1 + ks * 32 + 16);
+    const int c0 = ((2 * ks) ^ key) * 16, c1 = ((2 * ks + 1) ^ key) * 16;
+    const uint32_t b00 = lds32(k0 + c0), b01 = lds32(k0 + c1);
+    const uint32_t b10 = lds32(k1 + c0), b11 = lds32(k1 + c1);
 #pragma unroll
     for (int mi = 0; mi < MT; ++mi) {
       const uint4 ah = lds128(qhi + ((mi * KTq + ks) * 32 + lane) * 16);
@@ -1740,11 +1743,12 @@ __device__ __forceinline__ void warp_att_chunk(WarpAtt<MT, NTD>& st, const uint8
   }
   // ---- O += P V over this warp's dims; rows past n_valid of V are zeroed ----
   const int pk = p0 + 2 * tq;
-  const uint8_t* vrow = Vs + (size_t)(p0 + (lane & 15)) * pitch + (size_t)dim0 * 2;
+  const int vr = p0 + (lane & 15), vkey = (base + vr) & 7;
+  const uint8_t* vrow = Vs + (size_t)vr * pitch;
 #pragma unroll
   for (int nt = 0; nt < NTD; ++nt) {
     uint32_t b0, b1;
-    ldsm_x2_trans(vrow + nt * 16, b0, b1);
+    ldsm_x2_trans(vrow + (((dim0 >> 3) + nt) ^ vkey) * 16, b0, b1);
     if (pk >= n_valid) b0 = 0u;
     else if (pk + 1 >= n_valid) b0 &= 0xFFFFu;
     if (pk + 8 >= n_valid) b1 = 0u;
@@ -1822,15 +1826,16 @@ __device__ void attn_item(const Ctx& C, const Task t, uint32_t& it) {
         v1 = __float2bfloat16_rn(__ldcg(vr + i + half));
         __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(P.kv_k) + (head + pos) * d;
         __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(P.kv_v) + (head + pos) * d;
-        kc[i] = k0;
-        kc[i + half] = k1;
-        vc[i] = v0;
-        vc[i + half] = v1;
+        kc[kv_swz(pos, i)] = k0;
+        kc[kv_swz(pos, i + half)] = k1;
+        vc[kv_swz(pos, i)] = v0;
+        vc[kv_swz(pos, i + half)] = v1;
       }
-      *reinterpret_cast<__nv_bfloat16*>(nk + qi * pitch + i * 2) = k0;
-      *reinterpret_cast<__nv_bfloat16*>(nk + qi * pitch + (i + half) * 2) = k1;
-      *reinterpret_cast<__nv_bfloat16*>(nv + qi * pitch + i * 2) = v0;
-      *reinterpret_cast<__nv_bfloat16*>(nv + qi * pitch + (i + half) * 2) = v1;
+      // shared-memory row qi: permuted by qi (the reader's key for these rows)
+      *reinterpret_cast<__nv_bfloat16*>(nk + qi * pitch + kv_swz(qi, i) * 2) = k0;
+      *reinterpret_cast<__nv_bfloat16*>(nk + qi * pitch + kv_swz(qi, i + half) * 2) = k1;
+      *reinterpret_cast<__nv_bfloat16*>(nv + qi * pitch + kv_swz(qi, i) * 2) = v0;
+      *reinterpret_cast<__nv_bfloat16*>(nv + qi * pitch + kv_swz(qi, i + half) * 2) = v1;
     }
   }
   bar_consumers();
@@ -1854,11 +1859,15 @@ __device__ void attn_item(const Ctx& C, const Task t, uint32_t& it) {
     const int n = min(ATT_CT, b - t0);
     wait_full(C, it);
     const uint8_t* stage = C.ring + (size_t)(it % NSTAGE) * STAGE_BYTES;
-    warp_att_chunk<MT, NTD>(st, qhi, qlo, stage, stage + (size_t)ATT_CT * pitch, pitch, KTq, n, false, gh, p0, dim0);
+    // a warp takes its 16 positions of each 64-position half of the chunk
+    warp_att_chunk<MT, NTD>(st, qhi, qlo, stage, stage + (size_t)ATT_CT * pitch, pitch, KTq, n, false, gh, p0, dim0,
+                            t0);
+    warp_att_chunk<MT, NTD>(st, qhi, qlo, stage, stage + (size_t)ATT_CT * pitch, pitch, KTq, n, false, gh, p0 + 64,
+                            dim0, t0);
     release_stage(C, it);  // per warp: the ring's empty barrier counts the consumer warps
     ++it;
   }
-  if (last) warp_att_chunk<MT, NTD>(st, qhi, qlo, nk, nv, pitch, KTq, Q, true, gh, p0, dim0);
+  if (last) warp_att_chunk<MT, NTD>(st, qhi, qlo, nk, nv, pitch, KTq, Q, true, gh, p0, dim0, 0);
   bar_consumers();  // every warp is done with the query fragments: the scratch is reused below
   if (trc) {
     const long long t1 = clock64();
