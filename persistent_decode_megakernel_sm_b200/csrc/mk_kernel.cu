@@ -1185,6 +1185,26 @@ __device__ __forceinline__ void fp8_apply_scales(const Mat& m, int g0, int cb, f
   }
 }
 
+// Packed accumulators (M <= 4): column n < M holds the hi-part products of
+// activation row n, column n + M its lo-part products.  A lane holds columns
+// 2tq, 2tq + 1 of rows g and g + 8 (c0 c1 / c2 c3); the partner of column n
+// sits in lane tq' = (n + M) / 2 of the same quad, slot (n + M) & 1.  After
+// the fold, columns >= M are zero as in the unpacked layout.
+__device__ __forceinline__ void fold_lo_cols(float (&c)[4], int M, int tq, int lane) {
+  const bool odd = M & 1;
+  const int s0 = (lane & ~3) | ((tq + (M >> 1)) & 3);
+  const int s1 = (lane & ~3) | ((tq + ((M + 1) >> 1)) & 3);
+  const float u0 = __shfl_sync(0xffffffffu, odd ? c[1] : c[0], s0);
+  const float u1 = __shfl_sync(0xffffffffu, odd ? c[0] : c[1], s1);
+  const float u2 = __shfl_sync(0xffffffffu, odd ? c[3] : c[2], s0);
+  const float u3 = __shfl_sync(0xffffffffu, odd ? c[2] : c[3], s1);
+  const bool k0 = 2 * tq < M, k1 = 2 * tq + 1 < M;
+  c[0] = k0 ? c[0] + u0 : 0.f;
+  c[1] = k1 ? c[1] + u1 : 0.f;
+  c[2] = k0 ? c[2] + u2 : 0.f;
+  c[3] = k1 ? c[3] + u3 : 0.f;
+}
+
 template <int NR, bool FP8>
 __device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& mr, const GemvLane& Lr, uint32_t& itr,
                                         uint32_t& ixr, float* red, bool accum) {
@@ -1198,7 +1218,13 @@ __device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
 #pragma unroll
   for (int r = 0; r < NR; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
   const int lane = L.lane, g = L.g, tq = L.tq;
-  const bool xok = g < L.M;  // activation rows beyond M are zero
+  // M <= 4: the hi and lo parts of activation row n feed mma columns n and
+  // n + M, so one mma per tile covers both; the column pairs are summed once
+  // at the end.  Otherwise column n is row n and each tile takes two mmas.
+  const bool pk = L.M <= MAXM / 2;
+  const bool lo_col = pk && g >= L.M;
+  const int gr = lo_col ? g - L.M : g;
+  const bool xok = g < (pk ? 2 * L.M : L.M);  // other columns are zero
   long long tc0 = 0, tl0 = L.trc ? clock64() : 0;
   while (true) {
     const uint8_t* slot = C.xring + (size_t)(ix % XSLOTS) * XSLOT_BYTES;
@@ -1221,7 +1247,7 @@ __device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
     }
     wait_full(C, it);
     const uint8_t* stage = C.ring + (size_t)(it % NSTAGE) * STAGE_BYTES;
-    const uint8_t* xs = slot + (size_t)g * L.rowbytes + (size_t)(ci.c0 - ci.w0()) * 64 + tq * 16;
+    const uint8_t* xs = slot + (size_t)gr * L.rowbytes + (size_t)(ci.c0 - ci.w0()) * 64 + tq * 16;
     const int nc = ci.nc;
     if (L.trc) tc0 = clock64();
     // kept rolled: the instruction working set of the whole kernel must stay
@@ -1230,13 +1256,16 @@ __device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
 #pragma unroll 1
       for (int j = L.warp; j < nc; j += NCW) {
         const uint4 xf = xok ? lds128(xs + j * 64) : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t b0 = lo_col ? xf.z : xf.x, b1 = lo_col ? xf.w : xf.y;
         uint4 a[NR];
 #pragma unroll
         for (int r = 0; r < NR; ++r) a[r] = lds128(stage + ((size_t)r * nc + j) * TILE_BF16 + lane * 16);
 #pragma unroll
-        for (int r = 0; r < NR; ++r) mma_bf16(acc[r], a[r], xf.x, xf.y);
+        for (int r = 0; r < NR; ++r) mma_bf16(acc[r], a[r], b0, b1);
+        if (!pk) {
 #pragma unroll
-        for (int r = 0; r < NR; ++r) mma_bf16(acc[r], a[r], xf.z, xf.w);
+          for (int r = 0; r < NR; ++r) mma_bf16(acc[r], a[r], xf.z, xf.w);
+        }
       }
     } else {
       // fp8: each warp takes a contiguous run of the chunk's col tiles and
@@ -1256,14 +1285,15 @@ __device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
           cb = cbj;
         }
         const uint4 xf = xok ? lds128(xs + j * 64) : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t b0 = lo_col ? xf.z : xf.x, b1 = lo_col ? xf.w : xf.y;
         uint2 a8[NR];
 #pragma unroll
         for (int r = 0; r < NR; ++r) a8[r] = lds64(stage + ((size_t)r * nc + j) * TILE_FP8 + lane * 8);
 #pragma unroll
         for (int r = 0; r < NR; ++r) {
           const uint4 af = fp8_frag_to_f16(a8[r]);
-          mma_f16(raw[r], af, xf.x, xf.y);
-          mma_f16(raw[r], af, xf.z, xf.w);
+          mma_f16(raw[r], af, b0, b1);
+          if (!pk) mma_f16(raw[r], af, xf.z, xf.w);
         }
       }
       if (j0 < j1) fp8_apply_scales<NR>(m, ci.g0, cb, raw, acc);
@@ -1290,6 +1320,10 @@ __device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
     ci.next();
   }
   if (L.trc) C.ms->tr_loop += clock64() - tl0;
+  if (pk) {
+#pragma unroll
+    for (int r = 0; r < NR; ++r) fold_lo_cols(acc[r], L.M, tq, lane);
+  }
   // per-warp partial sums (added to the previous K segments' when accum)
 #pragma unroll
   for (int r = 0; r < NR; ++r) {

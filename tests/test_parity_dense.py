@@ -79,7 +79,7 @@ def test_tiny_prefill_and_greedy_decode(tiny):
     kv.close()
 
 
-@pytest.mark.parametrize("B", [1, 3, 8])
+@pytest.mark.parametrize("B", [1, 2, 3, 4, 8])
 def test_tiny_batched_ragged_positions(tiny, B):
     """B sequences at different positions over a synthetic context, gains != 1."""
     mc = synth.preset("tiny", gain_sigma=0.1)

@@ -203,7 +203,7 @@ def test_moe_no_shared_expert_and_top1():
     m.close()
 
 
-@pytest.mark.parametrize("B", [1, 8])
+@pytest.mark.parametrize("B", [1, 2, 8])
 def test_tiny_moe_fp8_experts(B):
     """Shared and routed expert weights as e4m3 codes with one fp32 scale per
     128 x 128 block (expert_ffn 192 gives a ragged second block)."""
@@ -233,3 +233,4 @@ def test_tiny_moe_fp8_experts(B):
     assert m.sync_status() == 0
     kv.close()
     m.close()
+
