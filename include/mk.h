@@ -184,12 +184,21 @@ mk_status mk_verify(mk_handle* h, const int32_t* tokens8, int n_prop, int32_t po
  * shape) in top-k order. */
 mk_status mk_set_router_trace(mk_handle* h, int32_t* idx_dev, float* w_dev);
 
-/* Debug trace of the next compute calls: for every task of every CTA the
- * kernel writes 8 int64 into trace_dev[cta][task][8]: %globaltimer (ns) at
- * task start, when its dependency was satisfied, and at its end; SM clock
- * cycles spent waiting for weight tiles, for activation slices; chunks and
- * weight bytes consumed; the task's type.  Tasks beyond max_tasks_per_cta
- * are not recorded.  NULL disables. */
+/* Debug trace of the next compute calls.  While a buffer is set, steps run
+ * an instrumented instance of the kernel (same arithmetic and results; the
+ * ordinary instance carries no tracing code).  For every task of every CTA it
+ * writes 20 int64 into trace_dev[cta][task][20]:
+ *   0-2   %globaltimer (ns) at task start, when its dependency was met, at its end;
+ *   3-4   SM cycles spent waiting for weight tiles, for activation slices;
+ *   5-7   chunks consumed, layer, type * 16 + epilogue;
+ *   8-11  cycles in fragment preparation, mma, epilogue, release;
+ *   12-15 (record 0) producer cycles blocked on a full ring, chunks issued,
+ *         first and last issue time (ns); (record 1) producer cycles and ns
+ *         over its lifetime (the SM clock); (later records) field 12 holds
+ *         the cycles spent waiting for the MoE route;
+ *   16-19 cycles in the chunk loop, before it, after it, signalling.
+ * The buffer holds ctas x max_tasks_per_cta records (mk_launch_info gives the
+ * CTA count); later tasks are not recorded.  NULL disables. */
 mk_status mk_set_trace(mk_handle* h, int64_t* trace_dev, int32_t max_tasks_per_cta);
 
 /* Read the device status word (call after the stream has been synchronised).

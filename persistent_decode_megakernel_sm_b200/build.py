@@ -6,20 +6,32 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libmk.so")
-SRC = [os.path.join(HERE, "csrc", f) for f in ("mk_kernel.cu", "mk_host.cu")]
+SRC = [os.path.join(HERE, "csrc", f) for f in ("mk_kernel.cu", "mk_kernel_traced.cu", "mk_host.cu")]
 DEPS = SRC + [os.path.join(HERE, "csrc", "mk_internal.h"), os.path.join(ROOT, "include", "mk.h"),
               os.path.join(ROOT, "synth", "synth.h")]
+DEPS.append(os.path.join(HERE, "csrc", "mk_kernel.cu"))  # included by mk_kernel_traced.cu
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
-         "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr",
+         "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I" + os.path.join(ROOT, "include")]
+OBJ_DIR = os.path.join(HERE, "_build")
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and os.path.exists(LIB) and all(os.path.getmtime(LIB) >= os.path.getmtime(p) for p in DEPS):
         return LIB
-    cmd = [NVCC] + FLAGS + (["-Xptxas", "-v"] if verbose else []) + ["-o", LIB] + SRC
-    subprocess.check_call(cmd)
+    os.makedirs(OBJ_DIR, exist_ok=True)
+    # the translation units compile in parallel, then link into one library
+    objs, procs = [], []
+    for src in SRC:
+        obj = os.path.join(OBJ_DIR, os.path.splitext(os.path.basename(src))[0] + ".o")
+        cmd = [NVCC] + FLAGS + (["-Xptxas", "-v"] if verbose else []) + ["-c", "-o", obj, src]
+        procs.append((subprocess.Popen(cmd), cmd))
+        objs.append(obj)
+    failed = [cmd for p, cmd in procs if p.wait() != 0]
+    if failed:
+        raise subprocess.CalledProcessError(1, failed[0])
+    subprocess.check_call([NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", LIB] + objs)
     return LIB
 
 

@@ -19,7 +19,9 @@
 #include "mk_internal.h"
 
 namespace mk {
-const void* step_kernel_for(bool mla, bool moe);  // the kernel instance of a model family
+// the kernel instance of a model family, without and with tracing compiled in
+namespace plain { const void* step_kernel_for(bool mla, bool moe); }
+namespace traced { const void* step_kernel_for(bool mla, bool moe); }
 }
 
 using namespace mk;
@@ -257,7 +259,8 @@ struct mk_handle {
   bool sticky = false;
   bool initialised = false;
   uint64_t noalloc_id = 0;  // identity of this handle for mk_decode_step_noalloc's installed task list
-  const void* kernel = nullptr;  // the step kernel instance of this model's family
+  const void* kernel = nullptr;         // the step kernel instance of this model's family
+  const void* kernel_traced = nullptr;  // ... with tracing compiled in (launched while a trace buffer is set)
   std::string err;
 };
 
@@ -593,15 +596,19 @@ mk_status mk_create(const mk_model_desc* desc, int device, mk_handle** out) {
       s = MK_ERR_CUDA;
       goto fail_out;
     }
-    h->kernel = step_kernel_for(d.kv_lora_rank > 0, d.n_routed > 0);
-    if (cudaFuncSetAttribute(h->kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess) {
+    h->kernel = plain::step_kernel_for(d.kv_lora_rank > 0, d.n_routed > 0);
+    h->kernel_traced = traced::step_kernel_for(d.kv_lora_rank > 0, d.n_routed > 0);
+    if (cudaFuncSetAttribute(h->kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(h->kernel_traced, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess) {
       s = MK_ERR_CUDA;
       h->err = std::string("cannot reserve dynamic shared memory: ") + cudaGetErrorString(cudaGetLastError());
       goto fail_out;
     }
     int occ = 0;
+    int occ_tr = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, h->kernel, NTHREADS, SMEM_BYTES) != cudaSuccess ||
-        occ < 1) {
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_tr, h->kernel_traced, NTHREADS, SMEM_BYTES) != cudaSuccess ||
+        occ < 1 || occ_tr < 1) {
       s = MK_ERR_CUDA;
       h->err = "kernel does not fit one CTA per SM (occupancy " + std::to_string(occ) + ", " +
                cudaGetErrorString(cudaGetLastError()) + ")";
@@ -1221,7 +1228,7 @@ static mk_status launch_step(mk_handle* h, mk_kv* kv, int S, int Q, const int32_
   P.trace_cap = h->task_trace_cap;
   h->stall_ns = 0;
   void* args[] = {&P};
-  cudaError_t e = cudaLaunchCooperativeKernel(h->kernel, dim3(h->ncta), dim3(NTHREADS), args,
+  cudaError_t e = cudaLaunchCooperativeKernel(P.trace ? h->kernel_traced : h->kernel, dim3(h->ncta), dim3(NTHREADS), args,
                                               SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(h, MK_ERR_CUDA, std::string("launch: ") + cudaGetErrorString(e));
   return MK_OK;
@@ -1451,7 +1458,7 @@ extern "C" mk_status mk_decode_step_noalloc(mk_handle* h, const int32_t* tokens,
   P.trace = h->task_trace;
   P.trace_cap = h->task_trace_cap;
   void* args[] = {&P};
-  const cudaError_t e = cudaLaunchCooperativeKernel(h->kernel, dim3(h->ncta), dim3(NTHREADS), args,
+  const cudaError_t e = cudaLaunchCooperativeKernel(P.trace ? h->kernel_traced : h->kernel, dim3(h->ncta), dim3(NTHREADS), args,
                                                     SMEM_BYTES, st);
   if (e != cudaSuccess) return fail(h, MK_ERR_CUDA, std::string("launch: ") + cudaGetErrorString(e));
   return MK_OK;

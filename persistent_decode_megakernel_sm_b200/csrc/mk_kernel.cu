@@ -8,7 +8,7 @@
 //   - grid = one CTA per SM (cooperative launch guarantees co-residency);
 //   - each CTA runs a host-planned task list (GEMV row tiles, attention items);
 //   - warp 8 is a producer: it walks the same task list and streams every
-//     weight tile and KV-cache row the CTA will consume into a 5-stage shared
+//     weight tile and KV-cache row the CTA will consume into a 2-stage shared
 //     memory ring with cp.async.bulk (TMA) + mbarrier complete_tx.  Weights do
 //     not depend on activations, so the producer never waits on another CTA:
 //     it runs ahead across task and layer boundaries (the cross-layer
@@ -28,7 +28,22 @@
 
 #include "mk_internal.h"
 
+// Tracing (per-task records and per-region cycle counts for the trace tool)
+// lives in separate instances of every kernel: mk_kernel_traced.cu compiles
+// this file again with MK_TRACE 1, into its own namespace.  The untraced
+// instances, which serve every ordinary step, carry none of its code: the
+// checks and counters cost about 4 % of the step time when compiled in.
+#ifndef MK_TRACE
+#define MK_TRACE 0
+#endif
+#if MK_TRACE
+#define MK_KNS traced
+#else
+#define MK_KNS plain
+#endif
+
 namespace mk {
+namespace MK_KNS {
 
 // ---------------------------------------------------------------------------
 // PTX helpers
@@ -783,7 +798,7 @@ __device__ void producer(const Ctx& C) {
     ++it;
   }
 drain:
-  if (lane == 0 && P.trace && P.trace_cap > 0) {
+  if (MK_TRACE && lane == 0 && P.trace && P.trace_cap > 0) {
     int64_t* rec = P.trace + (size_t)blockIdx.x * P.trace_cap * TRACE_FIELDS;
     rec[12] = blocked;
     rec[13] = it;
@@ -1039,7 +1054,7 @@ drain:
 __device__ __forceinline__ void wait_full(const Ctx& C, uint32_t it) {
   const int s = it % NSTAGE;
   const uint32_t par = (it / NSTAGE) & 1;
-  const bool tr = C.P->trace && threadIdx.x == 0;
+  const bool tr = MK_TRACE && C.P->trace && threadIdx.x == 0;
   const long long c0 = tr ? clock64() : 0;
   if (tr) C.ms->tr_chunks++;
   if ((threadIdx.x & 31) == 0) {
@@ -1124,7 +1139,7 @@ __device__ __forceinline__ void wait_x(const Ctx& C, uint32_t ix, bool landed = 
   const int s = ix % XSLOTS;
   const uint32_t par = (ix / XSLOTS) & 1;
   uint64_t* bar = landed ? &C.ms->xfull[s] : &C.ms->xready[s];
-  const bool tr = C.P->trace && threadIdx.x == 0;
+  const bool tr = MK_TRACE && C.P->trace && threadIdx.x == 0;
   const long long c0 = tr ? clock64() : 0;
   if ((threadIdx.x & 31) == 0) {
     uint32_t spins = 0;
@@ -1343,7 +1358,7 @@ __device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
 template <bool MOE>
 __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix) {
   const Launch& P = *C.P;
-  const long long tpre = (P.trace && threadIdx.x == 0) ? clock64() : 0;
+  const long long tpre = (MK_TRACE && P.trace && threadIdx.x == 0) ? clock64() : 0;
   const Model& md = *C.md;
   // Copies in registers: the barrier asm below clobbers "memory", which would
   // otherwise force a reload of every struct field on every chunk.
@@ -1363,7 +1378,7 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
   if (task_needs_route<MOE>(t)) {
     // the activation producer publishes the layer's route (it waits on the
     // router's counter anyway); the consumers only check that it is there
-    const long long tr0 = (P.trace && tid == 0) ? clock64() : 0;
+    const long long tr0 = (MK_TRACE && P.trace && tid == 0) ? clock64() : 0;
     if (tid == 0) {
       const uint64_t t0 = globaltimer();
       while (*reinterpret_cast<volatile int*>(&C.ms->route_layer) != t.layer + 1) {
@@ -1375,7 +1390,7 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
       }
       __threadfence_block();
     }
-    if (P.trace && tid == 0) C.ms->tr_route += clock64() - tr0;
+    if (MK_TRACE && P.trace && tid == 0) C.ms->tr_route += clock64() - tr0;
     bar_consumers();
     U = C.ms->rt_u[RR_XPROD];
   }
@@ -1394,7 +1409,7 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
   L.M = M;
   L.has_gain = has_gain;
   L.rowbytes = 0;
-  L.trc = P.trace && tid == 0;
+  L.trc = MK_TRACE && P.trace && tid == 0;
   L.coop = M > XCONV_M;
   L.conv = t.in_kind != IN_X_NORM && !frag_buf(t.in_buf);
   L.gain = t.gvec;
@@ -1801,7 +1816,7 @@ __device__ void attn_item(const Ctx& C, const Task t, uint32_t& it) {
   const Model& md = *C.md;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, tq = lane & 3;
-  const bool trc = P.trace && threadIdx.x == 0;
+  const bool trc = MK_TRACE && P.trace && threadIdx.x == 0;
   long long tA = trc ? clock64() : 0;
   const Item itm = decode_item(t.rt0, P.n_pairs, P.n_items);
   const int s = itm.pair / md.Hkv, kvh = itm.pair % md.Hkv;
@@ -2223,7 +2238,7 @@ __device__ __noinline__ void mla_task(const Ctx& C, const Task t, uint32_t& it) 
   const Model& md = *C.md;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, tq = lane & 3;
-  const bool trc = P.trace && threadIdx.x == 0;
+  const bool trc = MK_TRACE && P.trace && threadIdx.x == 0;
   long long tA = trc ? clock64() : 0;
   const Item itm = decode_item(t.rt0, P.n_pairs, P.n_items);
   const int mrow = itm.pair, Q = P.Q, s = mrow / Q, qi = mrow % Q;
@@ -2545,7 +2560,7 @@ __device__ void consumer(const Ctx& C) {
       const int lines = (C.md->H * 2 + 127) / 128;
       for (int i = threadIdx.x; i < lines; i += NCT) prefetch_l1(reinterpret_cast<const char*>(t.gnext) + i * 128);
     }
-    const bool tr = P.trace && (ti - beg) < P.trace_cap && threadIdx.x == 0;
+    const bool tr = MK_TRACE && P.trace && (ti - beg) < P.trace_cap && threadIdx.x == 0;
     uint64_t tb = 0, td = 0;
     if (tr) {
       tb = globaltimer();
@@ -2678,4 +2693,5 @@ const void* step_kernel_for(bool mla, bool moe) {
              : (moe ? (const void*)mk_step_kernel<false, true> : (const void*)mk_step_kernel<false, false>);
 }
 
+}  // namespace MK_KNS
 }  // namespace mk

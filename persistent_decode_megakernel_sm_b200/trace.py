@@ -32,10 +32,12 @@ def record(model, kv, tokens, positions, logits, argmax, cap: int = 512):
 
 
 def summarize(tr: np.ndarray, sm_clock_mhz: float = 0.0) -> dict:
-    """tr: [ctas][cap][16] = t_begin, t_dep, t_end (ns), wait_full, wait_x (cycles),
+    """tr: [ctas][cap][20] = t_begin, t_dep, t_end (ns), wait_full, wait_x (cycles),
     chunks, layer, type*16+epi, then cycles in fragment prep, mma, epilogue,
-    release (consumer thread 0); record 0 also carries the producer's cycles
-    blocked on a full ring, chunks issued, first and last issue time."""
+    release, [12..15] producer statistics (record 0: cycles blocked on a full
+    ring, chunks issued, first and last issue time; record 1: producer cycles
+    and ns, giving the SM clock), then cycles in the chunk loop, before it,
+    after it and signalling (consumer thread 0)."""
     if sm_clock_mhz <= 0:
         # measured: SM cycles / ns over each producer's lifetime (record 1)
         cyc, ns = tr[:, 1, 12].astype(np.float64), tr[:, 1, 13].astype(np.float64)

@@ -253,3 +253,33 @@ def test_host_argument_errors(tiny):
     with pytest.raises(mk.MkError):
         m.verify(_t([1] * 8), mc.max_ctx - 4, kv, None, am, am)   # positions past the cache
     kv.close()
+
+
+def test_task_trace_same_results_and_records(tiny):
+    """A step with the task trace on (the instrumented kernel instance) gives
+    bit-identical logits to the plain instance, and writes one record per
+    task: begin <= dependency met <= end, on every CTA."""
+    from persistent_decode_megakernel_sm_b200 import trace
+    mc, m = tiny
+    kv = m.kv_cache(2, mc.max_ctx)
+    toks, pos = _t([9, 10]), _t([40, 33])
+    outs = []
+    for traced in (False, True):
+        kv.fill_random(synth.SEED_KV, mc.kv_sigma, 40)
+        lg = torch.empty((2, mc.vocab), dtype=torch.float32, device=DEV)
+        am = torch.empty(2, dtype=torch.int32, device=DEV)
+        if traced:
+            tr = trace.record(m, kv, toks, pos, lg, am, cap=64)
+        else:
+            m.decode_step(toks, pos, kv, lg, am)
+            torch.cuda.synchronize()
+        outs.append(lg.cpu().numpy().copy())
+    assert np.array_equal(outs[0], outs[1])
+    assert m.sync_status() == 0
+    valid = tr[:, :, 2] > 0
+    assert valid[:, 0].all()  # every CTA ran at least its first task
+    tb, td, te = tr[:, :, 0][valid], tr[:, :, 1][valid], tr[:, :, 2][valid]
+    assert (tb <= td).all() and (td <= te).all()
+    s = trace.summarize(tr)
+    assert s["step_us"] > 0 and 0.0 < s["compute_fraction"] <= 1.0
+    kv.close()
