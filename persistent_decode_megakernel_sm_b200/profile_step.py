@@ -7,7 +7,9 @@ smaller vocabulary) for an external profiler: seeded weights and context,
 A cut keeps every per-layer shape of the workload, so the kernel's per-layer
 behaviour (tiles, chunks, attention splits) is the full model's; only the
 number of layers and the LM head / embedding rows shrink.  Prints the bytes
-the step must move (weights, cache rows, logits) for the cut."""
+the step must move (weights, cache rows, logits) for the cut.  For MoE models
+the weight figure counts every resident expert, an upper bound: a step reads
+only the shared experts and the routed experts its rows pick."""
 from __future__ import annotations
 
 import argparse
@@ -53,8 +55,9 @@ def main():
     weights = m.weight_bytes() - mc.vocab * mc.hidden * 2 + B * mc.hidden * 2
     kvt = (mc.kv_lora_rank + mc.rope_dim) * 2 if mc.mla else 2 * mc.n_kv_heads * mc.head_dim * 2
     cache = B * (mc.context + a.warmup) * kvt * mc.layers + B * kvt * mc.layers
+    key = "weight_bytes_resident_upper_bound" if mc.n_routed else "weight_bytes_streamed"
     print(json.dumps({"config": a.config, "layers": mc.layers, "vocab": mc.vocab, "batch": B,
-                      "weight_bytes_streamed": weights, "cache_bytes": cache, "logit_bytes": B * mc.vocab * 4,
+                      key: weights, "cache_bytes": cache, "logit_bytes": B * mc.vocab * 4,
                       "bytes_per_step_first_profiled": weights + cache + B * mc.vocab * 4}))
     kv.close()
     m.close()
