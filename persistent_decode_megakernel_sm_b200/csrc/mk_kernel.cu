@@ -229,7 +229,6 @@ struct Misc {
   uint64_t full[NSTAGE];
   uint64_t empty[NSTAGE];
   uint64_t xfull[XSLOTS];   // activation slice landed (bulk copy)
-  uint64_t xready[XSLOTS];  // ... and converted to mma fragments
   uint64_t xempty[XSLOTS];
   float scale[MAXM];
   float xscale[XSLOTS][MAXM];  // RMSNorm scale of the rows of the window in each activation slot
@@ -836,10 +835,14 @@ drain:
 // Convert an activation window in place into ready mma B fragments: col tile
 // jj of row m (16 fp32, 64 B) becomes, for each quad lane tq, 16 B =
 // {hi(k 2tq,2tq+1), hi(k 2tq+8,2tq+9), lo(..), lo(..)} of x * rms_scale * gain
-// (bf16 split; f16 for fp8 weights).  Threads t0, t0 + nt, ... share the work.
-__device__ __forceinline__ void convert_window(uint8_t* dst, int rb, int M, int wn, int w0, bool has_gain,
-                                               const uint16_t* gain, const float* scale, bool f16, int t0, int nt) {
-  for (int e = t0; e < M * wn; e += nt) {
+// (bf16 split; f16 for fp8 weights).  All consumer threads share the work.
+// Only inputs that no producer writes in fragment layout need it (the
+// absorbed-query GEMV of latent attention reads the raw QKV output).  Out of
+// line: keeps the GEMV inner loops small (one CTA runs every phase of the
+// step, so their instruction footprint matters).
+__device__ __noinline__ void convert_window_coop(uint8_t* dst, int rb, int M, int wn, int w0, bool has_gain,
+                                                 const uint16_t* gain, const float* scale, bool f16) {
+  for (int e = threadIdx.x; e < M * wn; e += NCT) {
     const int mm = e / wn, jj = e - mm * wn;
     float4* p4 = reinterpret_cast<float4*>(dst + (size_t)mm * rb + (size_t)jj * 64);
     float v[16];
@@ -880,17 +883,6 @@ __device__ __forceinline__ void convert_window(uint8_t* dst, int rb, int M, int 
   // the slot is written again by bulk copies (async proxy) once released
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-
-// Out of line for the consumers: keeps the GEMV inner loops small (one CTA
-// runs every phase of the step, so their instruction footprint matters).
-__device__ __noinline__ void convert_window_coop(uint8_t* dst, int rb, int M, int wn, int w0, bool has_gain,
-                                                 const uint16_t* gain, const float* scale, bool f16) {
-  convert_window(dst, rb, M, wn, w0, has_gain, gain, scale, f16, threadIdx.x, NCT);
-}
-
-// Windows of more than XCONV_M rows are converted by all consumer warps
-// together (a single warp would fall behind the tensor cores at M = 8).
-constexpr int XCONV_M = 0;
 
 __device__ bool xprod_reserve(const Ctx& C, uint32_t ix, uint32_t bytes) {
   const int lane = threadIdx.x & 31;
@@ -961,11 +953,10 @@ __device__ void xproducer(const Ctx& C) {
     if (!pc.init(rt0, rt1, gsz, nseg)) continue;
     // RMSNorm scale of every activation row (fixed-order reduction of the
     // per-CTA sums of squares), computed once the task's first activation
-    // copy is in flight, and the norm gain of this task
+    // copy is in flight
     float scale[MAXM];
     const bool has_gain = t.in_kind == IN_X_NORM;
     bool have_scale = !has_gain;
-    const uint16_t* gain = t.gvec;
 #pragma unroll
     for (int mm = 0; mm < MAXM; ++mm) scale[mm] = 1.f;
     do {
@@ -1005,28 +996,7 @@ __device__ void xproducer(const Ctx& C) {
           mbar_arrive(&C.ms->xfull[sl]);
         }
         __syncwarp();
-        if (M > XCONV_M || t.in_kind == IN_X_NORM || frag_buf(t.in_buf)) {
-          // the consumers convert this window themselves, or it needs no conversion
-          ++ix;
-          continue;
-        }
-        // wait for this warp's own copy, then convert the window in place
-        {
-          const uint32_t par = (ix / XSLOTS) & 1;
-          const uint64_t t0 = globaltimer();
-          bool landed = true;
-          while (!mbar_try_wait(&C.ms->xfull[sl], par)) {
-            if (C.ms->abort || globaltimer() - t0 > (uint64_t)P.timeout_ns * 2) { landed = false; break; }
-          }
-          if (!__all_sync(0xffffffffu, landed)) {
-            if (lane == 0 && !C.ms->abort) raise_error(P, C.ms, DERR_TIMEOUT, 0x60000 | sl);
-            goto drain;
-          }
-        }
-        convert_window(dst, rb, M, wn, w0, has_gain, gain, C.ms->xscale[sl], m.fp8 != 0, lane, 32);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&C.ms->xready[sl]);
-        ++ix;
+        ++ix;  // the consumers convert the window, where it needs converting
       } while (ci.next());
     } while (pc.next());
   }
@@ -1135,10 +1105,10 @@ __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z));
 
 // Wait for activation slot `ix`: converted by the activation producer
 // (`landed` false), or only landed, for the consumers to convert (true).
-__device__ __forceinline__ void wait_x(const Ctx& C, uint32_t ix, bool landed = false) {
+__device__ __forceinline__ void wait_x(const Ctx& C, uint32_t ix) {
   const int s = ix % XSLOTS;
   const uint32_t par = (ix / XSLOTS) & 1;
-  uint64_t* bar = landed ? &C.ms->xfull[s] : &C.ms->xready[s];
+  uint64_t* bar = &C.ms->xfull[s];
   const bool tr = MK_TRACE && C.P->trace && threadIdx.x == 0;
   const long long c0 = tr ? clock64() : 0;
   if ((threadIdx.x & 31) == 0) {
@@ -1151,7 +1121,7 @@ __device__ __forceinline__ void wait_x(const Ctx& C, uint32_t ix, bool landed = 
         uint64_t now = globaltimer();
         if (t0 == 0) t0 = now;
         else if (now - t0 > (uint64_t)C.P->timeout_ns * 2) {
-          raise_error(*C.P, C.ms, DERR_TIMEOUT, (landed ? 0x58000 : 0x50000) | s);
+          raise_error(*C.P, C.ms, DERR_TIMEOUT, 0x58000 | s);
           break;
         }
       }
@@ -1166,7 +1136,6 @@ __device__ __forceinline__ void wait_x(const Ctx& C, uint32_t ix, bool landed = 
 struct GemvLane {
   int warp, lane, g, tq, M, rowbytes;
   bool has_gain, trc;
-  bool coop;              // the consumers convert the activation windows (M > XCONV_M)
   bool conv;              // the windows need converting (false: the input buffer holds fragments)
   const uint16_t* gain;   // norm gain of the task's input
 };
@@ -1245,14 +1214,12 @@ __device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
     const uint8_t* slot = C.xring + (size_t)(ix % XSLOTS) * XSLOT_BYTES;
     if (ci.win_first()) {
       if (!L.conv) {
-        wait_x(C, ix, true);  // the window arrives in fragment layout: nothing to do
+        wait_x(C, ix);  // the window arrives in fragment layout: nothing to do
         // normed input: the rows' RMS scales, applied to the group's sums
         if (L.has_gain && ci.c0 == 0 && L.warp == 0 && lane < MAXM)
           C.ms->gscale[lane] = C.ms->xscale[ix % XSLOTS][lane];
-      } else if (!L.coop) {
-        wait_x(C, ix);  // the window arrives converted
       } else {
-        wait_x(C, ix, true);
+        wait_x(C, ix);
         const long long tv0 = L.trc ? clock64() : 0;
         convert_window_coop(const_cast<uint8_t*>(slot), L.rowbytes, L.M, ci.wn(), ci.w0(), L.has_gain, L.gain,
                             C.ms->xscale[ix % XSLOTS], FP8);
@@ -1410,7 +1377,6 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
   L.has_gain = has_gain;
   L.rowbytes = 0;
   L.trc = MK_TRACE && P.trace && tid == 0;
-  L.coop = M > XCONV_M;
   L.conv = t.in_kind != IN_X_NORM && !frag_buf(t.in_buf);
   L.gain = t.gvec;
   if (L.trc) C.ms->tr_pre += clock64() - tpre;
@@ -2656,7 +2622,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) mk_step_kernel(const __grid_const
     }
     for (int s = 0; s < XSLOTS; ++s) {
       mbar_init(&C.ms->xfull[s], 2);  // the copies' expect-tx arrival + the scales
-      mbar_init(&C.ms->xready[s], 1);
       mbar_init(&C.ms->xempty[s], NCW);
     }
     C.ms->abort = 0;
