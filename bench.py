@@ -51,6 +51,23 @@ def parse():
     return ap.parse_args()
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest of the ranks' values, on every rank (the job's time is its
+    slowest rank's); x itself when there is one rank."""
+    if world <= 1:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job throughput: the units all ranks processed (each rank the same
+    number, weak scaling) per second of the slowest rank's time."""
+    return world * units_per_rank / (ms / 1e3)
+
+
 def recorded_traffic(config: str, B: int):
     """DRAM bytes per launch recorded from an ncu capture under profiles/,
     valid only while the kernel sources are the ones it was taken on (the
@@ -224,11 +241,7 @@ def run_ours(args, rank, world, local_rank):
         clk = ck.stop() if ck else None
         assert model.sync_status() == 0, "device error in the timed region"
         per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
-        ms = ev[0].elapsed_time(ev[steps])
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            ms = float(t.item())
+        ms = max_over_ranks(ev[0].elapsed_time(ev[steps]), world, dev)
         unions = None
         if mc.n_routed:
             kv.fill_random(synth.SEED_KV, mc.kv_sigma, mc.context)
@@ -248,7 +261,7 @@ def run_ours(args, rank, world, local_rank):
         mean_bytes = statistics.mean(nbytes)
         launch_ms = statistics.mean(per)
         gbs = mean_bytes / (launch_ms / 1e3) / 1e9
-        out = {"tokens_per_s": world * B * steps / (ms / 1e3), "ms_per_step": ms / steps,
+        out = {"tokens_per_s": job_rate(B * steps, world, ms), "ms_per_step": ms / steps,
                "bytes_per_step": mean_bytes, "hbm_gbs": gbs, "frac_of_measured": gbs / peak, "frac_of_8tbs": gbs / 8000.0}
         if unions:
             out["routed_experts_per_layer_mean"] = statistics.mean(statistics.mean(u) for u in unions)
@@ -353,13 +366,9 @@ def run_ours(args, rank, world, local_rank):
         h_tok.copy_(h_out)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     assert model.sync_status() == 0
-    e2e = {"value": world * B * E / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": 2 * B * 4,
+    e2e = {"value": job_rate(B * E, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": 2 * B * 4,
            "d2h_bytes_per_step": B * 4}
     kv.close()
     model.close()
