@@ -9,7 +9,6 @@ LIB = os.path.join(HERE, "libmk.so")
 SRC = [os.path.join(HERE, "csrc", f) for f in ("mk_kernel.cu", "mk_kernel_traced.cu", "mk_host.cu")]
 DEPS = SRC + [os.path.join(HERE, "csrc", "mk_internal.h"), os.path.join(ROOT, "include", "mk.h"),
               os.path.join(ROOT, "synth", "synth.h")]
-DEPS.append(os.path.join(HERE, "csrc", "mk_kernel.cu"))  # included by mk_kernel_traced.cu
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
          "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
