@@ -78,3 +78,37 @@ def test_moe_one_layer(B):
 def test_mla_fp8_one_layer(B):
     mc = synth.preset("mla_fp8", layers=1, gain_sigma=0.1)
     _run(mc, B, mc.context)
+
+
+def test_moe_one_layer_verify():
+    """1 anchor + 7 seeded random proposals (the verify workload's input) at the
+    MoE model's full per-layer sizes over its 4096-position context: 8 causal
+    query rows of one sequence in one launch."""
+    mc = synth.preset("moe", layers=1, gain_sigma=0.1)
+    m = gpu_model(mc)
+    P = mc.context
+    kv = m.kv_cache(1, mc.max_ctx)
+    kv.fill_random(synth.SEED_KV, mc.kv_sigma, P)
+    orc = oracle.OracleModel(mc.replace(max_seqs=1))
+    orc.kv_fill_synthetic(synth.SEED_KV, P)
+    toks = [int(tokens_at(mc, 0, [P])[0])] + [int(x) for x in synth.proposals(synth.SEED_PROPOSALS, 0, 7, mc.vocab)]
+    logits = torch.empty((8, mc.vocab), dtype=torch.float32, device=DEV)
+    am = torch.empty(8, dtype=torch.int32, device=DEV)
+    acc = torch.full((1,), -1, dtype=torch.int32, device=DEV)
+    m.verify(_t(toks), P, kv, logits, am, acc)
+    ref = orc.step(toks, [P], Q=8)
+    torch.cuda.synchronize()
+    g = logits.cpu().numpy()
+    ga = am.cpu().numpy()
+    tied = [j for j in range(8) if (ref["router_margin"][:, j] < DELTA).any()]
+    for j in range(8):
+        if j in tied:
+            continue
+        ok, err, sc = logits_close(g[j], ref["logits"][j])
+        assert ok, (j, err, sc)
+        assert argmax_agrees(int(ga[j]), ref["logits"][j], int(ref["argmax"][j]), ref["argmax_margin"][j])
+    if not tied and all(int(ga[j]) == int(ref["argmax"][j]) for j in range(8)):
+        assert int(acc.item()) == oracle.accept(toks, ref["argmax"])
+    assert m.sync_status() == 0
+    kv.close()
+    m.close()
