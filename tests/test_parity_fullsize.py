@@ -80,11 +80,7 @@ def test_mla_fp8_one_layer(B):
     _run(mc, B, mc.context)
 
 
-def test_moe_one_layer_verify():
-    """1 anchor + 7 seeded random proposals (the verify workload's input) at the
-    MoE model's full per-layer sizes over its 4096-position context: 8 causal
-    query rows of one sequence in one launch."""
-    mc = synth.preset("moe", layers=1, gain_sigma=0.1)
+def _verify_one_layer(mc):
     m = gpu_model(mc)
     P = mc.context
     kv = m.kv_cache(1, mc.max_ctx)
@@ -96,7 +92,7 @@ def test_moe_one_layer_verify():
     am = torch.empty(8, dtype=torch.int32, device=DEV)
     acc = torch.full((1,), -1, dtype=torch.int32, device=DEV)
     m.verify(_t(toks), P, kv, logits, am, acc)
-    ref = orc.step(toks, [P], Q=8)
+    ref = orc.step(toks, [P], Q=8, absorbed=mc.mla)
     torch.cuda.synchronize()
     g = logits.cpu().numpy()
     ga = am.cpu().numpy()
@@ -104,11 +100,23 @@ def test_moe_one_layer_verify():
     for j in range(8):
         if j in tied:
             continue
-        ok, err, sc = logits_close(g[j], ref["logits"][j])
-        assert ok, (j, err, sc)
+        ok, err, sc = logits_close(g[j], ref["logits"][j], fp8=bool(mc.expert_fp8))
+        assert ok, (mc.name, j, err, sc)
         assert argmax_agrees(int(ga[j]), ref["logits"][j], int(ref["argmax"][j]), ref["argmax_margin"][j])
     if not tied and all(int(ga[j]) == int(ref["argmax"][j]) for j in range(8)):
         assert int(acc.item()) == oracle.accept(toks, ref["argmax"])
     assert m.sync_status() == 0
     kv.close()
     m.close()
+
+
+def test_moe_one_layer_verify():
+    """1 anchor + 7 seeded random proposals (the verify workload's input) at the
+    MoE model's full per-layer sizes over its 4096-position context: 8 causal
+    query rows of one sequence in one launch."""
+    _verify_one_layer(synth.preset("moe", layers=1, gain_sigma=0.1))
+
+
+def test_mla_fp8_one_layer_verify():
+    """The same with latent attention over 8192 cached positions and fp8 experts."""
+    _verify_one_layer(synth.preset("mla_fp8", layers=1, gain_sigma=0.1))
