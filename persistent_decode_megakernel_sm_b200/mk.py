@@ -52,7 +52,7 @@ class mk_tensor_src(ctypes.Structure):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libmk.so not built ({LIB_PATH}); run `python -m persistent_decode_megakernel_sm_b200.build`")
+        raise ImportError(f"libmk.so not built ({LIB_PATH}); run `python persistent_decode_megakernel_sm_b200/build.py`")
     L = ctypes.CDLL(LIB_PATH)
     vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
     st = ctypes.c_int
