@@ -36,7 +36,8 @@ def lib() -> ctypes.CDLL:
             getattr(L, f).argtypes = [vp]
             getattr(L, f).restype = vp
         L.orc_kv_fill_synthetic.argtypes = [vp, ctypes.c_uint64, i32]
-        L.orc_step.argtypes = [vp, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int]
+        L.orc_step.argtypes = [vp, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int,
+                               vp, dbl, vp]
         L.orc_step.restype = ctypes.c_int
         L.orc_forward_full.argtypes = [ctypes.POINTER(OrcCfg), ctypes.c_int, vp, vp]
         L.orc_forward_full.restype = ctypes.c_int
@@ -47,6 +48,8 @@ def lib() -> ctypes.CDLL:
         L.orc_silu.argtypes = [dbl]
         L.orc_silu.restype = dbl
         L.orc_router_select.argtypes = [ctypes.c_int, ctypes.c_int, vp, vp, vp, vp]
+        L.orc_router_select_follow.argtypes = [ctypes.c_int, ctypes.c_int, vp, vp, dbl, vp, vp, vp]
+        L.orc_router_select_follow.restype = ctypes.c_int
         L.orc_e4m3_value.argtypes = [ctypes.c_uint8]
         L.orc_e4m3_value.restype = dbl
         L.orc_bf16_round.argtypes = [dbl]
@@ -127,6 +130,19 @@ def router_select(logits, k):
     mg = np.empty(1, dtype=np.float64)
     lib().orc_router_select(len(lg), k, _p(lg), _p(idx), _p(w), _p(mg))
     return idx, w, float(mg[0])
+
+
+def router_select_follow(logits, k, follow, delta):
+    """Router selection with the near-tie protocol: `follow` is adopted only
+    when the oracle's own k-th / (k+1)-th gap is below delta and `follow` is a
+    valid choice at that tolerance.  Returns (idx, w, margin, followed)."""
+    lg = _d(logits)
+    fo = np.ascontiguousarray(follow, dtype=np.int32)
+    idx = np.empty(k, dtype=np.int32)
+    w = np.empty(k, dtype=np.float64)
+    mg = np.empty(1, dtype=np.float64)
+    fl = lib().orc_router_select_follow(len(lg), k, _p(lg), _p(fo), delta, _p(idx), _p(w), _p(mg))
+    return idx, w, float(mg[0]), bool(fl)
 
 
 def e4m3_value(code: int) -> float:
@@ -241,8 +257,26 @@ class OracleModel:
         v = np.ctypeslib.as_array(ctypes.cast(lib().orc_kv_v(self.h), ctypes.POINTER(ctypes.c_uint16)), shape=(n,))
         return k.reshape(shape), v.reshape(shape)
 
-    def step(self, tokens, pos0, Q: int = 1, want_logits: bool = True, absorbed: bool = False):
-        """One decode (Q=1) or verify (Q>1) step for S = len(pos0) sequences."""
+    def set_kv(self, gpu_logical: np.ndarray):
+        """Take a cache written elsewhere as this model's input (the layout of
+        the GPU library's logical copy-out: GQA keys then values, or latent
+        rows), for contexts prefilled by the GPU."""
+        flat = np.ascontiguousarray(gpu_logical).view(np.uint16).reshape(-1)
+        if self.mc.mla:
+            lat = self.kv_arrays()
+            assert flat.size == lat.size, (flat.size, lat.size)
+            lat.reshape(-1)[:] = flat
+        else:
+            k, v = self.kv_arrays()
+            assert flat.size == k.size + v.size, (flat.size, k.size, v.size)
+            k.reshape(-1)[:] = flat[:k.size]
+            v.reshape(-1)[:] = flat[k.size:]
+
+    def step(self, tokens, pos0, Q: int = 1, want_logits: bool = True, absorbed: bool = False,
+             follow=None, delta: float = 1e-3):
+        """One decode (Q=1) or verify (Q>1) step for S = len(pos0) sequences.
+        follow: router choices [layers][S*Q][top_k] of the implementation
+        under test, adopted only at near-ties (margin < delta)."""
         mc = self.mc
         tokens = np.ascontiguousarray(tokens, dtype=np.int32).reshape(-1)
         pos0 = np.ascontiguousarray(pos0, dtype=np.int32).reshape(-1)
@@ -256,12 +290,16 @@ class OracleModel:
         ridx = np.zeros((mc.layers, M, k), dtype=np.int32)
         rw = np.zeros((mc.layers, M, k), dtype=np.float64)
         rmargin = np.full((mc.layers, M), np.inf, dtype=np.float64)
+        fo = None
+        if follow is not None and mc.n_routed:
+            fo = np.ascontiguousarray(follow, dtype=np.int32).reshape(mc.layers, M, k)
+        followed = np.zeros((mc.layers, M), dtype=np.int32)
         rc = lib().orc_step(self.h, S, Q, _p(tokens), _p(pos0), _p(logits), _p(amax), _p(amargin),
-                            _p(ridx), _p(rw), _p(rmargin), int(absorbed))
+                            _p(ridx), _p(rw), _p(rmargin), int(absorbed), _p(fo), float(delta), _p(followed))
         if rc != 0:
             raise ValueError("oracle: bad step arguments")
         return dict(logits=logits, argmax=amax, argmax_margin=amargin,
-                    router_idx=ridx, router_w=rw, router_margin=rmargin)
+                    router_idx=ridx, router_w=rw, router_margin=rmargin, router_followed=followed.astype(bool))
 
 
 def forward_full(mc, tokens):

@@ -266,6 +266,44 @@ void orc_router_select(int E, int k, const double* logits, int32_t* idx, double*
   free(ord);
 }
 
+/* Near-tie protocol.  The pages fix no precision, so a router decision whose
+ * gap between the k-th and (k+1)-th logit is below `delta` has two correct
+ * answers at the precision of the arithmetic.  Another implementation's
+ * selection `follow` (k expert indices) is adopted at such a near-tie when it
+ * is a valid answer at that tolerance: every followed expert's logit is at
+ * least the k-th logit minus delta, no expert whose logit exceeds the k-th
+ * logit plus delta is left out, and no expert appears twice.  The weights
+ * are then this oracle's own softmax probabilities of the followed experts,
+ * renormalised over them.  Returns 1 when the selection was followed. */
+int orc_router_select_follow(int E, int k, const double* logits, const int32_t* follow, double delta,
+                             int32_t* idx, double* w, double* margin) {
+  double mg;
+  orc_router_select(E, k, logits, idx, w, &mg);
+  if (margin) *margin = mg;
+  if (!follow || !(mg < delta)) return 0;
+  /* the oracle's own k-th largest logit */
+  double kth = logits[idx[k - 1]];
+  for (int j = 0; j < k; ++j) {
+    int e = follow[j];
+    if (e < 0 || e >= E || logits[e] < kth - delta) return 0;
+    for (int q = 0; q < j; ++q)
+      if (follow[q] == e) return 0;
+  }
+  for (int e = 0; e < E; ++e) {
+    if (!(logits[e] > kth + delta)) continue;
+    int found = 0;
+    for (int j = 0; j < k; ++j) found |= (follow[j] == e);
+    if (!found) return 0;
+  }
+  double* p = (double*)malloc((size_t)E * sizeof(double));
+  orc_softmax(E, logits, p);
+  double s = 0.0;
+  for (int j = 0; j < k; ++j) { idx[j] = follow[j]; s += p[follow[j]]; }
+  for (int j = 0; j < k; ++j) w[j] = p[idx[j]] / s;
+  free(p);
+  return 1;
+}
+
 /* SwiGLU expert: y = W_d (silu(W_g x) * (W_u x)). */
 static void swiglu(const orc_mat* Wg, const orc_mat* Wu, const orc_mat* Wd, int M, const double* x, double* y) {
   int64_t I = Wg->rows;
@@ -291,11 +329,13 @@ void orc_swiglu_dense(int H, int I, const double* Wg, const double* Wu, const do
 static void moe_ffn(int H, int E, int k, int n_shared, const orc_mat* Wr,
                     const orc_mat* sg, const orc_mat* su, const orc_mat* sd, /* [n_shared] */
                     const orc_mat* eg, const orc_mat* eu, const orc_mat* ed, /* [E] */
-                    const double* x, double* y, int32_t* idx, double* w, double* margin) {
+                    const double* x, double* y, int32_t* idx, double* w, double* margin,
+                    const int32_t* follow, double delta, int32_t* followed) {
   double* lg = (double*)malloc((size_t)E * sizeof(double));
   double* t = (double*)malloc((size_t)H * sizeof(double));
   matvec(Wr, 1, x, lg);
-  orc_router_select(E, k, lg, idx, w, margin);
+  int fl = orc_router_select_follow(E, k, lg, follow, delta, idx, w, margin);
+  if (followed) *followed = fl;
   for (int i = 0; i < H; ++i) y[i] = 0.0;
   for (int j = 0; j < n_shared; ++j) {
     swiglu(&sg[j], &su[j], &sd[j], 1, x, t);
@@ -333,7 +373,7 @@ void orc_moe_ffn_dense(int H, int I, int E, int k, int n_shared, const double* W
     su[j] = (orc_mat){I, H, ORC_MAT_ARRAY, shu + (int64_t)j * I * H, 0, 0, 0.f, 0.f};
     sd[j] = (orc_mat){H, I, ORC_MAT_ARRAY, shd + (int64_t)j * H * I, 0, 0, 0.f, 0.f};
   }
-  moe_ffn(H, E, k, n_shared, &r, sg, su, sd, eg, eu, ed, x, y, idx, w, NULL);
+  moe_ffn(H, E, k, n_shared, &r, sg, su, sd, eg, eu, ed, x, y, idx, w, NULL, NULL, 0.0, NULL);
   free(eg); free(eu); free(ed); free(sg); free(su); free(sd);
 }
 
@@ -585,11 +625,15 @@ void orc_debug_mat_row(const orc_cfg* cfg, uint32_t kind, uint32_t layer, uint32
  * Row m = s*Q + j is sequence s at position pos0[s] + j with input tokens[m].
  * Outputs: logits [S*Q][V] (may be NULL), argmax [S*Q], argmax margin
  * (top1 - top2 logit), and per layer router trace [L][S*Q][k] when non-NULL.
+ * follow_idx ([L][S*Q][k] or NULL): another implementation's router choices,
+ * adopted only at near-ties of margin < follow_delta (orc_router_select_follow);
+ * followed ([L][S*Q] or NULL) records where that happened.
  * Returns 0, or -1 on an argument error.
  */
 int orc_step(orc_model* mdl, int S, int Q, const int32_t* tokens, const int32_t* pos0,
              double* logits, int32_t* amax, double* amargin,
-             int32_t* ridx, double* rw, double* rmargin, int mla_absorbed) {
+             int32_t* ridx, double* rw, double* rmargin, int mla_absorbed,
+             const int32_t* follow_idx, double follow_delta, int32_t* followed) {
   const orc_cfg* c = &mdl->c;
   int M = S * Q, H = c->hidden, L = c->layers, V = c->vocab;
   int Hq = c->n_q_heads, G = c->n_kv_heads, d = c->head_dim;
@@ -722,7 +766,10 @@ int orc_step(orc_model* mdl, int S, int Q, const int32_t* tokens, const int32_t*
       double* w = (double*)malloc((size_t)k * sizeof(double));
       for (int m = 0; m < M; ++m) {
         double mg;
-        moe_ffn(H, E, k, NS, &Wr, sg, su, sd, eg, eu, ed, h + (int64_t)m * H, t, idx, w, &mg);
+        int32_t fl = 0;
+        moe_ffn(H, E, k, NS, &Wr, sg, su, sd, eg, eu, ed, h + (int64_t)m * H, t, idx, w, &mg,
+                follow_idx ? follow_idx + ((int64_t)l * M + m) * k : NULL, follow_delta, &fl);
+        if (followed) followed[(int64_t)l * M + m] = fl;
         for (int i = 0; i < H; ++i) x[(int64_t)m * H + i] += t[i];
         if (ridx) for (int j = 0; j < k; ++j) ridx[((int64_t)l * M + m) * k + j] = idx[j];
         if (rw) for (int j = 0; j < k; ++j) rw[((int64_t)l * M + m) * k + j] = w[j];
@@ -873,7 +920,8 @@ int orc_forward_full(const orc_cfg* cfg, int T, const int32_t* tokens, double* l
       int32_t* idx = (int32_t*)malloc((size_t)k * sizeof(int32_t));
       double* w = (double*)malloc((size_t)k * sizeof(double));
       for (int p = 0; p < T; ++p)
-        moe_ffn(H, Ex, k, NS, &Wr, sg, su, sd, eg, eu, ed, h + (int64_t)p * H, t + (int64_t)p * H, idx, w, NULL);
+        moe_ffn(H, Ex, k, NS, &Wr, sg, su, sd, eg, eu, ed, h + (int64_t)p * H, t + (int64_t)p * H, idx, w, NULL,
+                NULL, 0.0, NULL);
       free(idx); free(w); free(eg); free(eu); free(ed); free(sg); free(su); free(sd);
     }
     for (int64_t i = 0; i < (int64_t)T * H; ++i) x[i] += t[i];

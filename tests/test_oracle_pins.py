@@ -254,6 +254,60 @@ def test_router_selection_is_stable_argsort():
         assert margin == srt[k - 1] - srt[k]
 
 
+def test_router_follow_only_at_valid_near_ties():
+    """The near-tie protocol: another selection is adopted only where the
+    oracle's own k-th / (k+1)-th gap is below delta, and only when it is a
+    correct top-k at that tolerance; the weights are then the oracle's own
+    softmax renormalised over the adopted experts."""
+    lg = np.array([3.0, 1.0, 2.0, 2.0 + 5e-4, 0.5, -1.0])
+    own, _, mg = oracle.router_select(lg, 2)
+    assert list(own) == [0, 3] and abs(mg - 5e-4) < 1e-15
+    idx, w, _, fl = oracle.router_select_follow(lg, 2, [0, 2], 1e-3)
+    p = scipy.special.softmax(lg)
+    assert fl and list(idx) == [0, 2]
+    assert np.allclose(w, p[[0, 2]] / p[[0, 2]].sum(), rtol=1e-14)
+    # not a near-tie at this delta: the oracle keeps its own choice
+    idx, w, _, fl = oracle.router_select_follow(lg, 2, [0, 2], 1e-4)
+    assert not fl and list(idx) == [0, 3]
+    # a near-tie, but the proposed expert is far below the k-th logit
+    idx, _, _, fl = oracle.router_select_follow(lg, 2, [0, 4], 1e-3)
+    assert not fl and list(idx) == [0, 3]
+    # a near-tie, but a clear winner (logit 3.0) is left out
+    idx, _, _, fl = oracle.router_select_follow(lg, 2, [2, 3], 1e-3)
+    assert not fl and list(idx) == [0, 3]
+    # a repeated expert is no selection
+    idx, _, _, fl = oracle.router_select_follow(lg, 2, [3, 3], 1e-3)
+    assert not fl and list(idx) == [0, 3]
+    # following its own choice changes nothing
+    idx, w2, _, _ = oracle.router_select_follow(lg, 2, own, 1e-3)
+    assert list(idx) == list(own) and np.allclose(w2, oracle.router_select(lg, 2)[1], rtol=0, atol=0)
+
+
+def test_model_follow_changes_only_near_tied_decisions():
+    """On a whole MoE step: following the oracle's own router choices is the
+    identity, and a different choice at a decision that is not a near-tie is
+    ignored (the step is bit-identical)."""
+    mc = synth.preset("tiny_moe", max_seqs=2, max_ctx=48)
+    toks, pos = [5, 77], [6, 3]
+    a = oracle.OracleModel(mc)
+    a.kv_fill_synthetic(synth.SEED_KV, 10)
+    ref = a.step(toks, pos)
+    b = oracle.OracleModel(mc)
+    b.kv_fill_synthetic(synth.SEED_KV, 10)
+    same = b.step(toks, pos, follow=ref["router_idx"])
+    assert np.array_equal(same["logits"], ref["logits"])
+    assert np.array_equal(same["router_idx"], ref["router_idx"])
+    bad = ref["router_idx"].copy()
+    l, r = np.unravel_index(np.argmax(ref["router_margin"]), ref["router_margin"].shape)
+    assert ref["router_margin"][l, r] > 1e-3
+    bad[l, r, -1] = [e for e in range(mc.n_routed) if e not in bad[l, r]][0]
+    c = oracle.OracleModel(mc)
+    c.kv_fill_synthetic(synth.SEED_KV, 10)
+    kept = c.step(toks, pos, follow=bad)
+    assert not kept["router_followed"][l, r]
+    assert np.array_equal(kept["logits"], ref["logits"])
+
+
 def test_router_k_equals_E_is_softmax():
     lg = rng.normal(size=16)
     idx, w, _ = oracle.router_select(lg, 16)
