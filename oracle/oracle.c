@@ -151,11 +151,26 @@ static void mat_row(const orc_mat* W, int64_t r, double* out) {
       for (int64_t c = 0; c < C; ++c) out[c] = bf16_to_double(syn_bf16_gain(W->key, (uint64_t)c, W->scale));
       break;
     case ORC_MAT_FP8: {
+      /* the same values as orc_e4m3_value(code) * block scale, element by
+       * element; the decode is looked up in a table of orc_e4m3_value and the
+       * scale is drawn once per 128-column block */
+      static double e4m3_tab[256];
+      static int e4m3_tab_ready = 0;
+      if (!e4m3_tab_ready) {
+#pragma omp critical(orc_e4m3_tab)
+        {
+          if (!e4m3_tab_ready) {
+            for (int q = 0; q < 256; ++q) e4m3_tab[q] = orc_e4m3_value((uint8_t)q);
+            __atomic_store_n(&e4m3_tab_ready, 1, __ATOMIC_RELEASE);
+          }
+        }
+      }
       int64_t nbc = (C + 127) / 128;
-      for (int64_t c = 0; c < C; ++c) {
-        double w = orc_e4m3_value(syn_e4m3_normal(W->key, (uint64_t)(r * C + c), W->scale));
-        double s = (double)syn_block_scale(W->skey, (uint64_t)((r / 128) * nbc + c / 128), W->base);
-        out[c] = w * s;
+      for (int64_t cb = 0; cb < nbc; ++cb) {
+        double s = (double)syn_block_scale(W->skey, (uint64_t)((r / 128) * nbc + cb), W->base);
+        int64_t c1 = (cb + 1) * 128 < C ? (cb + 1) * 128 : C;
+        for (int64_t c = cb * 128; c < c1; ++c)
+          out[c] = e4m3_tab[syn_e4m3_normal(W->key, (uint64_t)(r * C + c), W->scale)] * s;
       }
       break;
     }
