@@ -41,9 +41,13 @@ def parse():
     ap.add_argument("--config", default="dense27b")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--sweep", default="1,2,4,8", help="batch sizes timed for the by_batch table ('' = none)")
-    ap.add_argument("--workloads", default="moe,mla_fp8,verify",
+    ap.add_argument("--workloads", default="tiny,moe,verify,mla_fp8",
                     help="other workloads of the study timed after the headline ('' = none)")
     ap.add_argument("--verify-steps", type=int, default=256)
+    ap.add_argument("--sweep-steps", type=int, default=64,
+                    help="timed steps of each other batch size and workload (the study's configs use 64)")
+    ap.add_argument("--oracle-steps", type=int, default=3,
+                    help="full-depth oracle steps timed for cpu_baseline")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per launch of the kernel from an ncu capture of this build (null if none)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -196,19 +200,44 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.current_stream()
     peak, peak_kind = measured_peaks()
 
+    prefill_s = {}
+
     def load(config):
+        """The workload's model (seeded weights) and a cache of 8 sequences
+        whose context is sequence 0's seeded prompt run through the model on
+        the GPU (mk_prefill, 8 positions per launch), copied to the other
+        sequences.  Returns the model, the cache and a function that puts the
+        cache back to that context."""
         mc = synth.preset(config)
         model = Megakernel(mc, device=local_rank, max_batch=8)
         model.init_random(mc.seed, mc.w_sigma, mc.router_sigma, mc.gain_sigma, mc.fp8_block_base)
         kv = model.kv_cache(8, mc.max_ctx)
-        kv.fill_random(synth.SEED_KV, mc.kv_sigma, mc.context)
-        return mc, model, kv
+        prompt = torch.tensor(synth.seq_tokens(synth.SEED_TOKENS, 0, range(mc.context), mc.vocab), dtype=torch.int32,
+                              device=dev)
+        t0 = time.perf_counter()
+        model.prefill(prompt, 0, 0, kv, stream=stream)
+        torch.cuda.synchronize()
+        prefill_s[config] = time.perf_counter() - t0
+        assert model.sync_status() == 0, "device error in the prefill"
+        snap = kv.copy_out()
+        if mc.mla:
+            v = snap.view(mc.layers, 8, -1)
+            v[:, 1:] = v[:, :1]
+        else:
+            v = snap.view(2, mc.layers, 8, -1)
+            v[:, :, 1:] = v[:, :, :1]
+        kv.copy_in(snap)
+
+        def restore():
+            kv.copy_in(snap)
+
+        return mc, model, kv, restore
 
     def router_unions(mc, idx):
         a = idx.cpu().numpy()
         return [len(set(a[l].reshape(-1).tolist())) for l in range(mc.layers)]
 
-    def decode_run(mc, model, kv, B, steps, warmup, clocks=False):
+    def decode_run(mc, model, kv, restore, B, steps, warmup, clocks=False):
         """Greedy decode of B sequences from the synthetic context: `warmup`
         untimed steps, then `steps` steps timed with CUDA events on the
         launching stream.  For MoE models the same steps are replayed
@@ -220,7 +249,7 @@ def run_ours(args, rank, world, local_rank):
         toks = torch.tensor(synth.tokens(synth.SEED_TOKENS, B, mc.vocab), dtype=torch.int32, device=dev)
         am = [torch.zeros(B, dtype=torch.int32, device=dev) for _ in range(total)]
         logits = torch.empty((B, mc.vocab), dtype=torch.float32, device=dev)
-        kv.fill_random(synth.SEED_KV, mc.kv_sigma, mc.context)
+        restore()
         cur = toks
         for i in range(warmup):
             model.decode_step(cur, pos[i], kv, logits, am[i], stream)
@@ -244,7 +273,7 @@ def run_ours(args, rank, world, local_rank):
         ms = max_over_ranks(ev[0].elapsed_time(ev[steps]), world, dev)
         unions = None
         if mc.n_routed:
-            kv.fill_random(synth.SEED_KV, mc.kv_sigma, mc.context)
+            restore()
             idx = torch.zeros((mc.layers, B, mc.top_k), dtype=torch.int32, device=dev)
             w = torch.zeros((mc.layers, B, mc.top_k), dtype=torch.float32, device=dev)
             unions = []
@@ -267,14 +296,14 @@ def run_ours(args, rank, world, local_rank):
             out["routed_experts_per_layer_mean"] = statistics.mean(statistics.mean(u) for u in unions)
         return out, ms, per, clk, mean_bytes
 
-    def verify_run(mc, model, kv, steps, warmup):
+    def verify_run(mc, model, kv, restore, steps, warmup):
         """Speculative verify on one sequence: each step checks an anchor and
         7 seeded uniform proposals at position P over the synthetic context;
         the next anchor is the greedy token after the accepted prefix and P
         advances by accepted + 1 (rewound to the context end when the cache
         would overflow).  Device time per launch from CUDA events."""
         def one_pass(record_unions):
-            kv.fill_random(synth.SEED_KV, mc.kv_sigma, mc.context)
+            restore()
             anchor = int(synth.tokens(synth.SEED_TOKENS, 1, mc.vocab)[0])
             P = mc.context
             am = torch.zeros(8, dtype=torch.int32, device=dev)
@@ -324,23 +353,153 @@ def run_ours(args, rank, world, local_rank):
                 "routed_experts_per_layer_mean": statistics.mean(statistics.mean(u) for u in unions),
                 "proposals": "seeded uniform over the vocabulary"}
 
+    def tiny_latency():
+        """The small dense workload: 128 positions prefilled from seeded
+        tokens, then 16 greedy steps at B = 1, each timed alone (CUDA events
+        around each launch): step latency, no roofline claim (the model is
+        resident in L2)."""
+        tmc, tm, tkv, trestore = load("tiny")
+        n = 16
+        tok = torch.tensor(synth.seq_tokens(synth.SEED_TOKENS, 0, [tmc.context], tmc.vocab), dtype=torch.int32,
+                           device=dev)
+        ams = [torch.zeros(1, dtype=torch.int32, device=dev) for _ in range(n)]
+        times = []
+        for rep in range(2):  # the first pass warms up, the second is timed
+            trestore()
+            cur = tok
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * n)]
+            for i in range(n):
+                pos = torch.full((1,), tmc.context + i, dtype=torch.int32, device=dev)
+                ev[2 * i].record(stream)
+                tm.decode_step(cur, pos, tkv, None, ams[i], stream)
+                ev[2 * i + 1].record(stream)
+                cur = ams[i]
+            torch.cuda.synchronize()
+            times = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(n)]
+        assert tm.sync_status() == 0
+        tkv.close()
+        tm.close()
+        return {"greedy_steps": n, "ms_per_step_mean": statistics.mean(times), "ms_per_step_median": statistics.median(times),
+                "ms_per_step_max": max(times), "tokens_per_s": 1e3 / statistics.mean(times),
+                "note": "latency only: the 6 MB model is L2-resident, no roofline claim"}
+
+    def step_times(mc, model, kv, restore, B, steps, warmup, multikernel):
+        """Greedy decode of B sequences from the context: mean device time per
+        step (CUDA events on the launching stream) of the single persistent
+        kernel or of the multi-kernel comparison path (one kernel per phase in
+        a CUDA graph with programmatic dependent launch)."""
+        fn = model.decode_step_multikernel if multikernel else model.decode_step
+        total = warmup + steps
+        pos = torch.tensor([[mc.context + i] * B for i in range(total)], dtype=torch.int32, device=dev)
+        am = [torch.zeros(B, dtype=torch.int32, device=dev) for _ in range(total)]
+        restore()
+        cur = torch.tensor(synth.tokens(synth.SEED_TOKENS, B, mc.vocab), dtype=torch.int32, device=dev)
+        for i in range(warmup):
+            fn(cur, pos[i], kv, None, am[i], stream)
+            cur = am[i]
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(warmup, total):
+            fn(cur, pos[i], kv, None, am[i], stream)
+            cur = am[i]
+        e1.record(stream)
+        torch.cuda.synchronize()
+        assert model.sync_status() == 0
+        return e0.elapsed_time(e1) / steps, [int(a[0].item()) for a in am]
+
+    def compare_multikernel(mc, model, kv, restore, batches=(1, 8), steps=32):
+        out = {}
+        for b in batches:
+            one, t1 = step_times(mc, model, kv, restore, b, steps, 4, False)
+            multi, t2 = step_times(mc, model, kv, restore, b, steps, 4, True)
+            out[str(b)] = {"megakernel_ms_per_step": one, "multikernel_ms_per_step": multi,
+                           "megakernel_speedup": multi / one, "same_tokens": t1 == t2}
+        return out
+
+    def spec_run(mc, model, kv, restore, n_out=64, targets=(3, 6)):
+        """Speculative greedy generation (mk_spec_generate) on one sequence
+        from the end of the context, with a synthetic draft that proposes the
+        plain greedy chain (computed first by mk_decode_step) and corrupts
+        each proposal with a seeded probability chosen so that the mean
+        acceptance length (tokens emitted per verify launch) is the target.
+        Each run is timed with CUDA events around the whole call (it reads
+        every launch's accepted count on the host before the next launch)."""
+        import random
+        P = mc.context
+        anchor = int(synth.seq_tokens(synth.SEED_TOKENS, 0, [P], mc.vocab)[0])
+        restore()
+        chain = []
+        am = torch.zeros(1, dtype=torch.int32, device=dev)
+        cur = torch.tensor([anchor], dtype=torch.int32, device=dev)
+        for j in range(n_out + 8):
+            model.decode_step(cur, torch.tensor([P + j], dtype=torch.int32, device=dev), kv, None, am, stream)
+            cur = am.clone()
+            chain.append(cur)
+        chain = [int(x.item()) for x in chain]
+
+        def err_for(length):
+            # sum_{j=1..7} q^j = length - 1 (the mean of accepted + 1), q = 1 - err
+            lo, hi = 0.0, 1.0
+            for _ in range(60):
+                q = (lo + hi) / 2
+                if sum(q ** j for j in range(1, 8)) < length - 1:
+                    lo = q
+                else:
+                    hi = q
+            return 1.0 - lo
+
+        out = {}
+        for target in targets:
+            err = err_for(target)
+            rng = random.Random(1000 + target)
+
+            def draft(history, max_k):
+                e = len(history) - 1
+                props = []
+                for j in range(e, min(e + max_k, len(chain))):
+                    t = chain[j]
+                    if rng.random() < err:
+                        t = (t + 1 + rng.randrange(mc.vocab - 1)) % mc.vocab
+                    props.append(t)
+                return props
+
+            restore()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            toks, st = model.spec_generate(kv, anchor, P, n_out, draft, stream)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1)
+            out[f"acceptance_{target}"] = {
+                "per_proposal_error": err, "emitted": st["emitted"], "launches": st["launches"],
+                "acceptance_length_mean": st["emitted"] / st["launches"],
+                "emitted_tokens_per_s": st["emitted"] / (ms / 1e3), "ms_per_launch": ms / st["launches"],
+                "matches_plain_greedy": toks == chain[:n_out]}
+        assert model.sync_status() == 0
+        return out
+
     # ---- the headline workload ----
-    mc, model, kv = load(args.config)
+    mc, model, kv, restore = load(args.config)
     ctas, smem, threads = model.launch_info()
     B = args.batch
-    head, ms, per, clk, abytes = decode_run(mc, model, kv, B, args.steps, args.warmup, clocks=True)
+    head, ms, per, clk, abytes = decode_run(mc, model, kv, restore, B, args.steps, args.warmup, clocks=True)
     ms_step = ms / args.steps
     value = head["tokens_per_s"]
     launch_ms = statistics.mean(per)
     achieved = abytes / (launch_ms / 1e3) / 1e9
 
+    multikernel = {args.config: compare_multikernel(mc, model, kv, restore)}
+
+    # every timed run stays inside the cache: context + warm-up + steps <= max_ctx
+    sweep_steps = min(args.sweep_steps, mc.max_ctx - mc.context - 3)
     by_batch = {str(B): head}
     for b in [int(x) for x in args.sweep.split(",") if x]:
         if b != B:
-            by_batch[str(b)] = decode_run(mc, model, kv, b, max(8, args.steps // 4), 3)[0]
+            by_batch[str(b)] = decode_run(mc, model, kv, restore, b, sweep_steps, 3)[0]
 
     # ---- end to end through the public API with host buffers ----
-    kv.fill_random(synth.SEED_KV, mc.kv_sigma, mc.context)
+    restore()
     E = args.e2e_steps
     h_tok = torch.tensor(synth.tokens(synth.SEED_TOKENS, B, mc.vocab), dtype=torch.int32).pin_memory()
     h_pos = torch.tensor([mc.context] * B, dtype=torch.int32).pin_memory()
@@ -375,31 +534,47 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- the other workloads of the study (one GPU each, rank-local) ----
     workloads = {}
-    extra_steps = max(8, args.steps // 4)
+    cur_base, cur = None, None
     for name in [w for w in args.workloads.split(",") if w]:
+        if name == "tiny":
+            workloads["tiny"] = tiny_latency()
+            continue
+        base = "moe" if name == "verify" else name
+        if base != cur_base:
+            if cur:  # one model on the device at a time
+                cur[2].close()
+                cur[1].close()
+            cur, cur_base = load(base), base
+        wmc, wm, wkv, wrestore = cur
         if name == "verify":
-            wmc, wm, wkv = load("moe")
-            workloads["verify_moe"] = verify_run(wmc, wm, wkv, args.verify_steps, 4)
+            workloads["verify_moe"] = verify_run(wmc, wm, wkv, wrestore, args.verify_steps, 4)
+            workloads["spec_moe"] = spec_run(wmc, wm, wkv, wrestore)
         else:
-            wmc, wm, wkv = load(name)
             batches = (1, 2, 4, 8) if name == "moe" else (1, 8)
-            workloads[name] = {str(b): decode_run(wmc, wm, wkv, b, extra_steps, 3)[0] for b in batches}
-        wkv.close()
-        wm.close()
+            steps_w = min(args.sweep_steps, wmc.max_ctx - wmc.context - 3)
+            workloads[name] = {str(b): decode_run(wmc, wm, wkv, wrestore, b, steps_w, 3)[0] for b in batches}
+            if name == "moe":
+                multikernel["moe"] = compare_multikernel(wmc, wm, wkv, wrestore)
+    if cur:
+        cur[2].close()
+        cur[1].close()
 
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded random-init weights, seeded synthetic KV context)",
+        "data": "synthetic (seeded random-init weights; context = a seeded prompt prefilled through the model)",
         "config": {"workload": f"{args.config} decode, B={B}, context {mc.context} (+ positions advancing)",
                    "model": args.config, "global_batch": B * world, "seq_len": mc.context, "parallelism": f"dp{world}",
-                   "l2": "inputs larger than L2 (44 GB weights), no flush"},
+                   "l2": "inputs larger than L2 (44 GB weights), no flush",
+                   "context": "sequence 0's seeded prompt run through the model on the GPU, copied to the other sequences",
+                   "prefill_s": prefill_s, "sweep_steps": sweep_steps},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_kind": peak_kind,
                      "traffic": args.traffic if args.traffic is not None else recorded_traffic(args.config, B),
                      "frac_of_8tbs": achieved / 8000.0, "algorithmic_bytes_per_launch": abytes},
         "by_batch": by_batch,
         "workloads": workloads,
+        "multikernel_comparison": multikernel,
         "e2e": e2e,
         "gpu_launches": args.steps,
         "launch": {"ctas": ctas, "threads": threads, "smem_bytes": smem},
@@ -408,68 +583,57 @@ def run_ours(args, rank, world, local_rank):
     return res
 
 
-def cpu_baseline(config: str, sample_layers=(1, 4)):
-    """Time the fp64 oracle (as it stands) on the host cores for one B=1
-    decode step of the workload truncated to 1 and 4 layers (each the better
-    of two runs, so thread start-up is not counted), and extrapolate the
-    full-depth step linearly: head + L x layer."""
+def oracle_steps(config: str, steps: int, warmup: int = 0):
+    """Time the fp64 oracle (as it stands) on the host cores: `warmup`
+    untimed, then `steps` timed full-depth B=1 decode steps of the workload
+    (every layer, the LM head and the greedy argmax) at consecutive
+    positions past a seeded synthetic context (the oracle's own fill: its
+    prefill of thousands of positions would take hours, and the step's cost
+    does not depend on the context's values).  Returns the seconds of each
+    timed step."""
     import oracle
     import synth
     mc = synth.preset(config)
-    times = {}
-    for nl in sample_layers:
-        m = mc.replace(layers=nl, max_seqs=1)
-        om = oracle.OracleModel(m)
-        om.kv_fill_synthetic(synth.SEED_KV, mc.context)
-        tok = synth.tokens(synth.SEED_TOKENS, 1, mc.vocab)
-        best = float("inf")
-        for rep in range(2):
-            t0 = time.perf_counter()
-            om.step(tok, [mc.context + rep], want_logits=False)
-            best = min(best, time.perf_counter() - t0)
-        times[nl] = best
-        om.close()
-    lo, hi = sample_layers
-    t_layer = max((times[hi] - times[lo]) / (hi - lo), 1e-6)
-    t_head = max(times[lo] - lo * t_layer, 0.0)
-    full = t_head + mc.layers * t_layer
-    return {"value": 1.0 / full, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"one B=1 decode step of {config} truncated to {lo} and {hi} layers "
-                      f"({times[lo]:.2f} s, {times[hi]:.2f} s, best of 2); full {mc.layers}-layer step "
-                      f"extrapolated as head + {mc.layers} x layer = {full:.1f} s",
-            "t_layer_s": t_layer, "t_head_s": t_head}
+    om = oracle.OracleModel(mc.replace(max_seqs=1))
+    om.kv_fill_synthetic(synth.SEED_KV, mc.context)
+    tok = [int(synth.seq_tokens(synth.SEED_TOKENS, 0, [mc.context], mc.vocab)[0])]
+    times = []
+    for i in range(warmup + steps):
+        t0 = time.perf_counter()
+        r = om.step(tok, [mc.context + (i % 64)], want_logits=False, absorbed=mc.mla)
+        dt = time.perf_counter() - t0
+        tok = [int(r["argmax"][0])]
+        if i >= warmup:
+            times.append(dt)
+    om.close()
+    return times
+
+
+def cpu_baseline(config: str, steps: int = 3):
+    """The oracle timed over `steps` full-depth steps of the headline workload."""
+    import oracle
+    times = oracle_steps(config, steps)
+    mean = statistics.mean(times)
+    return {"value": 1.0 / mean, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{steps} full-depth B=1 decode steps of {config} (every layer, LM head, argmax) on a seeded "
+                      f"synthetic context, timed one by one: mean {mean:.2f} s per step",
+            "step_s": times}
 
 
 def run_reference(args):
-    """The reference arm: the fp64 CPU oracle on the host cores.  Each step
-    is a bounded sample - one B=1 decode step of the workload truncated to
-    one layer - scaled to the full depth with the head/layer split measured
-    by cpu_baseline (1- and 4-layer truncations)."""
+    """The reference arm: the fp64 CPU oracle on the host cores, W untimed
+    and K timed full-depth B=1 decode steps of the headline workload (each
+    step the whole model, as the GPU arm's)."""
     import oracle
     import synth
     mc = synth.preset(args.config)
-    fit = cpu_baseline(args.config)
-    t_layer, t_head = fit["t_layer_s"], fit["t_head_s"]
-    m1 = mc.replace(layers=1, max_seqs=1)
-    om = oracle.OracleModel(m1)
-    om.kv_fill_synthetic(synth.SEED_KV, mc.context)
-    tok = synth.tokens(synth.SEED_TOKENS, 1, mc.vocab)
-    for i in range(min(args.warmup, 2)):
-        om.step(tok, [mc.context + i], want_logits=False)
-    full = []
-    for i in range(args.steps):
-        t0 = time.perf_counter()
-        om.step(tok, [mc.context + (i % 8)], want_logits=False)
-        t1 = time.perf_counter() - t0
-        # this 1-layer step stands for head + L layers at the fitted ratio
-        full.append(t1 * (t_head + mc.layers * t_layer) / (t_head + t_layer))
-    om.close()
-    ms = 1e3 * sum(full) / len(full)
+    times = oracle_steps(args.config, args.steps, args.warmup)
+    ms = 1e3 * statistics.mean(times)
     value = 1e3 / ms
-    cpu = dict(fit)
-    cpu["value"] = value
-    cpu["sample"] = (f"{args.steps} decode steps of {args.config} truncated to 1 layer, each scaled to the full "
-                     f"{mc.layers}-layer step by the measured head/layer split; " + fit["sample"])
+    cpu = {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+           "sample": f"{args.steps} full-depth B=1 decode steps of {args.config} after {args.warmup} untimed ones "
+                     f"(every layer, LM head, argmax), seeded synthetic context, timed one by one",
+           "step_s": times}
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -497,7 +661,7 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     res = run_ours(args, rank, world, local_rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(args.config)
+        res["cpu_baseline"] = cpu_baseline(args.config, args.oracle_steps)
     if world > 1:
         import torch
         torch.distributed.barrier()

@@ -123,6 +123,12 @@ mk_status mk_kv_fill_random(mk_kv* kv, uint64_t seed, float sigma, int32_t lengt
 mk_status mk_kv_copy_out(mk_kv* kv, void* dst_dev);
 int64_t mk_kv_bytes(const mk_kv* kv);
 
+/* The inverse of mk_kv_copy_out: replace the whole cache with caller device
+ * memory of mk_kv_bytes() bytes in logical order (the copy-out layout), for
+ * example a context computed elsewhere.  The source is only read; the
+ * caller keeps it.  Synchronous. */
+mk_status mk_kv_copy_in(mk_kv* kv, const void* src_dev);
+
 /* One decode step for B sequences (B <= max_batch): sequence b consumes
  * tokens[b] at positions[b], writes its K/V there and attends over
  * positions 0..positions[b].
@@ -134,6 +140,26 @@ int64_t mk_kv_bytes(const mk_kv* kv);
  * [0, kv max_ctx). */
 mk_status mk_decode_step(mk_handle* h, const int32_t* tokens, const int32_t* positions, int B,
                          mk_kv* kv, float* logits_out, int32_t* argmax_out, void* stream);
+
+/* The same decode step as mk_decode_step, run the way the pages describe a
+ * GPU serving stack doing it ("Why megakernels?": one kernel per operation,
+ * launch overhead hidden with CUDA Graphs and programmatic dependent launch),
+ * for comparison with the persistent kernel.  The step's tasks are split at
+ * every phase boundary of the single kernel (each projection's row split,
+ * each layer's attention items, ...) into one launch of the same kernel code
+ * per phase; a phase waits for the previous one through the launch order,
+ * and its weight stream starts before that wait (programmatic dependent
+ * launch lets it begin while the previous phase drains).  The launches are
+ * recorded once per (batch size, cache, logits wanted, router trace) as a
+ * CUDA graph; each call copies tokens and positions into fixed device
+ * buffers, launches the graph and copies the argmax (and logits) out.  The
+ * arithmetic is the persistent kernel's, task for task: results are
+ * bit-identical to mk_decode_step.  Allocates on its first call (fixed
+ * buffers) and on the first call of each key (the graph).  Arguments as for
+ * mk_decode_step; the task trace and the stall hook are not supported
+ * (MK_ERR_STATE). */
+mk_status mk_decode_step_multikernel(mk_handle* h, const int32_t* tokens, const int32_t* positions, int B,
+                                     mk_kv* kv, float* logits_out, int32_t* argmax_out, void* stream);
 
 /* Size of the static device array behind mk_decode_step_noalloc, in bytes.
  * Every GPU that loads this library holds it until the process exits. */
@@ -158,12 +184,20 @@ mk_status mk_decode_step(mk_handle* h, const int32_t* tokens, const int32_t* pos
  *   memory, on `stream`) only when another handle or batch size used the
  *   array last.
  *   The first call on a device looks up the array's device address (a
- *   one-time set-up); make that first call before any stream capture.
+ *   one-time set-up); make that first call before any stream capture.  A
+ *   call that has to install a task list (its handle or batch size differs
+ *   from the last call's on this device) while `stream` is capturing returns
+ *   MK_ERR_STATE: the list is copied from host memory that the call frees.
+ *   Work enqueued by a call reads, when it runs on the GPU, whatever task
+ *   list the array holds then, so it is correct only while no call of
+ *   another handle or batch size has installed its own list in between.
  *   Calls that overlap on the GPU (other streams, other handles on the same
  *   device, or mk_decode_step_noalloc from several host threads without
  *   ordering their streams) race on the array: order them.
  *   A model and batch size whose scratch exceeds MK_NOALLOC_SCRATCH_BYTES
- *   are rejected with MK_ERR_INVALID (mk_last_error gives the bytes needed). */
+ *   are rejected with MK_ERR_INVALID (mk_last_error gives the bytes needed).
+ *   mk_debug_inject_stall does not apply to this entry point (its waits keep
+ *   their ordinary limit). */
 mk_status mk_decode_step_noalloc(mk_handle* h, const int32_t* tokens, const int32_t* positions, int B,
                                  mk_kv* kv, float* logits_out, int32_t* argmax_out, void* stream);
 
@@ -178,6 +212,50 @@ mk_status mk_decode_step_noalloc(mk_handle* h, const int32_t* tokens, const int3
  *                 tokens8[j] == argmax_out[j - 1] for all 1 <= j <= n. */
 mk_status mk_verify(mk_handle* h, const int32_t* tokens8, int n_prop, int32_t position, mk_kv* kv,
                     float* logits_out, int32_t* argmax_out, int32_t* accepted_out, void* stream);
+
+/* Prefill: run the model over a prompt of n tokens of cache sequence `seq`
+ * at positions start .. start + n - 1, writing their K/V (or latent rows)
+ * into the cache.  The prompt is processed in chunks of min(8, max_batch)
+ * positions, each one launch of the verify form (the positions of a chunk as
+ * the rows of one step, causal within the chunk; section "DSpark" of the
+ * pages checks 8 positions per launch the same way).  Asynchronous on
+ * `stream`; device errors as for mk_decode_step.
+ *   tokens: dev int32 [n]
+ *   argmax_last: dev int32 [1] (greedy token after the last position) or NULL
+ * Positions outside [0, kv max_ctx) or seq outside [0, kv max_seqs) are
+ * rejected on the host (MK_ERR_INVALID). */
+mk_status mk_prefill(mk_handle* h, const int32_t* tokens, int n, int seq, int32_t start, mk_kv* kv,
+                     int32_t* argmax_last, void* stream);
+
+/* Speculative greedy generation ("DSpark" section of the pages: each launch
+ * checks an anchor and up to 7 proposed continuations, keeps the accepted
+ * prefix plus one greedy "bonus" token, and rewinds the rest).  Runs on
+ * cache sequence 0, which holds positions 0 .. position - 1.
+ *
+ * The draft is the caller's: before every verify launch the library calls
+ *   draft(user, history, n_history, proposals, max_k)
+ * with history = the anchor followed by every token emitted so far (host
+ * memory, valid during the call); it writes up to max_k (<= 7) proposed
+ * next tokens into proposals (host) and returns how many it wrote (values
+ * outside [0, max_k] are clamped).  The verify launch (mk_verify) places the
+ * anchor at the current position and the proposals after it; with `a`
+ * proposals accepted, the emitted tokens are those a proposals and the greedy
+ * token after the last accepted one, which becomes the next anchor one
+ * position past them (later cache rows are overwritten by the next launch).
+ * The emitted sequence is the one plain greedy decoding (mk_decode_step fed
+ * its own argmax) produces, whatever the draft proposes.
+ *   out_tokens: host int32 [n_out], the emitted tokens in order
+ *   stats: host, optional: launches, proposed, accepted and emitted tokens
+ * Synchronous: the host reads each launch's accepted count before the next.
+ * MK_ERR_INVALID when the cache cannot hold the next launch's positions;
+ * device errors are returned as by mk_sync_status. */
+typedef int32_t (*mk_draft_fn)(void* user, const int32_t* history, int32_t n_history, int32_t* proposals,
+                               int32_t max_k);
+typedef struct {
+  int64_t launches, proposed, accepted, emitted;
+} mk_spec_stats;
+mk_status mk_spec_generate(mk_handle* h, mk_kv* kv, int32_t anchor, int32_t position, int32_t n_out,
+                           mk_draft_fn draft, void* user, int32_t* out_tokens, mk_spec_stats* stats, void* stream);
 
 /* Debug outputs of the next compute calls (dev pointers, or NULL to stop):
  * router expert indices int32 [layers][rows][top_k] and weights fp32 (same

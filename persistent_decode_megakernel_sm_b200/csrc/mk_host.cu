@@ -196,6 +196,17 @@ __global__ void unpermute_kv_kernel(uint16_t* dst, const uint16_t* src, int64_t 
   }
 }
 
+// The inverse: rows in logical order into the cache's permuted row layout.
+__global__ void permute_kv_kernel(uint16_t* dst, const uint16_t* src, int64_t rows, int Tmax, int d) {
+  const int64_t n = rows * d;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / d;
+    const int e = (int)(i - r * d);
+    const int t = (int)(r % Tmax);
+    dst[r * d + kv_swz(t, e)] = src[i];
+  }
+}
+
 // ---------------------------------------------------------------------------
 // handle
 // ---------------------------------------------------------------------------
@@ -215,6 +226,27 @@ struct Plan {
   int32_t* d_off = nullptr;
   int n_items = 0, n_pairs = 0;
   int n_tasks = 0;
+  // multi-kernel path: the non-empty phases, each CTA's task range per phase
+  std::vector<Task> host_tasks;
+  std::vector<int32_t> host_off;
+  int n_phases = 0;
+  int32_t* d_pbeg = nullptr;  // [phases][ncta]
+  int32_t* d_pend = nullptr;
+  int n_kphases = 0;
+};
+
+// One CUDA graph of the multi-kernel step per (batch, cache, logits wanted).
+struct GraphKey {
+  int S;
+  const void* kv;
+  bool logits;
+  const void* rtrace;  // router trace buffer (baked into the kernel arguments)
+  bool operator<(const GraphKey& o) const {
+    if (S != o.S) return S < o.S;
+    if (kv != o.kv) return kv < o.kv;
+    if (logits != o.logits) return logits < o.logits;
+    return rtrace < o.rtrace;
+  }
 };
 
 struct mk_handle {
@@ -249,7 +281,15 @@ struct mk_handle {
   int32_t* status = nullptr;
   float* logits_tmp = nullptr;
   int32_t* argmax_tmp = nullptr;
+  int32_t* spec_dev = nullptr;   // speculative generation: tokens [8] | argmax [8] | accepted [1]
   std::map<PlanKey, Plan> plans;
+  // multi-kernel comparison path: fixed step buffers and the captured graphs
+  int32_t* mk_tokens = nullptr;  // [MAXM]
+  int32_t* mk_pos = nullptr;     // [MAXM]
+  int32_t* mk_argmax = nullptr;  // [MAXM]
+  float* mk_logits = nullptr;    // [MAXM][vocab]
+  cudaStream_t mk_capture = nullptr;
+  std::map<GraphKey, cudaGraphExec_t> graphs;
   int32_t* trace_idx = nullptr;
   float* trace_w = nullptr;
   int64_t* task_trace = nullptr;
@@ -592,6 +632,7 @@ mk_status mk_create(const mk_model_desc* desc, int device, mk_handle** out) {
     TRY(dalloc(h, (void**)&h->status, 4 * sizeof(int32_t)));
     TRY(dalloc(h, (void**)&h->logits_tmp, 16));
     TRY(dalloc(h, (void**)&h->argmax_tmp, MAXM * sizeof(int32_t)));
+    TRY(dalloc(h, (void**)&h->spec_dev, 32 * sizeof(int32_t)));
     if (cudaMemset(h->ctr, 0, (size_t)h->n_ctr * 4) != cudaSuccess || cudaMemset(h->status, 0, 16) != cudaSuccess) {
       s = MK_ERR_CUDA;
       goto fail_out;
@@ -632,7 +673,11 @@ void mk_destroy(mk_handle* h) {
   for (auto& kv : h->plans) {
     cudaFree(kv.second.d_tasks);
     cudaFree(kv.second.d_off);
+    cudaFree(kv.second.d_pbeg);
+    cudaFree(kv.second.d_pend);
   }
+  for (auto& g : h->graphs) cudaGraphExecDestroy(g.second);
+  if (h->mk_capture) cudaStreamDestroy(h->mk_capture);
   for (void* p : h->allocs) cudaFree(p);
   delete h;
 }
@@ -888,6 +933,25 @@ mk_status mk_kv_copy_out(mk_kv* kv, void* dst) {
   return MK_OK;
 }
 
+mk_status mk_kv_copy_in(mk_kv* kv, const void* src) {
+  if (!kv || !src) return MK_ERR_INVALID;
+  mk_handle* h = kv->h;
+  cudaSetDevice(h->device);
+  if (!kv->v) {
+    CK(cudaMemcpy(kv->k, src, (size_t)kv->bytes, cudaMemcpyDeviceToDevice));
+    return MK_OK;
+  }
+  const size_t half = (size_t)kv->bytes / 2;
+  const int d = h->desc.head_dim;
+  const int64_t rows = (int64_t)(half / 2) / d;
+  permute_kv_kernel<<<148 * 16, 256>>>(kv->k, reinterpret_cast<const uint16_t*>(src), rows, kv->max_ctx, d);
+  permute_kv_kernel<<<148 * 16, 256>>>(kv->v, reinterpret_cast<const uint16_t*>(reinterpret_cast<const uint8_t*>(src) + half),
+                                       rows, kv->max_ctx, d);
+  CK(cudaGetLastError());
+  CK(cudaDeviceSynchronize());
+  return MK_OK;
+}
+
 // ---------------------------------------------------------------------------
 // planner: per-CTA task lists for a step of S sequences x Q positions
 // ---------------------------------------------------------------------------
@@ -928,7 +992,7 @@ static Task gemv(int layer, int mat, int rt0, int rt1, int in_kind, int in_buf, 
 // The task list of one step shape, built on the host: per-CTA task lists
 // flattened into `flat`, CTA c owning flat[off[c], off[c + 1]).
 static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>& flat, std::vector<int32_t>& off,
-                            int& n_items_out, int& n_pairs_out) {
+                            int& n_items_out, int& n_pairs_out, int& n_phases_out) {
   (void)Q;
   const mk_model_desc& d = h->desc;
   const int ncta = h->ncta, L = d.layers;
@@ -938,8 +1002,21 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
   auto C = [&](int l, int slot) { return l * NCTR_LAYER + slot; };
   std::vector<std::vector<Task>> per(ncta);
   int rot = 0;
+  // Phase of every task: the tasks pushed between two calls of next_phase()
+  // (one projection's row split over the CTAs, one layer's attention items,
+  // ...) form one kernel of the multi-kernel comparison path.
+  int phase = -1;
+  std::vector<size_t> mark(ncta, 0);
+  auto next_phase = [&]() {
+    for (int c = 0; c < ncta; ++c) {
+      for (size_t i = mark[c]; i < per[c].size(); ++i) per[c][i].phase = (int16_t)phase;
+      mark[c] = per[c].size();
+    }
+    ++phase;
+  };
   // embedding gather: every CTA writes its slice of the fp32 residual x and
   // the per-CTA sums of squares the first RMSNorm needs
+  next_phase();
   for (int c = 0; c < ncta; ++c) {
     Task t{};
     t.type = T_EMBED;
@@ -957,6 +1034,7 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
       // attention over the latent rows, per-head value up-projection, W_o
       const int hd = d.head_dim, dr = d.rope_dim, R = d.kv_lora_rank;
       auto rr = split_rows(h->mats[ly.m_qkv].m.RT, ncta, rot);
+      next_phase();
       for (int c = 0; c < ncta; ++c) {
         Task t = gemv(l, ly.m_qkv, rr[c].first, rr[c].second, IN_X_NORM, 0, EPI_STORE, B_QKV, 0,
                       l == 0 ? C(L, C_QKV) : C(l - 1, C_DOWN), ncta, C(l, C_QKV));
@@ -964,6 +1042,7 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
         per[c].push_back(t);
       }
       rr = split_rows(h->mats[ly.m_ukt].m.RT, ncta, rot);
+      next_phase();
       for (int c = 0; c < ncta; ++c) {
         // head g's rows read q_nope of head g: columns g * (dn + dr) of the QKV output
         Task t = gemv(l, ly.m_ukt, rr[c].first, rr[c].second, IN_BUF, B_QKV, EPI_STORE, B_QL, 0, C(l, C_QKV), ncta,
@@ -972,6 +1051,7 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
         t.xg_stride = hd + dr;
         per[c].push_back(t);
       }
+      next_phase();
       for (int i = 0; i < n_items; ++i) {
         // every item writes its partial (M, L, O) and counts itself done
         Task t{};
@@ -983,6 +1063,7 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
         t.sig_ctr = C(l, C_ATTN);
         per[i % ncta].push_back(t);
       }
+      next_phase();
       for (int c = 0; c < ncta; ++c) {
         // the split combine, a slice per CTA
         Task t{};
@@ -994,6 +1075,7 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
         per[c].push_back(t);
       }
       rr = split_rows(h->mats[ly.m_uv].m.RT, ncta, rot);
+      next_phase();
       for (int c = 0; c < ncta; ++c) {
         // head g's rows read the attention output of head g: columns g * R
         Task t = gemv(l, ly.m_uv, rr[c].first, rr[c].second, IN_BUF, B_OL, EPI_STORE, B_ATTN, 0, C(l, C_COMB),
@@ -1003,6 +1085,7 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
         per[c].push_back(t);
       }
       rr = split_rows(h->mats[ly.m_o].m.RT, ncta, rot);
+      next_phase();
       for (int c = 0; c < ncta; ++c) {
         Task t = gemv(l, ly.m_o, rr[c].first, rr[c].second, IN_BUF, B_ATTN, EPI_RESID, 0, 0, C(l, C_UV), ncta,
                       C(l, C_O));
@@ -1013,6 +1096,7 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
     // QKV projection (layer 0 reads the embedding rows directly)
     if (!mla) {
       auto rr = split_rows(h->mats[ly.m_qkv].m.RT, ncta, rot);
+      next_phase();
       for (int c = 0; c < ncta; ++c) {
         Task t = gemv(l, ly.m_qkv, rr[c].first, rr[c].second, IN_X_NORM, 0, EPI_STORE, B_QKV, 0,
                       l == 0 ? C(L, C_QKV) : C(l - 1, C_DOWN), ncta, C(l, C_QKV));
@@ -1021,6 +1105,7 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
       }
     }
     // attention items
+    next_phase();
     for (int i = 0; i < (mla ? 0 : n_items); ++i) {
       Task t{};
       t.type = T_ATTN;
@@ -1034,6 +1119,7 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
     // output projection + residual
     if (!mla) {
       auto rr = split_rows(h->mats[ly.m_o].m.RT, ncta, rot);
+      next_phase();
       for (int c = 0; c < ncta; ++c) {
         Task t = gemv(l, ly.m_o, rr[c].first, rr[c].second, IN_BUF, B_ATTN, EPI_RESID, 0, 0, C(l, C_ATTN), n_pairs,
                       C(l, C_O));
@@ -1045,6 +1131,7 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
       // gate/up + SwiGLU
       {
         auto rr = split_rows(h->mats[ly.m_gu].m.RT, ncta, rot);
+        next_phase();
         for (int c = 0; c < ncta; ++c) {
           Task t = gemv(l, ly.m_gu, rr[c].first, rr[c].second, IN_X_NORM, 0, EPI_SWIGLU, B_H, 1, C(l, C_O), ncta,
                         C(l, C_GU));
@@ -1055,6 +1142,7 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
       // down projection + residual
       {
         auto rr = split_rows(h->mats[ly.m_down].m.RT, ncta, rot);
+        next_phase();
         for (int c = 0; c < ncta; ++c) {
           Task t = gemv(l, ly.m_down, rr[c].first, rr[c].second, IN_BUF, B_H, EPI_RESID, 0, 0, C(l, C_GU), ncta,
                         C(l, C_DOWN));
@@ -1069,6 +1157,7 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
       // experts' (and the down) tiles wait for it.
       {
         auto rr = split_rows(h->mats[ly.m_router].m.RT, ncta, rot);
+        next_phase();
         for (int c = 0; c < ncta; ++c) {
           Task t = gemv(l, ly.m_router, rr[c].first, rr[c].second, IN_X_NORM, 0, EPI_STORE, B_RLOG, 1, C(l, C_O),
                         ncta, C(l, C_ROUTER));
@@ -1079,6 +1168,7 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
       if (d.n_shared > 0) {
         const MatHost& sh = h->mats[ly.m_shgu];
         auto rr = split_rows(sh.m.RT * sh.m.ne, ncta, rot);
+        next_phase();
         for (int c = 0; c < ncta; ++c) {
           Task t = gemv(l, ly.m_shgu, rr[c].first, rr[c].second, IN_X_NORM, 0, EPI_SWIGLU_MOE, B_H, 1, C(l, C_O),
                         ncta, C(l, C_GU));
@@ -1088,6 +1178,7 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
           per[c].push_back(t);
         }
       }
+      next_phase();
       for (int c = 0; c < ncta; ++c) {
         // rows decided on the device from the router's union of experts
         Task t = gemv(l, ly.m_exgu, 0, 0, IN_X_NORM, 0, EPI_SWIGLU_MOE, B_H, 1, C(l, C_ROUTER), ncta, C(l, C_GU));
@@ -1099,6 +1190,7 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
       {
         auto rr = split_rows(h->mats[ly.m_exdown].m.RT, ncta, rot);
         const int ngu = (d.n_shared > 0 ? 2 : 1) * ncta;
+        next_phase();
         for (int c = 0; c < ncta; ++c) {
           Task t = gemv(l, ly.m_exdown, rr[c].first, rr[c].second, IN_BUF, B_H, EPI_RESID, 0, 0, C(l, C_GU), ngu,
                         C(l, C_DOWN));
@@ -1113,6 +1205,7 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
   // final norm + LM head + argmax
   {
     auto rr = split_rows(h->mats[h->model.m_lm].m.RT, ncta, rot);
+    next_phase();
     for (int c = 0; c < ncta; ++c) {
       Task t = gemv(L - 1, h->model.m_lm, rr[c].first, rr[c].second, IN_X_NORM, 0, EPI_LOGITS, 0, 2,
                     C(L - 1, C_DOWN), ncta, -1);
@@ -1122,6 +1215,8 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
   }
   flat.clear();
   off.assign(ncta + 1, 0);
+  next_phase();  // tags the last phase's tasks
+  n_phases_out = phase;
   for (int c = 0; c < ncta; ++c) {
     off[c] = (int32_t)flat.size();
     flat.insert(flat.end(), per[c].begin(), per[c].end());
@@ -1160,11 +1255,15 @@ static mk_status get_plan(mk_handle* h, int S, int Q, Plan** out) {
   std::vector<Task> flat;
   std::vector<int32_t> off;
   int n_items = 0, n_pairs = 0;
-  build_plan_host(h, S, Q, flat, off, n_items, n_pairs);
+  int n_phases = 0;
+  build_plan_host(h, S, Q, flat, off, n_items, n_pairs, n_phases);
   Plan p;
   p.n_items = n_items;
   p.n_pairs = n_pairs;
   p.n_tasks = (int)flat.size();
+  p.n_phases = n_phases;
+  p.host_tasks = flat;
+  p.host_off = off;
   CK(cudaMalloc(&p.d_tasks, flat.size() * sizeof(Task)));
   CK(cudaMalloc(&p.d_off, off.size() * sizeof(int32_t)));
   CK(cudaMemcpy(p.d_tasks, flat.data(), flat.size() * sizeof(Task), cudaMemcpyHostToDevice));
@@ -1177,8 +1276,12 @@ static mk_status get_plan(mk_handle* h, int S, int Q, Plan** out) {
 // ---------------------------------------------------------------------------
 // compute entry points
 // ---------------------------------------------------------------------------
-static mk_status launch_step(mk_handle* h, mk_kv* kv, int S, int Q, const int32_t* tokens, const int32_t* positions,
-                             int32_t pos_const, float* logits, int32_t* argmax, int32_t* accepted, void* stream) {
+// The launch arguments of one step.  seq0: the cache sequence that step
+// sequence 0 maps to (sequences seq0 .. seq0 + S - 1 are used; the cache base
+// is offset, its strides are kept).
+static mk_status make_launch(mk_handle* h, mk_kv* kv, int S, int Q, const int32_t* tokens, const int32_t* positions,
+                             int32_t pos_const, float* logits, int32_t* argmax, int32_t* accepted, int seq0, Plan** plan_out,
+                             Launch* out) {
   if (h->sticky) return fail(h, MK_ERR_STATE, "a previous device error is pending; call mk_reset");
   if (!h->initialised) return fail(h, MK_ERR_STATE, "weights not initialised");
   cudaSetDevice(h->device);
@@ -1195,8 +1298,11 @@ static mk_status launch_step(mk_handle* h, mk_kv* kv, int S, int Q, const int32_
   P.S = S;
   P.Q = Q;
   P.M = S * Q;
-  P.kv_k = kv->k;
-  P.kv_v = kv->v;
+  const mk_model_desc& dd = h->desc;
+  const size_t seq_elems = dd.kv_lora_rank > 0 ? (size_t)kv->max_ctx * (dd.kv_lora_rank + dd.rope_dim)
+                                               : (size_t)dd.n_kv_heads * kv->max_ctx * dd.head_dim;
+  P.kv_k = kv->k + (size_t)seq0 * seq_elems;
+  P.kv_v = kv->v ? kv->v + (size_t)seq0 * seq_elems : nullptr;
   P.kv_seqs = kv->max_seqs;
   P.kv_ctx = kv->max_ctx;
   P.logits = logits;
@@ -1226,7 +1332,20 @@ static mk_status launch_step(mk_handle* h, mk_kv* kv, int S, int Q, const int32_
   P.n_pairs = plan->n_pairs;
   P.trace = h->task_trace;
   P.trace_cap = h->task_trace_cap;
+  P.task_end = nullptr;
+  P.phase_mode = 0;
   h->stall_ns = 0;
+  *out = P;
+  if (plan_out) *plan_out = plan;
+  return MK_OK;
+}
+
+static mk_status launch_step(mk_handle* h, mk_kv* kv, int S, int Q, const int32_t* tokens, const int32_t* positions,
+                             int32_t pos_const, float* logits, int32_t* argmax, int32_t* accepted, void* stream,
+                             int seq0 = 0) {
+  Launch P;
+  mk_status s = make_launch(h, kv, S, Q, tokens, positions, pos_const, logits, argmax, accepted, seq0, nullptr, &P);
+  if (s != MK_OK) return s;
   void* args[] = {&P};
   cudaError_t e = cudaLaunchCooperativeKernel(P.trace ? h->kernel_traced : h->kernel, dim3(h->ncta), dim3(NTHREADS), args,
                                               SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream));
@@ -1243,6 +1362,111 @@ mk_status mk_decode_step(mk_handle* h, const int32_t* tokens, const int32_t* pos
   return launch_step(h, kv, B, 1, tokens, positions, 0, logits_out, argmax_out, nullptr, stream);
 }
 
+// Per-phase task ranges of a plan, for the multi-kernel path (empty phases
+// are dropped).
+static mk_status ensure_phases(mk_handle* h, Plan* p) {
+  if (p->d_pbeg) return MK_OK;
+  const int ncta = h->ncta;
+  std::vector<int32_t> beg, end;
+  for (int ph = 0; ph < p->n_phases; ++ph) {
+    std::vector<int32_t> b(ncta), e(ncta);
+    bool any = false;
+    for (int c = 0; c < ncta; ++c) {
+      const int lo = p->host_off[c], hi = p->host_off[c + 1];
+      int i = lo;
+      while (i < hi && p->host_tasks[i].phase < ph) ++i;
+      int j = i;
+      while (j < hi && p->host_tasks[j].phase == ph) ++j;
+      b[c] = i;
+      e[c] = j;
+      any = any || j > i;
+    }
+    if (!any) continue;
+    beg.insert(beg.end(), b.begin(), b.end());
+    end.insert(end.end(), e.begin(), e.end());
+  }
+  p->n_kphases = (int)(beg.size() / ncta);
+  CK(cudaMalloc(&p->d_pbeg, beg.size() * sizeof(int32_t)));
+  CK(cudaMalloc(&p->d_pend, end.size() * sizeof(int32_t)));
+  CK(cudaMemcpy(p->d_pbeg, beg.data(), beg.size() * sizeof(int32_t), cudaMemcpyHostToDevice));
+  CK(cudaMemcpy(p->d_pend, end.data(), end.size() * sizeof(int32_t), cudaMemcpyHostToDevice));
+  return MK_OK;
+}
+
+mk_status mk_decode_step_multikernel(mk_handle* h, const int32_t* tokens, const int32_t* positions, int B, mk_kv* kv,
+                                     float* logits_out, int32_t* argmax_out, void* stream) {
+  if (!h) return MK_ERR_INVALID;
+  if (!tokens || !positions || !kv || !argmax_out) return fail(h, MK_ERR_INVALID, "null argument");
+  if (kv->h != h) return fail(h, MK_ERR_INVALID, "kv cache belongs to another model");
+  if (B < 1 || B > h->desc.max_batch || B > kv->max_seqs) return fail(h, MK_ERR_INVALID, "B out of range");
+  if (h->task_trace || h->stall_ns > 0)
+    return fail(h, MK_ERR_STATE, "the task trace and the stall hook apply to the single-kernel step only");
+  CK(cudaSetDevice(h->device));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const mk_model_desc& d = h->desc;
+  if (!h->mk_tokens) {
+    mk_status s;
+    if ((s = dalloc(h, (void**)&h->mk_tokens, MAXM * sizeof(int32_t))) != MK_OK) return s;
+    if ((s = dalloc(h, (void**)&h->mk_pos, MAXM * sizeof(int32_t))) != MK_OK) return s;
+    if ((s = dalloc(h, (void**)&h->mk_argmax, MAXM * sizeof(int32_t))) != MK_OK) return s;
+    if ((s = dalloc(h, (void**)&h->mk_logits, (size_t)MAXM * d.vocab * sizeof(float))) != MK_OK) return s;
+    CK(cudaStreamCreateWithFlags(&h->mk_capture, cudaStreamNonBlocking));
+  }
+  const GraphKey key{B, kv, logits_out != nullptr, h->trace_idx};
+  auto gi = h->graphs.find(key);
+  if (gi == h->graphs.end()) {
+    Launch P;
+    Plan* plan = nullptr;
+    mk_status s = make_launch(h, kv, B, 1, h->mk_tokens, h->mk_pos, 0, logits_out ? h->mk_logits : nullptr, h->mk_argmax,
+                              nullptr, 0, &plan, &P);
+    if (s != MK_OK) return s;
+    if ((s = ensure_phases(h, plan)) != MK_OK) return s;
+    // one kernel per phase, each allowed to start (programmatic dependent
+    // launch) while the previous one drains; recorded once as a graph
+    CK(cudaStreamBeginCapture(h->mk_capture, cudaStreamCaptureModeThreadLocal));
+    cudaError_t le = cudaSuccess;
+    for (int k = 0; k < plan->n_kphases && le == cudaSuccess; ++k) {
+      Launch Pk = P;
+      Pk.task_off = plan->d_pbeg + (size_t)k * h->ncta;
+      Pk.task_end = plan->d_pend + (size_t)k * h->ncta;
+      Pk.phase_mode = k + 1 == plan->n_kphases ? 2 : 1;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(h->ncta);
+      cfg.blockDim = dim3(NTHREADS);
+      cfg.dynamicSmemBytes = SMEM_BYTES;
+      cfg.stream = h->mk_capture;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = k > 0 ? 1 : 0;
+      void* args[] = {&Pk};
+      le = cudaLaunchKernelExC(&cfg, h->kernel, args);
+    }
+    cudaGraph_t graph = nullptr;
+    const cudaError_t ce = cudaStreamEndCapture(h->mk_capture, &graph);
+    if (le != cudaSuccess || ce != cudaSuccess) {
+      if (graph) cudaGraphDestroy(graph);
+      return fail(h, MK_ERR_CUDA, std::string("capture of the phase kernels: ") +
+                                      cudaGetErrorString(le != cudaSuccess ? le : ce));
+    }
+    cudaGraphExec_t exec = nullptr;
+    const cudaError_t ie = cudaGraphInstantiate(&exec, graph, 0);
+    cudaGraphDestroy(graph);
+    if (ie != cudaSuccess) return fail(h, MK_ERR_CUDA, std::string("graph instantiate: ") + cudaGetErrorString(ie));
+    gi = h->graphs.emplace(key, exec).first;
+  } else if (h->sticky) {
+    return fail(h, MK_ERR_STATE, "a previous device error is pending; call mk_reset");
+  }
+  CK(cudaMemcpyAsync(h->mk_tokens, tokens, (size_t)B * sizeof(int32_t), cudaMemcpyDeviceToDevice, st));
+  CK(cudaMemcpyAsync(h->mk_pos, positions, (size_t)B * sizeof(int32_t), cudaMemcpyDeviceToDevice, st));
+  CK(cudaGraphLaunch(gi->second, st));
+  CK(cudaMemcpyAsync(argmax_out, h->mk_argmax, (size_t)B * sizeof(int32_t), cudaMemcpyDeviceToDevice, st));
+  if (logits_out)
+    CK(cudaMemcpyAsync(logits_out, h->mk_logits, (size_t)B * d.vocab * sizeof(float), cudaMemcpyDeviceToDevice, st));
+  return MK_OK;
+}
+
 mk_status mk_verify(mk_handle* h, const int32_t* tokens8, int n_prop, int32_t position, mk_kv* kv, float* logits_out,
                     int32_t* argmax_out, int32_t* accepted_out, void* stream) {
   if (!h) return MK_ERR_INVALID;
@@ -1252,6 +1476,72 @@ mk_status mk_verify(mk_handle* h, const int32_t* tokens8, int n_prop, int32_t po
     return fail(h, MK_ERR_INVALID, "n_prop out of range");
   if (position < 0 || position + n_prop + 1 > kv->max_ctx) return fail(h, MK_ERR_INVALID, "position out of range");
   return launch_step(h, kv, 1, n_prop + 1, tokens8, nullptr, position, logits_out, argmax_out, accepted_out, stream);
+}
+
+mk_status mk_prefill(mk_handle* h, const int32_t* tokens, int n, int seq, int32_t start, mk_kv* kv,
+                     int32_t* argmax_last, void* stream) {
+  if (!h) return MK_ERR_INVALID;
+  if (!tokens || !kv) return fail(h, MK_ERR_INVALID, "null argument");
+  if (kv->h != h) return fail(h, MK_ERR_INVALID, "kv cache belongs to another model");
+  if (n < 1 || seq < 0 || seq >= kv->max_seqs) return fail(h, MK_ERR_INVALID, "n or seq out of range");
+  if (start < 0 || (int64_t)start + n > kv->max_ctx) return fail(h, MK_ERR_INVALID, "positions out of range");
+  const int chunk = std::min(h->desc.max_batch, MAXM);
+  for (int i = 0; i < n; i += chunk) {
+    const int q = std::min(chunk, n - i);
+    mk_status s = launch_step(h, kv, 1, q, tokens + i, nullptr, start + i, nullptr, h->argmax_tmp, nullptr, stream, seq);
+    if (s != MK_OK) return s;
+    if (i + q == n && argmax_last)
+      CK(cudaMemcpyAsync(argmax_last, h->argmax_tmp + (q - 1), sizeof(int32_t), cudaMemcpyDeviceToDevice,
+                         reinterpret_cast<cudaStream_t>(stream)));
+  }
+  return MK_OK;
+}
+
+mk_status mk_spec_generate(mk_handle* h, mk_kv* kv, int32_t anchor, int32_t position, int32_t n_out,
+                           mk_draft_fn draft, void* user, int32_t* out_tokens, mk_spec_stats* stats, void* stream) {
+  if (!h) return MK_ERR_INVALID;
+  if (!kv || !draft || !out_tokens) return fail(h, MK_ERR_INVALID, "null argument");
+  if (kv->h != h) return fail(h, MK_ERR_INVALID, "kv cache belongs to another model");
+  if (n_out < 1 || position < 0 || anchor < 0 || anchor >= h->desc.vocab)
+    return fail(h, MK_ERR_INVALID, "n_out, position or anchor out of range");
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int kcap = std::min(std::min(7, h->desc.max_batch - 1), MAXM - 1);
+  std::vector<int32_t> hist;
+  hist.reserve((size_t)n_out + 1);
+  hist.push_back(anchor);
+  mk_spec_stats sst{0, 0, 0, 0};
+  int32_t pos = position, emitted = 0;
+  int32_t props[8], toks[8], back[17];
+  while (emitted < n_out) {
+    const int kmax = std::min(kcap, kv->max_ctx - pos - 1);
+    if (kmax < 0) return fail(h, MK_ERR_INVALID, "mk_spec_generate: the cache is full");
+    int k = draft(user, hist.data(), (int32_t)hist.size(), props, kmax);
+    k = std::max(0, std::min(k, kmax));
+    toks[0] = anchor;
+    for (int j = 0; j < k; ++j) toks[j + 1] = props[j];
+    CK(cudaMemcpyAsync(h->spec_dev, toks, (size_t)(k + 1) * sizeof(int32_t), cudaMemcpyHostToDevice, st));
+    mk_status s = launch_step(h, kv, 1, k + 1, h->spec_dev, nullptr, pos, nullptr, h->spec_dev + 8, h->spec_dev + 16,
+                              stream);
+    if (s != MK_OK) return s;
+    CK(cudaMemcpyAsync(back, h->spec_dev + 8, 9 * sizeof(int32_t), cudaMemcpyDeviceToHost, st));
+    CK(cudaStreamSynchronize(st));
+    s = mk_sync_status(h);
+    if (s != MK_OK) return s;
+    const int a = std::max(0, std::min(back[8], k));
+    for (int j = 0; j <= a && emitted < n_out; ++j) {
+      const int32_t tkn = j < a ? props[j] : back[a];
+      out_tokens[emitted++] = tkn;
+      hist.push_back(tkn);
+    }
+    sst.launches += 1;
+    sst.proposed += k;
+    sst.accepted += a;
+    sst.emitted += a + 1;
+    anchor = back[a];
+    pos += a + 1;
+  }
+  if (stats) *stats = sst;
+  return MK_OK;
 }
 
 mk_status mk_set_router_trace(mk_handle* h, int32_t* idx_dev, float* w_dev) {
@@ -1366,7 +1656,16 @@ extern "C" mk_status mk_decode_step_noalloc(mk_handle* h, const int32_t* tokens,
   int n_items = nd.plan_items, n_pairs = nd.plan_pairs;
   size_t n_tasks = nd.plan_tasks;
   if (!installed) {
-    build_plan_host(h, B, 1, flat, off, n_items, n_pairs);
+    // Installing copies the task list from pageable host memory that is
+    // freed when this call returns; that copy must run now, not be recorded.
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    CK(cudaStreamIsCapturing(st, &cs));
+    if (cs != cudaStreamCaptureStatusNone)
+      return fail(h, MK_ERR_STATE,
+                  "mk_decode_step_noalloc: this handle and batch size must be installed by a call outside stream "
+                  "capture first");
+    int n_phases = 0;
+    build_plan_host(h, B, 1, flat, off, n_items, n_pairs, n_phases);
     n_tasks = flat.size();
   }
 

@@ -11,7 +11,8 @@ namespace mk {
 constexpr int NCW = 8;                       // consumer warps
 constexpr int WARP_WP = NCW;                 // weight producer warp
 constexpr int WARP_XP = NCW + 1;             // activation producer warp
-constexpr int NTHREADS = (NCW + 2) * 32;
+constexpr int WARP_MV = NCW + 2;             // tensor-memory mover warp
+constexpr int NTHREADS = (NCW + 3) * 32;
 constexpr int NCT = NCW * 32;                // consumer threads
 // Ring shape (tunable at build time).
 #ifndef MK_TILE_CAP
@@ -20,7 +21,19 @@ constexpr int NCT = NCW * 32;                // consumer threads
 #ifndef MK_NSTAGE
 #define MK_NSTAGE 2
 #endif
+// Second weight stage in tensor memory (TMEM, 256 KB per SM): bf16 GEMV
+// chunks are copied out of the shared-memory ring into TMEM slots as soon as
+// they land, which frees the ring for the next bulk copies; the consumers read
+// their mma A fragments from TMEM.  The producer can then run up to NSTAGE +
+// NTS chunks ahead of the consumers.  0 keeps every chunk in shared memory.
+#ifndef MK_TSLOTS
+#define MK_TSLOTS 0
+#endif
 constexpr int TILE_CAP = MK_TILE_CAP;        // weight tile bytes per GEMV chunk (gains follow)
+constexpr int NTS = MK_TSLOTS;               // TMEM slots
+constexpr int TSLOT_COLS = TILE_CAP / 512;   // TMEM columns per slot: 4 columns (16 B x 128 lanes) hold 4 tiles
+constexpr int TMEM_COLS = 512;               // the whole tensor memory of the SM (one CTA per SM)
+static_assert(NTS * TSLOT_COLS <= TMEM_COLS, "TMEM slots exceed the tensor memory");
 constexpr int STAGE_BYTES = (TILE_CAP + 1024 > 34816) ? TILE_CAP + 1024 : 34816;  // >= one attention chunk
 constexpr int NSTAGE = MK_NSTAGE;            // weight ring depth
 constexpr int XSLOTS = 2;                    // activation ring depth
@@ -136,7 +149,7 @@ struct Task {
   int16_t in_kind, epi;
   int16_t in_buf, out_buf;
   int16_t moe, gain;         // moe: 1 shared experts, 2 routed experts; gain: 0 attn, 1 ffn, 2 final
-  int16_t xg_rt, pad16;      // > 0: rows come in groups of xg_rt row tiles (one per head), each reading
+  int16_t xg_rt, phase;      // xg_rt > 0: rows come in groups of xg_rt row tiles (one per head), each reading
   int32_t xg_stride;         //      its own activation columns, xg_stride floats further per group
   int32_t mat;               // matrix table index
   int32_t rt0, rt1;          // row tiles (GEMV) / item index (ATTN)
@@ -219,6 +232,12 @@ struct Launch {
   int32_t n_pairs;           // S * Hkv
   int64_t* trace;            // [nCTA][trace_cap][8] or null
   int32_t trace_cap;
+  // One kernel per phase (the multi-kernel comparison path): this launch runs
+  // tasks [task_off[c], task_end[c]) of CTA c; phase_mode 1 = a phase that is
+  // not the step's last, 2 = the last (it clears the counters at exit).
+  // 0 = the whole step in one launch (task_end unused).
+  const int32_t* task_end;
+  int32_t phase_mode;
 };
 
 // counter slots inside one layer

@@ -45,6 +45,8 @@
 namespace mk {
 namespace MK_KNS {
 
+constexpr int NTSD = NTS > 0 ? NTS : 1;  // TMEM slot count as a divisor (the slot code is dead when NTS == 0)
+
 // ---------------------------------------------------------------------------
 // PTX helpers
 // ---------------------------------------------------------------------------
@@ -147,6 +149,49 @@ __device__ __forceinline__ uint32_t lds16(const void* p) {
   return v;
 }
 
+__device__ __forceinline__ void mbar_arrive_cnt(uint64_t* bar, uint32_t cnt) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(smem_u32(bar)), "r"(cnt)
+               : "memory");
+}
+
+// Tensor memory (tcgen05).  One warp allocates the CTA's columns at start and
+// frees them at exit.  Addresses are (lane << 16) | column.
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// Shared-memory matrix descriptor of 128 rows x 16 bytes stored contiguously
+// (no swizzle; 8-row core matrices 128 B apart).
+__device__ __forceinline__ uint64_t sdesc_rows16(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(128 >> 4) << 16) | ((uint64_t)(128 >> 4) << 32) |
+         (1ull << 46);
+}
+// Copy 128 rows x 16 bytes of shared memory into TMEM lanes 0..127, 4 columns.
+__device__ __forceinline__ void tmem_cp_rows16(uint32_t taddr, uint64_t desc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+}
+// Arrive (once) on `bar` when every earlier tcgen05 operation of this thread has completed.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+// This warp's 32 lanes x 4 columns: lane l receives the 16 bytes of TMEM lane (quarter base + l).
+__device__ __forceinline__ uint4 tmem_ld16(uint32_t taddr) {
+  uint4 v;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(taddr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
 __device__ __forceinline__ void mma_bf16(float (&d)[4], uint4 a, uint32_t b0, uint32_t b1) {
   asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
@@ -227,7 +272,11 @@ __device__ __forceinline__ uint4 fp8_frag_to_f16(uint2 v) {
 // ---------------------------------------------------------------------------
 struct Misc {
   uint64_t full[NSTAGE];
-  uint64_t empty[NSTAGE];
+  uint64_t empty[NSTAGE];   // consumers (NCW) + the mover (1); for TMEM chunks the mover's NCW + its copy commit
+  uint64_t tfull[NTS > 0 ? NTS : 1];   // TMEM slot written (copy commit)
+  uint64_t tempty[NTS > 0 ? NTS : 1];  // TMEM slot read by every consumer warp
+  uint32_t tmem_base;
+  int32_t cdesc[NSTAGE];    // per ring stage: 2 KB groups to move to TMEM (0: stays in shared memory; -1: end)
   uint64_t xfull[XSLOTS];   // activation slice landed (bulk copy)
   uint64_t xempty[XSLOTS];
   float scale[MAXM];
@@ -260,9 +309,21 @@ struct Ctx {
   uint8_t* att;
   uint8_t* newkv;
   int ncta;
+  uint32_t tmem;  // TMEM base address of the weight slots
 };
 
 __device__ __forceinline__ bool global_abort(const Launch& P) { return ld_volatile_i32(P.status + 1) != 0; }
+
+__device__ __forceinline__ int task_end_of(const Launch& P) {
+  return P.phase_mode ? P.task_end[blockIdx.x] : P.task_off[blockIdx.x + 1];
+}
+// Multi-kernel path: the activations and counters a phase reads were written
+// by earlier phase kernels; with programmatic dependent launch this kernel
+// may start before they finish, so every role that reads them waits here for
+// the preceding grid (the weight producer does not: weights are constant).
+__device__ __forceinline__ void phase_dependency_wait(const Launch& P) {
+  if (P.phase_mode) asm volatile("griddepcontrol.wait;" ::: "memory");
+}
 
 __device__ void raise_error(const Launch& P, Misc* ms, int code, int detail) {
   atomicCAS(P.status, 0, code);
@@ -277,6 +338,7 @@ __device__ void raise_error(const Launch& P, Misc* ms, int code, int detail) {
 struct ChunkIt {
   int rt1, KT, tb, gsz, xcap;
   int g0, nr, KC, WC, c0, nc, wb;  // wb: first col tile of the current activation window
+  bool tm;                         // the group's chunks go through the TMEM stage
   __device__ __forceinline__ void set_group() {
     nr = min(RMAX, rt1 - g0);
     if (gsz > 0) {
@@ -284,7 +346,12 @@ struct ChunkIt {
       nr = min(nr, nb - g0);
     }
     KC = min(min(KT, TILE_CAP / (nr * tb)), min(NCW * CPW, xcap));
+    if (KC < KT && KC >= 4) KC &= ~3;  // chunk widths in whole 4-tile groups
     WC = (xcap / KC) * KC;  // activation window: a whole number of chunks
+    // a chunk moves to TMEM in 2 KB groups of 4 consecutive tiles; with a
+    // width that is a multiple of 4, the tiles of col j (j = warp mod 8) sit
+    // in lane quarter warp mod 4, the only one the warp can read
+    tm = NTS > 0 && tb == TILE_BF16 && (KT & 3) == 0 && (KC & 3) == 0;
   }
   // xcap: most col tiles whose activation slice (M rows) fits one x slot
   __device__ __forceinline__ bool init(int rt0_, int rt1_, int KT_, int tb_, int gsz_, int xcap_) {
@@ -570,7 +637,8 @@ __device__ __forceinline__ bool gemv_like(const Task& t) {
 // ---------------------------------------------------------------------------
 // Reserve ring slot `it` for `bytes` (lane 0 waits for the consumers to free
 // it, then arms the full barrier).  Returns false on abort.
-__device__ bool prod_reserve(const Ctx& C, uint32_t it, uint32_t bytes, long long& blocked) {
+__device__ bool prod_reserve(const Ctx& C, uint32_t it, uint32_t bytes, long long& blocked, int desc = 0,
+                             bool end = false) {
   const int lane = threadIdx.x & 31;
   int ok = 1;
   if (lane == 0) {
@@ -596,7 +664,12 @@ __device__ bool prod_reserve(const Ctx& C, uint32_t it, uint32_t bytes, long lon
       }
     }
     blocked += clock64() - c0;
-    if (ok) mbar_arrive_expect_tx(&C.ms->full[s], bytes);
+    if (ok) {
+      // the mover reads the stage's descriptor once the stage's phase completes
+      if (NTS > 0) C.ms->cdesc[s] = end ? -1 : desc;
+      if (end) mbar_arrive(&C.ms->full[s]);
+      else mbar_arrive_expect_tx(&C.ms->full[s], bytes);
+    }
   }
   ok = __shfl_sync(0xffffffffu, ok, 0);
   return ok != 0;
@@ -639,6 +712,7 @@ struct Chunk {
   int kind;  // 1: GEMV tiles, 2: attention K/V rows, 3: latent cache rows (kb, n rows of d values)
   const uint8_t* w;
   int KT, tb, g0, nr, c0, nc;
+  int tm;    // GEMV tiles that go through the TMEM stage
   const uint16_t* kb;
   const uint16_t* vb;
   int n, d;
@@ -678,6 +752,7 @@ struct ChunkStream {
         c.nr = ci.nr;
         c.c0 = ci.c0;
         c.nc = ci.nc;
+        c.tm = ci.tm ? 1 : 0;
         if (!ci.next()) {
           if (!pc.next()) {
             state = 0;
@@ -691,6 +766,7 @@ struct ChunkStream {
       if (!MLA && state == 2) {
         if (t0 < b) {
           c.kind = 2;
+          c.tm = 0;
           c.kb = kb + (size_t)t0 * d;
           c.vb = vb + (size_t)t0 * d;
           c.n = min(ATT_CT, b - t0);
@@ -703,6 +779,7 @@ struct ChunkStream {
       if (MLA && state == 3) {
         if (t0 < b) {
           c.kind = 3;
+          c.tm = 0;
           c.kb = kb + (size_t)t0 * d;
           c.n = min(mla_ct(md.R, md.dr), b - t0);
           c.d = d;
@@ -762,7 +839,7 @@ __device__ void producer(const Ctx& C) {
   const int lane = threadIdx.x & 31;
   const uint64_t pol = policy_evict_first();
   uint32_t it = 0;
-  const int beg = P.task_off[blockIdx.x], end = P.task_off[blockIdx.x + 1];
+  const int beg = P.task_off[blockIdx.x], end = task_end_of(P);
   long long blocked = 0;
   const uint64_t t_first = globaltimer();
   const long long c_first = clock64();
@@ -774,7 +851,7 @@ __device__ void producer(const Ctx& C) {
     uint64_t* bar = &C.ms->full[it % NSTAGE];
     if (c.kind == 1) {
       const uint32_t tbytes = (uint32_t)(c.nr * c.nc * c.tb);
-      if (!prod_reserve(C, it, tbytes, blocked)) goto drain;
+      if (!prod_reserve(C, it, tbytes, blocked, c.tm ? (c.nr * c.nc) >> 2 : 0)) goto drain;
       if (lane < c.nr) {
         const uint8_t* srcp = c.w + ((size_t)(c.g0 + lane) * c.KT + c.c0) * c.tb;
         bulk_g2s(dst + (size_t)lane * c.nc * c.tb, srcp, (uint32_t)(c.nc * c.tb), bar, pol);
@@ -793,6 +870,12 @@ __device__ void producer(const Ctx& C) {
       if (lane == 0) bulk_g2s(dst, c.kb, rb, bar, pol);
       if (lane == 1) bulk_g2s(dst + (size_t)ATT_CT * pitch, c.vb, rb, bar, pol);
     }
+    __syncwarp();
+    ++it;
+  }
+  // end of the stream for the mover
+  if (NTS > 0) {
+    if (!prod_reserve(C, it, 0, blocked, 0, true)) goto drain;
     __syncwarp();
     ++it;
   }
@@ -823,6 +906,68 @@ drain:
     }
   }
   __syncwarp();
+}
+
+// ---------------------------------------------------------------------------
+// TMEM mover warp
+// ---------------------------------------------------------------------------
+// Follows the ring in order.  A stage whose descriptor says "TMEM" is copied
+// (tcgen05.cp, 2 KB per instruction) into the next TMEM slot once that slot
+// has been read by every consumer warp; the copy's completion both fills the
+// slot (tfull) and releases the stage to the producer (empty).  Any other
+// stage is only acknowledged: the consumers read it in place and release it.
+// Bounded waits end on the global abort flag or the time limit.
+__device__ bool mover_wait(const Ctx& C, uint64_t* bar, uint32_t par, int code) {
+  uint64_t t0 = 0;
+  uint32_t spins = 0;
+  while (!mbar_try_wait(bar, par)) {
+    if (++spins >= 64) {
+      spins = 0;
+      if (C.ms->abort || global_abort(*C.P)) return false;
+      const uint64_t now = globaltimer();
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > (uint64_t)C.P->timeout_ns * 2) {
+        raise_error(*C.P, C.ms, DERR_TIMEOUT, code);
+        return false;
+      }
+    }
+  }
+  return true;
+}
+
+__device__ void mover(const Ctx& C) {
+  if (NTS == 0) return;
+  if ((threadIdx.x & 31) != 0) return;
+  uint32_t i = 0, tc = 0;
+  while (true) {
+    const int s = i % NSTAGE;
+    if (!mover_wait(C, &C.ms->full[s], (i / NSTAGE) & 1, 0x90000 | s)) break;
+    const int d = C.ms->cdesc[s];
+    if (d < 0) break;
+    if (d > 0) {
+      const int t = tc % NTSD;
+      if (tc >= (uint32_t)NTSD && !mover_wait(C, &C.ms->tempty[t], ((tc / NTSD) + 1) & 1, 0xA0000 | t)) break;
+      tc_fence_after();
+      const uint32_t src = smem_u32(C.ring + (size_t)s * STAGE_BYTES);
+      const uint32_t dst = C.tmem + (uint32_t)(t * TSLOT_COLS);
+      for (int g = 0; g < d; ++g) tmem_cp_rows16(dst + 4 * g, sdesc_rows16(src + 2048 * g));
+      tc_commit(&C.ms->empty[s]);  // the stage is free once the copies have read it
+      tc_commit(&C.ms->tfull[t]);  // the slot is full
+      mbar_arrive_cnt(&C.ms->empty[s], NCW);
+      ++tc;
+    } else {
+      mbar_arrive(&C.ms->empty[s]);
+    }
+    ++i;
+  }
+  // every copy issued has completed before the CTA frees its tensor memory
+  if (tc > 0) {
+    const uint32_t last = tc - 1;
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(&C.ms->tfull[last % NTSD], (last / NTSD) & 1)) {
+      if (globaltimer() - t0 > (uint64_t)C.P->timeout_ns) break;
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -922,8 +1067,9 @@ __device__ void xproducer(const Ctx& C) {
   const int M = P.M;
   const uint64_t pol = policy_evict_last();
   uint32_t ix = 0;
-  const int beg = P.task_off[blockIdx.x], end = P.task_off[blockIdx.x + 1];
+  const int beg = P.task_off[blockIdx.x], end = task_end_of(P);
   if (P.stall_ctr >= 0) return;
+  phase_dependency_wait(P);
   for (int ti = beg; ti < end; ++ti) {
     const Task t = P.tasks[ti];
     if (!gemv_like<MOE>(t)) continue;
@@ -1052,6 +1198,35 @@ __device__ __forceinline__ void wait_full(const Ctx& C, uint32_t it) {
 __device__ __forceinline__ void release_stage(const Ctx& C, uint32_t it) {
   __syncwarp();
   if ((threadIdx.x & 31) == 0) mbar_arrive(&C.ms->empty[it % NSTAGE]);
+}
+
+// Wait for TMEM slot of TMEM chunk `tc` to be filled (the mover's copy commit).
+__device__ __forceinline__ void wait_tfull(const Ctx& C, uint32_t tc) {
+  const int t = tc % NTSD;
+  const uint32_t par = (tc / NTSD) & 1;
+  const bool tr = MK_TRACE && C.P->trace && threadIdx.x == 0;
+  const long long c0 = tr ? clock64() : 0;
+  if (tr) C.ms->tr_chunks++;
+  if ((threadIdx.x & 31) == 0) {
+    uint32_t spins = 0;
+    uint64_t t0 = 0;
+    while (!mbar_try_wait(&C.ms->tfull[t], par)) {
+      if (++spins >= 64) {
+        spins = 0;
+        if (C.ms->abort) break;
+        uint64_t now = globaltimer();
+        if (t0 == 0) t0 = now;
+        else if (now - t0 > (uint64_t)C.P->timeout_ns * 2) {
+          raise_error(*C.P, C.ms, DERR_TIMEOUT, 0xB0000 | t);
+          break;
+        }
+      }
+    }
+  }
+  __syncwarp();
+  if (!C.ms->abort) while (!mbar_try_wait(&C.ms->tfull[t], par)) {}
+  tc_fence_after();
+  if (tr) C.ms->tr_wf += clock64() - c0;
 }
 
 // Thread 0 decides, every consumer thread gets the same answer (a barrier
@@ -1191,13 +1366,13 @@ __device__ __forceinline__ void fold_lo_cols(float (&c)[4], int M, int tq, int l
 
 template <int NR, bool FP8>
 __device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& mr, const GemvLane& Lr, uint32_t& itr,
-                                        uint32_t& ixr, float* red, bool accum) {
+                                        uint32_t& ixr, uint32_t& tcr, float* red, bool accum) {
   // register copies (the arguments live in the caller's frame)
   const Ctx C = Cr;
   const Mat m = mr;
   const GemvLane L = Lr;
   ChunkIt ci = cir;
-  uint32_t it = itr, ix = ixr;
+  uint32_t it = itr, ix = ixr, tc = tcr;
   float acc[NR][4];
 #pragma unroll
   for (int r = 0; r < NR; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
@@ -1227,14 +1402,35 @@ __device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
         if (L.trc) C.ms->tr_frag += clock64() - tv0;
       }
     }
-    wait_full(C, it);
+    const bool tm = !FP8 && ci.tm;
+    if (tm) wait_tfull(C, tc);
+    else wait_full(C, it);
     const uint8_t* stage = C.ring + (size_t)(it % NSTAGE) * STAGE_BYTES;
     const uint8_t* xs = slot + (size_t)gr * L.rowbytes + (size_t)(ci.c0 - ci.w0()) * 64 + tq * 16;
     const int nc = ci.nc;
     if (L.trc) tc0 = clock64();
     // kept rolled: the instruction working set of the whole kernel must stay
     // small (one CTA executes every phase of every layer)
-    if (!FP8) {
+    if (tm) {
+      // tile (r, j) = tile r * nc + j of the chunk sits in 4-column group
+      // (r * nc + j) / 4, lane quarter j mod 4 = warp mod 4
+      const uint32_t tbase = C.tmem + (uint32_t)((tc % NTSD) * TSLOT_COLS) + ((uint32_t)(L.warp & 3) << 21);
+#pragma unroll 1
+      for (int j = L.warp; j < nc; j += NCW) {
+        const uint4 xf = xok ? lds128(xs + j * 64) : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t b0 = lo_col ? xf.z : xf.x, b1 = lo_col ? xf.w : xf.y;
+        uint4 a[NR];
+#pragma unroll
+        for (int r = 0; r < NR; ++r) a[r] = tmem_ld16(tbase + 4 * (uint32_t)((r * nc + j) >> 2));
+        tmem_ld_wait();
+#pragma unroll
+        for (int r = 0; r < NR; ++r) mma_bf16(acc[r], a[r], b0, b1);
+        if (!pk) {
+#pragma unroll
+          for (int r = 0; r < NR; ++r) mma_bf16(acc[r], a[r], xf.z, xf.w);
+        }
+      }
+    } else if (!FP8) {
 #pragma unroll 1
       for (int j = L.warp; j < nc; j += NCW) {
         const uint4 xf = xok ? lds128(xs + j * 64) : make_uint4(0u, 0u, 0u, 0u);
@@ -1289,13 +1485,16 @@ __device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
       C.ms->tr_mma += t1 - tc0;
       tc0 = t1;
     }
+    if (tm) tc_fence_before();
     __syncwarp();
     const bool xlast = ci.win_last();
     if (lane == 0) {
-      mbar_arrive(&C.ms->empty[it % NSTAGE]);
+      if (tm) mbar_arrive(&C.ms->tempty[tc % NTSD]);
+      else mbar_arrive(&C.ms->empty[it % NSTAGE]);
       if (xlast) mbar_arrive(&C.ms->xempty[ix % XSLOTS]);
     }
     ++it;
+    if (tm) ++tc;
     if (xlast) ++ix;
     if (L.trc) C.ms->tr_rel += clock64() - tc0;
     if (ci.group_done()) break;
@@ -1320,10 +1519,11 @@ __device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
   cir = ci;
   itr = it;
   ixr = ix;
+  tcr = tc;
 }
 
 template <bool MOE>
-__device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix) {
+__device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix, uint32_t& tc) {
   const Launch& P = *C.P;
   const long long tpre = (MK_TRACE && P.trace && threadIdx.x == 0) ? clock64() : 0;
   const Model& md = *C.md;
@@ -1393,25 +1593,25 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
     // weights exist only for experts, so only MoE kernels reach the fp8 ones)
     if (!MOE || !m.fp8) {
       switch (ci.nr) {
-        case 1: gemv_group<1, false>(C, ci, mg, L, it, ix, red, accum); break;
-        case 2: gemv_group<2, false>(C, ci, mg, L, it, ix, red, accum); break;
-        case 3: gemv_group<3, false>(C, ci, mg, L, it, ix, red, accum); break;
-        case 4: gemv_group<4, false>(C, ci, mg, L, it, ix, red, accum); break;
-        case 5: gemv_group<5, false>(C, ci, mg, L, it, ix, red, accum); break;
-        case 6: gemv_group<6, false>(C, ci, mg, L, it, ix, red, accum); break;
-        case 7: gemv_group<7, false>(C, ci, mg, L, it, ix, red, accum); break;
-        default: gemv_group<8, false>(C, ci, mg, L, it, ix, red, accum); break;
+        case 1: gemv_group<1, false>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        case 2: gemv_group<2, false>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        case 3: gemv_group<3, false>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        case 4: gemv_group<4, false>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        case 5: gemv_group<5, false>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        case 6: gemv_group<6, false>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        case 7: gemv_group<7, false>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        default: gemv_group<8, false>(C, ci, mg, L, it, ix, tc, red, accum); break;
       }
     } else {
       switch (ci.nr) {
-        case 1: gemv_group<1, true>(C, ci, mg, L, it, ix, red, accum); break;
-        case 2: gemv_group<2, true>(C, ci, mg, L, it, ix, red, accum); break;
-        case 3: gemv_group<3, true>(C, ci, mg, L, it, ix, red, accum); break;
-        case 4: gemv_group<4, true>(C, ci, mg, L, it, ix, red, accum); break;
-        case 5: gemv_group<5, true>(C, ci, mg, L, it, ix, red, accum); break;
-        case 6: gemv_group<6, true>(C, ci, mg, L, it, ix, red, accum); break;
-        case 7: gemv_group<7, true>(C, ci, mg, L, it, ix, red, accum); break;
-        default: gemv_group<8, true>(C, ci, mg, L, it, ix, red, accum); break;
+        case 1: gemv_group<1, true>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        case 2: gemv_group<2, true>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        case 3: gemv_group<3, true>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        case 4: gemv_group<4, true>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        case 5: gemv_group<5, true>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        case 6: gemv_group<6, true>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        case 7: gemv_group<7, true>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        default: gemv_group<8, true>(C, ci, mg, L, it, ix, tc, red, accum); break;
       }
     }
     if (pc.seg != pc.nseg - 1) {
@@ -2506,13 +2706,14 @@ __device__ __noinline__ void mla_comb_task(const Ctx& C, const Task t) {
 template <bool MLA, bool MOE>
 __device__ void consumer(const Ctx& C) {
   const Launch& P = *C.P;
-  uint32_t it = 0, ix = 0;
+  uint32_t it = 0, ix = 0, tc = 0;
   if (P.stall_ctr >= 0) {
     // test hook: a dependency that nothing signals
     wait_counter(C, P.stall_ctr, 1u);
     return;
   }
-  const int beg = P.task_off[blockIdx.x], end = P.task_off[blockIdx.x + 1];
+  const int beg = P.task_off[blockIdx.x], end = task_end_of(P);
+  phase_dependency_wait(P);
   for (int ti = beg; ti < end; ++ti) {
     const Task t = P.tasks[ti];
     // while this task waits and runs: the next task's record into L1, and
@@ -2539,7 +2740,7 @@ __device__ void consumer(const Ctx& C) {
     if (t.wait_ctr >= 0) wait_counter(C, t.wait_ctr, (uint32_t)t.wait_tgt);
     if (tr) td = globaltimer();
     if (gemv_like<MOE>(t)) {
-      gemv_task<MOE>(C, t, it, ix);
+      gemv_task<MOE>(C, t, it, ix, tc);
     } else if (!MLA && t.type == T_ATTN) {
       attn_task(C, t, it);
     } else if (MLA && t.type == T_MLA) {
@@ -2618,7 +2819,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) mk_step_kernel(const __grid_const
   if (tid == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(&C.ms->full[s], 1);
-      mbar_init(&C.ms->empty[s], NCW);
+      mbar_init(&C.ms->empty[s], NCW + (NTS > 0 ? 1 : 0));
+    }
+    for (int t = 0; t < NTS; ++t) {
+      mbar_init(&C.ms->tfull[t], 1);
+      mbar_init(&C.ms->tempty[t], NCW);
     }
     for (int s = 0; s < XSLOTS; ++s) {
       mbar_init(&C.ms->xfull[s], 2);  // the copies' expect-tx arrival + the scales
@@ -2628,14 +2833,29 @@ __global__ void __launch_bounds__(NTHREADS, 1) mk_step_kernel(const __grid_const
     C.ms->route_layer = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  // the next phase kernel may be scheduled as soon as SMs free up
+  if (P.phase_mode == 1) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (NTS > 0 && (tid >> 5) == WARP_MV) tmem_alloc(&C.ms->tmem_base, TMEM_COLS);
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  C.tmem = C.ms->tmem_base;
 
   if ((tid >> 5) == WARP_WP) producer<MLA, MOE>(C);
   else if ((tid >> 5) == WARP_XP) xproducer<MOE>(C);
+  else if ((tid >> 5) == WARP_MV) mover(C);
   else consumer<MLA, MOE>(C);
+  tc_fence_before();
   __syncthreads();
+  // every TMEM read and copy of the CTA has completed: free the columns
+  if (NTS > 0 && (tid >> 5) == WARP_MV) {
+    tc_fence_after();
+    tmem_dealloc(C.tmem, TMEM_COLS);
+  }
 
   // ---- teardown: the last CTA out zeroes every counter for the next launch ----
+  // (a phase kernel other than the step's last leaves them to later phases)
+  if (P.phase_mode == 1) return;
   if (tid == 0) {
     int last = 0;
     if (!global_abort(P)) {

@@ -20,9 +20,10 @@ STATUS_NAMES = {0: "MK_OK", 1: "MK_ERR_INVALID", 2: "MK_ERR_OOM", 3: "MK_ERR_CUD
 
 # Every symbol include/mk.h declares.
 EXPORTS = ("mk_create", "mk_init_random", "mk_load_weights", "mk_kv_create", "mk_kv_fill_random", "mk_kv_copy_out",
-           "mk_kv_bytes", "mk_decode_step", "mk_decode_step_noalloc", "mk_verify", "mk_set_router_trace", "mk_set_trace", "mk_sync_status", "mk_reset",
-           "mk_launch_info", "mk_weight_bytes", "mk_debug_inject_stall", "mk_last_error", "mk_kv_destroy",
-           "mk_destroy")
+           "mk_kv_copy_in", "mk_kv_bytes", "mk_decode_step", "mk_decode_step_noalloc", "mk_verify", "mk_prefill",
+           "mk_spec_generate", "mk_decode_step_multikernel",
+           "mk_set_router_trace", "mk_set_trace", "mk_sync_status", "mk_reset", "mk_launch_info", "mk_weight_bytes",
+           "mk_debug_inject_stall", "mk_last_error", "mk_kv_destroy", "mk_destroy")
 
 
 class MkError(RuntimeError):
@@ -44,6 +45,15 @@ class mk_synth_params(ctypes.Structure):
                 ("gain_sigma", ctypes.c_float), ("fp8_block_base", ctypes.c_float)]
 
 
+class mk_spec_stats(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in ("launches", "proposed", "accepted", "emitted")]
+
+
+# int32_t draft(void* user, const int32_t* history, int32_t n_history, int32_t* proposals, int32_t max_k)
+DRAFT_FN = ctypes.CFUNCTYPE(ctypes.c_int32, ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32), ctypes.c_int32,
+                            ctypes.POINTER(ctypes.c_int32), ctypes.c_int32)
+
+
 class mk_tensor_src(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int32), ("layer", ctypes.c_int32), ("expert", ctypes.c_int32),
                 ("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("data", ctypes.c_void_p),
@@ -63,10 +73,15 @@ def _load() -> ctypes.CDLL:
         "mk_kv_create": ([vp, ctypes.c_int, ctypes.c_int, ctypes.POINTER(vp)], st),
         "mk_kv_fill_random": ([vp, ctypes.c_uint64, ctypes.c_float, i32], st),
         "mk_kv_copy_out": ([vp, vp], st),
+        "mk_kv_copy_in": ([vp, vp], st),
         "mk_kv_bytes": ([vp], i64),
         "mk_decode_step": ([vp, vp, vp, ctypes.c_int, vp, vp, vp, vp], st),
         "mk_decode_step_noalloc": ([vp, vp, vp, ctypes.c_int, vp, vp, vp, vp], st),
+        "mk_decode_step_multikernel": ([vp, vp, vp, ctypes.c_int, vp, vp, vp, vp], st),
         "mk_verify": ([vp, vp, ctypes.c_int, i32, vp, vp, vp, vp, vp], st),
+        "mk_prefill": ([vp, vp, ctypes.c_int, ctypes.c_int, i32, vp, vp, vp], st),
+        "mk_spec_generate": ([vp, vp, i32, i32, i32, DRAFT_FN, vp, ctypes.POINTER(i32), ctypes.POINTER(mk_spec_stats),
+                              vp], st),
         "mk_set_router_trace": ([vp, vp, vp], st),
         "mk_set_trace": ([vp, vp, i32], st),
         "mk_sync_status": ([vp], st),
@@ -146,6 +161,10 @@ def mk_kv_copy_out(h: int, kv: int, dst) -> None:
     _check(h, lib.mk_kv_copy_out(kv, _ptr(dst)))
 
 
+def mk_kv_copy_in(h: int, kv: int, src) -> None:
+    _check(h, lib.mk_kv_copy_in(kv, _ptr(src)))
+
+
 def mk_kv_bytes(kv: int) -> int:
     return lib.mk_kv_bytes(kv)
 
@@ -162,10 +181,37 @@ def mk_decode_step_noalloc(h: int, tokens, positions, B: int, kv: int, logits_ou
                                          _stream(stream)))
 
 
+def mk_decode_step_multikernel(h: int, tokens, positions, B: int, kv: int, logits_out, argmax_out,
+                               stream=None) -> None:
+    """The decode step as one kernel per phase in a CUDA graph (include/mk.h)."""
+    _check(h, lib.mk_decode_step_multikernel(h, _ptr(tokens), _ptr(positions), B, kv, _ptr(logits_out),
+                                             _ptr(argmax_out), _stream(stream)))
+
+
 def mk_verify(h: int, tokens8, n_prop: int, position: int, kv: int, logits_out, argmax_out, accepted_out,
               stream=None) -> None:
     _check(h, lib.mk_verify(h, _ptr(tokens8), n_prop, position, kv, _ptr(logits_out), _ptr(argmax_out),
                             _ptr(accepted_out), _stream(stream)))
+
+
+def mk_prefill(h: int, tokens, n: int, seq: int, start: int, kv: int, argmax_last=None, stream=None) -> None:
+    _check(h, lib.mk_prefill(h, _ptr(tokens), n, seq, start, kv, _ptr(argmax_last), _stream(stream)))
+
+
+def mk_spec_generate(h: int, kv: int, anchor: int, position: int, n_out: int, draft, stream=None):
+    """draft(history: list[int], max_k: int) -> list[int] of proposals.
+    Returns (emitted tokens, stats dict)."""
+    def _cb(user, hist, n, props, max_k):
+        out = draft([hist[i] for i in range(n)], int(max_k))
+        k = min(len(out), int(max_k))
+        for i in range(k):
+            props[i] = int(out[i])
+        return k
+    cb = DRAFT_FN(_cb)
+    out = (ctypes.c_int32 * n_out)()
+    stats = mk_spec_stats()
+    _check(h, lib.mk_spec_generate(h, kv, anchor, position, n_out, cb, None, out, ctypes.byref(stats), _stream(stream)))
+    return list(out), {n: getattr(stats, n) for n, _ in mk_spec_stats._fields_}
 
 
 def mk_set_router_trace(h: int, idx_dev, w_dev) -> None:

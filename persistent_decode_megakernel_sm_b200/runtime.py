@@ -38,6 +38,11 @@ class KVCache:
         mk.mk_kv_copy_out(self.model.h, self.h, out)
         return out
 
+    def copy_in(self, src: torch.Tensor):
+        """Replace the cache with `src` (device, logical order, nbytes() bytes)."""
+        assert src.is_cuda and src.numel() * src.element_size() == self.nbytes()
+        mk.mk_kv_copy_in(self.model.h, self.h, src)
+
     def close(self):
         if self.h:
             mk.mk_kv_destroy(self.h)
@@ -67,9 +72,24 @@ class Megakernel:
         B = tokens.numel()
         mk.mk_decode_step(self.h, tokens, positions, B, kv.h, logits, argmax, stream)
 
+    def decode_step_multikernel(self, tokens: torch.Tensor, positions: torch.Tensor, kv: KVCache,
+                                logits: Optional[torch.Tensor], argmax: torch.Tensor, stream=None):
+        """The same step as one kernel per phase in a CUDA graph (comparison path)."""
+        mk.mk_decode_step_multikernel(self.h, tokens, positions, tokens.numel(), kv.h, logits, argmax, stream)
+
     def verify(self, tokens: torch.Tensor, position: int, kv: KVCache, logits: Optional[torch.Tensor],
                argmax: torch.Tensor, accepted: torch.Tensor, stream=None):
         mk.mk_verify(self.h, tokens, tokens.numel() - 1, position, kv.h, logits, argmax, accepted, stream)
+
+    def prefill(self, tokens: torch.Tensor, seq: int, start: int, kv: KVCache,
+                argmax_last: Optional[torch.Tensor] = None, stream=None):
+        """Write the K/V of tokens (positions start ..) of cache sequence seq."""
+        mk.mk_prefill(self.h, tokens, tokens.numel(), seq, start, kv.h, argmax_last, stream)
+
+    def spec_generate(self, kv: KVCache, anchor: int, position: int, n_out: int, draft, stream=None):
+        """Speculative greedy generation on cache sequence 0 (mk_spec_generate):
+        draft(history, max_k) -> proposals.  Returns (tokens, stats)."""
+        return mk.mk_spec_generate(self.h, kv.h, anchor, position, n_out, draft, stream)
 
     def set_router_trace(self, idx: Optional[torch.Tensor], w: Optional[torch.Tensor]):
         mk.mk_set_router_trace(self.h, idx, w)

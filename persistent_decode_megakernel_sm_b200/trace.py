@@ -81,6 +81,12 @@ def summarize(tr: np.ndarray, sm_clock_mhz: float = 0.0) -> dict:
         out["phases"][name] = {k: (v / ctas if k.endswith("_us") else v) for k, v in p.items()}
         out["phases"][name]["per_cta_us_note"] = "times summed over the CTA's tasks, averaged over CTAs"
     out["compute_fraction"] = busy / ctas / step_us
+    # SM idle between tasks: the part of the step a CTA spends outside task
+    # bodies (waiting for a task's dependency, or done before the step ends)
+    run_ns = np.where(valid, tr[:, :, 2] - tr[:, :, 1], 0).sum(axis=1).astype(np.float64)
+    idle = 1.0 - run_ns / float(t1 - t0)
+    out["idle_between_tasks_fraction"] = float(idle.mean())
+    out["idle_between_tasks_fraction_max_cta"] = float(idle.max())
     out["producer_blocked_us_per_cta"] = float(tr[:, 0, 12].mean()) / sm_clock_mhz
     out["producer_chunks_per_cta"] = float(tr[:, 0, 13].mean())
     out["producer_span_us"] = float((tr[:, 0, 15] - tr[:, 0, 14]).mean()) / 1e3

@@ -40,3 +40,81 @@ def gpu_model(mc, max_batch: int = 8):
 
 def tokens_at(mc, seq: int, positions):
     return synth.seq_tokens(synth.SEED_TOKENS, seq, positions, mc.vocab)
+
+
+# Router weights: fp32 softmax over fp32 logits on the GPU against fp64.
+RW_ATOL = 1e-3
+
+
+def check_router(mc, gidx, gw, ref, rows):
+    """Every router decision of every layer and row.  The oracle ran with
+    follow=gidx, so at its own near-ties it adopted the GPU's selection when
+    that selection is correct at tolerance DELTA; everywhere the two must
+    then pick the same experts (as a set), with the same renormalised
+    weights per expert.  Returns the number of decisions where the oracle
+    followed the GPU."""
+    gi, gwn = np.asarray(gidx), np.asarray(gw)
+    ri, rw = ref["router_idx"], ref["router_w"]
+    for l in range(mc.layers):
+        for r in range(rows):
+            a, b = [int(e) for e in gi[l, r]], [int(e) for e in ri[l, r]]
+            assert sorted(a) == sorted(b), ("router", l, r, a, b, float(ref["router_margin"][l, r]))
+            wa = dict(zip(a, gwn[l, r].tolist()))
+            wb = dict(zip(b, rw[l, r].tolist()))
+            err = max(abs(wa[e] - wb[e]) for e in a)
+            assert err <= RW_ATOL, ("router weight", l, r, err)
+    return int(ref["router_followed"][:, :rows].sum())
+
+
+def compare_rows(glogits, gargmax, ref, rows, fp8=False, what=""):
+    """Logits and greedy token of each row against the oracle (tolerances
+    above); asserts that at least one row was compared and returns the
+    largest error seen."""
+    worst, n = 0.0, 0
+    for b in rows:
+        ok, err, sc = logits_close(glogits[b], ref["logits"][b], fp8=fp8)
+        assert ok, (what, b, err, sc)
+        assert argmax_agrees(int(gargmax[b]), ref["logits"][b], int(ref["argmax"][b]), ref["argmax_margin"][b]), \
+            (what, b, int(gargmax[b]), int(ref["argmax"][b]), float(ref["argmax_margin"][b]))
+        worst = max(worst, err)
+        n += 1
+    assert n > 0, "nothing compared"
+    return worst
+
+
+# Absolute slack of a cache value, relative to the largest value of the
+# compared rows.  The GPU's K/V are fp32 dot products over thousands of terms
+# of an fp32 residual stream, so a value that is small through cancellation
+# carries the absolute error of the row's scale (~1e-5 of it per layer, and
+# the residual stream's error grows with depth: ~1e-4 after 64 layers), which
+# can exceed one bf16 step of the small value itself.
+KV_ATOL_REL = 1e-3
+
+
+def code_mismatch(a, b):
+    """Compare bf16 cache codes written by the GPU (fp32 arithmetic) and by
+    the oracle (fp64): each value must be within one bf16 step of the other,
+    up to KV_ATOL_REL of the rows' largest value, and returns the fraction of
+    codes that differ at all (a value whose exact result lies within the
+    GPU's rounding error of a bf16 rounding boundary can land on the
+    neighbouring code)."""
+    fa = synth.bf16_to_f32(np.ascontiguousarray(a)).astype(np.float64)
+    fb = synth.bf16_to_f32(np.ascontiguousarray(b)).astype(np.float64)
+    ulp = 2.0 ** -7 * np.maximum(np.abs(fa), np.abs(fb))
+    atol = KV_ATOL_REL * float(np.max(np.abs(fb)))
+    excess = np.abs(fa - fb) - ulp - atol
+    assert np.all(excess <= 0), (float(np.max(excess)), atol / KV_ATOL_REL)
+    rate = float(np.mean(a != b))
+    print(f"[cache codes differing: {rate:.3e} of {a.size}]")
+    return rate
+
+
+# Bound on the fraction of cache codes that differ after a few layers: a value
+# carried with a relative error of ~1e-6 (fp32 accumulation) falls on the
+# other side of a bf16 rounding boundary (spaced 2^-8 relative) for about
+# 2e-6 / 2^-8 = 5e-4 of values; the bound allows ten times that.
+CODE_MISMATCH_MAX = 5e-3
+# At full depth the residual stream's relative error (~1e-4 after 64 layers)
+# puts about 2e-4 / 2^-8 = 5 % of the deepest layers' codes within reach of a
+# boundary; bound for the whole-model tests.
+CODE_MISMATCH_MAX_DEEP = 0.1

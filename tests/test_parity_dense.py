@@ -5,7 +5,8 @@ import torch
 
 import oracle
 import synth
-from harness import argmax_agrees, gpu_model, logits_close, tokens_at
+from harness import (CODE_MISMATCH_MAX, argmax_agrees, check_router, code_mismatch, compare_rows, gpu_model,
+                     logits_close, tokens_at)
 
 pytestmark = pytest.mark.gpu
 
@@ -42,41 +43,112 @@ def test_tiny_prefill_and_greedy_decode(tiny):
             ok, err, sc = logits_close(logits.cpu().numpy()[0], ref["logits"][0])
             assert ok, (p, err, sc)
     assert m.sync_status() == 0
-    # greedy decode: each side feeds its own argmax
-    tok_g = tok_o = int(tokens_at(mc, 0, [mc.context])[0])
+    # greedy decode, teacher-forced: both sides consume the GPU's token, so
+    # a near-tie (where the two greedy choices may differ) does not end the run
+    tok = int(tokens_at(mc, 0, [mc.context])[0])
     for step in range(16):
         p = mc.context + step
-        m.decode_step(_t([tok_g]), _t([p]), kv, logits, am)
-        ref = orc.step([tok_o], [p])
+        m.decode_step(_t([tok]), _t([p]), kv, logits, am)
+        ref = orc.step([tok], [p])
         torch.cuda.synchronize()
         g = logits.cpu().numpy()[0]
-        ok, err, sc = logits_close(g, ref["logits"][0])
-        assert ok, (step, err, sc)
         ga = int(am.item())
         assert ga == int(np.argmax(g)) or g[ga] == g.max()
-        assert argmax_agrees(ga, ref["logits"][0], int(ref["argmax"][0]), ref["argmax_margin"][0]), step
-        if ga != int(ref["argmax"][0]):
-            break  # near-tie: the two greedy chains legitimately diverge here
-        tok_g, tok_o = ga, int(ref["argmax"][0])
+        compare_rows(logits.cpu().numpy(), am.cpu().numpy(), ref, range(1), False, f"greedy step {step}")
+        tok = ga
     assert m.sync_status() == 0
-    # KV cache: bf16 values written by both sides
+    # KV cache: bf16 values written by both sides, one code apart at most
     kk, vv = orc.kv_arrays()
     dev = kv.copy_out().cpu().numpy().view(np.uint16)
     half = dev.size // 2
     n_pos = mc.context + 16
     gk = dev[:half].reshape(kk.shape)[:, :, :, :n_pos]
     gv = dev[half:].reshape(vv.shape)[:, :, :, :n_pos]
-    for a, b in ((gk, kk[:, :, :, :n_pos]), (gv, vv[:, :, :, :n_pos])):
-        # Both sides round their own K/V to bf16 (fp32 on the GPU, fp64 in the
-        # oracle): a value within ~1e-5 of a rounding boundary may land on the
-        # neighbouring bf16 code.  Require at most one code apart, and rarely.
-        fa = synth.bf16_to_f32(np.ascontiguousarray(a)).astype(np.float64)
-        fb = synth.bf16_to_f32(np.ascontiguousarray(b)).astype(np.float64)
-        scale = np.max(np.abs(fb))
-        ulp = 2.0 ** -7 * np.maximum(np.abs(fa), np.abs(fb))
-        assert np.all(np.abs(fa - fb) <= ulp + 1e-3 * scale)
-        assert np.mean(a != b) < 0.1
+    rate = code_mismatch(np.stack([gk, gv]), np.stack([kk[:, :, :, :n_pos], vv[:, :, :, :n_pos]]))
+    assert rate <= CODE_MISMATCH_MAX, rate
     kv.close()
+
+
+@pytest.mark.parametrize("name", ["tiny", "tiny_moe", "tiny_mla"])
+def test_prefill_in_chunks_matches_oracle(name):
+    """mk_prefill runs a prompt 8 positions per launch (the verify form), for
+    cache sequence 0 and, in a second call, sequence 1.  The cache it writes
+    matches the oracle's position-by-position prefill code for code (within
+    the mismatch bound), its last greedy tokens are the oracle's, and a decode
+    step over the GPU-written cache (handed to the oracle) matches."""
+    mc = synth.preset(name, gain_sigma=0.1)
+    m = gpu_model(mc)
+    n = mc.context + 5  # a ragged last chunk
+    kv = m.kv_cache(2, mc.max_ctx)
+    toks = [tokens_at(mc, s, range(n + 1)) for s in range(2)]
+    last = [torch.full((1,), -1, dtype=torch.int32, device=DEV) for _ in range(2)]
+    for s in range(2):
+        m.prefill(_t(toks[s][:n]), s, 0, kv, last[s])
+    orc = oracle.OracleModel(mc.replace(max_seqs=2))
+    for p in range(n):
+        r = orc.step([toks[0][p], toks[1][p]], [p, p], want_logits=(p == n - 1))
+    torch.cuda.synchronize()
+    assert m.sync_status() == 0
+    for s in range(2):
+        assert argmax_agrees(int(last[s].item()), r["logits"][s], int(r["argmax"][s]), r["argmax_margin"][s]), s
+    dev = kv.copy_out().cpu().numpy().view(np.uint16)
+    if mc.mla:
+        lat = orc.kv_arrays()
+        rate = code_mismatch(dev.reshape(lat.shape)[:, :, :n], lat[:, :, :n])
+    else:
+        kk, vv = orc.kv_arrays()
+        half = dev.size // 2
+        gk, gv = dev[:half].reshape(kk.shape), dev[half:].reshape(vv.shape)
+        rate = code_mismatch(np.stack([gk[:, :, :, :n], gv[:, :, :, :n]]),
+                             np.stack([kk[:, :, :, :n], vv[:, :, :, :n]]))
+    assert rate <= CODE_MISMATCH_MAX, (name, rate)
+    orc.close()
+    # one decode step of both sequences over the GPU-written context
+    orc = oracle.OracleModel(mc.replace(max_seqs=2))
+    orc.set_kv(dev)
+    logits = torch.empty((2, mc.vocab), dtype=torch.float32, device=DEV)
+    am = torch.empty(2, dtype=torch.int32, device=DEV)
+    k = max(mc.top_k, 1)
+    idx = torch.full((mc.layers, 2, k), -1, dtype=torch.int32, device=DEV)
+    w = torch.zeros((mc.layers, 2, k), dtype=torch.float32, device=DEV)
+    if mc.n_routed:
+        m.set_router_trace(idx, w)
+    step_toks = [toks[0][n], toks[1][n]]
+    m.decode_step(_t(step_toks), _t([n, n]), kv, logits, am)
+    m.set_router_trace(None, None)
+    torch.cuda.synchronize()
+    assert m.sync_status() == 0
+    gidx = idx.cpu().numpy()
+    ref = orc.step(step_toks, [n, n], follow=gidx if mc.n_routed else None)
+    if mc.n_routed:
+        check_router(mc, gidx, w.cpu().numpy(), ref, 2)
+    compare_rows(logits.cpu().numpy(), am.cpu().numpy(), ref, range(2), bool(mc.expert_fp8), name)
+    orc.close()
+    kv.close()
+    m.close()
+
+
+def test_kv_copy_in_round_trip(tiny):
+    """mk_kv_copy_in is the inverse of mk_kv_copy_out (logical order in and
+    out), and a step over a copied-in cache equals the step over the original."""
+    mc, m = tiny
+    a = m.kv_cache(3, mc.max_ctx)
+    b = m.kv_cache(3, mc.max_ctx)
+    a.fill_random(synth.SEED_KV, mc.kv_sigma, 77)
+    img = a.copy_out()
+    b.copy_in(img)
+    assert torch.equal(b.copy_out(), img)
+    outs = []
+    for kv in (a, b):
+        lg = torch.empty((3, mc.vocab), dtype=torch.float32, device=DEV)
+        am = torch.empty(3, dtype=torch.int32, device=DEV)
+        m.decode_step(_t([4, 5, 6]), _t([77, 60, 10]), kv, lg, am)
+        torch.cuda.synchronize()
+        outs.append(lg.cpu().numpy().copy())
+    assert np.array_equal(outs[0], outs[1])
+    assert m.sync_status() == 0
+    a.close()
+    b.close()
 
 
 @pytest.mark.parametrize("B", [1, 2, 3, 4, 8])

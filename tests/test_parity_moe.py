@@ -7,7 +7,8 @@ import torch
 
 import oracle
 import synth
-from harness import DELTA, argmax_agrees, gpu_model, logits_close, tokens_at
+from harness import (CODE_MISMATCH_MAX, DELTA, check_router, code_mismatch, compare_rows, gpu_model,
+                     tokens_at)
 
 pytestmark = pytest.mark.gpu
 
@@ -24,21 +25,31 @@ def _router_buffers(mc, M):
     return idx, w
 
 
-def _check_router(mc, idx, w, ref, rows):
-    """Expert choices are exact unless the oracle's own k-th / (k+1)-th logit
-    gap is below DELTA (a near-tie).  Returns the rows whose choice is a
-    near-tie somewhere (their logits are then not comparable)."""
-    gi = idx.cpu().numpy()
-    gw = w.cpu().numpy()
-    tied = set()
-    for l in range(mc.layers):
-        for r in range(rows):
-            if ref["router_margin"][l, r] < DELTA:
-                tied.add(r)
-                continue
-            assert list(gi[l, r]) == list(ref["router_idx"][l, r]), (l, r, gi[l, r], ref["router_idx"][l, r])
-            assert np.allclose(gw[l, r], ref["router_w"][l, r], atol=5e-3), (l, r)
-    return tied
+def _gpu_step(m, mc, toks, pos, kv, Q=1):
+    """A traced GPU step: logits, greedy tokens, accepted (verify), router."""
+    M = len(toks)
+    logits = torch.empty((M, mc.vocab), dtype=torch.float32, device=DEV)
+    am = torch.empty(M, dtype=torch.int32, device=DEV)
+    acc = torch.full((1,), -1, dtype=torch.int32, device=DEV)
+    idx, w = _router_buffers(mc, M)
+    m.set_router_trace(idx, w)
+    if Q == 1:
+        m.decode_step(_t(toks), _t(pos), kv, logits, am)
+    else:
+        m.verify(_t(toks), pos[0], kv, logits, am, acc)
+    m.set_router_trace(None, None)
+    torch.cuda.synchronize()
+    return logits.cpu().numpy(), am.cpu().numpy(), int(acc.item()), idx.cpu().numpy(), w.cpu().numpy()
+
+
+def _compare(mc, orc, m, kv, toks, pos, Q=1, fp8=False, what=""):
+    """GPU step against the oracle's step on the same tokens (the oracle
+    follows the GPU's router at its own near-ties)."""
+    g, am, acc, gidx, gw = _gpu_step(m, mc, toks, pos, kv, Q)
+    ref = orc.step(toks, pos, Q=Q, follow=gidx, delta=DELTA)
+    check_router(mc, gidx, gw, ref, len(toks))
+    compare_rows(g, am, ref, range(len(toks)), fp8, what)
+    return g, am, acc, ref
 
 
 @pytest.fixture(scope="module")
@@ -62,72 +73,34 @@ def test_tiny_moe_batched_ragged(tiny_moe, B):
     for step in range(3):
         pp = [p + step for p in pos]
         toks = [int(tokens_at(mc, s, [pp[s]])[0]) for s in range(B)]
-        logits = torch.empty((B, mc.vocab), dtype=torch.float32, device=DEV)
-        am = torch.empty(B, dtype=torch.int32, device=DEV)
-        idx, w = _router_buffers(mc, B)
-        m.set_router_trace(idx, w)
-        m.decode_step(_t(toks), _t(pp), kv, logits, am)
-        m.set_router_trace(None, None)
-        ref = orc.step(toks, pp)
-        torch.cuda.synchronize()
-        tied = _check_router(mc, idx, w, ref, B)
-        g = logits.cpu().numpy()
-        for b in range(B):
-            if b in tied:
-                continue
-            ok, err, sc = logits_close(g[b], ref["logits"][b])
-            assert ok, (step, b, err, sc)
-            assert argmax_agrees(int(am[b].item()), ref["logits"][b], int(ref["argmax"][b]),
-                                 ref["argmax_margin"][b])
+        _compare(mc, orc, m, kv, toks, pp, what=f"B={B} step {step}")
     assert m.sync_status() == 0
     kv.close()
 
 
 def test_tiny_moe_prefill_and_greedy(tiny_moe):
     """Pre-fill from seeded tokens through the model on both sides, then
-    greedy steps; also compares the K/V both sides wrote."""
+    teacher-forced greedy steps (both sides consume the GPU's token); also
+    compares the K/V both sides wrote."""
     mc, m = tiny_moe
     kv = m.kv_cache(1, mc.max_ctx)
     orc = oracle.OracleModel(mc.replace(max_seqs=1))
     toks = tokens_at(mc, 0, range(mc.context))
-    logits = torch.empty((1, mc.vocab), dtype=torch.float32, device=DEV)
-    am = torch.empty(1, dtype=torch.int32, device=DEV)
     for p in range(mc.context):
-        m.decode_step(_t([toks[p]]), _t([p]), kv, logits, am)
-        ref = orc.step([toks[p]], [p], want_logits=(p % 16 == 15))
-        if p % 16 == 15:
-            torch.cuda.synchronize()
-            ok, err, sc = logits_close(logits.cpu().numpy()[0], ref["logits"][0])
-            if not (ref["router_margin"][:, 0] < DELTA).any():
-                assert ok, (p, err, sc)
-    tok_g = tok_o = int(tokens_at(mc, 0, [mc.context])[0])
+        _compare(mc, orc, m, kv, [toks[p]], [p], what=f"prefill {p}")
+    tok = int(tokens_at(mc, 0, [mc.context])[0])
     for step in range(8):
         p = mc.context + step
-        m.decode_step(_t([tok_g]), _t([p]), kv, logits, am)
-        ref = orc.step([tok_o], [p])
-        torch.cuda.synchronize()
-        g = logits.cpu().numpy()[0]
-        if (ref["router_margin"][:, 0] < DELTA).any():
-            break
-        ok, err, sc = logits_close(g, ref["logits"][0])
-        assert ok, (step, err, sc)
-        ga = int(am.item())
-        assert argmax_agrees(ga, ref["logits"][0], int(ref["argmax"][0]), ref["argmax_margin"][0]), step
-        if ga != int(ref["argmax"][0]):
-            break
-        tok_g, tok_o = ga, int(ref["argmax"][0])
+        g, am, _, _ = _compare(mc, orc, m, kv, [tok], [p], what=f"greedy {step}")
+        tok = int(am[0])
     assert m.sync_status() == 0
     kk, vv = orc.kv_arrays()
     dev = kv.copy_out().cpu().numpy().view(np.uint16)
     half = dev.size // 2
-    n = mc.context
-    for a, b in ((dev[:half].reshape(kk.shape)[:, :, :, :n], kk[:, :, :, :n]),
-                 (dev[half:].reshape(vv.shape)[:, :, :, :n], vv[:, :, :, :n])):
-        fa = synth.bf16_to_f32(np.ascontiguousarray(a)).astype(np.float64)
-        fb = synth.bf16_to_f32(np.ascontiguousarray(b)).astype(np.float64)
-        scale = np.max(np.abs(fb))
-        assert np.all(np.abs(fa - fb) <= 2.0 ** -7 * np.maximum(np.abs(fa), np.abs(fb)) + 1e-3 * scale)
-        assert np.mean(a != b) < 0.1
+    n = mc.context + 8
+    rate = code_mismatch(np.stack([dev[:half].reshape(kk.shape)[:, :, :, :n], dev[half:].reshape(vv.shape)[:, :, :, :n]]),
+                         np.stack([kk[:, :, :, :n], vv[:, :, :, :n]]))
+    assert rate <= CODE_MISMATCH_MAX, rate
     kv.close()
 
 
@@ -150,27 +123,11 @@ def test_tiny_moe_verify(tiny_moe):
     for case, props in (("planted", chain[1:]),
                         ("random", list(synth.proposals(synth.SEED_PROPOSALS, 0, 7, mc.vocab)))):
         toks = [anchor] + [int(x) for x in props]
-        logits = torch.empty((8, mc.vocab), dtype=torch.float32, device=DEV)
-        am = torch.empty(8, dtype=torch.int32, device=DEV)
-        acc = torch.full((1,), -1, dtype=torch.int32, device=DEV)
-        idx, w = _router_buffers(mc, 8)
-        m.set_router_trace(idx, w)
-        m.verify(_t(toks), P, kv, logits, am, acc)
-        m.set_router_trace(None, None)
-        ref = orc.step(toks, [P], Q=8)
-        torch.cuda.synchronize()
-        tied = _check_router(mc, idx, w, ref, 8)
-        g = logits.cpu().numpy()
-        for j in range(8):
-            if j in tied:
-                continue
-            ok, err, sc = logits_close(g[j], ref["logits"][j])
-            assert ok, (case, j, err, sc)
-        ga = am.cpu().numpy()
-        if not tied and all(int(ga[j]) == int(ref["argmax"][j]) for j in range(8)):
-            assert int(acc.item()) == oracle.accept(toks, ref["argmax"]), case
+        g, ga, acc, ref = _compare(mc, orc, m, kv, toks, [P], Q=8, what=case)
+        if all(int(ga[j]) == int(ref["argmax"][j]) for j in range(8)):
+            assert acc == oracle.accept(toks, ref["argmax"]), case
             if case == "planted":
-                assert int(acc.item()) == 7
+                assert acc == 7
     assert m.sync_status() == 0
     kv.close()
 
@@ -184,20 +141,11 @@ def test_moe_no_shared_expert_and_top1():
     orc = oracle.OracleModel(mc.replace(max_seqs=4))
     orc.kv_fill_synthetic(synth.SEED_KV, 20)
     toks, pos = [3, 99, 1500, 7], [20, 19, 18, 0]
-    logits = torch.empty((4, mc.vocab), dtype=torch.float32, device=DEV)
-    am = torch.empty(4, dtype=torch.int32, device=DEV)
-    idx, w = _router_buffers(mc, 4)
-    m.set_router_trace(idx, w)
-    m.decode_step(_t(toks), _t(pos), kv, logits, am)
-    ref = orc.step(toks, pos)
-    torch.cuda.synchronize()
-    tied = _check_router(mc, idx, w, ref, 4)
-    assert np.allclose(w.cpu().numpy(), 1.0)
-    g = logits.cpu().numpy()
-    for b in range(4):
-        if b not in tied:
-            ok, err, sc = logits_close(g[b], ref["logits"][b])
-            assert ok, (b, err, sc)
+    _, _, _, gidx, gw = _gpu_step(m, mc, toks, pos, kv)
+    ref = orc.step(toks, pos, follow=gidx, delta=DELTA)
+    check_router(mc, gidx, gw, ref, 4)
+    assert np.allclose(gw, 1.0)
+    g2, am2, _, ref2 = _compare(mc, orc, m, kv, toks, pos, what="top1")
     assert m.sync_status() == 0
     kv.close()
     m.close()
@@ -215,21 +163,7 @@ def test_tiny_moe_fp8_experts(B):
     orc.kv_fill_synthetic(synth.SEED_KV, mc.context)
     pp = [mc.context - 3 * s for s in range(B)]
     toks = [int(tokens_at(mc, s, [pp[s]])[0]) for s in range(B)]
-    logits = torch.empty((B, mc.vocab), dtype=torch.float32, device=DEV)
-    am = torch.empty(B, dtype=torch.int32, device=DEV)
-    idx, w = _router_buffers(mc, B)
-    m.set_router_trace(idx, w)
-    m.decode_step(_t(toks), _t(pp), kv, logits, am)
-    ref = orc.step(toks, pp)
-    torch.cuda.synchronize()
-    tied = _check_router(mc, idx, w, ref, B)
-    g = logits.cpu().numpy()
-    for b in range(B):
-        if b in tied:
-            continue
-        ok, err, sc = logits_close(g[b], ref["logits"][b], fp8=True)
-        assert ok, (b, err, sc)
-        assert argmax_agrees(int(am[b].item()), ref["logits"][b], int(ref["argmax"][b]), ref["argmax_margin"][b])
+    _compare(mc, orc, m, kv, toks, pp, fp8=True, what=f"fp8 B={B}")
     assert m.sync_status() == 0
     kv.close()
     m.close()
