@@ -1080,10 +1080,12 @@ __device__ void xproducer(const Ctx& C) {
     if (t.wait_ctr >= 0 && !warp_wait_counter(C, t.wait_ctr, (uint32_t)t.wait_tgt, 0x30000)) goto drain;
     int U = 0;
     if (task_needs_route<MOE>(t)) {
-      if (t.type == T_MOE_GU) {
+      // a one-kernel-per-phase launch starts the down projection with fresh
+      // shared memory, so it computes the layer's route again
+      if (t.type == T_MOE_GU || P.phase_mode) {
         // the layer's route, with the routed weights, for this warp and for
         // the consumers (published through shared memory)
-        U = moe_route(P, md, t.layer, C.ms, RR_XPROD, true, blockIdx.x == 0);
+        U = moe_route(P, md, t.layer, C.ms, RR_XPROD, true, blockIdx.x == 0 && t.type == T_MOE_GU);
         __syncwarp();
         if (lane == 0) {
           __threadfence_block();
@@ -1313,6 +1315,15 @@ struct GemvLane {
   bool has_gain, trc;
   bool conv;              // the windows need converting (false: the input buffer holds fragments)
   const uint16_t* gain;   // norm gain of the task's input
+  // K segments taken in one call (the MoE down projection: shared experts,
+  // then the routed experts of the union, each Ie wide); the fp8 block
+  // scales of segment s are those of shared expert s (s < NS) or of routed
+  // expert ex[s - NS]
+  int nseg, NS;
+  const float* sc_sh;
+  const float* sc_rt;
+  int64_t ss_sh, ss_rt;
+  const int16_t* ex;
 };
 
 // All chunks of one row group [g0, g0 + NR): each warp takes col tiles
@@ -1364,12 +1375,22 @@ __device__ __forceinline__ void fold_lo_cols(float (&c)[4], int M, int tq, int l
   c[3] = k1 ? c[3] + u3 : 0.f;
 }
 
+// The GEMV row-group loop: one out-of-line instance per row count (small
+// instruction footprint) or inlined into the task body (no call frame).
+#ifndef MK_GEMV_INLINE
+#define MK_GEMV_INLINE 0
+#endif
+#if MK_GEMV_INLINE
+#define MK_GEMV_ATTR __forceinline__
+#else
+#define MK_GEMV_ATTR __noinline__
+#endif
 template <int NR, bool FP8>
-__device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& mr, const GemvLane& Lr, uint32_t& itr,
+__device__ MK_GEMV_ATTR void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& mr, const GemvLane& Lr, uint32_t& itr,
                                         uint32_t& ixr, uint32_t& tcr, float* red, bool accum) {
   // register copies (the arguments live in the caller's frame)
   const Ctx C = Cr;
-  const Mat m = mr;
+  const Mat m0 = mr;
   const GemvLane L = Lr;
   ChunkIt ci = cir;
   uint32_t it = itr, ix = ixr, tc = tcr;
@@ -1385,6 +1406,12 @@ __device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
   const int gr = lo_col ? g - L.M : g;
   const bool xok = g < (pk ? 2 * L.M : L.M);  // other columns are zero
   long long tc0 = 0, tl0 = L.trc ? clock64() : 0;
+  const ChunkIt ci0 = ci;
+  for (int seg = 0; seg < L.nseg; ++seg) {
+  if (seg > 0) ci = ci0;
+  Mat m = m0;
+  if (FP8 && L.nseg > 1)
+    m.scales = seg < L.NS ? L.sc_sh + (size_t)seg * L.ss_sh : L.sc_rt + (size_t)L.ex[seg - L.NS] * L.ss_rt;
   while (true) {
     const uint8_t* slot = C.xring + (size_t)(ix % XSLOTS) * XSLOT_BYTES;
     if (ci.win_first()) {
@@ -1500,6 +1527,7 @@ __device__ __noinline__ void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
     if (ci.group_done()) break;
     ci.next();
   }
+  }
   if (L.trc) C.ms->tr_loop += clock64() - tl0;
   if (pk) {
 #pragma unroll
@@ -1579,6 +1607,11 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
   L.trc = MK_TRACE && P.trace && tid == 0;
   L.conv = t.in_kind != IN_X_NORM && !frag_buf(t.in_buf);
   L.gain = t.gvec;
+  L.nseg = 1;
+  L.NS = md.NS;
+  L.sc_sh = L.sc_rt = nullptr;
+  L.ss_sh = L.ss_rt = 0;
+  L.ex = C.ms->rt_ex[RR_XPROD];
   if (L.trc) C.ms->tr_pre += clock64() - tpre;
   while (have) {
     const PieceSrc src = piece_src<MOE>(md, t, m, m2, C.ms->rt_ex[RR_XPROD], pc);
@@ -1588,7 +1621,15 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
     Mat mg = (MOE && t.type == T_MOE_DOWN && pc.seg < md.NS) ? m2 : m;
     mg.w = src.w;
     mg.scales = src.scales;
-    const bool accum = pc.seg > 0;
+    const bool accum = false;
+    if (MOE && t.type == T_MOE_DOWN) {
+      // every K segment of the row group in one call, the sums kept in registers
+      L.nseg = pc.nseg;
+      L.sc_sh = m2.scales;
+      L.ss_sh = m2.sstride;
+      L.sc_rt = m.scales;
+      L.ss_rt = m.sstride;
+    }
     // one instance per row-tile count: every loop over rows is static (fp8
     // weights exist only for experts, so only MoE kernels reach the fp8 ones)
     if (!MOE || !m.fp8) {
@@ -1614,10 +1655,7 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
         default: gemv_group<8, true>(C, ci, mg, L, it, ix, tc, red, accum); break;
       }
     }
-    if (pc.seg != pc.nseg - 1) {
-      have = pc.next();
-      continue;
-    }
+    if (MOE && t.type == T_MOE_DOWN) pc.seg = pc.nseg - 1;  // the call took every segment
     const bool trc = L.trc;
     long long tc0 = trc ? clock64() : 0;
     {

@@ -26,6 +26,8 @@ def main():
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--steps", type=int, default=3)
     ap.add_argument("--warmup", type=int, default=2)
+    ap.add_argument("--verify", action="store_true",
+                    help="launch verify steps (1 anchor + 7 seeded proposals on sequence 0) instead of decode steps")
     a = ap.parse_args()
     sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
     import torch
@@ -42,19 +44,26 @@ def main():
     m.init_random(mc.seed, mc.w_sigma, mc.router_sigma, mc.gain_sigma, mc.fp8_block_base)
     kv = m.kv_cache(8, mc.max_ctx)
     kv.fill_random(synth.SEED_KV, mc.kv_sigma, mc.context)
-    B = a.batch
+    B = 8 if a.verify else a.batch
     tok = torch.tensor(synth.tokens(synth.SEED_TOKENS, B, mc.vocab), dtype=torch.int32, device=dev)
     lg = torch.empty((B, mc.vocab), dtype=torch.float32, device=dev)
     am = torch.empty(B, dtype=torch.int32, device=dev)
+    acc = torch.empty(1, dtype=torch.int32, device=dev)
     for i in range(a.warmup + a.steps):
-        pos = torch.full((B,), mc.context + i, dtype=torch.int32, device=dev)
-        m.decode_step(tok, pos, kv, lg, am)
-        tok = am.clone()
+        if a.verify:
+            props = synth.proposals(synth.SEED_PROPOSALS, i, 7, mc.vocab)
+            toks8 = torch.tensor([int(tok[0].item())] + [int(x) for x in props], dtype=torch.int32, device=dev)
+            m.verify(toks8, mc.context, kv, lg, am, acc)
+        else:
+            pos = torch.full((B,), mc.context + i, dtype=torch.int32, device=dev)
+            m.decode_step(tok, pos, kv, lg, am)
+            tok = am.clone()
     torch.cuda.synchronize()
     assert m.sync_status() == 0
     weights = m.weight_bytes() - mc.vocab * mc.hidden * 2 + B * mc.hidden * 2
     kvt = (mc.kv_lora_rank + mc.rope_dim) * 2 if mc.mla else 2 * mc.n_kv_heads * mc.head_dim * 2
-    cache = B * (mc.context + a.warmup) * kvt * mc.layers + B * kvt * mc.layers
+    cache = (mc.context * kvt * mc.layers + 8 * kvt * mc.layers if a.verify
+             else B * (mc.context + a.warmup) * kvt * mc.layers + B * kvt * mc.layers)
     key = "weight_bytes_resident_upper_bound" if mc.n_routed else "weight_bytes_streamed"
     print(json.dumps({"config": a.config, "layers": mc.layers, "vocab": mc.vocab, "batch": B,
                       key: weights, "cache_bytes": cache, "logit_bytes": B * mc.vocab * 4,

@@ -114,7 +114,9 @@ def code_mismatch(a, b):
 # other side of a bf16 rounding boundary (spaced 2^-8 relative) for about
 # 2e-6 / 2^-8 = 5e-4 of values; the bound allows ten times that.
 CODE_MISMATCH_MAX = 5e-3
-# At full depth the residual stream's relative error (~1e-4 after 64 layers)
-# puts about 2e-4 / 2^-8 = 5 % of the deepest layers' codes within reach of a
-# boundary; bound for the whole-model tests.
-CODE_MISMATCH_MAX_DEEP = 0.1
+# At full depth the residual stream's relative error grows with depth (~1e-4
+# after 64 layers), which puts a few percent of the deepest layers' codes
+# within reach of a boundary.  Measured on B200 over the rows one step writes
+# in every layer: 3.0 % / 3.3 % (dense 27B-shaped, B = 1 / 8), 1.2 - 1.5 %
+# (MoE), 1.8 - 2.0 % (latent attention); the 2-layer models 0.15 - 0.23 %.
+CODE_MISMATCH_MAX_DEEP = 0.06
