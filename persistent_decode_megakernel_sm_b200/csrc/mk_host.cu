@@ -412,6 +412,11 @@ static bool desc_ok(const mk_model_desc* d, std::string& why) {
     }
   }
   if (d->expert_fp8 && d->n_routed == 0) { why = "fp8 weights are supported for experts only"; return false; }
+  if (d->expert_fp8 && (d->hidden > 16384 || d->expert_ffn > 16384)) {
+    // the kernel stages a row group's block scales (<= 128 column blocks) in shared memory
+    why = "fp8 experts need hidden and expert_ffn <= 16384";
+    return false;
+  }
   return true;
 }
 
@@ -1217,6 +1222,43 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
   off.assign(ncta + 1, 0);
   next_phase();  // tags the last phase's tasks
   n_phases_out = phase;
+#ifndef MK_TAIL_PREFETCH
+#define MK_TAIL_PREFETCH 0
+#endif
+  // L2 requests one task ahead, issued by the weight producer when it starts
+  // the CTA's previous task:
+  //  - a CTA that streams one row tile more than the phase's even share ends
+  //    the phase late by that row's HBM time: that row is requested, so it
+  //    streams from L2;
+  //  - (mode 2) a projection that follows attention gets all of the CTA's rows
+  //    requested, since attention leaves HBM nearly idle.
+  if (MK_TAIL_PREFETCH) {
+    for (int c = 0; c < ncta; ++c) {
+      std::vector<Task>& v = per[c];
+      for (size_t i = 1; i < v.size(); ++i) {
+        const Task& t = v[i];
+        if (t.type != T_GEMV || t.rt1 <= t.rt0) continue;
+        const Mat& m = h->mats[t.mat].m;
+        const int16_t prev = v[i - 1].type;
+        const bool after_att = prev == T_ATTN || prev == T_MLA || prev == T_MLA_COMB;
+        int r0 = -1;
+        if (MK_TAIL_PREFETCH >= 2 && after_att) r0 = t.rt0;
+        else if (t.rt1 - t.rt0 > m.RT / ncta) r0 = t.rt1 - 1;
+        if (r0 < 0) continue;
+        Task pf{};
+        pf.type = T_PREFETCH;
+        pf.layer = t.layer;
+        pf.phase = v[i - 1].phase;
+        pf.mat = t.mat;
+        pf.rt0 = r0;
+        pf.rt1 = t.rt1;
+        pf.wait_ctr = -1;
+        pf.sig_ctr = -1;
+        v.insert(v.begin() + (i - 1), pf);
+        ++i;  // skip over the task just handled
+      }
+    }
+  }
   for (int c = 0; c < ncta; ++c) {
     off[c] = (int32_t)flat.size();
     flat.insert(flat.end(), per[c].begin(), per[c].end());

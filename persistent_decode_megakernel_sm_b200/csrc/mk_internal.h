@@ -34,7 +34,14 @@ constexpr int NTS = MK_TSLOTS;               // TMEM slots
 constexpr int TSLOT_COLS = TILE_CAP / 512;   // TMEM columns per slot: 4 columns (16 B x 128 lanes) hold 4 tiles
 constexpr int TMEM_COLS = 512;               // the whole tensor memory of the SM (one CTA per SM)
 static_assert(NTS * TSLOT_COLS <= TMEM_COLS, "TMEM slots exceed the tensor memory");
-constexpr int STAGE_BYTES = (TILE_CAP + 1024 > 34816) ? TILE_CAP + 1024 : 34816;  // >= one attention chunk
+// Cache positions per GQA attention chunk: 64 or 128 (K and V of a head_dim
+// 128 chunk fill 32 or 64 KB of one stage).
+#ifndef MK_ATT_CT
+#define MK_ATT_CT 128
+#endif
+constexpr int ATT_CT = MK_ATT_CT;
+static_assert(ATT_CT == 64 || ATT_CT == 128, "attention chunks of 64 or 128 positions");
+constexpr int STAGE_BYTES = (TILE_CAP > 2 * ATT_CT * 128 * 2) ? TILE_CAP : 2 * ATT_CT * 128 * 2;
 constexpr int NSTAGE = MK_NSTAGE;            // weight ring depth
 constexpr int XSLOTS = 2;                    // activation ring depth
 constexpr int XSLOT_BYTES = 22528;           // one activation window: M rows x (cols + pad)
@@ -46,7 +53,6 @@ constexpr int SMEM_BYTES = NSTAGE * STAGE_BYTES + XSLOTS * XSLOT_BYTES + ATT_BYT
 constexpr int RMAX = 8;                      // row tiles per chunk
 constexpr int CPW = 8;                       // col tiles per warp per chunk
 constexpr int MAXM = 8;                      // activation rows per step (S * Q)
-constexpr int ATT_CT = 128;                  // cache positions per attention chunk (K and V fill one stage)
 static_assert(2 * ATT_CT * 128 * 2 <= STAGE_BYTES, "a K/V chunk of head_dim 128 fills at most one stage");
 constexpr int TRACE_FIELDS = 20;             // int64 per traced task
 constexpr int TILE_BF16 = 512;               // 16x16 bf16 tile in A-fragment order
@@ -103,7 +109,7 @@ enum TaskType : int16_t {
   T_ATTN = 2,      // one split-KV attention item (GQA)
   T_MOE_GU = 3,    // expert gate/up row tiles (shared: static; routed: union of the router's picks)
   T_MOE_DOWN = 4,  // down projection, K = shared + selected experts' hidden units
-  T_TOPK = 5,      // (unused placeholder)
+  T_PREFETCH = 5,  // weight producer only: bring row tiles [rt0, rt1) of matrix `m` into L2 ahead of their task
   T_EMBED = 6,     // x[m][c0:c1) = embedding rows of the step's tokens (+ RMS partial sums)
   T_MLA = 7,       // one split-KV latent-attention item (one query row, all heads)
   T_MLA_COMB = 8,  // this CTA's slice of the latent-attention split combine

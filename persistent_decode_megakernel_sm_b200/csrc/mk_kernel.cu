@@ -82,6 +82,10 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
       : "memory");
 }
+// Bring `bytes` (a multiple of 16) at `src` into L2, with no completion to wait for.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void prefetch_l1(const void* p) {
   asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
 }
@@ -300,6 +304,14 @@ struct Misc {
 
 static_assert(sizeof(Misc) <= MISC_BYTES, "Misc must fit its shared-memory region");
 
+// The GEMV's cross-warp reduction uses the first RED_BYTES of the attention
+// scratch; fp8 block-scale tables (two alternating, FP8_SCALE_TAB floats each)
+// follow it.
+constexpr int RED_BYTES = NCW * RMAX * 32 * 16;
+constexpr int FP8_SCALE_OFF = RED_BYTES;
+constexpr int FP8_SCALE_TAB = 512;  // floats: 2 halves x 2 row blocks x 128 column blocks
+static_assert(FP8_SCALE_OFF + 2 * FP8_SCALE_TAB * 4 <= ATT_BYTES, "fp8 scale tables fit the attention scratch");
+
 struct Ctx {
   const Launch* P;
   const Model* md;
@@ -346,7 +358,7 @@ struct ChunkIt {
       nr = min(nr, nb - g0);
     }
     KC = min(min(KT, TILE_CAP / (nr * tb)), min(NCW * CPW, xcap));
-    if (KC < KT && KC >= 4) KC &= ~3;  // chunk widths in whole 4-tile groups
+    if (NTS > 0 && KC < KT && KC >= 4) KC &= ~3;  // chunk widths in whole 4-tile groups (TMEM stage)
     WC = (xcap / KC) * KC;  // activation window: a whole number of chunks
     // a chunk moves to TMEM in 2 KB groups of 4 consecutive tiles; with a
     // width that is a multiple of 4, the tiles of col j (j = warp mod 8) sit
@@ -818,6 +830,14 @@ struct ChunkStream {
         kb = P.kv_k + head * d;
         vb = P.kv_v + head * d;
         state = 2;
+      } else if (t.type == T_PREFETCH) {
+        // the rows this CTA streams beyond the phase's even share: requested
+        // into L2 one phase early, so that the CTA with an extra row tile does
+        // not set the phase's end at the HBM rate
+        if ((threadIdx.x & 31) == 0) {
+          const size_t rowb = (size_t)t.m.KT * (t.m.fp8 ? TILE_FP8 : TILE_BF16);
+          bulk_prefetch_l2(t.m.w + (size_t)t.rt0 * rowb, (uint32_t)((t.rt1 - t.rt0) * rowb));
+        }
       } else if (MLA && t.type == T_MLA) {
         // cached positions [0, T0) of the query row's sequence, split like GQA
         const Item itm = decode_item(t.rt0, P.n_pairs, P.n_items);
@@ -1334,18 +1354,18 @@ struct GemvLane {
 // is cleared).  Gate / up interleaved tiles take the gate scale for rows
 // 0-7 and the up scale for rows 8-15 of each tile.
 template <int NR>
-__device__ __forceinline__ void fp8_apply_scales(const Mat& m, int g0, int cb, float (&raw)[NR][4],
-                                                 float (&acc)[NR][4]) {
+__device__ __forceinline__ void fp8_apply_scales(const Mat& m, const float* sct, int rb0, int nrb, int g0, int cb,
+                                                 float (&raw)[NR][4], float (&acc)[NR][4]) {
 #pragma unroll
   for (int r = 0; r < NR; ++r) {
     const int rt = g0 + r;
     float s_top, s_bot;
     if (m.gu) {
-      const int rb = rt >> 4;
-      s_top = __ldg(m.scales + rb * m.nbc + cb);
-      s_bot = __ldg(m.scales + (size_t)m.nbr * m.nbc + rb * m.nbc + cb);
+      const int rb = (rt >> 4) - rb0;
+      s_top = sct[rb * m.nbc + cb];
+      s_bot = sct[(nrb + rb) * m.nbc + cb];
     } else {
-      s_top = s_bot = __ldg(m.scales + (rt >> 3) * m.nbc + cb);
+      s_top = s_bot = sct[((rt >> 3) - rb0) * m.nbc + cb];
     }
     acc[r][0] += s_top * raw[r][0];
     acc[r][1] += s_top * raw[r][1];
@@ -1378,7 +1398,7 @@ __device__ __forceinline__ void fold_lo_cols(float (&c)[4], int M, int tq, int l
 // The GEMV row-group loop: one out-of-line instance per row count (small
 // instruction footprint) or inlined into the task body (no call frame).
 #ifndef MK_GEMV_INLINE
-#define MK_GEMV_INLINE 0
+#define MK_GEMV_INLINE 1
 #endif
 #if MK_GEMV_INLINE
 #define MK_GEMV_ATTR __forceinline__
@@ -1412,6 +1432,23 @@ __device__ MK_GEMV_ATTR void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
   Mat m = m0;
   if (FP8 && L.nseg > 1)
     m.scales = seg < L.NS ? L.sc_sh + (size_t)seg * L.ss_sh : L.sc_rt + (size_t)L.ex[seg - L.NS] * L.ss_rt;
+  // fp8: the block scales of the group's rows (every column block) staged in
+  // shared memory once per segment, two tables alternating by segment; read
+  // through L1 they miss for every chunk (the L1 beside a 227 KB carve-out
+  // holds little)
+  const float* sct = reinterpret_cast<const float*>(C.att + FP8_SCALE_OFF) + (seg & 1) * FP8_SCALE_TAB;
+  int rb0 = 0, nrb = 1;
+  if (FP8) {
+    rb0 = m.gu ? (ci0.g0 >> 4) : (ci0.g0 >> 3);
+    nrb = (m.gu ? ((ci0.g0 + NR - 1) >> 4) : ((ci0.g0 + NR - 1) >> 3)) - rb0 + 1;
+    const int per = nrb * m.nbc, n = (m.gu ? 2 : 1) * per;
+    float* dst = const_cast<float*>(sct);
+    for (int i = threadIdx.x; i < n; i += NCT) {
+      const int hf = i >= per ? 1 : 0;
+      dst[i] = __ldg(m.scales + (size_t)hf * m.nbr * m.nbc + (size_t)rb0 * m.nbc + (i - hf * per));
+    }
+    bar_consumers();
+  }
   while (true) {
     const uint8_t* slot = C.xring + (size_t)(ix % XSLOTS) * XSLOT_BYTES;
     if (ci.win_first()) {
@@ -1486,7 +1523,7 @@ __device__ MK_GEMV_ATTR void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
       for (int j = j0; j < j1; ++j) {
         const int cbj = (ci.c0 + j) >> 3;
         if (cbj != cb) {
-          fp8_apply_scales<NR>(m, ci.g0, cb, raw, acc);
+          fp8_apply_scales<NR>(m, sct, rb0, nrb, ci.g0, cb, raw, acc);
           cb = cbj;
         }
         const uint4 xf = xok ? lds128(xs + j * 64) : make_uint4(0u, 0u, 0u, 0u);
@@ -1501,7 +1538,7 @@ __device__ MK_GEMV_ATTR void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
           if (!pk) mma_f16(raw[r], af, xf.z, xf.w);
         }
       }
-      if (j0 < j1) fp8_apply_scales<NR>(m, ci.g0, cb, raw, acc);
+      if (j0 < j1) fp8_apply_scales<NR>(m, sct, rb0, nrb, ci.g0, cb, raw, acc);
     }
     if (L.trc) {
       float sink = 0.f;
@@ -2035,48 +2072,54 @@ __device__ void attn_item(const Ctx& C, const Task t, uint32_t& it) {
   const float2* rope = md.rope;
   const int half = d / 2;
 
-  // ---- stage Q (RoPE, scaled to log2 units) as bf16 hi/lo A fragments ----
+  // ---- stage Q (RoPE, scaled to log2 units) as bf16 hi/lo A fragments; the
+  //      last split also appends the step's own new positions (RoPE(k), bf16)
+  //      to the cache.  One pass over both, so all their loads overlap. ----
   uint8_t* qhi = C.att;
   uint8_t* qlo = qhi + mt * KTq * 512;
-  for (int e = tid; e < mt * 16 * half; e += NCT) {
-    const int r = e / half, i = e % half;
-    float x0 = 0.f, x1 = 0.f;
-    if (r < nr) {
-      const int qi = r / gh, hh = r % gh;
-      const int mrow = s * Q + qi;
-      const int pos = T0 + qi;
-      const float* q = qkv + (size_t)mrow * ldq + (size_t)(kvh * gh + hh) * d;
-      const float a0 = __ldcg(q + i), a1 = __ldcg(q + i + half);
-      const float2 cs = __ldg(rope + (size_t)pos * half + i);
-      x0 = (a0 * cs.x - a1 * cs.y) * qscale;
-      x1 = (a0 * cs.y + a1 * cs.x) * qscale;
-    }
-    __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
-    __nv_bfloat16 l0 = __float2bfloat16_rn(x0 - __bfloat162float(h0));
-    __nv_bfloat16 l1 = __float2bfloat16_rn(x1 - __bfloat162float(h1));
-    *reinterpret_cast<__nv_bfloat16*>(qhi + frag_off(r, i, KTq)) = h0;
-    *reinterpret_cast<__nv_bfloat16*>(qhi + frag_off(r, i + half, KTq)) = h1;
-    *reinterpret_cast<__nv_bfloat16*>(qlo + frag_off(r, i, KTq)) = l0;
-    *reinterpret_cast<__nv_bfloat16*>(qlo + frag_off(r, i + half, KTq)) = l1;
-  }
-  // ---- the step's own new positions: RoPE(k), bf16, append to the cache ----
   uint8_t* nk = C.newkv;
   uint8_t* nv = C.newkv + 16 * pitch;
-  if (last) {
-    const size_t head = (((size_t)t.layer * P.kv_seqs + s) * md.Hkv + kvh) * (size_t)P.kv_ctx;
-    for (int e = tid; e < 16 * half; e += NCT) {
-      const int qi = e / half, i = e % half;
+  const size_t head = (((size_t)t.layer * P.kv_seqs + s) * md.Hkv + kvh) * (size_t)P.kv_ctx;
+  const int nq = mt * 16 * half, nkv = last ? 16 * half : 0;
+  for (int e = tid; e < max(nq, nkv); e += NCT) {
+    const int r = e / half, i = e % half;  // r: query row (Q part), or step position (K/V part)
+    const bool dq = e < nq && r < nr, dk = e < nkv && r < Q;
+    float qa0 = 0.f, qa1 = 0.f, ka0 = 0.f, ka1 = 0.f, va0 = 0.f, va1 = 0.f;
+    float2 qcs = make_float2(1.f, 0.f), kcs = make_float2(1.f, 0.f);
+    if (dq) {
+      const int qi = r / gh, hh = r % gh;
+      const float* q = qkv + (size_t)(s * Q + qi) * ldq + (size_t)(kvh * gh + hh) * d;
+      qa0 = __ldcg(q + i);
+      qa1 = __ldcg(q + i + half);
+      qcs = __ldg(rope + (size_t)(T0 + qi) * half + i);
+    }
+    if (dk) {
+      const float* kr = qkv + (size_t)(s * Q + r) * ldq + (size_t)(md.Hq + kvh) * d;
+      const float* vr = qkv + (size_t)(s * Q + r) * ldq + (size_t)(md.Hq + md.Hkv + kvh) * d;
+      ka0 = __ldcg(kr + i);
+      ka1 = __ldcg(kr + i + half);
+      va0 = __ldcg(vr + i);
+      va1 = __ldcg(vr + i + half);
+      kcs = __ldg(rope + (size_t)(T0 + r) * half + i);
+    }
+    if (e < nq) {
+      const float x0 = dq ? (qa0 * qcs.x - qa1 * qcs.y) * qscale : 0.f;
+      const float x1 = dq ? (qa0 * qcs.y + qa1 * qcs.x) * qscale : 0.f;
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
+      *reinterpret_cast<__nv_bfloat16*>(qhi + frag_off(r, i, KTq)) = h0;
+      *reinterpret_cast<__nv_bfloat16*>(qhi + frag_off(r, i + half, KTq)) = h1;
+      *reinterpret_cast<__nv_bfloat16*>(qlo + frag_off(r, i, KTq)) = __float2bfloat16_rn(x0 - __bfloat162float(h0));
+      *reinterpret_cast<__nv_bfloat16*>(qlo + frag_off(r, i + half, KTq)) =
+          __float2bfloat16_rn(x1 - __bfloat162float(h1));
+    }
+    if (e < nkv) {
       __nv_bfloat16 k0 = __float2bfloat16_rn(0.f), k1 = k0, v0 = k0, v1 = k0;
-      if (qi < Q) {
-        const int mrow = s * Q + qi, pos = T0 + qi;
-        const float* kr = qkv + (size_t)mrow * ldq + (size_t)(md.Hq + kvh) * d;
-        const float* vr = qkv + (size_t)mrow * ldq + (size_t)(md.Hq + md.Hkv + kvh) * d;
-        const float a0 = __ldcg(kr + i), a1 = __ldcg(kr + i + half);
-        const float2 cs = __ldg(rope + (size_t)pos * half + i);
-        k0 = __float2bfloat16_rn(a0 * cs.x - a1 * cs.y);
-        k1 = __float2bfloat16_rn(a0 * cs.y + a1 * cs.x);
-        v0 = __float2bfloat16_rn(__ldcg(vr + i));
-        v1 = __float2bfloat16_rn(__ldcg(vr + i + half));
+      if (dk) {
+        const int pos = T0 + r;
+        k0 = __float2bfloat16_rn(ka0 * kcs.x - ka1 * kcs.y);
+        k1 = __float2bfloat16_rn(ka0 * kcs.y + ka1 * kcs.x);
+        v0 = __float2bfloat16_rn(va0);
+        v1 = __float2bfloat16_rn(va1);
         __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(P.kv_k) + (head + pos) * d;
         __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(P.kv_v) + (head + pos) * d;
         kc[kv_swz(pos, i)] = k0;
@@ -2084,11 +2127,11 @@ __device__ void attn_item(const Ctx& C, const Task t, uint32_t& it) {
         vc[kv_swz(pos, i)] = v0;
         vc[kv_swz(pos, i + half)] = v1;
       }
-      // shared-memory row qi: permuted by qi (the reader's key for these rows)
-      *reinterpret_cast<__nv_bfloat16*>(nk + qi * pitch + kv_swz(qi, i) * 2) = k0;
-      *reinterpret_cast<__nv_bfloat16*>(nk + qi * pitch + kv_swz(qi, i + half) * 2) = k1;
-      *reinterpret_cast<__nv_bfloat16*>(nv + qi * pitch + kv_swz(qi, i) * 2) = v0;
-      *reinterpret_cast<__nv_bfloat16*>(nv + qi * pitch + kv_swz(qi, i + half) * 2) = v1;
+      // shared-memory row r: permuted by r (the reader's key for these rows)
+      *reinterpret_cast<__nv_bfloat16*>(nk + r * pitch + kv_swz(r, i) * 2) = k0;
+      *reinterpret_cast<__nv_bfloat16*>(nk + r * pitch + kv_swz(r, i + half) * 2) = k1;
+      *reinterpret_cast<__nv_bfloat16*>(nv + r * pitch + kv_swz(r, i) * 2) = v0;
+      *reinterpret_cast<__nv_bfloat16*>(nv + r * pitch + kv_swz(r, i + half) * 2) = v1;
     }
   }
   bar_consumers();
@@ -2112,11 +2155,11 @@ __device__ void attn_item(const Ctx& C, const Task t, uint32_t& it) {
     const int n = min(ATT_CT, b - t0);
     wait_full(C, it);
     const uint8_t* stage = C.ring + (size_t)(it % NSTAGE) * STAGE_BYTES;
-    // a warp takes its 16 positions of each 64-position half of the chunk
-    warp_att_chunk<MT, NTD>(st, qhi, qlo, stage, stage + (size_t)ATT_CT * pitch, pitch, KTq, n, false, gh, p0, dim0,
-                            t0);
-    warp_att_chunk<MT, NTD>(st, qhi, qlo, stage, stage + (size_t)ATT_CT * pitch, pitch, KTq, n, false, gh, p0 + 64,
-                            dim0, t0);
+    // a warp takes its 16 positions of each 64-position part of the chunk
+#pragma unroll
+    for (int h64 = 0; h64 < ATT_CT / 64; ++h64)
+      warp_att_chunk<MT, NTD>(st, qhi, qlo, stage, stage + (size_t)ATT_CT * pitch, pitch, KTq, n, false, gh,
+                              p0 + 64 * h64, dim0, t0);
     release_stage(C, it);  // per warp: the ring's empty barrier counts the consumer warps
     ++it;
   }

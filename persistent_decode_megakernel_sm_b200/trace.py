@@ -15,7 +15,7 @@ import sys
 
 import numpy as np
 
-TYPE_NAMES = {1: "gemv", 2: "attn", 3: "moe_gu", 4: "moe_down", 6: "embed", 7: "mla", 8: "mla_comb"}
+TYPE_NAMES = {1: "gemv", 2: "attn", 3: "moe_gu", 4: "moe_down", 5: "prefetch", 6: "embed", 7: "mla", 8: "mla_comb"}
 FIELDS = 20
 EPI_NAMES = {0: "store", 1: "resid", 2: "swiglu", 3: "logits", 4: "swiglu_moe"}
 
