@@ -104,52 +104,6 @@ def measured_peaks():
 
 
 # ---------------------------------------------------------------------------
-# algorithmic bytes of one decode step (what the method must move)
-# ---------------------------------------------------------------------------
-def _mat_bytes(rows, cols, fp8=False):
-    if not fp8:
-        return rows * cols * 2
-    return rows * cols + (-(-rows // 128)) * (-(-cols // 128)) * 4
-
-
-def expert_bytes(mc):
-    f8 = bool(mc.expert_fp8)
-    return 2 * _mat_bytes(mc.expert_ffn, mc.hidden, f8) + _mat_bytes(mc.hidden, mc.expert_ffn, f8)
-
-
-def step_bytes(mc, pos0, Q=1, unions=None, write_logits=True):
-    """Algorithmic bytes of one step: every weight the step needs (for MoE
-    layers the router, the shared experts and only the union of the routed
-    experts picked by the step's rows, `unions[l]`), B embedding rows, the
-    cached KV / latent rows attended (positions 0..p-1 of each sequence, read
-    once even in verify), the rows written and the logits written.
-    pos0: first position of each sequence; Q positions per sequence."""
-    H, L, V = mc.hidden, mc.layers, mc.vocab
-    Hq, d = mc.n_q_heads, mc.head_dim
-    M = len(pos0) * Q
-    total = _mat_bytes(V, H) + H * 2 + M * H * 2          # LM head, final norm, embedding rows
-    for l in range(L):
-        total += 2 * H * 2                                 # norm gains
-        if mc.mla:
-            R, dr = mc.kv_lora_rank, mc.rope_dim
-            total += (_mat_bytes(Hq * (d + dr) + R + dr, H) + _mat_bytes(Hq * R, d) + _mat_bytes(Hq * d, R)
-                      + _mat_bytes(H, Hq * d))
-        else:
-            total += _mat_bytes((Hq + 2 * mc.n_kv_heads) * d, H) + _mat_bytes(H, Hq * d)
-        if mc.n_routed == 0:
-            total += _mat_bytes(2 * mc.ffn, H) + _mat_bytes(H, mc.ffn)
-        else:
-            u = unions[l] if unions is not None else min(mc.n_routed, M * mc.top_k)
-            total += _mat_bytes(mc.n_routed, H) + (mc.n_shared + u) * expert_bytes(mc)
-    kvt = (mc.kv_lora_rank + mc.rope_dim) * 2 if mc.mla else 2 * mc.n_kv_heads * d * 2
-    total += sum(int(p) for p in pos0) * kvt * L           # cached rows read
-    total += M * kvt * L                                   # new rows written
-    if write_logits:
-        total += M * V * 4
-    return total
-
-
-# ---------------------------------------------------------------------------
 # clocks sampled during the timed region
 # ---------------------------------------------------------------------------
 class Clocks:
@@ -194,6 +148,7 @@ def run_ours(args, rank, world, local_rank):
     import torch
     import synth
     from persistent_decode_megakernel_sm_b200 import Megakernel
+    from persistent_decode_megakernel_sm_b200.traffic import router_unions, step_bytes
 
     torch.cuda.set_device(local_rank)
     dev = f"cuda:{local_rank}"
@@ -232,10 +187,6 @@ def run_ours(args, rank, world, local_rank):
             kv.copy_in(snap)
 
         return mc, model, kv, restore
-
-    def router_unions(mc, idx):
-        a = idx.cpu().numpy()
-        return [len(set(a[l].reshape(-1).tolist())) for l in range(mc.layers)]
 
     def decode_run(mc, model, kv, restore, B, steps, warmup, clocks=False):
         """Greedy decode of B sequences from the synthetic context: `warmup`

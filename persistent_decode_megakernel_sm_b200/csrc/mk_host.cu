@@ -1223,7 +1223,7 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
   next_phase();  // tags the last phase's tasks
   n_phases_out = phase;
 #ifndef MK_TAIL_PREFETCH
-#define MK_TAIL_PREFETCH 0
+#define MK_TAIL_PREFETCH 1
 #endif
   // L2 requests one task ahead, issued by the weight producer when it starts
   // the CTA's previous task:

@@ -7,9 +7,9 @@ smaller vocabulary) for an external profiler: seeded weights and context,
 A cut keeps every per-layer shape of the workload, so the kernel's per-layer
 behaviour (tiles, chunks, attention splits) is the full model's; only the
 number of layers and the LM head / embedding rows shrink.  Prints the bytes
-the step must move (weights, cache rows, logits) for the cut.  For MoE models
-the weight figure counts every resident expert, an upper bound: a step reads
-only the shared experts and the routed experts its rows pick."""
+the last step must move (weights, cache rows, logits) for the cut, counted
+as the benchmark counts them: for MoE models the routed experts are those the
+last step's rows picked (a router trace of that step)."""
 from __future__ import annotations
 
 import argparse
@@ -33,6 +33,7 @@ def main():
     import torch
     import synth
     from persistent_decode_megakernel_sm_b200 import Megakernel
+    from persistent_decode_megakernel_sm_b200.traffic import router_unions, step_bytes
 
     mc = synth.preset(a.config)
     if a.layers:
@@ -49,25 +50,36 @@ def main():
     lg = torch.empty((B, mc.vocab), dtype=torch.float32, device=dev)
     am = torch.empty(B, dtype=torch.int32, device=dev)
     acc = torch.empty(1, dtype=torch.int32, device=dev)
-    for i in range(a.warmup + a.steps):
+    n = a.warmup + a.steps
+    k = max(mc.top_k, 1)
+    idx = torch.full((mc.layers, B, k), -1, dtype=torch.int32, device=dev)
+    wts = torch.zeros((mc.layers, B, k), dtype=torch.float32, device=dev)
+    pos0 = None
+    for i in range(n):
+        last = i == n - 1
+        if last and mc.n_routed:
+            m.set_router_trace(idx, wts)
         if a.verify:
             props = synth.proposals(synth.SEED_PROPOSALS, i, 7, mc.vocab)
             toks8 = torch.tensor([int(tok[0].item())] + [int(x) for x in props], dtype=torch.int32, device=dev)
             m.verify(toks8, mc.context, kv, lg, am, acc)
+            pos0 = [mc.context]
         else:
             pos = torch.full((B,), mc.context + i, dtype=torch.int32, device=dev)
             m.decode_step(tok, pos, kv, lg, am)
             tok = am.clone()
+            pos0 = [mc.context + i] * B
+        if last and mc.n_routed:
+            m.set_router_trace(None, None)
     torch.cuda.synchronize()
     assert m.sync_status() == 0
-    weights = m.weight_bytes() - mc.vocab * mc.hidden * 2 + B * mc.hidden * 2
-    kvt = (mc.kv_lora_rank + mc.rope_dim) * 2 if mc.mla else 2 * mc.n_kv_heads * mc.head_dim * 2
-    cache = (mc.context * kvt * mc.layers + 8 * kvt * mc.layers if a.verify
-             else B * (mc.context + a.warmup) * kvt * mc.layers + B * kvt * mc.layers)
-    key = "weight_bytes_resident_upper_bound" if mc.n_routed else "weight_bytes_streamed"
-    print(json.dumps({"config": a.config, "layers": mc.layers, "vocab": mc.vocab, "batch": B,
-                      key: weights, "cache_bytes": cache, "logit_bytes": B * mc.vocab * 4,
-                      "bytes_per_step_first_profiled": weights + cache + B * mc.vocab * 4}))
+    Q = 8 if a.verify else 1
+    unions = router_unions(mc, idx) if mc.n_routed else None
+    out = {"config": a.config, "layers": mc.layers, "vocab": mc.vocab, "batch": B,
+           "launches": n, "algorithmic_bytes_last_step": step_bytes(mc, pos0, Q, unions, write_logits=True)}
+    if unions:
+        out["routed_experts_per_layer_last_step"] = unions
+    print(json.dumps(out))
     kv.close()
     m.close()
 

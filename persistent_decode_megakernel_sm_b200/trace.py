@@ -33,7 +33,7 @@ def record(model, kv, tokens, positions, logits, argmax, cap: int = 512):
 
 def summarize(tr: np.ndarray, sm_clock_mhz: float = 0.0) -> dict:
     """tr: [ctas][cap][20] = t_begin, t_dep, t_end (ns), wait_full, wait_x (cycles),
-    chunks, layer, type*16+epi, then cycles in fragment prep, mma, epilogue,
+    chunks, layer (+ phase << 16), type*16+epi, then cycles in fragment prep, mma, epilogue,
     release, [12..15] producer statistics (record 0: cycles blocked on a full
     ring, chunks issued, first and last issue time; record 1: producer cycles
     and ns, giving the SM clock), then cycles in the chunk loop, before it,
@@ -50,6 +50,9 @@ def summarize(tr: np.ndarray, sm_clock_mhz: float = 0.0) -> dict:
                                                   frag_us=0.0, mma_us=0.0, epi_us=0.0, rel_us=0.0,
                                                   loop_us=0.0, pre_us=0.0, post_us=0.0, sig_us=0.0))
     busy = 0.0
+    # wall span of each phase (the tasks between two dependency points):
+    # first dependency met to last task end
+    span = collections.defaultdict(lambda: [None, None])
     for c in range(tr.shape[0]):
         for k in range(tr.shape[1]):
             if not valid[c, k]:
@@ -59,6 +62,11 @@ def summarize(tr: np.ndarray, sm_clock_mhz: float = 0.0) -> dict:
             lo, pr, po, sg = tr[c, k, 16:20]
             name = TYPE_NAMES.get(int(te16) // 16, "?") + ("/" + EPI_NAMES[int(te16) % 16] if int(te16) // 16 in (1, 3) else "")
             p = phases[name]
+            phase = int(layer) >> 16
+            layer = int(layer) & 0xFFFF
+            sp = span[(phase, name)]
+            sp[0] = int(td) if sp[0] is None else min(sp[0], int(td))
+            sp[1] = int(te) if sp[1] is None else max(sp[1], int(te))
             p["n"] += 1
             p["dep_us"] += (td - tb) / 1e3
             p["run_us"] += (te - td) / 1e3
@@ -80,6 +88,10 @@ def summarize(tr: np.ndarray, sm_clock_mhz: float = 0.0) -> dict:
     for name, p in sorted(phases.items()):
         out["phases"][name] = {k: (v / ctas if k.endswith("_us") else v) for k, v in p.items()}
         out["phases"][name]["per_cta_us_note"] = "times summed over the CTA's tasks, averaged over CTAs"
+        # wall time: per phase, the first CTA's dependency met to the last
+        # CTA's end, summed over the step's phases of this kind (a prefetch
+        # task belongs to the phase before the task it serves)
+        out["phases"][name]["wall_us"] = sum((e - b) / 1e3 for (ph, nm), (b, e) in span.items() if nm == name)
     out["compute_fraction"] = busy / ctas / step_us
     # SM idle between tasks: the part of the step a CTA spends outside task
     # bodies (waiting for a task's dependency, or done before the step ends)

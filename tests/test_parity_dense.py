@@ -352,6 +352,11 @@ def test_task_trace_same_results_and_records(tiny):
     assert valid[:, 0].all()  # every CTA ran at least its first task
     tb, td, te = tr[:, :, 0][valid], tr[:, :, 1][valid], tr[:, :, 2][valid]
     assert (tb <= td).all() and (td <= te).all()
+    for c in range(tr.shape[0]):  # each CTA runs its tasks in phase order
+        ph = tr[c, :, 6][valid[c]] >> 16
+        assert (np.diff(ph) >= 0).all(), c
     s = trace.summarize(tr)
     assert s["step_us"] > 0 and 0.0 < s["compute_fraction"] <= 1.0
+    walls = [p["wall_us"] for p in s["phases"].values()]
+    assert min(walls) >= 0 and sum(walls) > 0
     kv.close()
