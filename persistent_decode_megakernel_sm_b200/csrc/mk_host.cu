@@ -20,8 +20,8 @@
 
 namespace mk {
 // the kernel instance of a model family, without and with tracing compiled in
-namespace plain { const void* step_kernel_for(bool mla, bool moe); }
-namespace traced { const void* step_kernel_for(bool mla, bool moe); }
+namespace plain { const void* step_kernel_for(bool mla, bool moe, bool fp8); }
+namespace traced { const void* step_kernel_for(bool mla, bool moe, bool fp8); }
 }
 
 using namespace mk;
@@ -642,8 +642,8 @@ mk_status mk_create(const mk_model_desc* desc, int device, mk_handle** out) {
       s = MK_ERR_CUDA;
       goto fail_out;
     }
-    h->kernel = plain::step_kernel_for(d.kv_lora_rank > 0, d.n_routed > 0);
-    h->kernel_traced = traced::step_kernel_for(d.kv_lora_rank > 0, d.n_routed > 0);
+    h->kernel = plain::step_kernel_for(d.kv_lora_rank > 0, d.n_routed > 0, d.n_routed > 0 && d.expert_fp8 != 0);
+    h->kernel_traced = traced::step_kernel_for(d.kv_lora_rank > 0, d.n_routed > 0, d.n_routed > 0 && d.expert_fp8 != 0);
     if (cudaFuncSetAttribute(h->kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(h->kernel_traced, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess) {
       s = MK_ERR_CUDA;
@@ -975,6 +975,26 @@ static std::vector<std::pair<int, int>> split_rows(int RT, int ncta, int& rot) {
   return r;
 }
 
+// As split_rows, over the CTAs whose `busy` entry is false only (the others
+// get empty ranges); all CTAs when every one is busy.
+static std::vector<std::pair<int, int>> split_rows_free(int RT, int ncta, int& rot, const std::vector<bool>& busy) {
+  std::vector<int> freec;
+  for (int c = 0; c < ncta; ++c)
+    if (!busy[c]) freec.push_back(c);
+  if (freec.empty()) return split_rows(RT, ncta, rot);
+  const int n = (int)freec.size();
+  std::vector<std::pair<int, int>> r(ncta, {0, 0});
+  const int base = RT / n, rem = RT % n;
+  int cur = 0;
+  for (int i = 0; i < n; ++i) {
+    const int extra = (((i - rot) % n + n) % n) < rem ? 1 : 0;
+    r[freec[i]] = {cur, cur + base + extra};
+    cur += base + extra;
+  }
+  rot = (rot + rem) % n;
+  return r;
+}
+
 static Task gemv(int layer, int mat, int rt0, int rt1, int in_kind, int in_buf, int epi, int out_buf, int gain,
                  int wait_ctr, int wait_tgt, int sig) {
   Task t{};
@@ -1160,8 +1180,13 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
       // -> down projection over all of them.  The shared expert's weights are
       // streamed while the router's choice is being made; only the routed
       // experts' (and the down) tiles wait for it.
+      // The few CTAs that compute the router's rows get no shared-expert rows:
+      // they start on the routed experts as soon as the route is known
+      // instead of after a shared-expert task as well.
+      std::vector<bool> routing(ncta, false);
       {
         auto rr = split_rows(h->mats[ly.m_router].m.RT, ncta, rot);
+        for (int c = 0; c < ncta; ++c) routing[c] = rr[c].second > rr[c].first;
         next_phase();
         for (int c = 0; c < ncta; ++c) {
           Task t = gemv(l, ly.m_router, rr[c].first, rr[c].second, IN_X_NORM, 0, EPI_STORE, B_RLOG, 1, C(l, C_O),
@@ -1172,7 +1197,7 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
       }
       if (d.n_shared > 0) {
         const MatHost& sh = h->mats[ly.m_shgu];
-        auto rr = split_rows(sh.m.RT * sh.m.ne, ncta, rot);
+        auto rr = split_rows_free(sh.m.RT * sh.m.ne, ncta, rot, routing);
         next_phase();
         for (int c = 0; c < ncta; ++c) {
           Task t = gemv(l, ly.m_shgu, rr[c].first, rr[c].second, IN_X_NORM, 0, EPI_SWIGLU_MOE, B_H, 1, C(l, C_O),

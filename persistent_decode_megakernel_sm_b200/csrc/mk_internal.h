@@ -50,7 +50,11 @@ constexpr int ATT_BYTES = 40960;             // GEMV reduction / attention scrat
 constexpr int NEWKV_BYTES = 8704;            // K/V rows of the step's own new positions
 constexpr int MISC_BYTES = 4096;
 constexpr int SMEM_BYTES = NSTAGE * STAGE_BYTES + XSLOTS * XSLOT_BYTES + ATT_BYTES + NEWKV_BYTES + MISC_BYTES;
-constexpr int RMAX = 8;                      // row tiles per chunk
+#ifndef MK_RMAX
+#define MK_RMAX 8
+#endif
+constexpr int RMAX = MK_RMAX;                // row tiles per chunk (4 or 8)
+static_assert(RMAX == 4 || RMAX == 8, "row tiles per chunk: 4 or 8");
 constexpr int CPW = 8;                       // col tiles per warp per chunk
 constexpr int MAXM = 8;                      // activation rows per step (S * Q)
 static_assert(2 * ATT_CT * 128 * 2 <= STAGE_BYTES, "a K/V chunk of head_dim 128 fills at most one stage");

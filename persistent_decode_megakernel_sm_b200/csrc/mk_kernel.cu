@@ -586,7 +586,7 @@ struct PieceSrc {
   int xcol0;  // first activation column (per-head groups of the latent-attention projections)
 };
 
-template <bool MOE>
+template <int MOE>
 __device__ __forceinline__ PieceSrc piece_src(const Model& md, const Task& t, const Mat& m, const Mat& m2,
                                               const int16_t* ex, const Pieces& pc) {
   PieceSrc r;
@@ -616,7 +616,7 @@ __device__ __forceinline__ PieceSrc piece_src(const Model& md, const Task& t, co
 }
 
 // Row range, expert-group size and K-segment count of a GEMV-like task.
-template <bool MOE>
+template <int MOE>
 __device__ __forceinline__ void task_rows(const Model& md, const Task& t, const Mat& m, int U, int& rt0, int& rt1,
                                           int& gsz, int& nseg) {
   rt0 = t.rt0;
@@ -635,11 +635,11 @@ __device__ __forceinline__ void task_rows(const Model& md, const Task& t, const 
   }
 }
 
-template <bool MOE>
+template <int MOE>
 __device__ __forceinline__ bool task_needs_route(const Task& t) {
   return MOE && ((t.type == T_MOE_GU && t.moe == 2) || t.type == T_MOE_DOWN);
 }
-template <bool MOE>
+template <int MOE>
 __device__ __forceinline__ bool gemv_like(const Task& t) {
   return t.type == T_GEMV || (MOE && (t.type == T_MOE_GU || t.type == T_MOE_DOWN));
 }
@@ -733,7 +733,7 @@ struct Chunk {
 // Walks a CTA's task list and yields its chunks in consumption order (the
 // enumeration the consumers use).  Routed-expert tasks first wait for the
 // router's counter: their tiles are the only ones that depend on activations.
-template <bool MLA, bool MOE>
+template <bool MLA, int MOE>
 struct ChunkStream {
   int ti, end, state;  // state 0: next task, 1: GEMV-like pieces, 2: attention, 3: latent attention
   Task t;
@@ -853,7 +853,7 @@ struct ChunkStream {
   }
 };
 
-template <bool MLA, bool MOE>
+template <bool MLA, int MOE>
 __device__ void producer(const Ctx& C) {
   const Launch& P = *C.P;
   const int lane = threadIdx.x & 31;
@@ -1079,7 +1079,7 @@ __device__ bool xprod_reserve(const Ctx& C, uint32_t ix, uint32_t bytes) {
   return ok != 0;
 }
 
-template <bool MOE>
+template <int MOE>
 __device__ void xproducer(const Ctx& C) {
   const Launch& P = *C.P;
   const Model& md = *C.md;
@@ -1355,9 +1355,10 @@ struct GemvLane {
 // 0-7 and the up scale for rows 8-15 of each tile.
 template <int NR>
 __device__ __forceinline__ void fp8_apply_scales(const Mat& m, const float* sct, int rb0, int nrb, int g0, int cb,
-                                                 float (&raw)[NR][4], float (&acc)[NR][4]) {
+                                                 float (&raw)[NR][4], float (&acc)[NR][4], int nrr) {
 #pragma unroll
   for (int r = 0; r < NR; ++r) {
+    if (r >= nrr) continue;
     const int rt = g0 + r;
     float s_top, s_bot;
     if (m.gu) {
@@ -1400,6 +1401,18 @@ __device__ __forceinline__ void fold_lo_cols(float (&c)[4], int M, int tq, int l
 #ifndef MK_GEMV_INLINE
 #define MK_GEMV_INLINE 1
 #endif
+#ifndef MK_FP8_UNROLL
+#define MK_FP8_UNROLL 1
+#endif
+// Row-group instances compiled (8: one per row count 1..RMAX; 4: 1, 2, 4 and
+// RMAX; 1: RMAX only), bf16 and fp8 weights: fewer instances, less code.
+#ifndef MK_GEMV_SET
+#define MK_GEMV_SET 8
+#endif
+#ifndef MK_FP8_SET
+#define MK_FP8_SET 8
+#endif
+constexpr int FP8_UNROLL = MK_FP8_UNROLL;
 #if MK_GEMV_INLINE
 #define MK_GEMV_ATTR __forceinline__
 #else
@@ -1414,6 +1427,10 @@ __device__ MK_GEMV_ATTR void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
   const GemvLane L = Lr;
   ChunkIt ci = cir;
   uint32_t it = itr, ix = ixr, tc = tcr;
+  // row tiles of this group: NR, or fewer when one instance serves several
+  // row counts (rows nrr..NR-1 then load and multiply nothing)
+  constexpr bool exact = NR == 1 || (FP8 ? MK_FP8_SET == 8 : MK_GEMV_SET == 8);
+  const int nrr = exact ? NR : ci.nr;
   float acc[NR][4];
 #pragma unroll
   for (int r = 0; r < NR; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
@@ -1440,7 +1457,7 @@ __device__ MK_GEMV_ATTR void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
   int rb0 = 0, nrb = 1;
   if (FP8) {
     rb0 = m.gu ? (ci0.g0 >> 4) : (ci0.g0 >> 3);
-    nrb = (m.gu ? ((ci0.g0 + NR - 1) >> 4) : ((ci0.g0 + NR - 1) >> 3)) - rb0 + 1;
+    nrb = (m.gu ? ((ci0.g0 + nrr - 1) >> 4) : ((ci0.g0 + nrr - 1) >> 3)) - rb0 + 1;
     const int per = nrb * m.nbc, n = (m.gu ? 2 : 1) * per;
     float* dst = const_cast<float*>(sct);
     for (int i = threadIdx.x; i < n; i += NCT) {
@@ -1485,13 +1502,16 @@ __device__ MK_GEMV_ATTR void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
         const uint32_t b0 = lo_col ? xf.z : xf.x, b1 = lo_col ? xf.w : xf.y;
         uint4 a[NR];
 #pragma unroll
-        for (int r = 0; r < NR; ++r) a[r] = tmem_ld16(tbase + 4 * (uint32_t)((r * nc + j) >> 2));
+        for (int r = 0; r < NR; ++r)
+          if (r < nrr) a[r] = tmem_ld16(tbase + 4 * (uint32_t)((r * nc + j) >> 2));
         tmem_ld_wait();
 #pragma unroll
-        for (int r = 0; r < NR; ++r) mma_bf16(acc[r], a[r], b0, b1);
+        for (int r = 0; r < NR; ++r)
+          if (r < nrr) mma_bf16(acc[r], a[r], b0, b1);
         if (!pk) {
 #pragma unroll
-          for (int r = 0; r < NR; ++r) mma_bf16(acc[r], a[r], xf.z, xf.w);
+          for (int r = 0; r < NR; ++r)
+            if (r < nrr) mma_bf16(acc[r], a[r], xf.z, xf.w);
         }
       }
     } else if (!FP8) {
@@ -1501,12 +1521,15 @@ __device__ MK_GEMV_ATTR void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
         const uint32_t b0 = lo_col ? xf.z : xf.x, b1 = lo_col ? xf.w : xf.y;
         uint4 a[NR];
 #pragma unroll
-        for (int r = 0; r < NR; ++r) a[r] = lds128(stage + ((size_t)r * nc + j) * TILE_BF16 + lane * 16);
+        for (int r = 0; r < NR; ++r)
+          if (r < nrr) a[r] = lds128(stage + ((size_t)r * nc + j) * TILE_BF16 + lane * 16);
 #pragma unroll
-        for (int r = 0; r < NR; ++r) mma_bf16(acc[r], a[r], b0, b1);
+        for (int r = 0; r < NR; ++r)
+          if (r < nrr) mma_bf16(acc[r], a[r], b0, b1);
         if (!pk) {
 #pragma unroll
-          for (int r = 0; r < NR; ++r) mma_bf16(acc[r], a[r], xf.z, xf.w);
+          for (int r = 0; r < NR; ++r)
+            if (r < nrr) mma_bf16(acc[r], a[r], xf.z, xf.w);
         }
       }
     } else {
@@ -1519,26 +1542,29 @@ __device__ MK_GEMV_ATTR void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
 #pragma unroll
       for (int r = 0; r < NR; ++r) raw[r][0] = raw[r][1] = raw[r][2] = raw[r][3] = 0.f;
       int cb = (ci.c0 + j0) >> 3;
-#pragma unroll 1
+#pragma unroll FP8_UNROLL
       for (int j = j0; j < j1; ++j) {
         const int cbj = (ci.c0 + j) >> 3;
         if (cbj != cb) {
-          fp8_apply_scales<NR>(m, sct, rb0, nrb, ci.g0, cb, raw, acc);
+          fp8_apply_scales<NR>(m, sct, rb0, nrb, ci.g0, cb, raw, acc, nrr);
           cb = cbj;
         }
         const uint4 xf = xok ? lds128(xs + j * 64) : make_uint4(0u, 0u, 0u, 0u);
         const uint32_t b0 = lo_col ? xf.z : xf.x, b1 = lo_col ? xf.w : xf.y;
         uint2 a8[NR];
 #pragma unroll
-        for (int r = 0; r < NR; ++r) a8[r] = lds64(stage + ((size_t)r * nc + j) * TILE_FP8 + lane * 8);
+        for (int r = 0; r < NR; ++r)
+          if (r < nrr) a8[r] = lds64(stage + ((size_t)r * nc + j) * TILE_FP8 + lane * 8);
 #pragma unroll
         for (int r = 0; r < NR; ++r) {
-          const uint4 af = fp8_frag_to_f16(a8[r]);
-          mma_f16(raw[r], af, b0, b1);
-          if (!pk) mma_f16(raw[r], af, xf.z, xf.w);
+          if (r < nrr) {
+            const uint4 af = fp8_frag_to_f16(a8[r]);
+            mma_f16(raw[r], af, b0, b1);
+            if (!pk) mma_f16(raw[r], af, xf.z, xf.w);
+          }
         }
       }
-      if (j0 < j1) fp8_apply_scales<NR>(m, sct, rb0, nrb, ci.g0, cb, raw, acc);
+      if (j0 < j1) fp8_apply_scales<NR>(m, sct, rb0, nrb, ci.g0, cb, raw, acc, nrr);
     }
     if (L.trc) {
       float sink = 0.f;
@@ -1587,7 +1613,23 @@ __device__ MK_GEMV_ATTR void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
   tcr = tc;
 }
 
-template <bool MOE>
+// fp8 row groups: the same loop, in its own function (MK_FP8_GEMV_NOINLINE)
+// or inlined like the bf16 ones.
+#ifndef MK_FP8_GEMV_NOINLINE
+#define MK_FP8_GEMV_NOINLINE 0
+#endif
+#if MK_FP8_GEMV_NOINLINE
+#define MK_FP8_GEMV_ATTR __noinline__
+#else
+#define MK_FP8_GEMV_ATTR __forceinline__
+#endif
+template <int NR>
+__device__ MK_FP8_GEMV_ATTR void gemv_group_fp8(const Ctx& C, ChunkIt& ci, const Mat& m, const GemvLane& L, uint32_t& it,
+                                                uint32_t& ix, uint32_t& tc, float* red, bool accum) {
+  gemv_group<NR, true>(C, ci, m, L, it, ix, tc, red, accum);
+}
+
+template <int MOE>
 __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix, uint32_t& tc) {
   const Launch& P = *C.P;
   const long long tpre = (MK_TRACE && P.trace && threadIdx.x == 0) ? clock64() : 0;
@@ -1668,28 +1710,53 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
       L.ss_rt = m.sstride;
     }
     // one instance per row-tile count: every loop over rows is static (fp8
-    // weights exist only for experts, so only MoE kernels reach the fp8 ones)
-    if (!MOE || !m.fp8) {
+    // weights exist only for experts, so only the fp8-expert MoE kernels
+    // (MOE == 2) hold the fp8 ones)
+    if (MOE != 2 || !m.fp8) {
       switch (ci.nr) {
+#if MK_GEMV_SET == 8
         case 1: gemv_group<1, false>(C, ci, mg, L, it, ix, tc, red, accum); break;
         case 2: gemv_group<2, false>(C, ci, mg, L, it, ix, tc, red, accum); break;
         case 3: gemv_group<3, false>(C, ci, mg, L, it, ix, tc, red, accum); break;
+#if MK_RMAX > 4
         case 4: gemv_group<4, false>(C, ci, mg, L, it, ix, tc, red, accum); break;
         case 5: gemv_group<5, false>(C, ci, mg, L, it, ix, tc, red, accum); break;
         case 6: gemv_group<6, false>(C, ci, mg, L, it, ix, tc, red, accum); break;
         case 7: gemv_group<7, false>(C, ci, mg, L, it, ix, tc, red, accum); break;
-        default: gemv_group<8, false>(C, ci, mg, L, it, ix, tc, red, accum); break;
+#endif
+        default: gemv_group<RMAX, false>(C, ci, mg, L, it, ix, tc, red, accum); break;
+#elif MK_GEMV_SET == 4
+        case 1: gemv_group<1, false>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        case 2: gemv_group<2, false>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        case 3:
+        case 4: gemv_group<4, false>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        default: gemv_group<RMAX, false>(C, ci, mg, L, it, ix, tc, red, accum); break;
+#else
+        default: gemv_group<RMAX, false>(C, ci, mg, L, it, ix, tc, red, accum); break;
+#endif
       }
-    } else {
+    } else if constexpr (MOE == 2) {
       switch (ci.nr) {
-        case 1: gemv_group<1, true>(C, ci, mg, L, it, ix, tc, red, accum); break;
-        case 2: gemv_group<2, true>(C, ci, mg, L, it, ix, tc, red, accum); break;
-        case 3: gemv_group<3, true>(C, ci, mg, L, it, ix, tc, red, accum); break;
-        case 4: gemv_group<4, true>(C, ci, mg, L, it, ix, tc, red, accum); break;
-        case 5: gemv_group<5, true>(C, ci, mg, L, it, ix, tc, red, accum); break;
-        case 6: gemv_group<6, true>(C, ci, mg, L, it, ix, tc, red, accum); break;
-        case 7: gemv_group<7, true>(C, ci, mg, L, it, ix, tc, red, accum); break;
-        default: gemv_group<8, true>(C, ci, mg, L, it, ix, tc, red, accum); break;
+#if MK_FP8_SET == 8
+        case 1: gemv_group_fp8<1>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        case 2: gemv_group_fp8<2>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        case 3: gemv_group_fp8<3>(C, ci, mg, L, it, ix, tc, red, accum); break;
+#if MK_RMAX > 4
+        case 4: gemv_group_fp8<4>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        case 5: gemv_group_fp8<5>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        case 6: gemv_group_fp8<6>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        case 7: gemv_group_fp8<7>(C, ci, mg, L, it, ix, tc, red, accum); break;
+#endif
+        default: gemv_group_fp8<RMAX>(C, ci, mg, L, it, ix, tc, red, accum); break;
+#elif MK_FP8_SET == 4
+        case 1: gemv_group_fp8<1>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        case 2: gemv_group_fp8<2>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        case 3:
+        case 4: gemv_group_fp8<4>(C, ci, mg, L, it, ix, tc, red, accum); break;
+        default: gemv_group_fp8<RMAX>(C, ci, mg, L, it, ix, tc, red, accum); break;
+#else
+        default: gemv_group_fp8<RMAX>(C, ci, mg, L, it, ix, tc, red, accum); break;
+#endif
       }
     }
     if (MOE && t.type == T_MOE_DOWN) pc.seg = pc.nseg - 1;  // the call took every segment
@@ -2804,7 +2871,7 @@ __device__ __noinline__ void mla_comb_task(const Ctx& C, const Task t) {
 // ---------------------------------------------------------------------------
 // consumer warps
 // ---------------------------------------------------------------------------
-template <bool MLA, bool MOE>
+template <bool MLA, int MOE>
 __device__ void consumer(const Ctx& C) {
   const Launch& P = *C.P;
   uint32_t it = 0, ix = 0, tc = 0;
@@ -2886,7 +2953,7 @@ __device__ void consumer(const Ctx& C) {
 // whole-step loop small.
 // 10 warps put 3 warps on two of the SM's four register-file partitions
 // (16K registers each), so a thread gets at most 168 registers.
-template <bool MLA, bool MOE>
+template <bool MLA, int MOE>
 __global__ void __launch_bounds__(NTHREADS, 1) mk_step_kernel(const __grid_constant__ Launch P) {
   extern __shared__ __align__(128) uint8_t smem[];
   Ctx C;
@@ -2974,9 +3041,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) mk_step_kernel(const __grid_const
 }
 
 // The host code (another translation unit) takes the kernel instances from here.
-const void* step_kernel_for(bool mla, bool moe) {
-  return mla ? (moe ? (const void*)mk_step_kernel<true, true> : (const void*)mk_step_kernel<true, false>)
-             : (moe ? (const void*)mk_step_kernel<false, true> : (const void*)mk_step_kernel<false, false>);
+const void* step_kernel_for(bool mla, bool moe, bool fp8) {
+  // MOE: 0 dense FFN, 1 MoE with bf16 experts, 2 MoE with fp8 experts
+  if (mla) {
+    if (!moe) return (const void*)mk_step_kernel<true, 0>;
+    return fp8 ? (const void*)mk_step_kernel<true, 2> : (const void*)mk_step_kernel<true, 1>;
+  }
+  if (!moe) return (const void*)mk_step_kernel<false, 0>;
+  return fp8 ? (const void*)mk_step_kernel<false, 2> : (const void*)mk_step_kernel<false, 1>;
 }
 
 }  // namespace MK_KNS
