@@ -20,7 +20,7 @@ FIELDS = 20
 EPI_NAMES = {0: "store", 1: "resid", 2: "swiglu", 3: "logits", 4: "swiglu_moe"}
 
 
-def record(model, kv, tokens, positions, logits, argmax, cap: int = 512):
+def record(model, kv, tokens, positions, logits, argmax, cap: int = 1024):
     import torch
     ctas, _, _ = model.launch_info()
     buf = torch.zeros((ctas, cap, FIELDS), dtype=torch.int64, device=tokens.device)
