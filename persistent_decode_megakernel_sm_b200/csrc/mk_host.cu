@@ -615,8 +615,11 @@ mk_status mk_create(const mk_model_desc* desc, int device, mk_handle** out) {
     const int hslots = d.n_routed ? d.n_shared + std::min(d.n_routed, MAXM * d.top_k) : 1;
     const int qkv_w = mla ? Hq * (hd + dr) + R + dr : (Hq + 2 * G) * hd;
     const int lat_w = mla ? Hq * R : 4;
+    // B_QL holds the absorbed queries as bf16 hi / lo attention fragments:
+    // 2 x (row tiles of 16 heads) x (R / 16) tiles x 512 B per query row
+    const int ql_w = mla ? ((Hq + 15) / 16) * 16 * R : 4;
     const int xf16_w = (d.n_routed && d.expert_fp8) ? H : 4;
-    const int widths[NBUF] = {H, qkv_w, Hq * hd, std::max(hw, 8), std::max(d.n_routed, 4), lat_w, lat_w, H, xf16_w};
+    const int widths[NBUF] = {H, qkv_w, Hq * hd, std::max(hw, 8), std::max(d.n_routed, 4), ql_w, lat_w, H, xf16_w};
     for (int b = 0; b < NBUF; ++b) {
       h->ld[b] = (widths[b] + 3) & ~3;
       const size_t rows = (b == B_H) ? (size_t)hslots * MB : (size_t)MB;

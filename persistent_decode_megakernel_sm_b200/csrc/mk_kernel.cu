@@ -237,6 +237,14 @@ __device__ __forceinline__ void split_f16(float a, float b, uint32_t& hi, uint32
 // col tile 64 bytes = for each quad lane tq, {hi(k 2tq, 2tq+1), hi(k 2tq+8,
 // 2tq+9), lo(..), lo(..)} (bf16 split, or f16 for fp8 weights), so that the
 // consuming GEMV copies them in and skips the conversion.
+__device__ __forceinline__ int frag_off(int r, int k, int KTn) {
+  // byte offset of element (row r, col k) in an A-fragment tile array [mt][KTn][32][8 x 2B]
+  const int mi = r >> 4, rr = r & 15, kt = k >> 4, kk = k & 15;
+  const int ln = (rr & 7) * 4 + ((kk & 7) >> 1);
+  const int e = (kk & 1) + 2 * (rr >> 3) + 4 * (kk >> 3);
+  return (((mi * KTn + kt) * 32 + ln) * 8 + e) * 2;
+}
+
 __device__ __forceinline__ bool frag_buf(int b) { return b == B_ATTN || b == B_H || b == B_OL; }
 __device__ __forceinline__ void st_frag(float* row, int k, float v, bool f16) {
   uint8_t* p = reinterpret_cast<uint8_t*>(row) + (size_t)(k >> 4) * 64 + ((k & 7) >> 1) * 16 + ((k >> 3) & 1) * 4 +
@@ -1629,7 +1637,7 @@ __device__ MK_FP8_GEMV_ATTR void gemv_group_fp8(const Ctx& C, ChunkIt& ci, const
   gemv_group<NR, true>(C, ci, m, L, it, ix, tc, red, accum);
 }
 
-template <int MOE>
+template <bool MLA, int MOE>
 __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix, uint32_t& tc) {
   const Launch& P = *C.P;
   const long long tpre = (MK_TRACE && P.trace && threadIdx.x == 0) ? clock64() : 0;
@@ -1790,7 +1798,25 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
           if (t.epi == EPI_STORE) {
             float* out = P.buf[t.out_buf];
             const int ld = P.ld[t.out_buf];
-            if (frag_buf(t.out_buf)) {  // feeds the next GEMV only (bf16 weights)
+            if (MLA && t.out_buf == B_QL) {
+              // absorbed queries: written as the latent attention's bf16 hi / lo
+              // A fragments (row = head, col = latent dim), scaled to log2 units
+              const int R = md.R, KWl = R >> 4, hiblk = ((md.Hq + 15) >> 4) * KWl * 512;
+              const float qs = rsqrtf((float)(md.d + md.dr)) * 1.4426950408889634f;
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int row = (q < 2) ? row0 : row1;
+                const int mm = (q & 1) ? m1 : m0;
+                if (row < m.rows && mm < M) {
+                  uint8_t* blk = reinterpret_cast<uint8_t*>(out + (size_t)mm * ld);
+                  const int off = frag_off(row / R, row - (row / R) * R, KWl);
+                  const float x = v[q] * qs;
+                  const __nv_bfloat16 hb = __float2bfloat16_rn(x);
+                  *reinterpret_cast<__nv_bfloat16*>(blk + off) = hb;
+                  *reinterpret_cast<__nv_bfloat16*>(blk + hiblk + off) = __float2bfloat16_rn(x - __bfloat162float(hb));
+                }
+              }
+            } else if (frag_buf(t.out_buf)) {  // feeds the next GEMV only (bf16 weights)
               if (row0 < m.rows) {
                 if (m0 < M) st_frag(out + (size_t)m0 * ld, row0, v[0], false);
                 if (m1 < M) st_frag(out + (size_t)m1 * ld, row0, v[1], false);
@@ -2001,13 +2027,6 @@ __device__ void lm_finish(const Ctx& C) {
 //   Q fragments (hi, lo): [mt][d/16][32 lanes][16 B]
 //   P fragments (hi, lo): [mt][64/16][32 lanes][16 B]
 //   smax: [2][NCW][48] fp32
-__device__ __forceinline__ int frag_off(int r, int k, int KTn) {
-  // byte offset of element (row r, col k) in an A-fragment tile array [mt][KTn][32][8 x 2B]
-  const int mi = r >> 4, rr = r & 15, kt = k >> 4, kk = k & 15;
-  const int ln = (rr & 7) * 4 + ((kk & 7) >> 1);
-  const int e = (kk & 1) + 2 * (rr >> 3) + 4 * (kk >> 3);
-  return (((mi * KTn + kt) * 32 + ln) * 8 + e) * 2;
-}
 
 // Each consumer warp owns 16 positions of every 64-position chunk (position
 // group w & 3) and half of the head dims (w >> 2), and runs its own online
@@ -2593,26 +2612,11 @@ __device__ MK_MLA_ATTR void mla_task(const Ctx& C, const Task t, uint32_t& it) {
   uint8_t* qhi = base + lay.qhi;
   uint8_t* qlo = base + lay.qlo;
 
-  // ---- queries: absorbed latent part, then the rotary part (RoPE at this row's
-  //      position), scaled to log2 units, as bf16 hi / lo A fragments ----
-  {
-    // 4 consecutive latent dims per thread and step, 4 steps in flight
-    const int R4 = R / 4, n4 = mt * 16 * R4;
-#pragma unroll 4
-    for (int e = tid; e < n4; e += NCT) {
-      const int r = e / R4, k = (e - r * R4) * 4;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r < Hq) v = __ldcg(reinterpret_cast<const float4*>(qa + (size_t)mrow * lda + (size_t)r * R + k));
-      const float xs[4] = {v.x * qscale, v.y * qscale, v.z * qscale, v.w * qscale};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const __nv_bfloat16 h = __float2bfloat16_rn(xs[q]);
-        *reinterpret_cast<__nv_bfloat16*>(qhi + frag_off(r, k + q, KW)) = h;
-        *reinterpret_cast<__nv_bfloat16*>(qlo + frag_off(r, k + q, KW)) =
-            __float2bfloat16_rn(xs[q] - __bfloat162float(h));
-      }
-    }
-  }
+  // ---- queries as bf16 hi / lo A fragments scaled to log2 units: first the
+  //      rotary part (RoPE at this row's position) and the step's own latent
+  //      rows, which need only the QKV projection (done: this CTA's absorbing
+  //      projection task waited for it), then, once every CTA's absorbing
+  //      projection is done, the absorbed latent part ----
   const int pos = T0 + qi;
   for (int e = tid; e < mt * 16 * half; e += NCT) {
     const int r = e / half, i = e - r * half;
@@ -2658,6 +2662,33 @@ __device__ MK_MLA_ATTR void mla_task(const Ctx& C, const Task t, uint32_t& it) {
           cache[R + i] = k0;
           cache[R + i + half] = k1;
         }
+      }
+    }
+  }
+  if (t.wait_ctr >= 0) wait_counter(C, t.wait_ctr, (uint32_t)t.wait_tgt);
+  {
+    // the latent part arrives in fragment layout (written by the absorbing
+    // projection's epilogue): per row tile, R / 16 contiguous tiles, hi then lo
+    const int KWl = R >> 4, tiles = mt * KWl, n16 = tiles * 32;  // 16-byte pieces per part
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(qa + (size_t)mrow * lda);
+    // every item of the step reads these same bytes at the same moment: each
+    // CTA starts at its own offset so the requests spread over the L2 slices
+    const int rot = (int)((blockIdx.x * 97u) % (unsigned)(2 * n16));
+#pragma unroll 4
+    for (int e0 = tid; e0 < 2 * n16; e0 += NCT) {
+      const int e = e0 + rot < 2 * n16 ? e0 + rot : e0 + rot - 2 * n16;
+      const int hl = e >= n16 ? 1 : 0, f = e - hl * n16;
+      const int tile = f >> 5, mi = tile / KWl, kt = tile - mi * KWl;
+      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(src + (size_t)hl * tiles * 512 + (size_t)f * 16));
+      *reinterpret_cast<uint4*>((hl ? qlo : qhi) + ((size_t)(mi * KW + kt) * 512) + (f & 31) * 16) = v;
+    }
+    if (Hq < mt * 16) {  // rows past the last head: zero (nothing writes them)
+      bar_consumers();
+      const __nv_bfloat16 z = __float2bfloat16_rn(0.f);
+      for (int e = tid; e < (mt * 16 - Hq) * R; e += NCT) {
+        const int r = Hq + e / R, k = e % R;
+        *reinterpret_cast<__nv_bfloat16*>(qhi + frag_off(r, k, KW)) = z;
+        *reinterpret_cast<__nv_bfloat16*>(qlo + frag_off(r, k, KW)) = z;
       }
     }
   }
@@ -2905,10 +2936,12 @@ __device__ void consumer(const Ctx& C) {
       C.ms->tr_route = 0;
       C.ms->tr_chunks = 0;
     }
-    if (t.wait_ctr >= 0) wait_counter(C, t.wait_ctr, (uint32_t)t.wait_tgt);
+    // a latent-attention item stages what it can before its dependency and
+    // waits inside
+    if (t.wait_ctr >= 0 && !(MLA && t.type == T_MLA)) wait_counter(C, t.wait_ctr, (uint32_t)t.wait_tgt);
     if (tr) td = globaltimer();
     if (gemv_like<MOE>(t)) {
-      gemv_task<MOE>(C, t, it, ix, tc);
+      gemv_task<MLA, MOE>(C, t, it, ix, tc);
     } else if (!MLA && t.type == T_ATTN) {
       attn_task(C, t, it);
     } else if (MLA && t.type == T_MLA) {
