@@ -308,6 +308,11 @@ struct Misc {
   long long tr_wf, tr_wx, tr_bytes, tr_route;
   long long tr_frag, tr_mma, tr_epi, tr_rel, tr_loop, tr_pre, tr_post, tr_sig;
   int tr_chunks;
+  // shared-memory copies, so that reading them costs no global (or spilled
+  // local) round trip: the model description (every role), and the task the
+  // consumer warps are on
+  Model cmodel;
+  Task ctask;
 };
 
 static_assert(sizeof(Misc) <= MISC_BYTES, "Misc must fit its shared-memory region");
@@ -1638,7 +1643,7 @@ __device__ MK_FP8_GEMV_ATTR void gemv_group_fp8(const Ctx& C, ChunkIt& ci, const
 }
 
 template <bool MLA, int MOE>
-__device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix, uint32_t& tc) {
+__device__ void gemv_task(const Ctx& C, const Task& t, uint32_t& it, uint32_t& ix, uint32_t& tc) {
   const Launch& P = *C.P;
   const long long tpre = (MK_TRACE && P.trace && threadIdx.x == 0) ? clock64() : 0;
   const Model& md = *C.md;
@@ -1939,7 +1944,7 @@ __device__ void gemv_task(const Ctx& C, const Task t, uint32_t& it, uint32_t& ix
 // Embedding gather: this CTA's column slice [c0, c1) of x[m] = E[token_m],
 // widened exactly to fp32, and its per-row sums of squares for the first
 // RMSNorm (fixed-order reduction).
-__device__ void embed_task(const Ctx& C, const Task t) {
+__device__ void embed_task(const Ctx& C, const Task& t) {
   const Launch& P = *C.P;
   const Model& md = *C.md;
   const int tid = threadIdx.x, M = P.M;
@@ -2138,7 +2143,7 @@ __device__ __forceinline__ void warp_att_chunk(WarpAtt<MT, NTD>& st, const uint8
 }
 
 template <int MT, int NTD>
-__device__ void attn_item(const Ctx& C, const Task t, uint32_t& it) {
+__device__ void attn_item(const Ctx& C, const Task& t, uint32_t& it) {
   const Launch& P = *C.P;
   const Model& md = *C.md;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -2430,7 +2435,7 @@ __device__ void attn_item(const Ctx& C, const Task t, uint32_t& it) {
 #else
 #define MK_MLA_ATTR __noinline__
 #endif
-__device__ MK_ATTN_ATTR void attn_task(const Ctx& C, const Task t, uint32_t& it) {
+__device__ MK_ATTN_ATTR void attn_task(const Ctx& C, const Task& t, uint32_t& it) {
   const Model& md = *C.md;
   const int nr = C.P->Q * (md.Hq / md.Hkv);
   const int mt = (nr + 15) >> 4;
@@ -2586,7 +2591,7 @@ __device__ __forceinline__ void mla_chunk(const Ctx& C, MlaState& st, const uint
   }
 }
 
-__device__ MK_MLA_ATTR void mla_task(const Ctx& C, const Task t, uint32_t& it) {
+__device__ MK_MLA_ATTR void mla_task(const Ctx& C, const Task& t, uint32_t& it) {
   const Launch& P = *C.P;
   const Model& md = *C.md;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -2795,7 +2800,7 @@ __device__ MK_MLA_ATTR void mla_task(const Ctx& C, const Task t, uint32_t& it) {
 // CTAs: CTA c owns a contiguous slice of the outputs [pair][head][R] and
 // forms each as sum_j exp2(M_j - M*) O_j / sum_j exp2(M_j - M*) L_j over the
 // pair's splits j (fixed order).
-__device__ __noinline__ void mla_comb_task(const Ctx& C, const Task t) {
+__device__ __noinline__ void mla_comb_task(const Ctx& C, const Task& t) {
   const Launch& P = *C.P;
   const Model& md = *C.md;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -2914,7 +2919,14 @@ __device__ void consumer(const Ctx& C) {
   const int beg = P.task_off[blockIdx.x], end = task_end_of(P);
   phase_dependency_wait(P);
   for (int ti = beg; ti < end; ++ti) {
-    const Task t = P.tasks[ti];
+    // the task record into shared memory, once every consumer thread is done
+    // with the previous one (not every task ends with a barrier: a task
+    // without a signal, or thread 0's trace record after it)
+    bar_consumers();
+    for (int i = threadIdx.x; i < (int)(sizeof(Task) / 4); i += NCT)
+      reinterpret_cast<uint32_t*>(&C.ms->ctask)[i] = __ldg(reinterpret_cast<const uint32_t*>(P.tasks + ti) + i);
+    bar_consumers();
+    const Task& t = C.ms->ctask;
     // while this task waits and runs: the next task's record into L1, and
     // the gain that this task's x updates are multiplied by for the next norm
     if (ti + 1 < end && threadIdx.x < 3) {
@@ -3017,6 +3029,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) mk_step_kernel(const __grid_const
     }
     return;
   }
+  for (int i = tid; i < (int)(sizeof(Model) / 4); i += NTHREADS)
+    reinterpret_cast<uint32_t*>(&C.ms->cmodel)[i] = __ldg(reinterpret_cast<const uint32_t*>(P.model) + i);
   if (tid == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(&C.ms->full[s], 1);
@@ -3041,6 +3055,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) mk_step_kernel(const __grid_const
   __syncthreads();
   tc_fence_after();
   C.tmem = C.ms->tmem_base;
+  C.md = &C.ms->cmodel;
 
   if ((tid >> 5) == WARP_WP) producer<MLA, MOE>(C);
   else if ((tid >> 5) == WARP_XP) xproducer<MOE>(C);

@@ -133,7 +133,7 @@ def main():
     assert m.sync_status() == 0
     s = summarize(tr)
     if a.out:
-        np.save(a.out, tr)
+        np.savez_compressed(a.out, tr=tr)
     print(json.dumps(s, indent=1))
 
 
