@@ -27,8 +27,8 @@ class Pair:
     """One model with two identical caches: one stepped by mk_decode_step,
     the other by mk_decode_step_noalloc."""
 
-    def __init__(self, name):
-        self.mc = mc = synth.preset(name, gain_sigma=0.1)
+    def __init__(self, name, **over):
+        self.mc = mc = synth.preset(name, gain_sigma=0.1, **over)
         self.m = gpu_model(mc)
         self.kv = {}
         for key in ("ref", "noalloc"):
@@ -60,11 +60,17 @@ class Pair:
         self.m.close()
 
 
-@pytest.mark.parametrize("name,B", [("tiny", 3), ("tiny_moe", 8)])
-def test_noalloc_matches_decode_step_two_calls(name, B):
+# a dense model whose projections have more row tiles than CTAs, with a
+# remainder (160 row tiles: some CTAs take one more)
+MID = dict(layers=2, hidden=2560, n_q_heads=20, n_kv_heads=4, head_dim=128, ffn=6912, vocab=8192, max_ctx=600)
+
+
+@pytest.mark.parametrize("name,B,over", [("tiny", 3, {}), ("tiny_moe", 8, {}), ("tiny", 3, MID)],
+                         ids=["tiny", "tiny_moe", "mid_dense"])
+def test_noalloc_matches_decode_step_two_calls(name, B, over):
     """Two calls in a row on one handle and batch size: bit-identical logits
     and greedy tokens to mk_decode_step."""
-    p = Pair(name)
+    p = Pair(name, **over)
     p.step_and_compare(B)
     p.step_and_compare(B)
     p.close()
