@@ -1149,7 +1149,7 @@ static void build_plan_host(const mk_handle* h, int S, int Q, std::vector<Task>&
       auto rr = split_rows(h->mats[ly.m_o].m.RT, ncta, rot);
       next_phase();
       for (int c = 0; c < ncta; ++c) {
-        Task t = gemv(l, ly.m_o, rr[c].first, rr[c].second, IN_BUF, B_ATTN, EPI_RESID, 0, 0, C(l, C_ATTN), n_pairs,
+        Task t = gemv(l, ly.m_o, rr[c].first, rr[c].second, IN_BUF, B_ATTN, EPI_RESID, 0, 0, C(l, C_ATTN), n_items,
                       C(l, C_O));
         t.ss_dst = 0;
         per[c].push_back(t);

@@ -2333,85 +2333,97 @@ __device__ void attn_item(const Ctx& C, const Task& t, uint32_t& it) {
     tA = t1;
   }
 
-  // ---- the last item of this (sequence, kv head) combines all splits ----
-  int lastc = 0;
+  // ---- the split combine, spread over the pair's items: each item counts
+  //      itself in (publishing its partial), waits until every item of its
+  //      (sequence, kv head) has, then merges a slice of the pair's outputs.
+  //      Eight threads per output (4 dims of one row), each over every 8th
+  //      split, with an online max; one round of loads, then quad-octet
+  //      shuffles.  Each item has at most one CTA's worth of work per layer
+  //      whenever a pair has more than one item (n_items = max(pairs, CTAs)),
+  //      so no item waits for an item queued behind it. ----
   if (tid == 0 && !C.ms->abort) {
-    const int pc = P.ctr_pair_base + t.layer * P.n_pairs + itm.pair;
-    const uint32_t old = atom_add_acqrel(P.ctr + pc, 1u);
-    lastc = (old == (uint32_t)itm.ns - 1) ? 1 : 0;
+    uint32_t* pc = P.ctr + P.ctr_pair_base + t.layer * P.n_pairs + itm.pair;
+    red_release_add(pc, 1u);
+    const uint64_t w0 = globaltimer();
+    uint32_t spins = 0;
+    while (ld_acquire(pc) < (uint32_t)itm.ns) {
+      if (C.ms->abort) break;
+      if (++spins >= 16) {
+        spins = 0;
+        if (global_abort(P)) { C.ms->abort = 1; break; }
+        if (globaltimer() - w0 > (uint64_t)P.timeout_ns) {
+          raise_error(P, C.ms, DERR_TIMEOUT, 0xE0000 | itm.pair);
+          break;
+        }
+      }
+    }
   }
+  bar_consumers();
   if (trc) {
     const long long t1 = clock64();
     C.ms->tr_post += t1 - tA;
     tA = t1;
   }
-  if (broadcast_from0(C, lastc)) {
+  {
     float* out = P.buf[B_ATTN];
     const int ldo = P.ld[B_ATTN];
-    // per (row, split) weight exp2(m_j - m*) / L*, one warp per row
-    float* wsh = reinterpret_cast<float*>(C.att);
-    const int ns = itm.ns;
-    for (int r = warp; r < nr; r += NCW) {
-      float mj[5], lj[5];
-      float mx = -INFINITY;
-#pragma unroll
-      for (int q = 0; q < 5; ++q) {
-        const int jj = lane + 32 * q;
-        mj[q] = -INFINITY;
-        lj[q] = 0.f;
-        if (jj < ns) {
-          const float* pp = P.att_part + ((size_t)(itm.first + jj) * rows_max + r) * dP + d;
-          mj[q] = __ldcg(pp);
-          lj[q] = __ldcg(pp + 1);
-        }
-        mx = fmaxf(mx, mj[q]);
-      }
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      float den = 0.f, w[5];
-#pragma unroll
-      for (int q = 0; q < 5; ++q) {
-        w[q] = (mj[q] == -INFINITY) ? 0.f : exp2f(mj[q] - mx);
-        den += w[q] * lj[q];
-      }
-      for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-#pragma unroll
-      for (int q = 0; q < 5; ++q) {
-        const int jj = lane + 32 * q;
-        if (jj < ns) wsh[r * 160 + jj] = w[q] / den;
-      }
-    }
-    bar_consumers();
-    // 4 consecutive dims per thread, the splits' loads 16 at a time in flight
-    const int d4 = d / 4;
-    for (int e = tid; e < nr * d4; e += NCT) {
-      const int r = e / d4, k = (e - r * d4) * 4;
-      const float* wr = wsh + r * 160;
-      const float* src = P.att_part + ((size_t)itm.first * rows_max + r) * dP + k;
-      const size_t js = (size_t)rows_max * dP;
+    const int ns = itm.ns, d4 = d / 4, U = nr * d4;
+    const int u0 = (int)(((int64_t)itm.j * U) / ns), u1 = (int)(((int64_t)(itm.j + 1) * U) / ns);
+    const int sub = tid & 7;
+    const size_t js = (size_t)rows_max * dP;
+    for (int base = u0; base < u1; base += NCT / 8) {
+      const int u = base + (tid >> 3);
+      const bool act = u < u1;
+      const int r = act ? u / d4 : 0, k = act ? (u - r * d4) * 4 : 0;
+      const float* src = P.att_part + ((size_t)itm.first * rows_max + r) * dP;
+      float mr = -INFINITY, den = 0.f;
       float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 16
-      for (int jj = 0; jj < ns; ++jj) {
-        const float w = wr[jj];
-        const float4 q = __ldcg(reinterpret_cast<const float4*>(src + jj * js));
-        num.x += w * q.x;
-        num.y += w * q.y;
-        num.z += w * q.z;
-        num.w += w * q.w;
+      if (act) {
+#pragma unroll 4
+        for (int jj = sub; jj < ns; jj += 8) {
+          const float2 ml = __ldcg(reinterpret_cast<const float2*>(src + jj * js + d));
+          const float4 o = __ldcg(reinterpret_cast<const float4*>(src + jj * js + k));
+          if (ml.x == -INFINITY) continue;
+          const float mn = fmaxf(mr, ml.x);
+          const float a = mr == -INFINITY ? 0.f : exp2f(mr - mn), b = exp2f(ml.x - mn);
+          den = den * a + b * ml.y;
+          num.x = num.x * a + b * o.x;
+          num.y = num.y * a + b * o.y;
+          num.z = num.z * a + b * o.z;
+          num.w = num.w * a + b * o.w;
+          mr = mn;
+        }
       }
-      const int qi = r / gh, hh = r % gh;
-      float* orow = out + (size_t)(s * Q + qi) * ldo;
-      const int kc = (kvh * gh + hh) * d + k;
-      st_frag(orow, kc, num.x, false);
-      st_frag(orow, kc + 1, num.y, false);
-      st_frag(orow, kc + 2, num.z, false);
-      st_frag(orow, kc + 3, num.w, false);
+#pragma unroll
+      for (int off = 1; off < 8; off <<= 1) {
+        const float mo = __shfl_xor_sync(0xffffffffu, mr, off);
+        const float dno = __shfl_xor_sync(0xffffffffu, den, off);
+        const float nx = __shfl_xor_sync(0xffffffffu, num.x, off), ny = __shfl_xor_sync(0xffffffffu, num.y, off);
+        const float nz = __shfl_xor_sync(0xffffffffu, num.z, off), nw = __shfl_xor_sync(0xffffffffu, num.w, off);
+        const float mn = fmaxf(mr, mo);
+        const float a = mr == -INFINITY ? 0.f : exp2f(mr - mn), b = mo == -INFINITY ? 0.f : exp2f(mo - mn);
+        den = den * a + dno * b;
+        num.x = num.x * a + nx * b;
+        num.y = num.y * a + ny * b;
+        num.z = num.z * a + nz * b;
+        num.w = num.w * a + nw * b;
+        mr = mn;
+      }
+      if (act && sub == 0) {
+        const float inv = 1.f / den;
+        const int qi = r / gh, hh = r % gh;
+        float* orow = out + (size_t)(s * Q + qi) * ldo;
+        const int kc = (kvh * gh + hh) * d + k;
+        st_frag(orow, kc, num.x * inv, false);
+        st_frag(orow, kc + 1, num.y * inv, false);
+        st_frag(orow, kc + 2, num.z * inv, false);
+        st_frag(orow, kc + 3, num.w * inv, false);
+      }
     }
-    bar_consumers();
-    if (tid == 0 && !C.ms->abort) {
-      red_release_add(P.ctr + t.layer * P.ctr_layer_stride + C_ATTN, 1u);
-    }
-    if (trc) C.ms->tr_epi += clock64() - tA;
   }
+  bar_consumers();
+  if (tid == 0 && !C.ms->abort) red_release_add(P.ctr + t.layer * P.ctr_layer_stride + C_ATTN, 1u);
+  if (trc) C.ms->tr_epi += clock64() - tA;
 }
 
 
