@@ -313,6 +313,9 @@ struct Misc {
   // consumer warps are on
   Model cmodel;
   Task ctask;
+  // latent attention: bulk copy of the absorbed queries (completion, uses so far)
+  uint64_t qbar;
+  uint32_t qpar;
 };
 
 static_assert(sizeof(Misc) <= MISC_BYTES, "Misc must fit its shared-memory region");
@@ -2685,22 +2688,42 @@ __device__ MK_MLA_ATTR void mla_task(const Ctx& C, const Task& t, uint32_t& it) 
   if (t.wait_ctr >= 0) wait_counter(C, t.wait_ctr, (uint32_t)t.wait_tgt);
   {
     // the latent part arrives in fragment layout (written by the absorbing
-    // projection's epilogue): per row tile, R / 16 contiguous tiles, hi then lo
-    const int KWl = R >> 4, tiles = mt * KWl, n16 = tiles * 32;  // 16-byte pieces per part
+    // projection's epilogue): per row tile, R / 16 contiguous tiles, hi then
+    // lo; four bulk copies (every item of the step reads these same bytes at
+    // once, which the copy engine serves far better than per-thread loads)
+    const int KWl = R >> 4, tiles = mt * KWl;
     const uint8_t* src = reinterpret_cast<const uint8_t*>(qa + (size_t)mrow * lda);
-    // every item of the step reads these same bytes at the same moment: each
-    // CTA starts at its own offset so the requests spread over the L2 slices
-    const int rot = (int)((blockIdx.x * 97u) % (unsigned)(2 * n16));
-#pragma unroll 4
-    for (int e0 = tid; e0 < 2 * n16; e0 += NCT) {
-      const int e = e0 + rot < 2 * n16 ? e0 + rot : e0 + rot - 2 * n16;
-      const int hl = e >= n16 ? 1 : 0, f = e - hl * n16;
-      const int tile = f >> 5, mi = tile / KWl, kt = tile - mi * KWl;
-      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(src + (size_t)hl * tiles * 512 + (size_t)f * 16));
-      *reinterpret_cast<uint4*>((hl ? qlo : qhi) + ((size_t)(mi * KW + kt) * 512) + (f & 31) * 16) = v;
+    uint64_t* qb = &C.ms->qbar;
+    const uint32_t par = C.ms->qpar & 1u;
+    if (tid == 0 && !C.ms->abort) {
+      // earlier generic-proxy accesses of this scratch precede the copies
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive_expect_tx(qb, (uint32_t)(2 * tiles * 512));
+      const uint64_t pol = policy_evict_last();
+      for (int hl = 0; hl < 2; ++hl)
+        for (int mi = 0; mi < mt; ++mi)
+          bulk_g2s((hl ? qlo : qhi) + (size_t)mi * KW * 512, src + ((size_t)hl * tiles + (size_t)mi * KWl) * 512,
+                   (uint32_t)(KWl * 512), qb, pol);
     }
+    if (lane == 0 && !C.ms->abort) {
+      uint32_t spins = 0;
+      uint64_t w0 = 0;
+      while (!mbar_try_wait(qb, par)) {
+        if (++spins >= 64) {
+          spins = 0;
+          if (C.ms->abort) break;
+          const uint64_t now = globaltimer();
+          if (w0 == 0) w0 = now;
+          else if (now - w0 > (uint64_t)P.timeout_ns * 2) {
+            raise_error(P, C.ms, DERR_TIMEOUT, 0x5A000);
+            break;
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (!C.ms->abort) while (!mbar_try_wait(qb, par)) {}
     if (Hq < mt * 16) {  // rows past the last head: zero (nothing writes them)
-      bar_consumers();
       const __nv_bfloat16 z = __float2bfloat16_rn(0.f);
       for (int e = tid; e < (mt * 16 - Hq) * R; e += NCT) {
         const int r = Hq + e / R, k = e % R;
@@ -2710,6 +2733,7 @@ __device__ MK_MLA_ATTR void mla_task(const Ctx& C, const Task& t, uint32_t& it) 
     }
   }
   bar_consumers();
+  if (tid == 0) C.ms->qpar += 1;  // every thread has read it; read again after the next item's dependency barrier
   if (trc) {
     const long long t1 = clock64();
     C.ms->tr_pre += t1 - tA;
@@ -3056,6 +3080,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) mk_step_kernel(const __grid_const
       mbar_init(&C.ms->xfull[s], 2);  // the copies' expect-tx arrival + the scales
       mbar_init(&C.ms->xempty[s], NCW);
     }
+    mbar_init(&C.ms->qbar, 1);
+    C.ms->qpar = 0;
     C.ms->abort = 0;
     C.ms->route_layer = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
