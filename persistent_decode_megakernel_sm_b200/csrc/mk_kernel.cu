@@ -2585,15 +2585,19 @@ __device__ __forceinline__ void mla_chunk(const Ctx& C, MlaState& st, const uint
         al[mi] = lds128(plo + ((mi * 4 + ks) * 32 + lane) * 16);
       }
     }
+    // B fragments of C by transposed 8x8 matrix loads; lanes 0-15 address
+    // the 16 positions of the k-step (clamped to the valid rows: the rows
+    // past n_valid are masked below), 16-byte aligned since the pitch is
+    const uint8_t* vrow = rows + (size_t)min(ks * 16 + (lane & 15), n_valid - 1) * pitch;
 #pragma unroll
     for (int jn = 0; jn < 8; ++jn) {
       if (jn < NTW) {
-        const uint8_t* vc = rows + ((warp * NTW + jn) * 8 + g) * 2;
-        const uint32_t v0 = pk < n_valid ? lds16(vc + (size_t)pk * pitch) : 0u;
-        const uint32_t v1 = pk + 1 < n_valid ? lds16(vc + (size_t)(pk + 1) * pitch) : 0u;
-        const uint32_t v8 = pk + 8 < n_valid ? lds16(vc + (size_t)(pk + 8) * pitch) : 0u;
-        const uint32_t v9 = pk + 9 < n_valid ? lds16(vc + (size_t)(pk + 9) * pitch) : 0u;
-        const uint32_t b0 = v0 | (v1 << 16), b1 = v8 | (v9 << 16);
+        uint32_t b0, b1;
+        ldsm_x2_trans(vrow + (size_t)((warp * NTW + jn) * 8) * 2, b0, b1);
+        if (pk >= n_valid) b0 = 0u;
+        else if (pk + 1 >= n_valid) b0 &= 0xFFFFu;
+        if (pk + 8 >= n_valid) b1 = 0u;
+        else if (pk + 9 >= n_valid) b1 &= 0xFFFFu;
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi) {
           if (mi < mt) {
