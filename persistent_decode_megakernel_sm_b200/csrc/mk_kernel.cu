@@ -1460,21 +1460,33 @@ __device__ MK_GEMV_ATTR void gemv_group(const Ctx& Cr, ChunkIt& cir, const Mat& 
   const bool xok = g < (pk ? 2 * L.M : L.M);  // other columns are zero
   long long tc0 = 0, tl0 = L.trc ? clock64() : 0;
   const ChunkIt ci0 = ci;
+  // fp8: the block scales of the group's rows (every column block) staged in
+  // shared memory; read through L1 they miss for every chunk (the L1 beside a
+  // 227 KB carve-out holds little).  A call over several K segments (the MoE
+  // down projection: one per expert) stages every segment's rows in one pass
+  // when they fit (one global round trip instead of one per segment), else
+  // one segment at a time in two tables alternating by segment.
+  const int rb0 = FP8 ? (m0.gu ? (ci0.g0 >> 4) : (ci0.g0 >> 3)) : 0;
+  const int nrb = FP8 ? (m0.gu ? ((ci0.g0 + nrr - 1) >> 4) : ((ci0.g0 + nrr - 1) >> 3)) - rb0 + 1 : 1;
+  const int sc_per = nrb * m0.nbc;
+  const bool sc_all = FP8 && L.nseg > 1 && !m0.gu && L.nseg * sc_per <= 2 * FP8_SCALE_TAB;
+  float* const sc_base = reinterpret_cast<float*>(C.att + FP8_SCALE_OFF);
+  if (sc_all) {
+    for (int i = threadIdx.x; i < L.nseg * sc_per; i += NCT) {
+      const int sg = i / sc_per, j = i - sg * sc_per;
+      const float* scs = sg < L.NS ? L.sc_sh + (size_t)sg * L.ss_sh : L.sc_rt + (size_t)L.ex[sg - L.NS] * L.ss_rt;
+      sc_base[i] = __ldg(scs + (size_t)rb0 * m0.nbc + j);
+    }
+    bar_consumers();
+  }
   for (int seg = 0; seg < L.nseg; ++seg) {
   if (seg > 0) ci = ci0;
   Mat m = m0;
   if (FP8 && L.nseg > 1)
     m.scales = seg < L.NS ? L.sc_sh + (size_t)seg * L.ss_sh : L.sc_rt + (size_t)L.ex[seg - L.NS] * L.ss_rt;
-  // fp8: the block scales of the group's rows (every column block) staged in
-  // shared memory once per segment, two tables alternating by segment; read
-  // through L1 they miss for every chunk (the L1 beside a 227 KB carve-out
-  // holds little)
-  const float* sct = reinterpret_cast<const float*>(C.att + FP8_SCALE_OFF) + (seg & 1) * FP8_SCALE_TAB;
-  int rb0 = 0, nrb = 1;
-  if (FP8) {
-    rb0 = m.gu ? (ci0.g0 >> 4) : (ci0.g0 >> 3);
-    nrb = (m.gu ? ((ci0.g0 + nrr - 1) >> 4) : ((ci0.g0 + nrr - 1) >> 3)) - rb0 + 1;
-    const int per = nrb * m.nbc, n = (m.gu ? 2 : 1) * per;
+  const float* sct = sc_all ? sc_base + seg * sc_per : sc_base + (seg & 1) * FP8_SCALE_TAB;
+  if (FP8 && !sc_all) {
+    const int per = sc_per, n = (m.gu ? 2 : 1) * per;
     float* dst = const_cast<float*>(sct);
     for (int i = threadIdx.x; i < n; i += NCT) {
       const int hf = i >= per ? 1 : 0;
