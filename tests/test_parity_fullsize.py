@@ -58,6 +58,15 @@ def _run(mc, B, context, steps=2):
     m.close()
 
 
+def test_more_kv_pairs_than_ctas():
+    """32 kv heads at B = 8: 256 (sequence, kv head) pairs, more than CTAs, so
+    every pair is one attention item (no split to combine) and some CTAs run
+    two items of a layer."""
+    mc = synth.preset("tiny", layers=2, hidden=2048, n_q_heads=32, n_kv_heads=32, head_dim=64, ffn=4096,
+                      vocab=4096, max_ctx=300, context=256, gain_sigma=0.1)
+    _run(mc, 8, 256)
+
+
 def test_mid_dense_split_phases():
     """Hidden 2560 (160 row tiles over the CTAs), 2 layers, B = 3."""
     mc = synth.preset("tiny", layers=2, hidden=2560, n_q_heads=20, n_kv_heads=4, head_dim=128, ffn=6912,
