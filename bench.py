@@ -49,7 +49,7 @@ def parse():
     ap.add_argument("--oracle-steps", type=int, default=3,
                     help="full-depth oracle steps timed for cpu_baseline")
     ap.add_argument("--traffic", type=float, default=None,
-                    help="DRAM bytes per launch of the kernel from an ncu capture of this build (null if none)")
+                    help="DRAM bytes per launch of the kernel from an ncu capture of the current kernel sources (null if none)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=16)
     return ap.parse_args()
