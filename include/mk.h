@@ -268,7 +268,9 @@ mk_status mk_set_router_trace(mk_handle* h, int32_t* idx_dev, float* w_dev);
  * writes 20 int64 into trace_dev[cta][task][20]:
  *   0-2   %globaltimer (ns) at task start, when its dependency was met, at its end;
  *   3-4   SM cycles spent waiting for weight tiles, for activation slices;
- *   5-7   chunks consumed, layer, type * 16 + epilogue;
+ *   5-7   chunks consumed, layer (+ the task's phase << 16: the tasks between
+ *         two dependency points, one kernel of the multi-kernel path),
+ *         type * 16 + epilogue;
  *   8-11  cycles in fragment preparation, mma, epilogue, release;
  *   12-15 (record 0) producer cycles blocked on a full ring, chunks issued,
  *         first and last issue time (ns); (record 1) producer cycles and ns
