@@ -589,8 +589,11 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{args.config} decode, B=1, context {mc.context}", "model": args.config,
-                   "global_batch": 1, "seq_len": mc.context, "parallelism": "none (host cores)"},
+        "config": {"workload": f"{args.config} decode, B=1, context {mc.context} (+ positions advancing)",
+                   "model": args.config, "global_batch": 1, "seq_len": mc.context,
+                   "parallelism": "none (host cores)",
+                   "context": "a seeded synthetic cache (the oracle's own fill; the step's cost does not depend on "
+                              "the cached values)"},
         "cpu_baseline": cpu,
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
