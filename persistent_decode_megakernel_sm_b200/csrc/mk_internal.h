@@ -55,7 +55,13 @@ constexpr int SMEM_BYTES = NSTAGE * STAGE_BYTES + XSLOTS * XSLOT_BYTES + ATT_BYT
 #endif
 constexpr int RMAX = MK_RMAX;                // row tiles per chunk (4 or 8)
 static_assert(RMAX == 4 || RMAX == 8, "row tiles per chunk: 4 or 8");
-constexpr int CPW = 8;                       // col tiles per warp per chunk
+// Most col tiles per warp in one GEMV chunk; the ring stage and the
+// activation window cap a chunk too.  16 lets a one-row group at B = 1 fill
+// a whole 64 KB stage (128 bf16 col tiles) instead of half of one.
+#ifndef MK_CPW
+#define MK_CPW 16
+#endif
+constexpr int CPW = MK_CPW;
 constexpr int MAXM = 8;                      // activation rows per step (S * Q)
 static_assert(2 * ATT_CT * 128 * 2 <= STAGE_BYTES, "a K/V chunk of head_dim 128 fills at most one stage");
 constexpr int TRACE_FIELDS = 20;             // int64 per traced task
