@@ -46,6 +46,10 @@ def summarize(tr: np.ndarray, sm_clock_mhz: float = 0.0) -> dict:
     valid = tr[:, :, 2] > 0
     t0 = tr[:, :, 0][valid].min()
     t1 = tr[:, :, 2][valid].max()
+    # a prefetch record is an L2 request the weight producer issued ahead of
+    # a task (no consumer work, no phase of its own): counted, kept out of the
+    # phases and of the CTAs' busy time
+    work = valid & (tr[:, :, 7] // 16 != 5)
     phases = collections.defaultdict(lambda: dict(n=0, dep_us=0.0, run_us=0.0, wf_us=0.0, wx_us=0.0, chunks=0,
                                                   frag_us=0.0, mma_us=0.0, epi_us=0.0, rel_us=0.0,
                                                   loop_us=0.0, pre_us=0.0, post_us=0.0, sig_us=0.0))
@@ -55,7 +59,7 @@ def summarize(tr: np.ndarray, sm_clock_mhz: float = 0.0) -> dict:
     span = collections.defaultdict(lambda: [None, None])
     for c in range(tr.shape[0]):
         for k in range(tr.shape[1]):
-            if not valid[c, k]:
+            if not work[c, k]:
                 continue
             tb, td, te, wf, wx, ch, layer, te16 = tr[c, k, :8]
             fr, mm, ep, rl = tr[c, k, 8:12]
@@ -89,16 +93,16 @@ def summarize(tr: np.ndarray, sm_clock_mhz: float = 0.0) -> dict:
         out["phases"][name] = {k: (v / ctas if k.endswith("_us") else v) for k, v in p.items()}
         out["phases"][name]["per_cta_us_note"] = "times summed over the CTA's tasks, averaged over CTAs"
         # wall time: per phase, the first CTA's dependency met to the last
-        # CTA's end, summed over the step's phases of this kind (a prefetch
-        # task belongs to the phase before the task it serves)
+        # CTA's end, summed over the step's phases of this kind
         out["phases"][name]["wall_us"] = sum((e - b) / 1e3 for (ph, nm), (b, e) in span.items() if nm == name)
     out["compute_fraction"] = busy / ctas / step_us
     # SM idle between tasks: the part of the step a CTA spends outside task
     # bodies (waiting for a task's dependency, or done before the step ends)
-    run_ns = np.where(valid, tr[:, :, 2] - tr[:, :, 1], 0).sum(axis=1).astype(np.float64)
+    run_ns = np.where(work, tr[:, :, 2] - tr[:, :, 1], 0).sum(axis=1).astype(np.float64)
     idle = 1.0 - run_ns / float(t1 - t0)
     out["idle_between_tasks_fraction"] = float(idle.mean())
     out["idle_between_tasks_fraction_max_cta"] = float(idle.max())
+    out["prefetch_requests"] = int((valid & ~work).sum())
     out["producer_blocked_us_per_cta"] = float(tr[:, 0, 12].mean()) / sm_clock_mhz
     out["producer_chunks_per_cta"] = float(tr[:, 0, 13].mean())
     out["producer_span_us"] = float((tr[:, 0, 15] - tr[:, 0, 14]).mean()) / 1e3
