@@ -112,18 +112,32 @@ class Clocks:
         q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        self.start = 0
         try:
             self.p = subprocess.Popen(["nvidia-smi", f"--id={index}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
-                                       "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+                                       "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.p = None
+            return
+        # the sampler takes a moment to start: wait for its first sample (it
+        # is started before the warm-up steps, so that it runs through them)
+        t0 = time.time()
+        while time.time() - t0 < 3.0 and self.p.poll() is None:
+            if os.path.getsize(self.f.name) > 0:
+                break
+            time.sleep(0.01)
+
+    def mark(self):
+        """Start of the timed region: only the samples written after this count."""
+        if self.p is not None:
+            self.start = os.path.getsize(self.f.name)
 
     def stop(self):
         if self.p is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.p.terminate()
         self.p.wait()
-        self.f.seek(0)
+        self.f.seek(self.start)
         sm, mx, reasons = [], None, set()
         for line in self.f:
             parts = [x.strip() for x in line.split(",")]
@@ -201,6 +215,7 @@ def run_ours(args, rank, world, local_rank):
         am = [torch.zeros(B, dtype=torch.int32, device=dev) for _ in range(total)]
         logits = torch.empty((B, mc.vocab), dtype=torch.float32, device=dev)
         restore()
+        ck = Clocks(local_rank) if clocks else None
         cur = toks
         for i in range(warmup):
             model.decode_step(cur, pos[i], kv, logits, am[i], stream)
@@ -210,8 +225,9 @@ def run_ours(args, rank, world, local_rank):
         if world > 1:
             torch.distributed.barrier()
         torch.cuda.synchronize()
-        ck = Clocks(local_rank) if clocks else None
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+        if ck:
+            ck.mark()
         ev[0].record(stream)
         for i in range(steps):
             model.decode_step(cur, pos[warmup + i], kv, logits, am[warmup + i], stream)
